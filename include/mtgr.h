@@ -1,0 +1,246 @@
+/*
+ * mtgr.h — C ABI of libmtgr.so: the forward pass of the MTGR HSTU block and
+ * block stack over user-aggregated, jagged token sequences, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "MTGR: Industrial-Scale Generative Recommendation Framework in
+ * Meituan" (summary page, section "Method"; fun-rec "MTGR: Hybrid Paradigm
+ * Modeling", 7.3.1 data organisation, 7.3.3 Group Layer Normalization,
+ * 7.3.4 Dynamic Masking). Each user request is one sample
+ * D = [U, S, R, [C,I]_1..K]; users are packed back to back; one HSTU block is
+ *   X~ = GroupLN_1(X);  Q|K|V|U = X~ W_qkvu^T
+ *   G  = (silu(Q K^T) (.) M / N) V (.) U          (per head, no 1/sqrt(dh))
+ *   X  <- MLP(GroupLN_2(G)) + X,   MLP = Linear -> SiLU -> Linear
+ * with the three-rule mask M and N the user's total token count.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named d_* are DEVICE pointers (CUDA global memory) on the
+ *    current device; the caller owns and frees all memory. The library never
+ *    allocates or frees device memory and keeps no state between calls other
+ *    than cached device attributes.
+ *  - All work is enqueued asynchronously on the given stream (a cudaStream_t;
+ *    NULL is the legacy default stream). Entry points do not synchronise.
+ *  - Return value: MTGR_OK or an error code for errors the host can see
+ *    (bad arguments, unsupported shapes, launch failures). Errors that depend
+ *    on device data (inconsistent lengths, capacity overflow, an internal
+ *    wait that timed out) are written to the caller's device status word
+ *    (int32, 0 = ok; the first error wins) and must be read after the stream
+ *    is synchronised. No entry point prints, traps or throws.
+ *  - Token layout: user b occupies rows [user_off[b], user_off[b+1]) in the
+ *    order U, S, R, C. Group ids: 0 = U, 1 = S, 2 = R, 3 = C.
+ *  - Timestamps are int64, one per token; entries of U tokens are ignored.
+ *  - Thread safety: calls on different streams may run concurrently; calls
+ *    sharing a workspace must be ordered by the caller.
+ */
+#ifndef MTGR_H
+#define MTGR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MTGR_API __attribute__((visibility("default")))
+
+/* status codes */
+#define MTGR_OK 0
+#define MTGR_ERR_INVALID_ARG 1        /* null pointer, bad size or inconsistent argument */
+#define MTGR_ERR_CUDA 2               /* a CUDA runtime call or kernel launch failed */
+#define MTGR_ERR_UNSUPPORTED 3        /* dtype / head size / architecture not supported */
+#define MTGR_ERR_CAPACITY 4           /* an output or workspace buffer is too small */
+#define MTGR_ERR_TIMEOUT 5            /* device: an internal wait exceeded its limit */
+#define MTGR_ERR_DEVICE_VALIDATION 6  /* device: lengths negative or not summing to T */
+
+/* element types */
+#define MTGR_F32 0
+#define MTGR_BF16 1
+#define MTGR_F16 2
+
+/* canonical mask-metadata tile (rows x columns of the user-relative grid) */
+#define MTGR_TILE_M 128
+#define MTGR_TILE_N 128
+
+typedef void* mtgr_stream_t; /* a cudaStream_t */
+
+/* Human-readable name of a status code. Never returns NULL. */
+MTGR_API const char* mtgr_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+MTGR_API int mtgr_version(void);
+
+/*
+ * Jagged packing (summary page, Method: D = [U, S, R, [C,I]_1..K]; chenhuiyu
+ * blog: sequence packing keeps users from attending to one another).
+ *   d_lens     [B][4] int32: N_U, N_S, N_R, K of each user (read)
+ *   T          total token count the caller expects (= sum of d_lens)
+ *   d_seg_off  [4B+1] int32: row where U, S, R, C of each user start; last = T
+ *   d_user_off [B+1] int32
+ *   d_group_id [T] int8
+ *   d_status   device int32 status word (MTGR_ERR_DEVICE_VALIDATION when a
+ *              length is negative or the lengths do not sum to T)
+ * B = 0 is valid (writes seg_off[0] = user_off[0] = 0).
+ */
+MTGR_API int mtgr_pack_offsets(int32_t B, const int32_t* d_lens, int32_t T, int32_t* d_seg_off,
+                               int32_t* d_user_off, int8_t* d_group_id, int32_t* d_status,
+                               mtgr_stream_t stream);
+
+/* Bytes of device workspace mtgr_build_mask_meta needs. */
+MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_capacity);
+
+/*
+ * Mask metadata: the canonical list of non-empty 128x128 tiles of every
+ * user's mask M (fun-rec 7.3.4 Rules 1-3; summary page, Method, mask rules).
+ *   Rule 1: keys in U and S are visible to every query of the user.
+ *   Rule 2: a key j in R is visible to query i iff t_j < t_i or j == i
+ *           (U queries carry no time and never see R keys).
+ *   Rule 3: a candidate key is visible only to itself.
+ * Tiles lie on the user-relative grid (q-tile qt covers user rows
+ * [128 qt, 128 qt + 128)); only cells inside the user count. A tile is EMPTY
+ * (omitted) if no cell is visible, FULL if every cell is, PARTIAL otherwise.
+ *   d_seg_off    [4B+1] from mtgr_pack_offsets
+ *   d_ts         [T] int64 timestamps
+ *   q_capacity   rows available in d_qtile_desc/d_order (>= sum ceil(N_b/128))
+ *   kt_capacity  >= max_b ceil(N_b/128)
+ *   e_capacity   entries available in d_entries
+ *   d_qtile_desc [q_capacity][2] int32: (user, qt), user-major, qt ascending
+ *   d_row_ptr    [q_capacity+1] int32: CSR row pointers into d_entries
+ *   d_entries    [e_capacity] int32: (kt << 1) | partial, kt ascending per row
+ *   d_order      [q_capacity] int32: q-tile indices by descending entry count,
+ *                ties by ascending index (the attention's work order)
+ *   d_counts     [3] int64: Q (q-tiles), E (entries), visible (query,key) pairs
+ *   d_ws, ws_bytes  workspace of mtgr_mask_meta_workspace_bytes() bytes
+ *   d_status     device status word (MTGR_ERR_CAPACITY if Q, E or a user's
+ *                tile count exceed the capacities; outputs are then invalid)
+ */
+MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int64_t* d_ts,
+                                  int32_t q_capacity, int32_t kt_capacity, int32_t e_capacity,
+                                  int32_t* d_qtile_desc, int32_t* d_row_ptr, int32_t* d_entries,
+                                  int32_t* d_order, int64_t* d_counts, void* d_ws,
+                                  size_t ws_bytes, int32_t* d_status, mtgr_stream_t stream);
+
+/*
+ * Group-Layer Normalization (fun-rec 7.3.3, the GLN formula):
+ *   y_i = (x_i - mean_i) / sqrt(var_i + eps) * gamma[g(i)] + beta[g(i)]
+ * with mean and biased variance of token i over its d features and g(i) the
+ * token's group id.
+ *   x_dtype / y_dtype: (MTGR_F32, MTGR_F32), (MTGR_F32, MTGR_BF16) or
+ *                      (MTGR_BF16, MTGR_BF16); x, y [T][d] row-major
+ *   d_group_id [T] int8 in [0, G)
+ *   d_gamma, d_beta [G][d] float32
+ * d must be a multiple of 8 and at most 8192.
+ */
+MTGR_API int mtgr_group_layernorm(int32_t T, int32_t d, int32_t x_dtype, const void* d_x,
+                                  const int8_t* d_group_id, int32_t G, const float* d_gamma,
+                                  const float* d_beta, float eps, int32_t y_dtype, void* d_y,
+                                  mtgr_stream_t stream);
+
+/* A packed batch plus its mask metadata (all device pointers). */
+typedef struct mtgr_batch {
+  int32_t B;                  /* users */
+  int32_t T;                  /* tokens */
+  int32_t q_capacity;         /* rows of qtile_desc/order (launch bound, >= Q) */
+  int32_t kt_capacity;        /* >= max_b ceil(N_b/128) */
+  const int32_t* seg_off;     /* [4B+1] */
+  const int32_t* user_off;    /* [B+1] */
+  const int8_t* group_id;     /* [T] */
+  const int64_t* ts;          /* [T] */
+  const int32_t* qtile_desc;  /* [q_capacity][2] */
+  const int32_t* row_ptr;     /* [q_capacity+1] */
+  const int32_t* entries;     /* [E] */
+  const int32_t* order;       /* [q_capacity] */
+  const int64_t* counts;      /* [3] Q, E, visible pairs */
+  const float* norm;          /* optional [B] normaliser override; NULL = user length */
+  int32_t* status;            /* device status word */
+} mtgr_batch;
+
+/*
+ * Masked pointwise SiLU attention with the 1/N normaliser and the U gate
+ * (summary page, Method: V~ = silu(K^T Q)/(N_U+N_S+N_R+N_I) M V; the gate
+ * V~ (.) U of the block update):
+ *   G[i, h] = (1/N_b) sum_j silu(q_i,h . k_j,h) M_ij v_j,h  (.)  u_i,h
+ *   d_qkvu   [T][4d] row-major, column blocks Q | K | V | U, head h at
+ *            columns [h dh, (h+1) dh) of each block; qkvu_dtype MTGR_BF16 or
+ *            MTGR_F16 (tensor-core path, dh = 64) or MTGR_F32 (exact SIMT path,
+ *            dh in {32, 64})
+ *   d_g      [T][d] output, out_dtype MTGR_F32 or MTGR_BF16 (MTGR_F32 only for
+ *            the f32 path)
+ * The mask is evaluated tile by tile from the metadata and the timestamps and
+ * is never stored. d = H * dh, d % 64 == 0 for the tensor-core path.
+ */
+MTGR_API int mtgr_hstu_attention_fwd(const mtgr_batch* batch, int32_t d, int32_t H,
+                                     int32_t qkvu_dtype, const void* d_qkvu, int32_t out_dtype,
+                                     void* d_g, mtgr_stream_t stream);
+
+/* Parameters of one HSTU block (device pointers; PyTorch Linear [out][in] layout). */
+typedef struct mtgr_block_params {
+  int32_t d;                  /* d_model */
+  int32_t H;                  /* heads, dh = d / H */
+  int32_t d_ff;               /* MLP hidden width */
+  int32_t dtype;              /* MTGR_BF16: bf16 weights, tensor cores; MTGR_F32: f32 SIMT */
+  float eps;                  /* GroupLN epsilon */
+  int32_t reserved;
+  const float* gln1_gamma;    /* [4][d] */
+  const float* gln1_beta;     /* [4][d] */
+  const float* gln2_gamma;    /* [4][d] */
+  const float* gln2_beta;     /* [4][d] */
+  const void* w_qkvu;         /* [4d][d] (dtype) */
+  const void* w1;             /* [d_ff][d] (dtype) */
+  const void* w2;             /* [d][d_ff] (dtype) */
+  const float* b_qkvu;        /* [4d] or NULL */
+  const float* b1;            /* [d_ff] or NULL */
+  const float* b2;            /* [d] or NULL */
+} mtgr_block_params;
+
+/* Workspace bytes of mtgr_hstu_block_fwd for T tokens (0 on invalid params). */
+MTGR_API size_t mtgr_block_workspace_bytes(int32_t T, const mtgr_block_params* p);
+
+/*
+ * One HSTU block (summary page, Method, the update equations). The residual
+ * stream is float32 on both paths: d_x_in, d_x_out [T][d] float32 (distinct
+ * buffers). dtype MTGR_BF16: GroupLN outputs and GEMM operands in bf16,
+ * Q|K|V|U and the attention probabilities in fp16, fp32 accumulation
+ * (d % 64 == 0, dh == 64, d_ff % 64 == 0). dtype MTGR_F32: every step in fp32
+ * on CUDA cores (dh in {32, 64}).
+ */
+MTGR_API int mtgr_hstu_block_fwd(const mtgr_block_params* p, const mtgr_batch* batch,
+                                 const float* d_x_in, float* d_x_out, void* d_ws,
+                                 size_t ws_bytes, mtgr_stream_t stream);
+
+/* Workspace bytes of mtgr_stack_fwd (0 on invalid params). */
+MTGR_API size_t mtgr_stack_workspace_bytes(int32_t T, const mtgr_block_params* layers, int32_t L);
+
+/*
+ * L stacked HSTU blocks (summary page, Method: the L-layer stack). The mask
+ * metadata in *batch is shared by all layers. d_x_in and d_x_out [T][d]
+ * float32, distinct. All layers must share d, H and dtype.
+ */
+MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mtgr_batch* batch,
+                            const float* d_x_in, float* d_x_out, void* d_ws, size_t ws_bytes,
+                            mtgr_stream_t stream);
+
+/*
+ * Dense GEMM with the block's epilogues, exposed for testing:
+ *   out[m][n] = epi( sum_k a[m][k] * b[n][k] + bias[n] )
+ *   epi = MTGR_EPI_NONE (out dtype MTGR_F16/MTGR_BF16/MTGR_F32),
+ *         MTGR_EPI_SILU (out MTGR_BF16/MTGR_F32),
+ *         MTGR_EPI_RESID (adds d_resid[m][n] float32; out MTGR_F32)
+ *   ab_dtype MTGR_BF16: tcgen05 tensor cores (K % 64 == 0, N % 32 == 0);
+ *   ab_dtype MTGR_F32: CUDA cores. a [M][K], b [N][K] row-major; bias may
+ *   be NULL. q_cols > 0 multiplies output columns [0, q_cols) by 0.5 before
+ *   the epilogue conversion (used to pre-halve Q for the attention).
+ */
+#define MTGR_EPI_NONE 0
+#define MTGR_EPI_SILU 1
+#define MTGR_EPI_RESID 2
+MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const void* d_a,
+                       const void* d_b, const float* d_bias, int32_t epi, const float* d_resid,
+                       int32_t q_cols, int32_t out_dtype, void* d_out, int32_t* d_status,
+                       mtgr_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MTGR_H */
