@@ -1,0 +1,41 @@
+"""MTGR HSTU-block forward for NVIDIA B200 (sm_100a).
+
+The forward pass of the HSTU block and block stack of "MTGR: Industrial-Scale
+Generative Recommendation Framework in Meituan" over user-aggregated, jagged
+token sequences, implemented in libmtgr.so (hand-written CUDA for sm_100a)
+behind a C ABI (include/mtgr.h). This package is the Python binding.
+"""
+
+from ._lib import (  # noqa: F401
+    MTGR_BF16,
+    MTGR_EPI_NONE,
+    MTGR_EPI_RESID,
+    MTGR_EPI_SILU,
+    MTGR_F16,
+    MTGR_F32,
+    MTGRError,
+    load,
+    mtgr_block_workspace_bytes,
+    mtgr_build_mask_meta,
+    mtgr_gemm,
+    mtgr_group_layernorm,
+    mtgr_hstu_attention_fwd,
+    mtgr_hstu_block_fwd,
+    mtgr_mask_meta_workspace_bytes,
+    mtgr_pack_offsets,
+    mtgr_stack_fwd,
+    mtgr_stack_workspace_bytes,
+    mtgr_version,
+    status_string,
+)
+from .api import (  # noqa: F401
+    BlockWeights,
+    PackedBatch,
+    capacities,
+    gemm,
+    group_layernorm,
+    hstu_attention,
+    hstu_block_forward,
+    hstu_stack_forward,
+    stack_workspace,
+)

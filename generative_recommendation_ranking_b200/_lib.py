@@ -1,0 +1,231 @@
+"""ctypes binding of libmtgr.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and takes
+torch tensors (device tensors for the d_* arguments) plus an optional
+torch.cuda.Stream. Non-zero host status raises MTGRError. Loading fails loudly
+when the shared library is missing: there is no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmtgr.so")
+
+MTGR_OK = 0
+MTGR_ERR_INVALID_ARG = 1
+MTGR_ERR_CUDA = 2
+MTGR_ERR_UNSUPPORTED = 3
+MTGR_ERR_CAPACITY = 4
+MTGR_ERR_TIMEOUT = 5
+MTGR_ERR_DEVICE_VALIDATION = 6
+
+MTGR_F32 = 0
+MTGR_BF16 = 1
+MTGR_F16 = 2
+
+MTGR_EPI_NONE = 0
+MTGR_EPI_SILU = 1
+MTGR_EPI_RESID = 2
+
+TILE_M = 128
+TILE_N = 128
+
+_TORCH_DTYPE = {MTGR_F32: torch.float32, MTGR_BF16: torch.bfloat16, MTGR_F16: torch.float16}
+_MTGR_DTYPE = {v: k for k, v in _TORCH_DTYPE.items()}
+
+
+class MTGRError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+        self.status = status
+
+
+c_i32, c_i64, c_size, c_vp, c_float = (ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                                       ctypes.c_void_p, ctypes.c_float)
+
+
+class MtgrBatch(ctypes.Structure):
+    _fields_ = [("B", c_i32), ("T", c_i32), ("q_capacity", c_i32), ("kt_capacity", c_i32),
+                ("seg_off", c_vp), ("user_off", c_vp), ("group_id", c_vp), ("ts", c_vp),
+                ("qtile_desc", c_vp), ("row_ptr", c_vp), ("entries", c_vp), ("order", c_vp),
+                ("counts", c_vp), ("norm", c_vp), ("status", c_vp)]
+
+
+class MtgrBlockParams(ctypes.Structure):
+    _fields_ = [("d", c_i32), ("H", c_i32), ("d_ff", c_i32), ("dtype", c_i32), ("eps", c_float),
+                ("reserved", c_i32), ("gln1_gamma", c_vp), ("gln1_beta", c_vp),
+                ("gln2_gamma", c_vp), ("gln2_beta", c_vp), ("w_qkvu", c_vp), ("w1", c_vp),
+                ("w2", c_vp), ("b_qkvu", c_vp), ("b1", c_vp), ("b2", c_vp)]
+
+
+_SIGNATURES = {
+    "mtgr_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mtgr_version": (ctypes.c_int, []),
+    "mtgr_pack_offsets": (ctypes.c_int, [c_i32, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "mtgr_mask_meta_workspace_bytes": (c_size, [c_i32, c_i32]),
+    "mtgr_build_mask_meta": (ctypes.c_int, [c_i32, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp,
+                                            c_vp, c_vp, c_vp, c_vp, c_size, c_vp, c_vp]),
+    "mtgr_group_layernorm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp,
+                                            c_float, c_i32, c_vp, c_vp]),
+    "mtgr_hstu_attention_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_i32, c_i32, c_i32,
+                                               c_vp, c_i32, c_vp, c_vp]),
+    "mtgr_block_workspace_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams)]),
+    "mtgr_hstu_block_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams),
+                                           ctypes.POINTER(MtgrBatch), c_vp, c_vp, c_vp, c_size,
+                                           c_vp]),
+    "mtgr_stack_workspace_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams), c_i32]),
+    "mtgr_stack_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams), c_i32,
+                                      ctypes.POINTER(MtgrBatch), c_vp, c_vp, c_vp, c_size, c_vp]),
+    "mtgr_gemm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32,
+                                 c_i32, c_vp, c_vp, c_vp]),
+    "mtgr_timer_create": (c_vp, []),
+    "mtgr_timer_destroy": (None, [c_vp]),
+    "mtgr_timer_attach": (ctypes.c_int, [c_vp]),
+    "mtgr_timer_read": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_double),
+                                       ctypes.POINTER(ctypes.c_int64)]),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libmtgr.so (built in-tree). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python -m generative_recommendation_ranking_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().mtgr_status_string(int(status)).decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MTGR_OK:
+        raise MTGRError(fn, rc)
+
+
+def dtype_code(t: torch.dtype) -> int:
+    return _MTGR_DTYPE[t]
+
+
+def mtgr_version() -> int:
+    return load().mtgr_version()
+
+
+def mtgr_pack_offsets(B, d_lens, T, d_seg_off, d_user_off, d_group_id, d_status, stream=None):
+    _check("mtgr_pack_offsets", load().mtgr_pack_offsets(
+        B, _ptr(d_lens), T, _ptr(d_seg_off), _ptr(d_user_off), _ptr(d_group_id), _ptr(d_status),
+        _stream(stream)))
+
+
+def mtgr_mask_meta_workspace_bytes(q_capacity: int, kt_capacity: int) -> int:
+    return load().mtgr_mask_meta_workspace_bytes(q_capacity, kt_capacity)
+
+
+def mtgr_build_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, d_qtile_desc,
+                         d_row_ptr, d_entries, d_order, d_counts, d_ws, d_status, stream=None):
+    ws_bytes = 0 if d_ws is None else d_ws.numel() * d_ws.element_size()
+    _check("mtgr_build_mask_meta", load().mtgr_build_mask_meta(
+        B, _ptr(d_seg_off), _ptr(d_ts), q_capacity, kt_capacity, e_capacity, _ptr(d_qtile_desc),
+        _ptr(d_row_ptr), _ptr(d_entries), _ptr(d_order), _ptr(d_counts), _ptr(d_ws), ws_bytes,
+        _ptr(d_status), _stream(stream)))
+
+
+def mtgr_group_layernorm(T, d, d_x, d_group_id, G, d_gamma, d_beta, eps, d_y, stream=None):
+    _check("mtgr_group_layernorm", load().mtgr_group_layernorm(
+        T, d, dtype_code(d_x.dtype), _ptr(d_x), _ptr(d_group_id), G, _ptr(d_gamma), _ptr(d_beta),
+        float(eps), dtype_code(d_y.dtype), _ptr(d_y), _stream(stream)))
+
+
+def mtgr_hstu_attention_fwd(batch: MtgrBatch, d, H, d_qkvu, d_g, stream=None):
+    _check("mtgr_hstu_attention_fwd", load().mtgr_hstu_attention_fwd(
+        ctypes.byref(batch), d, H, dtype_code(d_qkvu.dtype), _ptr(d_qkvu),
+        dtype_code(d_g.dtype), _ptr(d_g), _stream(stream)))
+
+
+def mtgr_block_workspace_bytes(T: int, p: MtgrBlockParams) -> int:
+    return load().mtgr_block_workspace_bytes(T, ctypes.byref(p))
+
+
+def mtgr_hstu_block_fwd(p: MtgrBlockParams, batch: MtgrBatch, d_x_in, d_x_out, d_ws, stream=None):
+    _check("mtgr_hstu_block_fwd", load().mtgr_hstu_block_fwd(
+        ctypes.byref(p), ctypes.byref(batch), _ptr(d_x_in), _ptr(d_x_out), _ptr(d_ws),
+        d_ws.numel() * d_ws.element_size(), _stream(stream)))
+
+
+def mtgr_stack_workspace_bytes(T: int, layers) -> int:
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    return load().mtgr_stack_workspace_bytes(T, arr, len(layers))
+
+
+def mtgr_stack_fwd(layers, batch: MtgrBatch, d_x_in, d_x_out, d_ws, stream=None):
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    _check("mtgr_stack_fwd", load().mtgr_stack_fwd(
+        arr, len(layers), ctypes.byref(batch), _ptr(d_x_in), _ptr(d_x_out), _ptr(d_ws),
+        d_ws.numel() * d_ws.element_size(), _stream(stream)))
+
+
+TIMER_CLASSES = ("pack", "mask_meta", "gln", "gemm_qkvu", "attention", "gemm_mlp1", "gemm_mlp2")
+
+
+class Timer:
+    """Per-kernel-class CUDA-event timer (mtgr_timer_*). While attached to the
+    calling thread, every library launch is bracketed by events and counted."""
+
+    def __init__(self):
+        self.h = load().mtgr_timer_create()
+        if not self.h:
+            raise MemoryError("mtgr_timer_create failed")
+
+    def attach(self):
+        load().mtgr_timer_attach(self.h)
+
+    def detach(self):
+        load().mtgr_timer_attach(None)
+
+    def read(self) -> dict:
+        n = len(TIMER_CLASSES)
+        ms = (ctypes.c_double * n)()
+        cnt = (ctypes.c_int64 * n)()
+        _check("mtgr_timer_read", load().mtgr_timer_read(self.h, ms, cnt))
+        return {c: (ms[i], cnt[i]) for i, c in enumerate(TIMER_CLASSES)}
+
+    def __del__(self):
+        h, self.h = getattr(self, "h", None), None
+        if h and _lib is not None:
+            _lib.mtgr_timer_destroy(h)
+
+
+def mtgr_gemm(d_a, d_b, d_bias, epi, d_resid, q_cols, d_out, d_status, stream=None):
+    M, K = d_a.shape
+    N = d_b.shape[0]
+    _check("mtgr_gemm", load().mtgr_gemm(
+        M, N, K, dtype_code(d_a.dtype), _ptr(d_a), _ptr(d_b), _ptr(d_bias), epi, _ptr(d_resid),
+        q_cols, dtype_code(d_out.dtype), _ptr(d_out), _ptr(d_status), _stream(stream)))

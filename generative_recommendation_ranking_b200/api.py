@@ -1,0 +1,182 @@
+"""User-facing API over libmtgr.so: device buffers (through PyTorch) plus calls
+into the C ABI. Every step of the forward runs in the library's CUDA kernels;
+this module only sizes and allocates buffers and marshals arguments.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import (MTGR_BF16, MTGR_F16, MTGR_F32, MtgrBatch, MtgrBlockParams, TILE_M, TILE_N)
+
+EPS = 1e-5
+
+
+def capacities(lens: np.ndarray) -> tuple:
+    """Host-side buffer sizes of the mask metadata for per-user lengths [B,4]:
+    q-tiles, largest per-user k-tile count, and an upper bound on entries."""
+    n = np.asarray(lens, dtype=np.int64).reshape(-1, 4).sum(axis=1)
+    nq = (n + TILE_M - 1) // TILE_M
+    nk = (n + TILE_N - 1) // TILE_N
+    q_cap = int(nq.sum())
+    kt_cap = int(nk.max()) if nk.size else 0
+    e_cap = int((nq * nk).sum())
+    return q_cap, kt_cap, e_cap
+
+
+class PackedBatch:
+    """A packed batch of users on one device with its mask metadata.
+
+    ``lens`` int [B,4] (N_U, N_S, N_R, K per user; host) and ``ts`` int64 [T]
+    (host array or device tensor). ``norm`` optionally overrides each user's
+    normaliser N. Runs mtgr_pack_offsets and mtgr_build_mask_meta on
+    ``stream``.
+    """
+
+    def __init__(self, lens, ts, device="cuda", norm=None, stream=None):
+        lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(-1, 4))
+        self.lens = lens
+        self.B = int(lens.shape[0])
+        self.T = int(lens.sum())
+        self.device = torch.device(device)
+        dev = self.device
+        self.q_cap, self.kt_cap, self.e_cap = capacities(lens)
+        self.d_lens = torch.from_numpy(lens).to(dev, non_blocking=True)
+        self.d_ts = (ts if isinstance(ts, torch.Tensor) else torch.from_numpy(
+            np.ascontiguousarray(ts, dtype=np.int64))).to(dev, dtype=torch.int64, non_blocking=True)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.seg_off = torch.empty(4 * self.B + 1, **i32)
+        self.user_off = torch.empty(self.B + 1, **i32)
+        self.group_id = torch.empty(max(self.T, 1), dtype=torch.int8, device=dev)
+        self.status = torch.zeros(1, **i32)
+        self.qtile_desc = torch.empty(max(self.q_cap, 1), 2, **i32)
+        self.row_ptr = torch.empty(self.q_cap + 1, **i32)
+        self.entries = torch.empty(max(self.e_cap, 1), **i32)
+        self.order = torch.empty(max(self.q_cap, 1), **i32)
+        self.counts = torch.zeros(3, dtype=torch.int64, device=dev)
+        ws_bytes = _lib.mtgr_mask_meta_workspace_bytes(self.q_cap, self.kt_cap)
+        self.meta_ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        self.norm = None
+        if norm is not None:
+            self.norm = torch.as_tensor(np.asarray(norm, dtype=np.float32)).to(dev)
+        _lib.mtgr_pack_offsets(self.B, self.d_lens, self.T, self.seg_off, self.user_off,
+                               self.group_id, self.status, stream)
+        _lib.mtgr_build_mask_meta(self.B, self.seg_off, self.d_ts, self.q_cap, self.kt_cap,
+                                  self.e_cap, self.qtile_desc, self.row_ptr, self.entries,
+                                  self.order, self.counts, self.meta_ws, self.status, stream)
+        self.c = MtgrBatch(
+            B=self.B, T=self.T, q_capacity=self.q_cap, kt_capacity=self.kt_cap,
+            seg_off=self.seg_off.data_ptr(), user_off=self.user_off.data_ptr(),
+            group_id=self.group_id.data_ptr(), ts=self.d_ts.data_ptr(),
+            qtile_desc=self.qtile_desc.data_ptr(), row_ptr=self.row_ptr.data_ptr(),
+            entries=self.entries.data_ptr(), order=self.order.data_ptr(),
+            counts=self.counts.data_ptr(),
+            norm=None if self.norm is None else self.norm.data_ptr(),
+            status=self.status.data_ptr())
+
+    def check(self) -> None:
+        """Synchronise and raise if a kernel recorded a device-side error."""
+        torch.cuda.synchronize(self.device)
+        st = int(self.status.item())
+        if st != 0:
+            raise _lib.MTGRError("device status", st)
+
+    def meta(self) -> dict:
+        """Mask metadata copied to the host (for inspection and tests)."""
+        torch.cuda.synchronize(self.device)
+        Q, E, V = (int(v) for v in self.counts.cpu())
+        return dict(
+            seg_off=self.seg_off.cpu().numpy(), user_off=self.user_off.cpu().numpy(),
+            group_id=self.group_id[:self.T].cpu().numpy(),
+            qtile_desc=self.qtile_desc[:Q].cpu().numpy(),
+            row_ptr=self.row_ptr[:Q + 1].cpu().numpy(), entries=self.entries[:E].cpu().numpy(),
+            order=self.order[:Q].cpu().numpy(), visible_pairs=V, Q=Q, E=E)
+
+
+class BlockWeights:
+    """One HSTU block's parameters on the device (PyTorch Linear layouts).
+
+    ``dtype`` "bf16" keeps W_qkvu, W1, W2 in bf16 (tensor-core path); "f32"
+    keeps everything in fp32 (CUDA-core path). GroupLN parameters are fp32.
+    """
+
+    def __init__(self, p: dict, H: int, dtype: str = "bf16", device="cuda", eps: float = EPS):
+        dev = torch.device(device)
+        wdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+
+        def f32(a):
+            return None if a is None else torch.as_tensor(np.asarray(a, np.float32)).to(dev).contiguous()
+
+        def w(a):
+            return torch.as_tensor(np.asarray(a, np.float32)).to(dev).to(wdt).contiguous()
+
+        self.t = dict(gln1_gamma=f32(p["gln1_gamma"]), gln1_beta=f32(p["gln1_beta"]),
+                      gln2_gamma=f32(p["gln2_gamma"]), gln2_beta=f32(p["gln2_beta"]),
+                      w_qkvu=w(p["w_qkvu"]), w1=w(p["w1"]), w2=w(p["w2"]),
+                      b_qkvu=f32(p.get("b_qkvu")), b1=f32(p.get("b1")), b2=f32(p.get("b2")))
+        d = self.t["w_qkvu"].shape[1]
+        d_ff = self.t["w1"].shape[0]
+        ptr = {k: (None if v is None else v.data_ptr()) for k, v in self.t.items()}
+        self.c = MtgrBlockParams(d=d, H=H, d_ff=d_ff,
+                                 dtype=MTGR_BF16 if dtype == "bf16" else MTGR_F32, eps=eps,
+                                 reserved=0, **ptr)
+        self.d, self.H, self.d_ff, self.dtype = d, H, d_ff, dtype
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def hstu_block_forward(w: BlockWeights, batch: PackedBatch, x: torch.Tensor, out=None, ws=None,
+                       stream=None) -> torch.Tensor:
+    """One HSTU block: x [T, d] float32 on the device -> new [T, d] float32."""
+    if out is None:
+        out = torch.empty_like(x)
+    need = _lib.mtgr_block_workspace_bytes(batch.T, w.c)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x.device)
+    _lib.mtgr_hstu_block_fwd(w.c, batch.c, x, out, ws, stream)
+    return out
+
+
+def stack_workspace(layers, batch: PackedBatch) -> torch.Tensor:
+    return _ws(_lib.mtgr_stack_workspace_bytes(batch.T, [l.c for l in layers]), batch.device)
+
+
+def hstu_stack_forward(layers, batch: PackedBatch, x: torch.Tensor, out=None, ws=None,
+                       stream=None) -> torch.Tensor:
+    """L stacked HSTU blocks sharing the batch's mask metadata."""
+    if out is None:
+        out = torch.empty_like(x)
+    if ws is None:
+        ws = stack_workspace(layers, batch)
+    _lib.mtgr_stack_fwd([l.c for l in layers], batch.c, x, out, ws, stream)
+    return out
+
+
+def hstu_attention(batch: PackedBatch, qkvu: torch.Tensor, d: int, H: int,
+                   out_dtype=torch.float32, stream=None) -> torch.Tensor:
+    """G = (silu(Q K^T) (.) M / N) V (.) U for qkvu [T, 4d] (bf16, f16 or f32)."""
+    g = torch.empty(batch.T, d, dtype=out_dtype, device=qkvu.device)
+    _lib.mtgr_hstu_attention_fwd(batch.c, d, H, qkvu, g, stream)
+    return g
+
+
+def group_layernorm(x: torch.Tensor, group_id: torch.Tensor, gamma: torch.Tensor,
+                    beta: torch.Tensor, eps: float = EPS, out_dtype=None, stream=None):
+    T, d = x.shape
+    y = torch.empty(T, d, dtype=out_dtype or x.dtype, device=x.device)
+    _lib.mtgr_group_layernorm(T, d, x, group_id, gamma.shape[0], gamma, beta, eps, y, stream)
+    return y
+
+
+def gemm(a: torch.Tensor, b: torch.Tensor, bias=None, epi: int = 0, resid=None, q_cols: int = 0,
+         out_dtype=torch.float32, status=None, stream=None) -> torch.Tensor:
+    """out = epi(a b^T + bias); a [M, K], b [N, K]."""
+    out = torch.empty(a.shape[0], b.shape[0], dtype=out_dtype, device=a.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=a.device)
+    _lib.mtgr_gemm(a, b, bias, epi, resid, q_cols, out, status, stream)
+    return out

@@ -1,0 +1,360 @@
+// extern "C" entry points of libmtgr.so: argument validation, workspace
+// layout and the launch sequence of the HSTU block and stack.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "timer.h"
+
+namespace mtgr {
+int launch_pack(int32_t B, const int32_t* lens, int32_t T, int32_t* seg_off, int32_t* user_off,
+                int8_t* group_id, int32_t* status, cudaStream_t s);
+size_t mask_meta_ws_bytes(int32_t q_cap, int32_t kt_cap);
+int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32_t q_cap,
+                     int32_t kt_cap, int32_t e_cap, int32_t* qtile_desc, int32_t* row_ptr,
+                     int32_t* entries, int32_t* order, int64_t* counts, void* ws, int32_t* status,
+                     cudaStream_t s);
+int launch_gln(int32_t T, int32_t d, int32_t x_dtype, const void* x, const int8_t* gid, int32_t G,
+               const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
+               cudaStream_t s);
+int launch_gemm_f32(int M, int N, int K, const float* a, const float* b, const float* bias, int epi,
+                    const float* resid, int q_cols, int32_t out_dtype, void* out, cudaStream_t s);
+int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
+                   const float* resid, int q_cols, int32_t out_dtype, void* out, int32_t* status,
+                   cudaStream_t s);
+int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu, float* g,
+                    cudaStream_t s);
+int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
+                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s);
+}  // namespace mtgr
+
+using namespace mtgr;
+
+namespace {
+
+constexpr int32_t kMaxKtCapacity = 4096;  // users up to 4096 * 128 tokens
+constexpr int32_t kMaxD = 8192;
+
+inline cudaStream_t as_stream(mtgr_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool batch_ok(const mtgr_batch* b) {
+  if (b == nullptr) return false;
+  if (b->B < 0 || b->T < 0 || b->q_capacity < 0 || b->kt_capacity < 0) return false;
+  if (b->kt_capacity > kMaxKtCapacity) return false;
+  if (b->seg_off == nullptr || b->user_off == nullptr || b->ts == nullptr) return false;
+  if (b->q_capacity > 0 && (b->qtile_desc == nullptr || b->row_ptr == nullptr ||
+                            b->entries == nullptr || b->order == nullptr))
+    return false;
+  if (b->counts == nullptr || b->status == nullptr) return false;
+  return true;
+}
+
+// Validates a layer's parameters; returns MTGR_OK or the error code.
+int params_check(const mtgr_block_params* p) {
+  if (p == nullptr) return MTGR_ERR_INVALID_ARG;
+  if (p->d <= 0 || p->H <= 0 || p->d_ff <= 0 || p->d > kMaxD || p->d % p->H != 0)
+    return MTGR_ERR_INVALID_ARG;
+  if (!(p->eps >= 0.0f)) return MTGR_ERR_INVALID_ARG;
+  if (p->gln1_gamma == nullptr || p->gln1_beta == nullptr || p->gln2_gamma == nullptr ||
+      p->gln2_beta == nullptr || p->w_qkvu == nullptr || p->w1 == nullptr || p->w2 == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  const int dh = p->d / p->H;
+  if (p->dtype == MTGR_BF16) {
+    if (dh != 64 || p->d % 64 != 0 || p->d_ff % 64 != 0) return MTGR_ERR_UNSUPPORTED;
+    if (!aligned16(p->w_qkvu) || !aligned16(p->w1) || !aligned16(p->w2)) return MTGR_ERR_INVALID_ARG;
+  } else if (p->dtype == MTGR_F32) {
+    if (dh != 32 && dh != 64) return MTGR_ERR_UNSUPPORTED;
+    if (p->d % 8 != 0) return MTGR_ERR_UNSUPPORTED;
+  } else {
+    return MTGR_ERR_UNSUPPORTED;
+  }
+  return MTGR_OK;
+}
+
+struct BlockWs {
+  void* xt;    // GroupLN output [T][d]
+  void* qkvu;  // [T][4d]
+  void* g;     // attention output [T][d]
+  void* h;     // MLP hidden [T][d_ff]
+  size_t bytes;
+};
+
+BlockWs block_ws_layout(int32_t T, const mtgr_block_params* p, void* base) {
+  const size_t e = p->dtype == MTGR_BF16 ? 2 : 4;
+  const size_t t = (size_t)T;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  BlockWs w;
+  size_t off = 0;
+  w.xt = b + off;   off += align_up(t * p->d * e, 256);
+  w.qkvu = b + off; off += align_up(t * 4 * p->d * e, 256);
+  w.g = b + off;    off += align_up(t * p->d * e, 256);
+  w.h = b + off;    off += align_up(t * p->d_ff * e, 256);
+  w.bytes = off;
+  return w;
+}
+
+int block_fwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_in, float* x_out,
+              void* ws, cudaStream_t s) {
+  const int32_t T = bt->T, d = p->d, H = p->H, dff = p->d_ff;
+  if (T == 0) return MTGR_OK;
+  BlockWs w = block_ws_layout(T, p, ws);
+  int rc;
+  if (p->dtype == MTGR_BF16) {
+    {
+      TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+      if ((rc = launch_gln(T, d, MTGR_F32, x_in, bt->group_id, 4, p->gln1_gamma, p->gln1_beta,
+                           p->eps, MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
+    }
+    {
+      // Q|K|V|U in f16 with the Q columns halved (silu's tanh form takes s/2)
+      TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
+      if ((rc = launch_gemm_tc(T, 4 * d, d, w.xt, p->w_qkvu, p->b_qkvu, MTGR_EPI_NONE, nullptr, d,
+                               MTGR_F16, w.qkvu, bt->status, s)) != MTGR_OK) return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
+      if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, w.qkvu, MTGR_BF16, w.g, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+      if ((rc = launch_gln(T, d, MTGR_BF16, w.g, bt->group_id, 4, p->gln2_gamma, p->gln2_beta,
+                           p->eps, MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
+      if ((rc = launch_gemm_tc(T, dff, d, w.xt, p->w1, p->b1, MTGR_EPI_SILU, nullptr, 0, MTGR_BF16,
+                               w.h, bt->status, s)) != MTGR_OK) return rc;
+    }
+    TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
+    return launch_gemm_tc(T, d, dff, w.h, p->w2, p->b2, MTGR_EPI_RESID, x_in, 0, MTGR_F32, x_out,
+                          bt->status, s);
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(T, d, MTGR_F32, x_in, bt->group_id, 4, p->gln1_gamma, p->gln1_beta, p->eps,
+                         MTGR_F32, w.xt, s)) != MTGR_OK) return rc;
+  }
+  const float* xt = static_cast<const float*>(w.xt);
+  {
+    TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
+    if ((rc = launch_gemm_f32(T, 4 * d, d, xt, static_cast<const float*>(p->w_qkvu), p->b_qkvu,
+                              MTGR_EPI_NONE, nullptr, 0, MTGR_F32, w.qkvu, s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
+    if ((rc = launch_attn_f32(bt, d, H, static_cast<const float*>(w.qkvu),
+                              static_cast<float*>(w.g), s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(T, d, MTGR_F32, w.g, bt->group_id, 4, p->gln2_gamma, p->gln2_beta, p->eps,
+                         MTGR_F32, w.xt, s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
+    if ((rc = launch_gemm_f32(T, dff, d, xt, static_cast<const float*>(p->w1), p->b1, MTGR_EPI_SILU,
+                              nullptr, 0, MTGR_F32, w.h, s)) != MTGR_OK)
+      return rc;
+  }
+  TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
+  return launch_gemm_f32(T, d, dff, static_cast<const float*>(w.h),
+                         static_cast<const float*>(p->w2), p->b2, MTGR_EPI_RESID, x_in, 0,
+                         MTGR_F32, x_out, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+MTGR_API const char* mtgr_status_string(int status) {
+  switch (status) {
+    case MTGR_OK: return "ok";
+    case MTGR_ERR_INVALID_ARG: return "invalid argument";
+    case MTGR_ERR_CUDA: return "CUDA error";
+    case MTGR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MTGR_ERR_CAPACITY: return "capacity exceeded";
+    case MTGR_ERR_TIMEOUT: return "device wait timed out";
+    case MTGR_ERR_DEVICE_VALIDATION: return "device-side validation failed";
+    default: return "unknown status";
+  }
+}
+
+MTGR_API int mtgr_version(void) { return 100; }
+
+MTGR_API int mtgr_pack_offsets(int32_t B, const int32_t* d_lens, int32_t T, int32_t* d_seg_off,
+                               int32_t* d_user_off, int8_t* d_group_id, int32_t* d_status,
+                               mtgr_stream_t stream) {
+  if (B < 0 || T < 0) return MTGR_ERR_INVALID_ARG;
+  if ((B > 0 && d_lens == nullptr) || d_seg_off == nullptr || d_user_off == nullptr ||
+      (T > 0 && d_group_id == nullptr) || d_status == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  TimedScope tsc(MTGR_TIMER_PACK, as_stream(stream), T > 0 ? 2 : 1);
+  return launch_pack(B, d_lens, T, d_seg_off, d_user_off, d_group_id, d_status, as_stream(stream));
+}
+
+MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_capacity) {
+  if (q_capacity < 0 || kt_capacity < 0) return 0;
+  return mask_meta_ws_bytes(q_capacity, kt_capacity);
+}
+
+MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int64_t* d_ts,
+                                  int32_t q_capacity, int32_t kt_capacity, int32_t e_capacity,
+                                  int32_t* d_qtile_desc, int32_t* d_row_ptr, int32_t* d_entries,
+                                  int32_t* d_order, int64_t* d_counts, void* d_ws,
+                                  size_t ws_bytes, int32_t* d_status, mtgr_stream_t stream) {
+  if (B < 0 || q_capacity < 0 || kt_capacity < 0 || e_capacity < 0 ||
+      kt_capacity > kMaxKtCapacity)
+    return MTGR_ERR_INVALID_ARG;
+  if (d_seg_off == nullptr || d_row_ptr == nullptr || d_counts == nullptr || d_status == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  if (q_capacity > 0 && (d_ts == nullptr || d_qtile_desc == nullptr || d_order == nullptr ||
+                         (e_capacity > 0 && d_entries == nullptr)))
+    return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < mask_meta_ws_bytes(q_capacity, kt_capacity)) return MTGR_ERR_CAPACITY;
+  if (q_capacity > 0 && kt_capacity > 0 && d_ws == nullptr) return MTGR_ERR_INVALID_ARG;
+  TimedScope tsc(MTGR_TIMER_MASK_META, as_stream(stream), q_capacity > 0 ? 4 : 2);
+  return launch_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, d_qtile_desc,
+                          d_row_ptr, d_entries, d_order, d_counts, d_ws, d_status,
+                          as_stream(stream));
+}
+
+MTGR_API int mtgr_group_layernorm(int32_t T, int32_t d, int32_t x_dtype, const void* d_x,
+                                  const int8_t* d_group_id, int32_t G, const float* d_gamma,
+                                  const float* d_beta, float eps, int32_t y_dtype, void* d_y,
+                                  mtgr_stream_t stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || d > kMaxD || G <= 0 || !(eps >= 0.0f))
+    return MTGR_ERR_INVALID_ARG;
+  if (T > 0 && (d_x == nullptr || d_group_id == nullptr || d_gamma == nullptr ||
+                d_beta == nullptr || d_y == nullptr))
+    return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x) || !aligned16(d_y) || !aligned16(d_gamma) || !aligned16(d_beta))
+    return MTGR_ERR_INVALID_ARG;
+  TimedScope tsc(MTGR_TIMER_GLN, as_stream(stream), T > 0 ? 1 : 0);
+  return launch_gln(T, d, x_dtype, d_x, d_group_id, G, d_gamma, d_beta, eps, y_dtype, d_y,
+                    as_stream(stream));
+}
+
+MTGR_API int mtgr_hstu_attention_fwd(const mtgr_batch* batch, int32_t d, int32_t H,
+                                     int32_t qkvu_dtype, const void* d_qkvu, int32_t out_dtype,
+                                     void* d_g, mtgr_stream_t stream) {
+  if (!batch_ok(batch) || d <= 0 || H <= 0 || d % H != 0 || d > kMaxD) return MTGR_ERR_INVALID_ARG;
+  if (batch->T > 0 && (d_qkvu == nullptr || d_g == nullptr)) return MTGR_ERR_INVALID_ARG;
+  const int dh = d / H;
+  TimedScope tsc(MTGR_TIMER_ATTENTION, as_stream(stream), 1);
+  if (qkvu_dtype == MTGR_F32) {
+    if (out_dtype != MTGR_F32 || (dh != 32 && dh != 64)) return MTGR_ERR_UNSUPPORTED;
+    return launch_attn_f32(batch, d, H, static_cast<const float*>(d_qkvu),
+                           static_cast<float*>(d_g), as_stream(stream));
+  }
+  if (qkvu_dtype != MTGR_BF16 && qkvu_dtype != MTGR_F16) return MTGR_ERR_UNSUPPORTED;
+  if (out_dtype != MTGR_F32 && out_dtype != MTGR_BF16) return MTGR_ERR_UNSUPPORTED;
+  if (dh != 64 || d % 64 != 0) return MTGR_ERR_UNSUPPORTED;
+  if (!aligned16(d_qkvu) || !aligned16(d_g)) return MTGR_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  return launch_attn_tc(batch, d, H, qkvu_dtype, false, d_qkvu, out_dtype, d_g, as_stream(stream));
+}
+
+MTGR_API size_t mtgr_block_workspace_bytes(int32_t T, const mtgr_block_params* p) {
+  if (T < 0 || params_check(p) != MTGR_OK) return 0;
+  return block_ws_layout(T, p, nullptr).bytes;
+}
+
+MTGR_API int mtgr_hstu_block_fwd(const mtgr_block_params* p, const mtgr_batch* batch,
+                                 const float* d_x_in, float* d_x_out, void* d_ws, size_t ws_bytes,
+                                 mtgr_stream_t stream) {
+  int rc = params_check(p);
+  if (rc != MTGR_OK) return rc;
+  if (!batch_ok(batch) || (batch->T > 0 && (batch->group_id == nullptr || d_x_in == nullptr ||
+                                            d_x_out == nullptr || d_ws == nullptr)))
+    return MTGR_ERR_INVALID_ARG;
+  if (d_x_in == d_x_out && batch->T > 0) return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x_in) || !aligned16(d_x_out) || !aligned16(d_ws)) return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < block_ws_layout(batch->T, p, nullptr).bytes) return MTGR_ERR_CAPACITY;
+  if (p->dtype == MTGR_BF16 && !device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  return block_fwd(p, batch, d_x_in, d_x_out, d_ws, as_stream(stream));
+}
+
+MTGR_API size_t mtgr_stack_workspace_bytes(int32_t T, const mtgr_block_params* layers, int32_t L) {
+  if (T < 0 || L <= 0 || layers == nullptr) return 0;
+  size_t m = 0;
+  for (int32_t l = 0; l < L; ++l) {
+    if (params_check(&layers[l]) != MTGR_OK) return 0;
+    const size_t b = block_ws_layout(T, &layers[l], nullptr).bytes;
+    m = b > m ? b : m;
+  }
+  return m + (L > 1 ? align_up((size_t)T * layers[0].d * sizeof(float), 256) : 0);
+}
+
+MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mtgr_batch* batch,
+                            const float* d_x_in, float* d_x_out, void* d_ws, size_t ws_bytes,
+                            mtgr_stream_t stream) {
+  if (layers == nullptr || L <= 0) return MTGR_ERR_INVALID_ARG;
+  for (int32_t l = 0; l < L; ++l) {
+    const int rc = params_check(&layers[l]);
+    if (rc != MTGR_OK) return rc;
+    if (layers[l].d != layers[0].d || layers[l].H != layers[0].H ||
+        layers[l].dtype != layers[0].dtype)
+      return MTGR_ERR_INVALID_ARG;
+  }
+  if (!batch_ok(batch) || (batch->T > 0 && (batch->group_id == nullptr || d_x_in == nullptr ||
+                                            d_x_out == nullptr || d_ws == nullptr)))
+    return MTGR_ERR_INVALID_ARG;
+  if (d_x_in == d_x_out && batch->T > 0) return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x_in) || !aligned16(d_x_out) || !aligned16(d_ws)) return MTGR_ERR_INVALID_ARG;
+  const size_t need = mtgr_stack_workspace_bytes(batch->T, layers, L);
+  if (need == 0 && batch->T > 0) return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < need) return MTGR_ERR_CAPACITY;
+  if (layers[0].dtype == MTGR_BF16 && !device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  const cudaStream_t s = as_stream(stream);
+  // ping-pong: layer l writes x_out when (L-1-l) is even, the spare buffer otherwise,
+  // so the last layer lands in x_out and no layer reads its own output buffer
+  size_t block_bytes = 0;
+  for (int32_t l = 0; l < L; ++l) {
+    const size_t b = block_ws_layout(batch->T, &layers[l], nullptr).bytes;
+    block_bytes = b > block_bytes ? b : block_bytes;
+  }
+  float* spare = reinterpret_cast<float*>(static_cast<uint8_t*>(d_ws) + block_bytes);
+  const float* in = d_x_in;
+  for (int32_t l = 0; l < L; ++l) {
+    float* out = ((L - 1 - l) % 2 == 0) ? d_x_out : spare;
+    const int rc = block_fwd(&layers[l], batch, in, out, d_ws, s);
+    if (rc != MTGR_OK) return rc;
+    in = out;
+  }
+  return MTGR_OK;
+}
+
+MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const void* d_a,
+                       const void* d_b, const float* d_bias, int32_t epi, const float* d_resid,
+                       int32_t q_cols, int32_t out_dtype, void* d_out, int32_t* d_status,
+                       mtgr_stream_t stream) {
+  if (M < 0 || N < 0 || K <= 0 || q_cols < 0) return MTGR_ERR_INVALID_ARG;
+  if (epi != MTGR_EPI_NONE && epi != MTGR_EPI_SILU && epi != MTGR_EPI_RESID)
+    return MTGR_ERR_INVALID_ARG;
+  if (M > 0 && N > 0 && (d_a == nullptr || d_b == nullptr || d_out == nullptr))
+    return MTGR_ERR_INVALID_ARG;
+  if (epi == MTGR_EPI_RESID && (d_resid == nullptr || out_dtype != MTGR_F32))
+    return MTGR_ERR_INVALID_ARG;
+  TimedScope tsc(MTGR_TIMER_GEMM_QKVU, as_stream(stream), 1);
+  if (ab_dtype == MTGR_F32) {
+    return launch_gemm_f32(M, N, K, static_cast<const float*>(d_a), static_cast<const float*>(d_b),
+                           d_bias, epi, d_resid, q_cols, out_dtype, d_out, as_stream(stream));
+  }
+  if (ab_dtype != MTGR_BF16) return MTGR_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || N % 32 != 0) return MTGR_ERR_UNSUPPORTED;
+  if (!aligned16(d_a) || !aligned16(d_b) || !aligned16(d_out) || !aligned16(d_bias) ||
+      !aligned16(d_resid))
+    return MTGR_ERR_INVALID_ARG;
+  if (d_status == nullptr) return MTGR_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  return launch_gemm_tc(M, N, K, d_a, d_b, d_bias, epi, d_resid, q_cols, out_dtype, d_out,
+                        d_status, as_stream(stream));
+}
+
+}  // extern "C"

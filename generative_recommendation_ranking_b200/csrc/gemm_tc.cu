@@ -1,0 +1,248 @@
+// bf16 GEMM on the 5th-generation tensor cores (tcgen05) for the HSTU block's
+// three projections: Q|K|V|U = X~ W_qkvu^T, H = silu(G~ W1^T), and
+// X_out = H W2^T + X (summary page, "Method": the block update equations).
+//
+//   out[m][n] = epi(sum_k a[m][k] b[n][k] + bias[n])
+//
+// Design: a persistent kernel, one CTA per SM, 128x256 output tiles, 64-deep
+// k-blocks staged by TMA (128-byte swizzle) through a 4-stage mbarrier
+// pipeline. Warp 0 issues TMA loads, one thread of warp 1 issues
+// tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM), warps 2-5 drain
+// the accumulator (tcgen05.ld), apply the epilogue and store. The 512 TMEM
+// columns hold two accumulators so the epilogue of tile i overlaps the main
+// loop of tile i+1.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace mtgr {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int NUM_THREADS = 192;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+
+struct GemmArgs {
+  int M, N, K;
+  const float* bias;
+  const float* resid;
+  void* out;
+  int q_cols;
+  int32_t* status;
+};
+
+__device__ __forceinline__ float u32_as_f(uint32_t v) { return __uint_as_float(v); }
+
+// Epilogue of 32 consecutive columns [col0, col0+32) of one row.
+template <int EPI, int OUT>
+__device__ __forceinline__ void epilogue_store(const GemmArgs& a, int row, int col0,
+                                               const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = u32_as_f(r[c]);
+  if (a.bias != nullptr) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 4) {
+      const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.bias + col0 + c));
+      v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
+    }
+  }
+  if (col0 < a.q_cols) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] *= 0.5f;
+  }
+  if (EPI == MTGR_EPI_SILU) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = silu_fast(v[c]);
+  }
+  const int64_t off = (int64_t)row * a.N + col0;
+  if (EPI == MTGR_EPI_RESID) {
+    const float4* rp = reinterpret_cast<const float4*>(a.resid + off);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 x = __ldg(rp + c);
+      v[4 * c] += x.x; v[4 * c + 1] += x.y; v[4 * c + 2] += x.z; v[4 * c + 3] += x.w;
+    }
+  }
+  if (OUT == MTGR_F32) {
+    float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + off);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) op[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  } else {
+    uint32_t w[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      w[c] = OUT == MTGR_F16 ? cvt_f16x2(v[2 * c], v[2 * c + 1]) : cvt_bf16x2(v[2 * c], v[2 * c + 1]);
+    uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + off);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) op[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+  }
+}
+
+template <int EPI, int OUT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int M = args.M, N = args.N, K = args.K;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int kblocks = K / BK;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool timed_out = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !timed_out; tile += gridDim.x) {
+        const int mb = tile / n_tiles, nb = tile % n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { timed_out = true; break; }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(&tmA, &full[stage], sA + stage * A_BYTES, kb * BK, mb * BM);
+          tma_load_2d(&tmB, &full[stage], sB + stage * B_BYTES, kb * BK, nb * BN);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(BM, BN, 1u, false, false);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !timed_out; tile += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { timed_out = true; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { timed_out = true; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_ss(d_tmem, sdesc_sw128(a_addr + 32 * k, 16, 1024),
+                      sdesc_sw128(b_addr + 32 * k, 16, 1024), idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (timed_out) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile / n_tiles, nb = tile % n_tiles;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
+      if (!ok) { timed_out = true; break; }
+      tc_fence_after();
+      const int row = mb * BM + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nb * BN + c * 32;
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        tmem_ld_wait();
+        if (row < M && col0 < N) epilogue_store<EPI, OUT>(args, row, col0, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  if (timed_out) set_status(args.status, MTGR_ERR_TIMEOUT);
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int EPI, int OUT>
+int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, cudaStream_t s) {
+  auto kern = gemm_tc_kernel<EPI, OUT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+      cudaSuccess)
+    return MTGR_ERR_CUDA;
+  const int tiles = ((args.M + BM - 1) / BM) * ((args.N + BN - 1) / BN);
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, args);
+  return launch_status();
+}
+
+}  // namespace
+
+// a [M][K] bf16, b [N][K] bf16; K % 64 == 0, N % 32 == 0, rows 16-byte aligned.
+int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
+                   const float* resid, int q_cols, int32_t out_dtype, void* out, int32_t* status,
+                   cudaStream_t s) {
+  if (M == 0 || N == 0) return MTGR_OK;
+  CUtensorMap ta, tb;
+  int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
+  if (rc != MTGR_OK) return rc;
+  GemmArgs args{M, N, K, bias, resid, out, q_cols, status};
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_NONE, MTGR_F16>(ta, tb, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_NONE, MTGR_BF16>(ta, tb, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_NONE, MTGR_F32>(ta, tb, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_SILU, MTGR_BF16>(ta, tb, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, args, s);
+  if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, args, s);
+  return MTGR_ERR_UNSUPPORTED;
+}
+
+}  // namespace mtgr

@@ -1,0 +1,190 @@
+// Group-Layer Normalization (fun-rec 7.3.3, the GLN formula; summary page,
+// "Method": GroupLN before the projection and before the MLP):
+//   y_i = (x_i - mean_i) / sqrt(var_i + eps) * gamma[g(i)] + beta[g(i)]
+// Statistics are per token over its d features (biased variance); gamma and
+// beta are the rows of the token's group. One warp per token, 128-bit loads,
+// the row held in registers between the two passes. HBM-bound: it reads
+// d * sizeof(x) and writes d * sizeof(y) bytes per token.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace mtgr {
+
+namespace {
+
+// 8 consecutive elements <-> float[8]
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+    w[k] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// VPL = 8-element vectors per lane (ceil(d / 256)); the row stays in registers.
+template <typename Tin, typename Tout, int VPL>
+__global__ void __launch_bounds__(256) gln_reg_kernel(int32_t T, int32_t d, const Tin* __restrict__ x,
+                                                      const int8_t* __restrict__ gid, int32_t G,
+                                                      const float* __restrict__ gamma,
+                                                      const float* __restrict__ beta, float eps,
+                                                      Tout* __restrict__ y) {
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int nv = d >> 3;
+  const Tin* xr = x + t * d;
+  float v[VPL][8];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      load8(xr + 8 * vi, v[k]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[k][e];
+    }
+  }
+  const float mean = warp_sum(s) / (float)d;
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    if (lane + 32 * k < nv) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float c = v[k][e] - mean;
+        q += c * c;
+      }
+    }
+  }
+  const float var = warp_sum(q) / (float)d;
+  const float rstd = 1.0f / sqrtf(var + eps);
+  int g = gid[t];
+  g = g < 0 ? 0 : (g >= G ? G - 1 : g);
+  const float* ga = gamma + (int64_t)g * d;
+  const float* be = beta + (int64_t)g * d;
+  Tout* yr = y + t * d;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      float gm[8], bt[8], o[8];
+      load8(ga + 8 * vi, gm);
+      load8(be + 8 * vi, bt);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (v[k][e] - mean) * rstd * gm[e] + bt[e];
+      store8(yr + 8 * vi, o);
+    }
+  }
+}
+
+// d > 1024: two passes over the row (the second from cache), Welford-free:
+// the mean first, then the centred sum of squares.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) gln_loop_kernel(int32_t T, int32_t d, const Tin* __restrict__ x,
+                                                       const int8_t* __restrict__ gid, int32_t G,
+                                                       const float* __restrict__ gamma,
+                                                       const float* __restrict__ beta, float eps,
+                                                       Tout* __restrict__ y) {
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int nv = d >> 3;
+  const Tin* xr = x + t * d;
+  float s = 0.f;
+  for (int vi = lane; vi < nv; vi += 32) {
+    float v[8];
+    load8(xr + 8 * vi, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += v[e];
+  }
+  const float mean = warp_sum(s) / (float)d;
+  float q = 0.f;
+  for (int vi = lane; vi < nv; vi += 32) {
+    float v[8];
+    load8(xr + 8 * vi, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float c = v[e] - mean;
+      q += c * c;
+    }
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(q) / (float)d + eps);
+  int g = gid[t];
+  g = g < 0 ? 0 : (g >= G ? G - 1 : g);
+  const float* ga = gamma + (int64_t)g * d;
+  const float* be = beta + (int64_t)g * d;
+  Tout* yr = y + t * d;
+  for (int vi = lane; vi < nv; vi += 32) {
+    float v[8], gm[8], bt[8], o[8];
+    load8(xr + 8 * vi, v);
+    load8(ga + 8 * vi, gm);
+    load8(be + 8 * vi, bt);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = (v[e] - mean) * rstd * gm[e] + bt[e];
+    store8(yr + 8 * vi, o);
+  }
+}
+
+template <typename Tin, typename Tout>
+int launch_gln_t(int32_t T, int32_t d, const void* x, const int8_t* gid, int32_t G,
+                 const float* gamma, const float* beta, float eps, void* y, cudaStream_t s) {
+  const unsigned grid = (unsigned)((T + 7) / 8);
+  const Tin* xi = static_cast<const Tin*>(x);
+  Tout* yo = static_cast<Tout*>(y);
+  const int vpl = (d + 255) / 256;
+  switch (vpl) {
+    case 1: gln_reg_kernel<Tin, Tout, 1><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 2: gln_reg_kernel<Tin, Tout, 2><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 3: gln_reg_kernel<Tin, Tout, 3><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 4: gln_reg_kernel<Tin, Tout, 4><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    default: gln_loop_kernel<Tin, Tout><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+int launch_gln(int32_t T, int32_t d, int32_t x_dtype, const void* x, const int8_t* gid, int32_t G,
+               const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
+               cudaStream_t s) {
+  if (T == 0) return MTGR_OK;
+  if (x_dtype == MTGR_F32 && y_dtype == MTGR_F32)
+    return launch_gln_t<float, float>(T, d, x, gid, G, gamma, beta, eps, y, s);
+  if (x_dtype == MTGR_F32 && y_dtype == MTGR_BF16)
+    return launch_gln_t<float, __nv_bfloat16>(T, d, x, gid, G, gamma, beta, eps, y, s);
+  if (x_dtype == MTGR_BF16 && y_dtype == MTGR_BF16)
+    return launch_gln_t<__nv_bfloat16, __nv_bfloat16>(T, d, x, gid, G, gamma, beta, eps, y, s);
+  return MTGR_ERR_UNSUPPORTED;
+}
+
+}  // namespace mtgr

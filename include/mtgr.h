@@ -239,6 +239,32 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
                        int32_t q_cols, int32_t out_dtype, void* d_out, int32_t* d_status,
                        mtgr_stream_t stream);
 
+/*
+ * Kernel timing. A timer attached to the calling host thread makes every
+ * entry point bracket its kernels with CUDA events on its stream and count
+ * them, per class: MTGR_TIMER_PACK (2 kernels per call), MTGR_TIMER_MASK_META
+ * (4), MTGR_TIMER_GLN, MTGR_TIMER_GEMM_QKVU, MTGR_TIMER_ATTENTION,
+ * MTGR_TIMER_GEMM_MLP1, MTGR_TIMER_GEMM_MLP2 (1 each; mtgr_gemm counts as
+ * MTGR_TIMER_GEMM_QKVU). mtgr_timer_read synchronises on the recorded events,
+ * writes the summed milliseconds and launch counts per class into
+ * ms[MTGR_TIMER_CLASSES] and launches[MTGR_TIMER_CLASSES] (host arrays) and
+ * clears the records. Attaching NULL detaches. Not for use during CUDA graph
+ * capture.
+ */
+#define MTGR_TIMER_PACK 0
+#define MTGR_TIMER_MASK_META 1
+#define MTGR_TIMER_GLN 2
+#define MTGR_TIMER_GEMM_QKVU 3
+#define MTGR_TIMER_ATTENTION 4
+#define MTGR_TIMER_GEMM_MLP1 5
+#define MTGR_TIMER_GEMM_MLP2 6
+#define MTGR_TIMER_CLASSES 7
+typedef struct mtgr_timer mtgr_timer;
+MTGR_API mtgr_timer* mtgr_timer_create(void);
+MTGR_API void mtgr_timer_destroy(mtgr_timer* timer);
+MTGR_API int mtgr_timer_attach(mtgr_timer* timer);
+MTGR_API int mtgr_timer_read(mtgr_timer* timer, double* ms, int64_t* launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,81 @@
+"""The C ABI library on the CPU: it loads, exports every entry point the header
+declares, and rejects bad arguments on the host before touching a device."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from generative_recommendation_ranking_b200 import _lib, api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "mtgr.h")).read()
+    return sorted(set(re.findall(r"MTGR_API\s+[\w\s\*]+?\b(mtgr_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from generative_recommendation_ranking_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib._SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert _lib.status_string(code) != "unknown status"
+    assert _lib.status_string(99) == "unknown status"
+    assert lib.mtgr_version() >= 100
+
+
+def test_host_validation_without_device(lib):
+    E = _lib.MTGR_ERR_INVALID_ARG
+    assert lib.mtgr_pack_offsets(-1, None, 0, None, None, None, None, None) == E
+    assert lib.mtgr_pack_offsets(2, None, 10, None, None, None, None, None) == E
+    assert lib.mtgr_build_mask_meta(1, None, None, 1, 1, 1, None, None, None, None, None, None, 0,
+                                    None, None) == E
+    assert lib.mtgr_group_layernorm(4, 12, 0, None, None, 4, None, None, 1e-5, 0, None, None) == E
+    assert lib.mtgr_hstu_attention_fwd(None, 64, 2, 0, None, 0, None, None) == E
+    assert lib.mtgr_stack_fwd(None, 0, None, None, None, None, 0, None) == E
+    assert lib.mtgr_gemm(-1, 2, 64, 1, None, None, None, 0, None, 0, 0, None, None, None) == E
+
+
+def _params(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16):
+    fake = 0x100000  # 16-byte aligned stand-in addresses; never dereferenced
+    return _lib.MtgrBlockParams(d=d, H=H, d_ff=d_ff, dtype=dtype, eps=1e-5, reserved=0,
+                                gln1_gamma=fake, gln1_beta=fake, gln2_gamma=fake, gln2_beta=fake,
+                                w_qkvu=fake, w1=fake, w2=fake, b_qkvu=None, b1=None, b2=None)
+
+
+def test_workspace_sizes(lib):
+    T = 1000
+    p = _params()
+    want = sum(-(-T * n * 2 // 256) * 256 for n in (512, 2048, 512, 2048))
+    assert _lib.mtgr_block_workspace_bytes(T, p) == want
+    assert _lib.mtgr_block_workspace_bytes(T, _params(H=4)) == 0        # dh = 128 unsupported
+    assert _lib.mtgr_block_workspace_bytes(T, _params(d=100, H=2)) == 0  # d % 64 != 0
+    f = _params(d=64, H=2, d_ff=256, dtype=_lib.MTGR_F32)
+    assert _lib.mtgr_block_workspace_bytes(T, f) > 0
+    two = _lib.mtgr_stack_workspace_bytes(T, [p, p])
+    assert two == want + -(-T * 512 * 4 // 256) * 256
+    assert _lib.mtgr_stack_workspace_bytes(T, [p]) == want
+    assert _lib.mtgr_mask_meta_workspace_bytes(100, 8) == 1024
+
+
+def test_capacities_host_logic():
+    lens = np.array([[4, 32, 8, 8], [16, 300, 50, 100], [0, 0, 0, 0]])
+    q, kt, e = api.capacities(lens)
+    assert (q, kt, e) == (1 + 4 + 0, 4, 1 + 16)
