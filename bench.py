@@ -263,11 +263,8 @@ def run_ours(args, world, rank, local):
     batch.check()
 
     def step(lens_d, ts_d, x_d, out_d):
-        _lib.mtgr_pack_offsets(batch.B, lens_d, batch.T, batch.seg_off, batch.user_off,
-                               batch.group_id, batch.status, stream)
-        _lib.mtgr_build_mask_meta(batch.B, batch.seg_off, ts_d, batch.q_cap, batch.kt_cap,
-                                  batch.e_cap, batch.qtile_desc, batch.row_ptr, batch.entries,
-                                  batch.order, batch.counts, batch.meta_ws, batch.status, stream)
+        batch.pack(stream, d_lens=lens_d)
+        batch.build_meta(stream, d_ts=ts_d)
         _lib.mtgr_stack_fwd([l.c for l in layers], batch.c, x_d, out_d, ws, stream)
 
     for _ in range(args.warmup):

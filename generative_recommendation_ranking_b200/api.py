@@ -16,14 +16,20 @@ EPS = 1e-5
 
 def capacities(lens: np.ndarray) -> tuple:
     """Host-side buffer sizes of the mask metadata for per-user lengths [B,4]:
-    q-tiles, largest per-user k-tile count, and an upper bound on entries."""
-    n = np.asarray(lens, dtype=np.int64).reshape(-1, 4).sum(axis=1)
+    q-tiles, largest per-user k-tile count, an upper bound on tile entries, and
+    the rank-table entries (64-column groups holding R keys x (N_R + 1))."""
+    lens = np.asarray(lens, dtype=np.int64).reshape(-1, 4)
+    n = lens.sum(axis=1)
     nq = (n + TILE_M - 1) // TILE_M
     nk = (n + TILE_N - 1) // TILE_N
     q_cap = int(nq.sum())
     kt_cap = int(nk.max()) if nk.size else 0
     e_cap = int((nq * nk).sum())
-    return q_cap, kt_cap, e_cap
+    n_us = lens[:, 0] + lens[:, 1]
+    c_lo = n_us + lens[:, 2]
+    groups = np.where(lens[:, 2] > 0, (c_lo - 1) // 64 - n_us // 64 + 1, 0)
+    rt_cap = int((groups * (lens[:, 2] + 1)).sum())
+    return q_cap, kt_cap, e_cap, rt_cap
 
 
 class PackedBatch:
@@ -42,7 +48,7 @@ class PackedBatch:
         self.T = int(lens.sum())
         self.device = torch.device(device)
         dev = self.device
-        self.q_cap, self.kt_cap, self.e_cap = capacities(lens)
+        self.q_cap, self.kt_cap, self.e_cap, self.rt_cap = capacities(lens)
         self.d_lens = torch.from_numpy(lens).to(dev, non_blocking=True)
         self.d_ts = (ts if isinstance(ts, torch.Tensor) else torch.from_numpy(
             np.ascontiguousarray(ts, dtype=np.int64))).to(dev, dtype=torch.int64, non_blocking=True)
@@ -56,6 +62,9 @@ class PackedBatch:
         self.entries = torch.empty(max(self.e_cap, 1), **i32)
         self.order = torch.empty(max(self.q_cap, 1), **i32)
         self.counts = torch.zeros(3, dtype=torch.int64, device=dev)
+        self.rt_cnt = torch.empty(max(self.T, 1), **i32)
+        self.rt_off = torch.empty(self.B + 1, dtype=torch.int64, device=dev)
+        self.rt_mask = torch.empty(max(self.rt_cap, 1), dtype=torch.int64, device=dev)
         ws_bytes = _lib.mtgr_mask_meta_workspace_bytes(self.q_cap, self.kt_cap)
         self.meta_ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
         self.norm = None
@@ -63,18 +72,30 @@ class PackedBatch:
             self.norm = torch.as_tensor(np.asarray(norm, dtype=np.float32)).to(dev)
         _lib.mtgr_pack_offsets(self.B, self.d_lens, self.T, self.seg_off, self.user_off,
                                self.group_id, self.status, stream)
-        _lib.mtgr_build_mask_meta(self.B, self.seg_off, self.d_ts, self.q_cap, self.kt_cap,
-                                  self.e_cap, self.qtile_desc, self.row_ptr, self.entries,
-                                  self.order, self.counts, self.meta_ws, self.status, stream)
+        self.build_meta(stream)
         self.c = MtgrBatch(
             B=self.B, T=self.T, q_capacity=self.q_cap, kt_capacity=self.kt_cap,
             seg_off=self.seg_off.data_ptr(), user_off=self.user_off.data_ptr(),
             group_id=self.group_id.data_ptr(), ts=self.d_ts.data_ptr(),
             qtile_desc=self.qtile_desc.data_ptr(), row_ptr=self.row_ptr.data_ptr(),
             entries=self.entries.data_ptr(), order=self.order.data_ptr(),
-            counts=self.counts.data_ptr(),
+            counts=self.counts.data_ptr(), rt_cnt=self.rt_cnt.data_ptr(),
+            rt_off=self.rt_off.data_ptr(), rt_mask=self.rt_mask.data_ptr(),
             norm=None if self.norm is None else self.norm.data_ptr(),
             status=self.status.data_ptr())
+
+    def pack(self, stream=None, d_lens=None) -> None:
+        """(Re)run mtgr_pack_offsets into this batch's buffers."""
+        _lib.mtgr_pack_offsets(self.B, self.d_lens if d_lens is None else d_lens, self.T,
+                               self.seg_off, self.user_off, self.group_id, self.status, stream)
+
+    def build_meta(self, stream=None, d_ts=None) -> None:
+        """(Re)run mtgr_build_mask_meta into this batch's buffers."""
+        _lib.mtgr_build_mask_meta(self.B, self.seg_off, self.d_ts if d_ts is None else d_ts,
+                                  self.q_cap, self.kt_cap, self.e_cap, self.rt_cap,
+                                  self.qtile_desc, self.row_ptr, self.entries, self.order,
+                                  self.counts, self.rt_cnt, self.rt_off, self.rt_mask,
+                                  self.meta_ws, self.status, stream)
 
     def check(self) -> None:
         """Synchronise and raise if a kernel recorded a device-side error."""
@@ -92,7 +113,9 @@ class PackedBatch:
             group_id=self.group_id[:self.T].cpu().numpy(),
             qtile_desc=self.qtile_desc[:Q].cpu().numpy(),
             row_ptr=self.row_ptr[:Q + 1].cpu().numpy(), entries=self.entries[:E].cpu().numpy(),
-            order=self.order[:Q].cpu().numpy(), visible_pairs=V, Q=Q, E=E)
+            order=self.order[:Q].cpu().numpy(), visible_pairs=V, Q=Q, E=E,
+            rt_cnt=self.rt_cnt[:self.T].cpu().numpy(), rt_off=self.rt_off.cpu().numpy(),
+            rt_mask=self.rt_mask[:self.rt_cap].cpu().numpy().view(np.uint64))
 
 
 class BlockWeights:

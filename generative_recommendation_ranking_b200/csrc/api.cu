@@ -11,9 +11,10 @@ int launch_pack(int32_t B, const int32_t* lens, int32_t T, int32_t* seg_off, int
                 int8_t* group_id, int32_t* status, cudaStream_t s);
 size_t mask_meta_ws_bytes(int32_t q_cap, int32_t kt_cap);
 int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32_t q_cap,
-                     int32_t kt_cap, int32_t e_cap, int32_t* qtile_desc, int32_t* row_ptr,
-                     int32_t* entries, int32_t* order, int64_t* counts, void* ws, int32_t* status,
-                     cudaStream_t s);
+                     int32_t kt_cap, int32_t e_cap, int64_t rt_cap, int32_t* qtile_desc,
+                     int32_t* row_ptr, int32_t* entries, int32_t* order, int64_t* counts,
+                     int32_t* rt_cnt, int64_t* rt_off, uint64_t* rt_mask, void* ws,
+                     int32_t* status, cudaStream_t s);
 int launch_gln(int32_t T, int32_t d, int32_t x_dtype, const void* x, const int8_t* gid, int32_t G,
                const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
                cudaStream_t s);
@@ -48,6 +49,7 @@ bool batch_ok(const mtgr_batch* b) {
                             b->entries == nullptr || b->order == nullptr))
     return false;
   if (b->counts == nullptr || b->status == nullptr) return false;
+  if (b->T > 0 && (b->rt_cnt == nullptr || b->rt_off == nullptr)) return false;
   return true;
 }
 
@@ -205,23 +207,27 @@ MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_ca
 
 MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int64_t* d_ts,
                                   int32_t q_capacity, int32_t kt_capacity, int32_t e_capacity,
-                                  int32_t* d_qtile_desc, int32_t* d_row_ptr, int32_t* d_entries,
-                                  int32_t* d_order, int64_t* d_counts, void* d_ws,
-                                  size_t ws_bytes, int32_t* d_status, mtgr_stream_t stream) {
-  if (B < 0 || q_capacity < 0 || kt_capacity < 0 || e_capacity < 0 ||
+                                  int64_t rt_capacity, int32_t* d_qtile_desc, int32_t* d_row_ptr,
+                                  int32_t* d_entries, int32_t* d_order, int64_t* d_counts,
+                                  int32_t* d_rt_cnt, int64_t* d_rt_off, uint64_t* d_rt_mask,
+                                  void* d_ws, size_t ws_bytes, int32_t* d_status,
+                                  mtgr_stream_t stream) {
+  if (B < 0 || q_capacity < 0 || kt_capacity < 0 || e_capacity < 0 || rt_capacity < 0 ||
       kt_capacity > kMaxKtCapacity)
     return MTGR_ERR_INVALID_ARG;
-  if (d_seg_off == nullptr || d_row_ptr == nullptr || d_counts == nullptr || d_status == nullptr)
+  if (d_seg_off == nullptr || d_row_ptr == nullptr || d_counts == nullptr || d_status == nullptr ||
+      d_rt_off == nullptr)
     return MTGR_ERR_INVALID_ARG;
   if (q_capacity > 0 && (d_ts == nullptr || d_qtile_desc == nullptr || d_order == nullptr ||
-                         (e_capacity > 0 && d_entries == nullptr)))
+                         d_rt_cnt == nullptr || (e_capacity > 0 && d_entries == nullptr) ||
+                         (rt_capacity > 0 && d_rt_mask == nullptr)))
     return MTGR_ERR_INVALID_ARG;
   if (ws_bytes < mask_meta_ws_bytes(q_capacity, kt_capacity)) return MTGR_ERR_CAPACITY;
   if (q_capacity > 0 && kt_capacity > 0 && d_ws == nullptr) return MTGR_ERR_INVALID_ARG;
-  TimedScope tsc(MTGR_TIMER_MASK_META, as_stream(stream), q_capacity > 0 ? 4 : 2);
-  return launch_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, d_qtile_desc,
-                          d_row_ptr, d_entries, d_order, d_counts, d_ws, d_status,
-                          as_stream(stream));
+  TimedScope tsc(MTGR_TIMER_MASK_META, as_stream(stream), q_capacity > 0 ? 6 : 4);
+  return launch_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, rt_capacity,
+                          d_qtile_desc, d_row_ptr, d_entries, d_order, d_counts, d_rt_cnt,
+                          d_rt_off, d_rt_mask, d_ws, d_status, as_stream(stream));
 }
 
 MTGR_API int mtgr_group_layernorm(int32_t T, int32_t d, int32_t x_dtype, const void* d_x,

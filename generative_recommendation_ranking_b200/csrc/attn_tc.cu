@@ -14,7 +14,8 @@
 //   warp 0      TMA producer: Q tile once per item, K and V tiles per k-tile
 //   warp 1      MMA issuer:  S = Q K^T (SS, M=128 N=128 K=16) into TMEM,
 //                            O += P V  (TS: P read from TMEM, M=128 N=64)
-//   warps 2-9   SiLU: S from TMEM -> mask -> P = silu(S) in f16 -> TMEM
+//   warps 2-9   SiLU, two groups of 4 warps taking alternate k-tiles: S from
+//               TMEM -> mask -> P = silu(S) in f16 -> TMEM
 //   warps 10-13 epilogue: O from TMEM -> O / N (.) U -> global; and, for bf16
 //               inputs, the in-place bf16 -> f16 conversion of V tiles
 // TMEM (512 columns): S[2] (128 each), P[2] (64 each, f16 pairs), O[2] (64).
@@ -44,7 +45,7 @@ namespace {
 constexpr int DH = 64;
 constexpr int TM = MTGR_TILE_M;  // 128 query rows per item
 constexpr int TN = MTGR_TILE_N;  // 128 keys per k-tile
-constexpr int KV_STAGES = 3;
+constexpr int KV_STAGES = 5;
 constexpr int TILE_BYTES = TM * DH * 2;  // 16 KB (Q, K or V tile)
 constexpr int NUM_SILU_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
@@ -65,6 +66,9 @@ struct AttnArgs {
   const int32_t* entries;
   const int32_t* order;
   const int64_t* counts;
+  const int32_t* rt_cnt;
+  const int64_t* rt_off;
+  const uint64_t* rt_mask;
   const float* norm;
   int32_t q_cap;
   void* out;  // [T][d] f32 or bf16
@@ -73,6 +77,7 @@ struct AttnArgs {
 
 struct Item {
   int32_t h, us, n, n_u, n_us, c_lo, qt, b, e0, e1;
+  int64_t rt_base;
 };
 
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int32_t w) {
@@ -90,6 +95,7 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int32_t w) {
   it.c_lo = so[3] - so[0];
   it.e0 = a.row_ptr[q];
   it.e1 = a.row_ptr[q + 1];
+  it.rt_base = a.rt_off[it.b];
   return it;
 }
 
@@ -107,14 +113,15 @@ __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
   return m << lo;
 }
 
-// Visibility of keys [j0, j0 + 64) (user-relative) to query row i.
-__device__ __forceinline__ uint64_t visible_bits(const Item& it, const int64_t* ts, int32_t i,
-                                                 bool has_time, int64_t t_i, int32_t j0) {
+// Visibility of keys [j0, j0 + 64) (user-relative, j0 a multiple of 64) to
+// query row i, whose rank-table index is cnt_i (rule 2 as a table lookup).
+__device__ __forceinline__ uint64_t visible_bits(const Item& it, const uint64_t* rt_mask,
+                                                 int32_t i, int32_t cnt_i, int32_t j0) {
   uint64_t vis = range_bits(0, it.n_us - j0);  // rule 1: U and S keys
-  const int r0 = max(it.n_us - j0, 0), r1 = min(it.c_lo - j0, 64);
-  const int64_t* tk = ts + it.us + j0;
-  for (int c = r0; c < r1; ++c) {  // rule 2: R keys strictly earlier (warp-uniform loads)
-    if (has_time && __ldg(tk + c) < t_i) vis |= 1ull << c;
+  const int32_t n_r = it.c_lo - it.n_us;
+  if (n_r > 0 && j0 + 64 > it.n_us && j0 < it.c_lo) {  // rule 2: R keys earlier than t_i
+    const int32_t gidx = j0 / 64 - it.n_us / 64;
+    vis |= __ldg(rt_mask + it.rt_base + (int64_t)gidx * (n_r + 1) + cnt_i);
   }
   const int dc = i - j0;  // the diagonal: every token sees itself (rules 1-3)
   if (dc >= 0 && dc < 64) vis |= 1ull << dc;
@@ -167,8 +174,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], NUM_SILU_WARPS);
-      mbar_init(&p_full[i], NUM_SILU_WARPS);
+      mbar_init(&s_free[i], NUM_SILU_WARPS / 2);
+      mbar_init(&p_full[i], NUM_SILU_WARPS / 2);
       mbar_init(&p_free[i], 1);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], NUM_EPI_WARPS);
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
       constexpr uint32_t idesc_o = idesc_f16(TM, DH, 0u, false, true);
-      struct Pend { int32_t g, li, st; bool first, last, valid; } pend{0, 0, 0, false, false, false};
+      struct Pend { int32_t g, li, st; bool first, last, valid; };
       auto issue_pv = [&](const Pend& p) -> bool {
         const int pb = p.g & 1, ob = p.li & 1;
         if (p.first && !mbar_wait(&o_free[ob], ((p.li >> 1) & 1) ^ 1)) return false;
@@ -237,14 +244,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (p.last) tc_commit(&o_full[ob]);
         return true;
       };
+      // Issue order S_0, S_1, S_2, PV_0, S_3, PV_1, ...: S runs two k-tiles ahead
+      // of P V, so each SiLU group finds its next S computed when it finishes.
+      constexpr int LAG = 2;
+      Pend ring[LAG + 1];
+      int n_pend = 0, head = 0;
+      auto push = [&](const Pend& p) -> bool {
+        ring[(head + n_pend) % (LAG + 1)] = p;
+        if (++n_pend <= LAG) return true;
+        const bool ok = issue_pv(ring[head]);
+        head = (head + 1) % (LAG + 1);
+        --n_pend;
+        return ok;
+      };
       int32_t g = 0, li = 0;
       for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += gridDim.x, ++li) {
         const Item it = load_item(a, w);
         const int qb = li & 1, ob = li & 1;
         const int32_t nnz = it.e1 - it.e0;
         if (nnz <= 0) {  // cannot happen for valid metadata (the diagonal tile)
-          if (pend.valid && !issue_pv(pend)) { timed_out = true; break; }
-          pend.valid = false;
+          while (n_pend > 0 && !timed_out) {
+            if (!issue_pv(ring[head])) timed_out = true;
+            head = (head + 1) % (LAG + 1);
+            --n_pend;
+          }
+          if (timed_out) break;
           if (!mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
           tc_commit(&q_empty[qb]);
           if (!mbar_wait(&o_free[ob], ((li >> 1) & 1) ^ 1)) { timed_out = true; break; }
@@ -266,63 +290,76 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_commit(&s_full[sb]);
           if (t == nnz - 1) tc_commit(&q_empty[qb]);
-          if (pend.valid && !issue_pv(pend)) { timed_out = true; break; }
-          pend = Pend{g, li, st, t == 0, t == nnz - 1, true};
+          if (!push(Pend{g, li, st, t == 0, t == nnz - 1, true})) { timed_out = true; break; }
         }
       }
-      if (!timed_out && pend.valid && !issue_pv(pend)) timed_out = true;
+      while (!timed_out && n_pend > 0) {
+        if (!issue_pv(ring[head])) timed_out = true;
+        head = (head + 1) % (LAG + 1);
+        --n_pend;
+      }
     }
   } else if (warp < 2 + NUM_SILU_WARPS) {
     // -------------------------------------------------------- SiLU warps --
+    // group gb takes the k-tiles g with g % 2 == gb (S and P buffer gb); each
+    // warp covers its 32 query rows across all 128 keys of the tile
     const int quarter = warp & 3;
-    const int hf = (warp - 2) >> 2;  // which 64-key half of the tile
+    const int gb = (warp - 2) >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     int32_t g = 0;
     for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += gridDim.x) {
       const Item it = load_item(a, w);
       const int32_t i = it.qt * TM + quarter * 32 + lane;  // user-relative query row
-      const bool row_ok = i < it.n;
-      const bool has_time = row_ok && i >= it.n_u;
-      const int64_t t_i = row_ok ? a.ts[it.us + i] : 0;
+      const int32_t cnt_i = i < it.n ? a.rt_cnt[it.us + i] : 0;
       for (int32_t e = it.e0; e < it.e1; ++e, ++g) {
+        if ((g & 1) != gb) continue;
         const int32_t ent = a.entries[e];
-        const int32_t j0 = (ent >> 1) * TN + hf * 64;
-        const int sb = g & 1;
-        if (!warp_wait(&s_full[sb], (g >> 1) & 1)) { timed_out = true; break; }
+        const int32_t kt = ent >> 1;
+        const uint32_t r = static_cast<uint32_t>(g >> 1);
+        if (!warp_wait(&s_full[gb], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-        uint32_t s0[32], s1[32];
-        tmem_ld32(tmem + lane_base + s_col(sb) + hf * 64, s0);
-        tmem_ld32(tmem + lane_base + s_col(sb) + hf * 64 + 32, s1);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[sb]);
-        uint32_t p[32];
-        if ((ent & 1) || j0 + 64 > it.n) {
-          const uint64_t vis = visible_bits(it, a.ts, i, has_time, t_i, j0);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float x0 = (vis >> (2 * c)) & 1ull ? __uint_as_float(s0[2 * c]) : 0.f;
-            const float x1 = (vis >> (2 * c + 1)) & 1ull ? __uint_as_float(s0[2 * c + 1]) : 0.f;
-            p[c] = silu_pair<HALVE>(x0, x1);
-            const float y0 = (vis >> (32 + 2 * c)) & 1ull ? __uint_as_float(s1[2 * c]) : 0.f;
-            const float y1 = (vis >> (33 + 2 * c)) & 1ull ? __uint_as_float(s1[2 * c + 1]) : 0.f;
-            p[16 + c] = silu_pair<HALVE>(y0, y1);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          const int32_t j0 = kt * TN + half * 64;
+          uint32_t s0[32], s1[32];
+          tmem_ld32(tmem + lane_base + s_col(gb) + half * 64, s0);
+          tmem_ld32(tmem + lane_base + s_col(gb) + half * 64 + 32, s1);
+          tmem_ld_wait();
+          if (half == 1) {  // all of S read: the MMA may overwrite this buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[gb]);
           }
-        } else {
+          uint32_t p[32];
+          if ((ent & 1) || j0 + 64 > it.n) {
+            const uint64_t vis = visible_bits(it, a.rt_mask, i, cnt_i, j0);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            p[c] = silu_pair<HALVE>(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1]));
-            p[16 + c] = silu_pair<HALVE>(__uint_as_float(s1[2 * c]), __uint_as_float(s1[2 * c + 1]));
+            for (int c = 0; c < 16; ++c) {
+              const float x0 = (vis >> (2 * c)) & 1ull ? __uint_as_float(s0[2 * c]) : 0.f;
+              const float x1 = (vis >> (2 * c + 1)) & 1ull ? __uint_as_float(s0[2 * c + 1]) : 0.f;
+              p[c] = silu_pair<HALVE>(x0, x1);
+              const float y0 = (vis >> (32 + 2 * c)) & 1ull ? __uint_as_float(s1[2 * c]) : 0.f;
+              const float y1 = (vis >> (33 + 2 * c)) & 1ull ? __uint_as_float(s1[2 * c + 1]) : 0.f;
+              p[16 + c] = silu_pair<HALVE>(y0, y1);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              p[c] = silu_pair<HALVE>(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1]));
+              p[16 + c] = silu_pair<HALVE>(__uint_as_float(s1[2 * c]), __uint_as_float(s1[2 * c + 1]));
+            }
           }
+          if (half == 0) {  // P buffer free once the previous P V of this buffer is done
+            if (!warp_wait(&p_free[gb], (r & 1) ^ 1)) { timed_out = true; break; }
+            tc_fence_after();
+          }
+          tmem_st32(tmem + lane_base + p_col(gb) + half * 32, p);
         }
-        if (!warp_wait(&p_free[sb], ((g >> 1) & 1) ^ 1)) { timed_out = true; break; }
-        tc_fence_after();
-        tmem_st32(tmem + lane_base + p_col(sb) + hf * 32, p);
+        if (timed_out) break;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sb]);
+        if (lane == 0) mbar_arrive(&p_full[gb]);
       }
     }
   } else {
@@ -434,8 +471,8 @@ int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype,
   int rc = make_tmap_2d_16b(&tm, qkvu, (uint64_t)4 * d, (uint64_t)bt->T, (uint64_t)8 * d, DH, TM);
   if (rc != MTGR_OK) return rc;
   AttnArgs a{d, H, static_cast<const uint16_t*>(qkvu), bt->seg_off, bt->ts, bt->qtile_desc,
-             bt->row_ptr, bt->entries, bt->order, bt->counts, bt->norm, bt->q_capacity, out,
-             bt->status};
+             bt->row_ptr, bt->entries, bt->order, bt->counts, bt->rt_cnt, bt->rt_off,
+             bt->rt_mask, bt->norm, bt->q_capacity, out, bt->status};
   const int64_t items = (int64_t)bt->q_capacity * H;
   const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
   const bool f32 = out_dtype == MTGR_F32;

@@ -126,24 +126,40 @@ __device__ __forceinline__ UserSeg load_user(const int32_t* seg_off, int32_t b) 
   return u;
 }
 
-// q-tiles of every user, user-major: qtile_desc[q] = (user, qt)
+// Number of 64-column groups of a user's key range that hold R keys.
+__device__ __forceinline__ int32_t rt_groups(int32_t n_us, int32_t c_lo) {
+  return c_lo > n_us ? (c_lo - 1) / 64 - n_us / 64 + 1 : 0;
+}
+
+constexpr int32_t kMaxRt = 4096;  // R keys per user handled by the rank tables
+
+// q-tiles of every user, user-major: qtile_desc[q] = (user, qt); and the
+// offsets of each user's R rank tables: rt_off[b] = sum over earlier users of
+// groups * (N_R + 1).
 __global__ void __launch_bounds__(kScanThreads) meta_qtiles_kernel(
-    int32_t B, const int32_t* seg_off, int32_t q_cap, int32_t kt_cap, int32_t* qtile_desc,
-    int32_t* row_ptr, int64_t* counts, int32_t* status) {
+    int32_t B, const int32_t* seg_off, int32_t q_cap, int32_t kt_cap, int64_t rt_cap,
+    int32_t* qtile_desc, int32_t* row_ptr, int64_t* rt_off, int64_t* counts, int32_t* status) {
   __shared__ int64_t warp_tot[32];
-  int64_t carry = 0;
+  int64_t carry = 0, rt_carry = 0;
   bool over = false;
   for (int32_t base = 0; base < B; base += kScanThreads) {
     const int32_t b = base + threadIdx.x;
     int32_t nq = 0;
+    int64_t rt = 0;
     if (b < B) {
-      const int32_t n = seg_off[4 * (int64_t)b + 4] - seg_off[4 * (int64_t)b];
+      const int32_t* so = seg_off + 4 * (int64_t)b;
+      const int32_t n = so[4] - so[0];
       nq = (n + MTGR_TILE_M - 1) / MTGR_TILE_M;
       if ((n + MTGR_TILE_N - 1) / MTGR_TILE_N > kt_cap) over = true;
+      const int32_t n_r = so[3] - so[2];
+      if (n_r > kMaxRt) over = true;
+      rt = (int64_t)rt_groups(so[2] - so[0], so[3] - so[0]) * (n_r + 1);
     }
-    int64_t excl;
+    int64_t excl, rt_excl;
     const int64_t chunk = block_exclusive_scan(nq, warp_tot, excl);
+    const int64_t rt_chunk = block_exclusive_scan(rt, warp_tot, rt_excl);
     if (b < B) {
+      rt_off[b] = rt_carry + rt_excl;
       for (int32_t qt = 0; qt < nq; ++qt) {
         const int64_t q = carry + excl + qt;
         if (q < q_cap) {
@@ -153,16 +169,70 @@ __global__ void __launch_bounds__(kScanThreads) meta_qtiles_kernel(
       }
     }
     carry += chunk;
+    rt_carry += rt_chunk;
   }
   // any overflow: record it and publish zero q-tiles, so no later kernel reads
   // past a buffer the caller sized
-  const int any_over = __syncthreads_or(over || carry > q_cap);
+  const int any_over = __syncthreads_or(over || carry > q_cap || rt_carry > rt_cap);
   if (threadIdx.x == 0) {
+    rt_off[B] = rt_carry;
     counts[0] = any_over ? 0 : carry;
     counts[1] = 0;
     counts[2] = 0;
     row_ptr[0] = 0;
     if (any_over) set_status(status, MTGR_ERR_CAPACITY);
+  }
+}
+
+// Rank tables of rule 2, one CTA per user. Order the user's R keys by
+// (timestamp, index); then the R keys with t_j < t_i are exactly those whose
+// rank is below cnt_i = #{R keys k : t_k < t_i}. Written:
+//   rt_cnt[token]  = cnt_i (0 for U tokens, which carry no time)
+//   rt_mask[rt_off[b] + g * (N_R + 1) + r] = bits (within 64-column group g
+//       of the user's R key range) of the R keys with rank < r.
+// So an R key j in group g is visible to query i (j != i) iff bit (j mod 64)
+// of rt_mask[.. g .. cnt_i] is set.
+__global__ void __launch_bounds__(256) meta_rt_kernel(const int32_t* seg_off, const int64_t* ts,
+                                                      const int64_t* rt_off,
+                                                      const int64_t* counts, int32_t* rt_cnt,
+                                                      uint64_t* rt_mask) {
+  extern __shared__ int64_t tsR[];  // [n_r], then int32 ranks [n_r]
+  if (counts[0] == 0) return;  // no q-tiles: empty batch, or a capacity overflow
+  const int32_t b = blockIdx.x;
+  const int32_t* so = seg_off + 4 * (int64_t)b;
+  const int32_t us = so[0], n = so[4] - so[0], n_u = so[1] - so[0], n_us = so[2] - so[0],
+                c_lo = so[3] - so[0];
+  const int32_t n_r = min(c_lo - n_us, kMaxRt);
+  int32_t* rankR = reinterpret_cast<int32_t*>(tsR + kMaxRt);
+  for (int32_t k = threadIdx.x; k < n_r; k += blockDim.x) tsR[k] = ts[us + n_us + k];
+  __syncthreads();
+  for (int32_t j = threadIdx.x; j < n_r; j += blockDim.x) {
+    const int64_t t = tsR[j];
+    int32_t r = 0;
+    for (int32_t k = 0; k < n_r; ++k) r += (tsR[k] < t || (tsR[k] == t && k < j)) ? 1 : 0;
+    rankR[j] = r;
+  }
+  for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+    int32_t c = 0;
+    if (i >= n_u) {
+      const int64_t t = ts[us + i];
+      for (int32_t k = 0; k < n_r; ++k) c += tsR[k] < t ? 1 : 0;
+    }
+    rt_cnt[us + i] = c;
+  }
+  __syncthreads();
+  const int32_t G = rt_groups(n_us, c_lo);
+  const int64_t base = rt_off[b];
+  const int32_t g0 = n_us / 64;
+  for (int32_t e = threadIdx.x; e < G * (n_r + 1); e += blockDim.x) {
+    const int32_t g = e / (n_r + 1), r = e - g * (n_r + 1);
+    const int32_t col0 = (g0 + g) * 64;
+    uint64_t m = 0;
+    for (int p = 0; p < 64; ++p) {
+      const int32_t j = col0 + p;
+      if (j >= n_us && j < c_lo && rankR[j - n_us] < r) m |= 1ull << p;
+    }
+    rt_mask[base + e] = m;
   }
 }
 
@@ -220,6 +290,9 @@ __global__ void __launch_bounds__(MTGR_TILE_M) meta_classify_kernel(
     nnz += any_vis ? 1 : 0;
     __syncthreads();
   }
+  // k-tiles past this user's end are EMPTY (the workspace is not pre-cleared)
+  for (int32_t kt = KT + threadIdx.x; kt < kt_cap; kt += blockDim.x)
+    codes[(int64_t)q * kt_cap + kt] = 0;
   if (threadIdx.x == 0) {
     row_ptr[q + 1] = nnz;
     atomicAdd(reinterpret_cast<unsigned long long*>(&counts[2]),
@@ -227,26 +300,17 @@ __global__ void __launch_bounds__(MTGR_TILE_M) meta_classify_kernel(
   }
 }
 
-// Exclusive scan of the per-q-tile counts into row_ptr, E, and the work order
-// (q-tiles by descending count, ties by ascending index).
-constexpr int kMaxHist = 4096;
-__global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, int32_t kt_cap,
-                                                                 int32_t e_cap, int32_t* row_ptr,
-                                                                 int32_t* order, int64_t* counts,
+// Exclusive scan of the per-q-tile counts into row_ptr, and E.
+__global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, int32_t e_cap,
+                                                                 int32_t* row_ptr, int64_t* counts,
                                                                  int32_t* status) {
   __shared__ int64_t warp_tot[32];
-  __shared__ int32_t hist[kMaxHist + 1];
-  __shared__ int32_t bucket_start[kMaxHist + 1];
   const int64_t Qd = counts[0];
   const int32_t Q = (int32_t)(Qd < (int64_t)q_cap ? Qd : (int64_t)q_cap);
-  const int32_t nb = min(kt_cap, kMaxHist) + 1;
-  for (int v = threadIdx.x; v < nb; v += blockDim.x) hist[v] = 0;
-  __syncthreads();
   int64_t carry = 0;
   for (int32_t base = 0; base < Q; base += kScanThreads) {
     const int32_t q = base + threadIdx.x;
     const int32_t c = q < Q ? row_ptr[q + 1] : 0;
-    if (q < Q) atomicAdd(&hist[min(c, nb - 1)], 1);
     int64_t excl;
     const int64_t chunk = block_exclusive_scan(c, warp_tot, excl);
     __syncthreads();  // all reads of row_ptr[q+1] in this chunk are done
@@ -255,7 +319,6 @@ __global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, 
     __syncthreads();
   }
   if (carry > e_cap) {  // entries would overflow: publish zero q-tiles
-    __syncthreads();
     if (threadIdx.x == 0) {
       counts[0] = 0;
       counts[1] = 0;
@@ -263,30 +326,29 @@ __global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, 
     }
     return;
   }
-  if (threadIdx.x == 0) {
-    counts[1] = carry;
-    int32_t s = 0;  // bucket starts in descending count order
-    for (int v = nb - 1; v >= 0; --v) {
-      bucket_start[v] = s;
-      s += hist[v];
+  if (threadIdx.x == 0) counts[1] = carry;
+}
+
+// Work order: users by descending length (ties by ascending index), each
+// user's q-tiles contiguous and by ascending qt, so that every item of a user
+// (all its q-tiles and heads) runs close in time and its keys and values stay
+// in L2. One thread per user ranks it against all users.
+__global__ void __launch_bounds__(kScanThreads) meta_order_kernel(int32_t B, const int32_t* seg_off,
+                                                                  int32_t q_cap, int32_t* order,
+                                                                  const int64_t* counts) {
+  if (counts[0] == 0) return;
+  for (int32_t b = threadIdx.x; b < B; b += blockDim.x) {
+    const int32_t n = seg_off[4 * (int64_t)b + 4] - seg_off[4 * (int64_t)b];
+    int64_t pos = 0, qstart = 0;
+    for (int32_t k = 0; k < B; ++k) {
+      const int32_t nk = seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
+      const int32_t nqk = (nk + MTGR_TILE_M - 1) / MTGR_TILE_M;
+      if (k < b) qstart += nqk;
+      if (nk > n || (nk == n && k < b)) pos += nqk;
     }
-  }
-  __syncthreads();
-  // stable placement: warp w handles the non-empty buckets k with k % 32 == w
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int k = 0;
-  for (int v = nb - 1; v >= 0; --v) {
-    if (hist[v] == 0) continue;
-    if ((k++ & 31) != wid) continue;
-    int32_t pos = bucket_start[v];
-    for (int32_t base = 0; base < Q; base += 32) {
-      const int32_t q = base + lane;
-      const int32_t c = q < Q ? row_ptr[q + 1] - row_ptr[q] : -1;
-      const bool hit = q < Q && min(c, nb - 1) == v;
-      const uint32_t m = __ballot_sync(0xffffffffu, hit);
-      if (hit) order[pos + __popc(m & ((1u << lane) - 1u))] = q;
-      pos += __popc(m);
-    }
+    const int32_t nq = (n + MTGR_TILE_M - 1) / MTGR_TILE_M;
+    for (int32_t qt = 0; qt < nq; ++qt)
+      if (pos + qt < q_cap) order[pos + qt] = (int32_t)(qstart + qt);
   }
 }
 
@@ -327,21 +389,31 @@ size_t mask_meta_ws_bytes(int32_t q_cap, int32_t kt_cap) {
 }
 
 int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32_t q_cap,
-                     int32_t kt_cap, int32_t e_cap, int32_t* qtile_desc, int32_t* row_ptr,
-                     int32_t* entries, int32_t* order, int64_t* counts, void* ws,
+                     int32_t kt_cap, int32_t e_cap, int64_t rt_cap, int32_t* qtile_desc,
+                     int32_t* row_ptr, int32_t* entries, int32_t* order, int64_t* counts,
+                     int32_t* rt_cnt, int64_t* rt_off, uint64_t* rt_mask, void* ws,
                      int32_t* status, cudaStream_t s) {
   uint8_t* codes = static_cast<uint8_t*>(ws);
-  meta_qtiles_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, kt_cap, qtile_desc, row_ptr,
-                                               counts, status);
+  meta_qtiles_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, kt_cap, rt_cap, qtile_desc,
+                                               row_ptr, rt_off, counts, status);
   int rc = launch_status();
   if (rc != MTGR_OK) return rc;
+  if (B > 0) {
+    const size_t smem = (size_t)kMaxRt * (sizeof(int64_t) + sizeof(int32_t));
+    if (cudaFuncSetAttribute(meta_rt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MTGR_ERR_CUDA;
+    meta_rt_kernel<<<B, 256, smem, s>>>(seg_off, ts, rt_off, counts, rt_cnt, rt_mask);
+    if ((rc = launch_status()) != MTGR_OK) return rc;
+  }
   if (q_cap > 0) {
     meta_classify_kernel<<<q_cap, MTGR_TILE_M, 0, s>>>(seg_off, ts, qtile_desc, q_cap, kt_cap,
                                                       codes, row_ptr, counts);
     if ((rc = launch_status()) != MTGR_OK) return rc;
   }
-  meta_scan_kernel<<<1, kScanThreads, 0, s>>>(q_cap, kt_cap, e_cap, row_ptr, order, counts,
-                                             status);
+  meta_scan_kernel<<<1, kScanThreads, 0, s>>>(q_cap, e_cap, row_ptr, counts, status);
+  if ((rc = launch_status()) != MTGR_OK) return rc;
+  meta_order_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, order, counts);
   if ((rc = launch_status()) != MTGR_OK) return rc;
   if (q_cap > 0) {
     meta_fill_kernel<<<(q_cap + 7) / 8, 256, 0, s>>>(q_cap, kt_cap, e_cap, codes, row_ptr,
@@ -350,5 +422,4 @@ int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32
   }
   return rc;
 }
-
 }  // namespace mtgr

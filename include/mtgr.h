@@ -107,18 +107,34 @@ MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_ca
  *   d_qtile_desc [q_capacity][2] int32: (user, qt), user-major, qt ascending
  *   d_row_ptr    [q_capacity+1] int32: CSR row pointers into d_entries
  *   d_entries    [e_capacity] int32: (kt << 1) | partial, kt ascending per row
- *   d_order      [q_capacity] int32: q-tile indices by descending entry count,
- *                ties by ascending index (the attention's work order)
+ *   d_order      [q_capacity] int32: the attention's work order: q-tiles user
+ *                by user, users by descending length (ties by ascending user
+ *                index), each user's q-tiles by ascending qt
  *   d_counts     [3] int64: Q (q-tiles), E (entries), visible (query,key) pairs
+ *   rt_capacity  entries available in d_rt_mask (>= sum over users of
+ *                G_b (N_R,b + 1), G_b = number of 64-column groups of the
+ *                user's key range [N_U+N_S, N_U+N_S+N_R) that hold R keys)
+ *   d_rt_cnt     [T] int32: cnt_i = number of R keys of token i's user with a
+ *                timestamp strictly below t_i (0 for U tokens)
+ *   d_rt_off     [B+1] int64: start of each user's rank tables in d_rt_mask
+ *   d_rt_mask    [rt_capacity] uint64: rule 2 as prefix tables. With the
+ *                user's R keys ordered by (timestamp, index), entry
+ *                rt_off[b] + g (N_R + 1) + r holds the bits (column mod 64
+ *                within the user-relative 64-column group N_U+N_S rounded down
+ *                to 64, plus g) of the R keys ranked below r. R key j != i is
+ *                visible to query i iff its bit is set in the entry at r = cnt_i.
  *   d_ws, ws_bytes  workspace of mtgr_mask_meta_workspace_bytes() bytes
- *   d_status     device status word (MTGR_ERR_CAPACITY if Q, E or a user's
- *                tile count exceed the capacities; outputs are then invalid)
+ *   d_status     device status word (MTGR_ERR_CAPACITY if Q, E, the rank
+ *                tables or a user's tile count exceed the capacities, or a
+ *                user has more than 4096 R tokens; no q-tile is then published)
  */
 MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int64_t* d_ts,
                                   int32_t q_capacity, int32_t kt_capacity, int32_t e_capacity,
-                                  int32_t* d_qtile_desc, int32_t* d_row_ptr, int32_t* d_entries,
-                                  int32_t* d_order, int64_t* d_counts, void* d_ws,
-                                  size_t ws_bytes, int32_t* d_status, mtgr_stream_t stream);
+                                  int64_t rt_capacity, int32_t* d_qtile_desc, int32_t* d_row_ptr,
+                                  int32_t* d_entries, int32_t* d_order, int64_t* d_counts,
+                                  int32_t* d_rt_cnt, int64_t* d_rt_off, uint64_t* d_rt_mask,
+                                  void* d_ws, size_t ws_bytes, int32_t* d_status,
+                                  mtgr_stream_t stream);
 
 /*
  * Group-Layer Normalization (fun-rec 7.3.3, the GLN formula):
@@ -151,6 +167,9 @@ typedef struct mtgr_batch {
   const int32_t* entries;     /* [E] */
   const int32_t* order;       /* [q_capacity] */
   const int64_t* counts;      /* [3] Q, E, visible pairs */
+  const int32_t* rt_cnt;      /* [T] rank-table index of each token */
+  const int64_t* rt_off;      /* [B+1] */
+  const uint64_t* rt_mask;    /* rank tables of rule 2 */
   const float* norm;          /* optional [B] normaliser override; NULL = user length */
   int32_t* status;            /* device status word */
 } mtgr_batch;
@@ -243,7 +262,7 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
  * Kernel timing. A timer attached to the calling host thread makes every
  * entry point bracket its kernels with CUDA events on its stream and count
  * them, per class: MTGR_TIMER_PACK (2 kernels per call), MTGR_TIMER_MASK_META
- * (4), MTGR_TIMER_GLN, MTGR_TIMER_GEMM_QKVU, MTGR_TIMER_ATTENTION,
+ * (6), MTGR_TIMER_GLN, MTGR_TIMER_GEMM_QKVU, MTGR_TIMER_ATTENTION,
  * MTGR_TIMER_GEMM_MLP1, MTGR_TIMER_GEMM_MLP2 (1 each; mtgr_gemm counts as
  * MTGR_TIMER_GEMM_QKVU). mtgr_timer_read synchronises on the recorded events,
  * writes the summed milliseconds and launch counts per class into

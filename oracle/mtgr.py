@@ -191,8 +191,9 @@ def mask_meta(lens: np.ndarray, ts: np.ndarray, bm: int = BM, bn: int = BN):
     tile with no visible cell is EMPTY and omitted; FULL if every in-range cell
     is visible; PARTIAL otherwise. Q-tiles are listed user-major with the
     q-tile index ascending, and entries of a q-tile by ascending k-tile; each
-    entry is (kt << 1) | partial. ``order`` lists q-tile indices by descending
-    entry count, ties by ascending index. Returns dict with qtile_desc int32
+    entry is (kt << 1) | partial. ``order`` lists the q-tiles user by user,
+    users by descending length (ties by ascending user index), each user's
+    q-tiles by ascending qt. Returns dict with qtile_desc int32
     [Q,2] (user, qt), row_ptr int32 [Q+1], entries int32 [E], order int32 [Q]
     and the visible-pair count.
     """
@@ -218,8 +219,8 @@ def mask_meta(lens: np.ndarray, ts: np.ndarray, bm: int = BM, bn: int = BN):
             desc.append((b, qt))
             row_ptr.append(len(entries))
     Q = len(desc)
-    nnz = np.diff(np.asarray(row_ptr, dtype=np.int64))
-    order = sorted(range(Q), key=lambda q: (-int(nnz[q]), q))
+    n_user = lens.sum(axis=1)
+    order = sorted(range(Q), key=lambda q: (-int(n_user[desc[q][0]]), desc[q][0], desc[q][1]))
     return dict(
         qtile_desc=np.asarray(desc, dtype=np.int32).reshape(-1, 2),
         row_ptr=np.asarray(row_ptr, dtype=np.int32),

@@ -20,6 +20,21 @@ def assert_close_rms(gpu, ref, tol, what=""):
     return err / max(rms, 1e-300)
 
 
+def assert_close_bf16_out(gpu, ref, what="", tol=1e-2):
+    """Bar for an intermediate tensor stored in bf16: within one bf16 rounding
+    of the exact value (|rounded - x| <= 2^-8 |x| for round-to-nearest) plus a
+    computation error of ``tol`` x RMS."""
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite GPU values"
+    rms = float(np.sqrt(np.mean(r ** 2))) if r.size else 0.0
+    excess = np.abs(g - r) - 2.0 ** -8 * np.abs(r)
+    worst = float(excess.max()) if r.size else 0.0
+    assert worst <= tol * rms, f"{what}: error beyond bf16 rounding {worst:.3e} > {tol} x RMS {rms:.3e}"
+    return worst / max(rms, 1e-300)
+
+
 def user_rows(lens, users):
     """Row indices (in the packed layout) of the given users, in order."""
     n = np.asarray(lens, np.int64).reshape(-1, 4).sum(1)

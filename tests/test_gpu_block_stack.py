@@ -26,7 +26,8 @@ def _gpu_stack(w, layers=None, x=None, lens=None, ts=None, norm=None):
     b = mt.PackedBatch(lens, ts, norm=norm)
     ws = [mt.BlockWeights(p, w["H"], dtype=w["dtype"]) for p in layers]
     xin = torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev)
-    y = mt.hstu_stack_forward(ws, b, xin)
+    scratch = mt.stack_workspace(ws, b).fill_(0xFF)  # NaN bit patterns: results must not read stale workspace
+    y = mt.hstu_stack_forward(ws, b, xin, ws=scratch)
     b.check()
     return to_host(y)
 

@@ -15,6 +15,13 @@ mt = pytest.importorskip("generative_recommendation_ranking_b200")
 def _check_batch(lens, ts):
     b = mt.PackedBatch(lens, ts)
     b.check()
+    # rebuild over dirty buffers: nothing may depend on pre-cleared memory
+    for t in (b.meta_ws, b.qtile_desc, b.row_ptr, b.entries, b.order, b.counts, b.seg_off,
+              b.user_off, b.group_id, b.rt_cnt, b.rt_off, b.rt_mask):
+        t.view(torch.uint8).fill_(0xA7)
+    b.pack()
+    b.build_meta()
+    b.check()
     m = b.meta()
     seg_off, user_off, gid = oracle.pack_offsets(lens)
     np.testing.assert_array_equal(m["seg_off"], seg_off)
@@ -26,7 +33,33 @@ def _check_batch(lens, ts):
     np.testing.assert_array_equal(m["entries"], ref["entries"])
     np.testing.assert_array_equal(m["order"], ref["order"])
     assert m["visible_pairs"] == ref["visible_pairs"]
+    _check_rank_tables(lens, ts, m)
     return b
+
+
+def _check_rank_tables(lens, ts, m):
+    """Rule 2 as tables: for every query row i and every 64-column group g
+    holding R keys, the table entry at cnt_i must equal the R columns of that
+    group visible to i in the oracle's explicit M, the diagonal excluded."""
+    _, user_off, _ = oracle.pack_offsets(lens)
+    for b, (n_u, n_s, n_r, n_k) in enumerate(np.asarray(lens, np.int64)):
+        s, e = int(user_off[b]), int(user_off[b + 1])
+        if n_r == 0 or e == s:
+            continue
+        n_us, c_lo = n_u + n_s, n_u + n_s + n_r
+        M = oracle.user_mask(int(n_u), int(n_s), int(n_r), int(n_k), ts[s:e]).copy()
+        np.fill_diagonal(M, False)
+        cnt = m["rt_cnt"][s:e].astype(np.int64)
+        g0, g1 = n_us // 64, (c_lo - 1) // 64
+        for g in range(g1 - g0 + 1):
+            tab = m["rt_mask"][m["rt_off"][b] + g * (n_r + 1): m["rt_off"][b] + (g + 1) * (n_r + 1)]
+            assert tab.shape[0] == n_r + 1
+            cols = np.arange((g0 + g) * 64, (g0 + g + 1) * 64)
+            in_r = (cols >= n_us) & (cols < c_lo)
+            sub = M[:, np.clip(cols, 0, e - s - 1)] & in_r[None, :]
+            weights = np.left_shift(np.uint64(1), np.arange(64, dtype=np.uint64))
+            want = (sub.astype(np.uint64) * weights[None, :]).sum(axis=1, dtype=np.uint64)
+            np.testing.assert_array_equal(tab[cnt], want)
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2, 3])
@@ -102,9 +135,11 @@ def test_capacity_overflow_sets_device_status():
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     i32 = dict(dtype=torch.int32, device=dev)
     ws = torch.empty(mt.mtgr_mask_meta_workspace_bytes(3, 3), dtype=torch.uint8, device=dev)
+    i64 = dict(dtype=torch.int64, device=dev)
     # e_capacity 2 < the 9 tiles this user has
-    mt.mtgr_build_mask_meta(1, b.seg_off, b.d_ts, 3, 3, 2, torch.empty(3, 2, **i32),
+    mt.mtgr_build_mask_meta(1, b.seg_off, b.d_ts, 3, 3, 2, b.rt_cap, torch.empty(3, 2, **i32),
                             torch.empty(4, **i32), torch.empty(2, **i32), torch.empty(3, **i32),
-                            torch.zeros(3, dtype=torch.int64, device=dev), ws, st)
+                            torch.zeros(3, **i64), torch.empty(b.T, **i32), torch.empty(2, **i64),
+                            torch.empty(max(b.rt_cap, 1), **i64), ws, st)
     torch.cuda.synchronize()
     assert int(st.item()) == mt._lib.MTGR_ERR_CAPACITY

@@ -45,8 +45,8 @@ def test_host_validation_without_device(lib):
     E = _lib.MTGR_ERR_INVALID_ARG
     assert lib.mtgr_pack_offsets(-1, None, 0, None, None, None, None, None) == E
     assert lib.mtgr_pack_offsets(2, None, 10, None, None, None, None, None) == E
-    assert lib.mtgr_build_mask_meta(1, None, None, 1, 1, 1, None, None, None, None, None, None, 0,
-                                    None, None) == E
+    assert lib.mtgr_build_mask_meta(1, None, None, 1, 1, 1, 1, None, None, None, None, None, None,
+                                    None, None, None, 0, None, None) == E
     assert lib.mtgr_group_layernorm(4, 12, 0, None, None, 4, None, None, 1e-5, 0, None, None) == E
     assert lib.mtgr_hstu_attention_fwd(None, 64, 2, 0, None, 0, None, None) == E
     assert lib.mtgr_stack_fwd(None, 0, None, None, None, None, 0, None) == E
@@ -76,6 +76,9 @@ def test_workspace_sizes(lib):
 
 
 def test_capacities_host_logic():
-    lens = np.array([[4, 32, 8, 8], [16, 300, 50, 100], [0, 0, 0, 0]])
-    q, kt, e = api.capacities(lens)
-    assert (q, kt, e) == (1 + 4 + 0, 4, 1 + 16)
+    lens = np.array([[4, 32, 8, 8], [16, 300, 50, 100], [0, 0, 0, 0], [0, 60, 10, 0]])
+    q, kt, e, rt = api.capacities(lens)
+    assert (q, kt, e) == (1 + 4 + 0 + 1, 4, 1 + 16 + 1)
+    # R groups: user 0 cols [36, 44) -> 1 group; user 1 [316, 366) -> groups 4, 5;
+    # user 3 [60, 70) -> groups 0, 1
+    assert rt == 1 * 9 + 2 * 51 + 0 + 2 * 11

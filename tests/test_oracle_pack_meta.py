@@ -72,12 +72,12 @@ def test_mask_meta_brute_force_small_tiles(seed):
     flat = [e for r in rows for e in r]
     np.testing.assert_array_equal(mm["entries"], flat)
     np.testing.assert_array_equal(np.diff(mm["row_ptr"]), [len(r) for r in rows])
-    # order: by descending count, ties by ascending index
-    cnt = np.diff(mm["row_ptr"])
+    # order: users by descending length (ties by index), q-tiles ascending
     order = mm["order"]
     assert sorted(order.tolist()) == list(range(len(rows)))
-    for a, b in zip(order[:-1], order[1:]):
-        assert cnt[a] > cnt[b] or (cnt[a] == cnt[b] and a < b)
+    n_user = lens.sum(1)
+    key = [(-int(n_user[desc[q][0]]), desc[q][0], desc[q][1]) for q in order]
+    assert key == sorted(key)
     assert mm["visible_pairs"] == oracle.visible_pairs(lens, ts)
 
 
