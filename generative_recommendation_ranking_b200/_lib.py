@@ -53,7 +53,9 @@ class MtgrBatch(ctypes.Structure):
                 ("seg_off", c_vp), ("user_off", c_vp), ("group_id", c_vp), ("ts", c_vp),
                 ("qtile_desc", c_vp), ("row_ptr", c_vp), ("entries", c_vp), ("order", c_vp),
                 ("counts", c_vp), ("rt_cnt", c_vp), ("rt_off", c_vp), ("rt_mask", c_vp),
-                ("norm", c_vp), ("status", c_vp)]
+                ("work", c_vp), ("norm", c_vp), ("status", c_vp)]
+
+WORK_ITEM_BYTES = 48  # sizeof(mtgr_work_item)
 
 
 class MtgrBlockParams(ctypes.Structure):
@@ -69,8 +71,8 @@ _SIGNATURES = {
     "mtgr_pack_offsets": (ctypes.c_int, [c_i32, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "mtgr_mask_meta_workspace_bytes": (c_size, [c_i32, c_i32]),
     "mtgr_build_mask_meta": (ctypes.c_int, [c_i32, c_vp, c_vp, c_i32, c_i32, c_i32, c_i64, c_vp,
-                                            c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_size,
-                                            c_vp, c_vp]),
+                                            c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                            c_size, c_vp, c_vp]),
     "mtgr_group_layernorm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp,
                                             c_float, c_i32, c_vp, c_vp]),
     "mtgr_hstu_attention_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_i32, c_i32, c_i32,
@@ -153,13 +155,13 @@ def mtgr_mask_meta_workspace_bytes(q_capacity: int, kt_capacity: int) -> int:
 
 def mtgr_build_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, rt_capacity,
                          d_qtile_desc, d_row_ptr, d_entries, d_order, d_counts, d_rt_cnt, d_rt_off,
-                         d_rt_mask, d_ws, d_status, stream=None):
+                         d_rt_mask, d_work, d_ws, d_status, stream=None):
     ws_bytes = 0 if d_ws is None else d_ws.numel() * d_ws.element_size()
     _check("mtgr_build_mask_meta", load().mtgr_build_mask_meta(
         B, _ptr(d_seg_off), _ptr(d_ts), q_capacity, kt_capacity, e_capacity, rt_capacity,
         _ptr(d_qtile_desc), _ptr(d_row_ptr), _ptr(d_entries), _ptr(d_order), _ptr(d_counts),
-        _ptr(d_rt_cnt), _ptr(d_rt_off), _ptr(d_rt_mask), _ptr(d_ws), ws_bytes, _ptr(d_status),
-        _stream(stream)))
+        _ptr(d_rt_cnt), _ptr(d_rt_off), _ptr(d_rt_mask), _ptr(d_work), _ptr(d_ws), ws_bytes,
+        _ptr(d_status), _stream(stream)))
 
 
 def mtgr_group_layernorm(T, d, d_x, d_group_id, G, d_gamma, d_beta, eps, d_y, stream=None):

@@ -65,6 +65,8 @@ class PackedBatch:
         self.rt_cnt = torch.empty(max(self.T, 1), **i32)
         self.rt_off = torch.empty(self.B + 1, dtype=torch.int64, device=dev)
         self.rt_mask = torch.empty(max(self.rt_cap, 1), dtype=torch.int64, device=dev)
+        self.work = torch.empty(max(self.q_cap, 1) * _lib.WORK_ITEM_BYTES, dtype=torch.uint8,
+                                device=dev)
         ws_bytes = _lib.mtgr_mask_meta_workspace_bytes(self.q_cap, self.kt_cap)
         self.meta_ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
         self.norm = None
@@ -81,7 +83,7 @@ class PackedBatch:
             entries=self.entries.data_ptr(), order=self.order.data_ptr(),
             counts=self.counts.data_ptr(), rt_cnt=self.rt_cnt.data_ptr(),
             rt_off=self.rt_off.data_ptr(), rt_mask=self.rt_mask.data_ptr(),
-            norm=None if self.norm is None else self.norm.data_ptr(),
+            work=self.work.data_ptr(), norm=None if self.norm is None else self.norm.data_ptr(),
             status=self.status.data_ptr())
 
     def pack(self, stream=None, d_lens=None) -> None:
@@ -95,7 +97,7 @@ class PackedBatch:
                                   self.q_cap, self.kt_cap, self.e_cap, self.rt_cap,
                                   self.qtile_desc, self.row_ptr, self.entries, self.order,
                                   self.counts, self.rt_cnt, self.rt_off, self.rt_mask,
-                                  self.meta_ws, self.status, stream)
+                                  self.work, self.meta_ws, self.status, stream)
 
     def check(self) -> None:
         """Synchronise and raise if a kernel recorded a device-side error."""
@@ -115,7 +117,8 @@ class PackedBatch:
             row_ptr=self.row_ptr[:Q + 1].cpu().numpy(), entries=self.entries[:E].cpu().numpy(),
             order=self.order[:Q].cpu().numpy(), visible_pairs=V, Q=Q, E=E,
             rt_cnt=self.rt_cnt[:self.T].cpu().numpy(), rt_off=self.rt_off.cpu().numpy(),
-            rt_mask=self.rt_mask[:self.rt_cap].cpu().numpy().view(np.uint64))
+            rt_mask=self.rt_mask[:self.rt_cap].cpu().numpy().view(np.uint64),
+            work=self.work[:Q * _lib.WORK_ITEM_BYTES].cpu().numpy().view(np.int32).reshape(Q, 12))
 
 
 class BlockWeights:

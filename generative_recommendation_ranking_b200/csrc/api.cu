@@ -13,8 +13,8 @@ size_t mask_meta_ws_bytes(int32_t q_cap, int32_t kt_cap);
 int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32_t q_cap,
                      int32_t kt_cap, int32_t e_cap, int64_t rt_cap, int32_t* qtile_desc,
                      int32_t* row_ptr, int32_t* entries, int32_t* order, int64_t* counts,
-                     int32_t* rt_cnt, int64_t* rt_off, uint64_t* rt_mask, void* ws,
-                     int32_t* status, cudaStream_t s);
+                     int32_t* rt_cnt, int64_t* rt_off, uint64_t* rt_mask, mtgr_work_item* work,
+                     void* ws, int32_t* status, cudaStream_t s);
 int launch_gln(int32_t T, int32_t d, int32_t x_dtype, const void* x, const int8_t* gid, int32_t G,
                const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
                cudaStream_t s);
@@ -46,7 +46,7 @@ bool batch_ok(const mtgr_batch* b) {
   if (b->kt_capacity > kMaxKtCapacity) return false;
   if (b->seg_off == nullptr || b->user_off == nullptr || b->ts == nullptr) return false;
   if (b->q_capacity > 0 && (b->qtile_desc == nullptr || b->row_ptr == nullptr ||
-                            b->entries == nullptr || b->order == nullptr))
+                            b->entries == nullptr || b->order == nullptr || b->work == nullptr))
     return false;
   if (b->counts == nullptr || b->status == nullptr) return false;
   if (b->T > 0 && (b->rt_cnt == nullptr || b->rt_off == nullptr)) return false;
@@ -210,8 +210,8 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
                                   int64_t rt_capacity, int32_t* d_qtile_desc, int32_t* d_row_ptr,
                                   int32_t* d_entries, int32_t* d_order, int64_t* d_counts,
                                   int32_t* d_rt_cnt, int64_t* d_rt_off, uint64_t* d_rt_mask,
-                                  void* d_ws, size_t ws_bytes, int32_t* d_status,
-                                  mtgr_stream_t stream) {
+                                  mtgr_work_item* d_work, void* d_ws, size_t ws_bytes,
+                                  int32_t* d_status, mtgr_stream_t stream) {
   if (B < 0 || q_capacity < 0 || kt_capacity < 0 || e_capacity < 0 || rt_capacity < 0 ||
       kt_capacity > kMaxKtCapacity)
     return MTGR_ERR_INVALID_ARG;
@@ -219,7 +219,8 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
       d_rt_off == nullptr)
     return MTGR_ERR_INVALID_ARG;
   if (q_capacity > 0 && (d_ts == nullptr || d_qtile_desc == nullptr || d_order == nullptr ||
-                         d_rt_cnt == nullptr || (e_capacity > 0 && d_entries == nullptr) ||
+                         d_rt_cnt == nullptr || d_work == nullptr ||
+                         (e_capacity > 0 && d_entries == nullptr) ||
                          (rt_capacity > 0 && d_rt_mask == nullptr)))
     return MTGR_ERR_INVALID_ARG;
   if (ws_bytes < mask_meta_ws_bytes(q_capacity, kt_capacity)) return MTGR_ERR_CAPACITY;
@@ -227,7 +228,7 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
   TimedScope tsc(MTGR_TIMER_MASK_META, as_stream(stream), q_capacity > 0 ? 6 : 4);
   return launch_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, rt_capacity,
                           d_qtile_desc, d_row_ptr, d_entries, d_order, d_counts, d_rt_cnt,
-                          d_rt_off, d_rt_mask, d_ws, d_status, as_stream(stream));
+                          d_rt_off, d_rt_mask, d_work, d_ws, d_status, as_stream(stream));
 }
 
 MTGR_API int mtgr_group_layernorm(int32_t T, int32_t d, int32_t x_dtype, const void* d_x,

@@ -59,15 +59,10 @@ constexpr size_t SMEM_BYTES = 1024 + 2 * TILE_BYTES + KV_STAGES * 2 * TILE_BYTES
 struct AttnArgs {
   int32_t d, H;
   const uint16_t* qkvu;  // [T][4d] 16-bit
-  const int32_t* seg_off;
-  const int64_t* ts;
-  const int32_t* qtile_desc;
-  const int32_t* row_ptr;
   const int32_t* entries;
-  const int32_t* order;
+  const mtgr_work_item* work;
   const int64_t* counts;
   const int32_t* rt_cnt;
-  const int64_t* rt_off;
   const uint64_t* rt_mask;
   const float* norm;
   int32_t q_cap;
@@ -76,26 +71,22 @@ struct AttnArgs {
 };
 
 struct Item {
-  int32_t h, us, n, n_u, n_us, c_lo, qt, b, e0, e1;
-  int64_t rt_base;
+  mtgr_work_item w;
+  int32_t h;
 };
 
+// Item w = (work-list slot w / H, head w % H): a single 48-byte record, so
+// the load has no dependent chain and can be issued one item ahead.
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int32_t w) {
   Item it;
   const int32_t slot = w / a.H;
   it.h = w - slot * a.H;
-  const int32_t q = a.order[slot];
-  it.b = a.qtile_desc[2 * q];
-  it.qt = a.qtile_desc[2 * q + 1];
-  const int32_t* so = a.seg_off + 4 * (int64_t)it.b;
-  it.us = so[0];
-  it.n = so[4] - so[0];
-  it.n_u = so[1] - so[0];
-  it.n_us = so[2] - so[0];
-  it.c_lo = so[3] - so[0];
-  it.e0 = a.row_ptr[q];
-  it.e1 = a.row_ptr[q + 1];
-  it.rt_base = a.rt_off[it.b];
+  const int4* p = reinterpret_cast<const int4*>(a.work + slot);
+  const int4 x0 = __ldg(p), x1 = __ldg(p + 1), x2 = __ldg(p + 2);
+  it.w.us = x0.x; it.w.n = x0.y; it.w.n_u = x0.z; it.w.n_us = x0.w;
+  it.w.c_lo = x1.x; it.w.qt = x1.y; it.w.b = x1.z; it.w.e0 = x1.w;
+  it.w.e1 = x2.x; it.w.reserved = x2.y;
+  it.w.rt_base = (int64_t)(uint32_t)x2.z | ((int64_t)x2.w << 32);
   return it;
 }
 
@@ -113,9 +104,19 @@ __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
   return m << lo;
 }
 
+template <bool HALVE>
+__device__ __forceinline__ uint32_t silu_pair(float a, float b) {
+  if (HALVE) {
+    a *= 0.5f;
+    b *= 0.5f;
+  }
+  const uint32_t h = cvt_f16x2(a, b);
+  return fma_f16x2(h, tanh_f16x2(h), h);
+}
+
 // Visibility of keys [j0, j0 + 64) (user-relative, j0 a multiple of 64) to
 // query row i, whose rank-table index is cnt_i (rule 2 as a table lookup).
-__device__ __forceinline__ uint64_t visible_bits(const Item& it, const uint64_t* rt_mask,
+__device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, const uint64_t* rt_mask,
                                                  int32_t i, int32_t cnt_i, int32_t j0) {
   uint64_t vis = range_bits(0, it.n_us - j0);  // rule 1: U and S keys
   const int32_t n_r = it.c_lo - it.n_us;
@@ -128,15 +129,24 @@ __device__ __forceinline__ uint64_t visible_bits(const Item& it, const uint64_t*
   return vis & range_bits(0, it.n - j0);  // keys past the user's end
 }
 
+// P for 32 consecutive keys [j0, j0 + 32) of one query row: 16 f16 pairs.
 template <bool HALVE>
-__device__ __forceinline__ uint32_t silu_pair(float a, float b) {
-  if (HALVE) {
-    a *= 0.5f;
-    b *= 0.5f;
+__device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p)[16], bool masked,
+                                           uint32_t vis) {
+  if (masked) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const float x0 = (vis >> (2 * c)) & 1u ? __uint_as_float(s[2 * c]) : 0.f;
+      const float x1 = (vis >> (2 * c + 1)) & 1u ? __uint_as_float(s[2 * c + 1]) : 0.f;
+      p[c] = silu_pair<HALVE>(x0, x1);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      p[c] = silu_pair<HALVE>(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
   }
-  const uint32_t h = cvt_f16x2(a, b);
-  return fma_f16x2(h, tanh_f16x2(h), h);
 }
+
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
@@ -197,26 +207,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const int32_t n_items = num_items(a);
   const int32_t d = a.d;
+  const int32_t stride = gridDim.x;
   bool timed_out = false;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       int32_t g = 0, li = 0;
-      for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += gridDim.x, ++li) {
-        const Item it = load_item(a, w);
+      Item nxt;
+      if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
+      for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
+        const Item it = nxt;
+        if (w + stride < n_items) nxt = load_item(a, w + stride);
         const int qb = li & 1;
+        const int32_t row_q = it.w.us + it.w.qt * TM;
         if (!mbar_wait(&q_empty[qb], ((li >> 1) & 1) ^ 1)) { timed_out = true; break; }
         mbar_arrive_expect_tx(&q_full[qb], TILE_BYTES);
-        tma_load_2d(&tm, &q_full[qb], sQ + qb * TILE_BYTES, it.h * DH, it.us + it.qt * TM);
-        for (int32_t e = it.e0; e < it.e1; ++e, ++g) {
-          const int32_t kt = a.entries[e] >> 1;
+        tma_load_2d(&tm, &q_full[qb], sQ + qb * TILE_BYTES, it.h * DH, row_q);
+        int32_t ent = it.w.e0 < it.w.e1 ? __ldg(a.entries + it.w.e0) : 0;
+        for (int32_t e = it.w.e0; e < it.w.e1; ++e, ++g) {
+          const int32_t kt = ent >> 1;
+          if (e + 1 < it.w.e1) ent = __ldg(a.entries + e + 1);
           const int st = g % KV_STAGES;
           if (!mbar_wait(&kv_empty[st], ((g / KV_STAGES) & 1) ^ 1)) { timed_out = true; break; }
           uint8_t* sk = sKV + st * 2 * TILE_BYTES;
           mbar_arrive_expect_tx(&kv_full[st], 2 * TILE_BYTES);
-          tma_load_2d(&tm, &kv_full[st], sk, d + it.h * DH, it.us + kt * TN);
-          tma_load_2d(&tm, &kv_full[st], sk + TILE_BYTES, 2 * d + it.h * DH, it.us + kt * TN);
+          tma_load_2d(&tm, &kv_full[st], sk, d + it.h * DH, it.w.us + kt * TN);
+          tma_load_2d(&tm, &kv_full[st], sk + TILE_BYTES, 2 * d + it.h * DH, it.w.us + kt * TN);
         }
       }
     }
@@ -225,7 +242,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
       constexpr uint32_t idesc_o = idesc_f16(TM, DH, 0u, false, true);
-      struct Pend { int32_t g, li, st; bool first, last, valid; };
+      struct Pend { int32_t g, li, st; bool first, last; };
       auto issue_pv = [&](const Pend& p) -> bool {
         const int pb = p.g & 1, ob = p.li & 1;
         if (p.first && !mbar_wait(&o_free[ob], ((p.li >> 1) & 1) ^ 1)) return false;
@@ -249,25 +266,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr int LAG = 2;
       Pend ring[LAG + 1];
       int n_pend = 0, head = 0;
-      auto push = [&](const Pend& p) -> bool {
-        ring[(head + n_pend) % (LAG + 1)] = p;
-        if (++n_pend <= LAG) return true;
+      auto pop = [&]() -> bool {
         const bool ok = issue_pv(ring[head]);
         head = (head + 1) % (LAG + 1);
         --n_pend;
         return ok;
       };
       int32_t g = 0, li = 0;
-      for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += gridDim.x, ++li) {
-        const Item it = load_item(a, w);
+      Item nxt;
+      if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
+      for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
+        const Item it = nxt;
+        if (w + stride < n_items) nxt = load_item(a, w + stride);
         const int qb = li & 1, ob = li & 1;
-        const int32_t nnz = it.e1 - it.e0;
+        const int32_t nnz = it.w.e1 - it.w.e0;
         if (nnz <= 0) {  // cannot happen for valid metadata (the diagonal tile)
-          while (n_pend > 0 && !timed_out) {
-            if (!issue_pv(ring[head])) timed_out = true;
-            head = (head + 1) % (LAG + 1);
-            --n_pend;
-          }
+          while (n_pend > 0 && !timed_out)
+            if (!pop()) timed_out = true;
           if (timed_out) break;
           if (!mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
           tc_commit(&q_empty[qb]);
@@ -290,77 +305,87 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_commit(&s_full[sb]);
           if (t == nnz - 1) tc_commit(&q_empty[qb]);
-          if (!push(Pend{g, li, st, t == 0, t == nnz - 1, true})) { timed_out = true; break; }
+          ring[(head + n_pend) % (LAG + 1)] = Pend{g, li, st, t == 0, t == nnz - 1};
+          if (++n_pend > LAG && !pop()) { timed_out = true; break; }
         }
       }
-      while (!timed_out && n_pend > 0) {
-        if (!issue_pv(ring[head])) timed_out = true;
-        head = (head + 1) % (LAG + 1);
-        --n_pend;
-      }
+      while (!timed_out && n_pend > 0)
+        if (!pop()) timed_out = true;
     }
   } else if (warp < 2 + NUM_SILU_WARPS) {
     // -------------------------------------------------------- SiLU warps --
-    // group gb takes the k-tiles g with g % 2 == gb (S and P buffer gb); each
-    // warp covers its 32 query rows across all 128 keys of the tile
+    // Group gb takes the k-tiles g with g % 2 == gb (S and P buffer gb); each
+    // warp covers its 32 query rows across all 128 keys, in four 32-key
+    // chunks with the TMEM load of chunk k+1 in flight while chunk k is
+    // computed.
     const int quarter = warp & 3;
     const int gb = (warp - 2) >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int32_t g = 0;
-    for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += gridDim.x) {
-      const Item it = load_item(a, w);
-      const int32_t i = it.qt * TM + quarter * 32 + lane;  // user-relative query row
-      const int32_t cnt_i = i < it.n ? a.rt_cnt[it.us + i] : 0;
-      for (int32_t e = it.e0; e < it.e1; ++e, ++g) {
-        if ((g & 1) != gb) continue;
-        const int32_t ent = a.entries[e];
+    int32_t g0 = 0;  // CTA-wide index of the current item's first k-tile
+    Item nxt;
+    int32_t cnt_nxt = 0;
+    auto cnt_of = [&](const Item& x) -> int32_t {
+      const int32_t i = x.w.qt * TM + quarter * 32 + lane;
+      return i < x.w.n ? __ldg(a.rt_cnt + x.w.us + i) : 0;
+    };
+    if ((int32_t)blockIdx.x < n_items) {
+      nxt = load_item(a, blockIdx.x);
+      cnt_nxt = cnt_of(nxt);
+    }
+    for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride) {
+      const Item it = nxt;
+      const int32_t cnt_i = cnt_nxt;
+      if (w + stride < n_items) {
+        nxt = load_item(a, w + stride);
+        cnt_nxt = cnt_of(nxt);
+      }
+      const int32_t i = it.w.qt * TM + quarter * 32 + lane;  // user-relative query row
+      const int32_t nnz = it.w.e1 - it.w.e0;
+      int32_t t = ((g0 & 1) == gb) ? 0 : 1;  // this group's first k-tile of the item
+      int32_t ent = t < nnz ? __ldg(a.entries + it.w.e0 + t) : 0;
+      for (; t < nnz; t += 2) {
+        const int32_t g = g0 + t;
         const int32_t kt = ent >> 1;
+        const bool partial = ent & 1;
+        if (t + 2 < nnz) ent = __ldg(a.entries + it.w.e0 + t + 2);
         const uint32_t r = static_cast<uint32_t>(g >> 1);
+        const bool masked = partial || kt * TN + TN > it.w.n;
+        uint64_t vis_lo = 0, vis_hi = 0;
+        if (masked) {
+          vis_lo = visible_bits(it.w, a.rt_mask, i, cnt_i, kt * TN);
+          vis_hi = visible_bits(it.w, a.rt_mask, i, cnt_i, kt * TN + 64);
+        }
         if (!warp_wait(&s_full[gb], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          const int32_t j0 = kt * TN + half * 64;
-          uint32_t s0[32], s1[32];
-          tmem_ld32(tmem + lane_base + s_col(gb) + half * 64, s0);
-          tmem_ld32(tmem + lane_base + s_col(gb) + half * 64 + 32, s1);
-          tmem_ld_wait();
-          if (half == 1) {  // all of S read: the MMA may overwrite this buffer
+        const uint32_t s_addr = tmem + lane_base + s_col(gb);
+        const uint32_t p_addr = tmem + lane_base + p_col(gb);
+        uint32_t sa[32], sbuf[32];
+        tmem_ld32(s_addr, sa);
+        tmem_ld_wait();
+        if (!warp_wait(&p_free[gb], (r & 1) ^ 1)) { timed_out = true; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t (&cur)[32] = (k & 1) ? sbuf : sa;
+          uint32_t (&ahead)[32] = (k & 1) ? sa : sbuf;
+          if (k < 3) tmem_ld32(s_addr + 32 * (k + 1), ahead);
+          const uint64_t vv = k < 2 ? vis_lo : vis_hi;
+          uint32_t p[16];
+          silu_chunk<HALVE>(cur, p, masked, (uint32_t)(vv >> (32 * (k & 1))));
+          tmem_st16(p_addr + 16 * k, p);
+          if (k < 3) tmem_ld_wait();
+          if (k == 2) {  // all of S is in registers: the MMA may overwrite it
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[gb]);
           }
-          uint32_t p[32];
-          if ((ent & 1) || j0 + 64 > it.n) {
-            const uint64_t vis = visible_bits(it, a.rt_mask, i, cnt_i, j0);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float x0 = (vis >> (2 * c)) & 1ull ? __uint_as_float(s0[2 * c]) : 0.f;
-              const float x1 = (vis >> (2 * c + 1)) & 1ull ? __uint_as_float(s0[2 * c + 1]) : 0.f;
-              p[c] = silu_pair<HALVE>(x0, x1);
-              const float y0 = (vis >> (32 + 2 * c)) & 1ull ? __uint_as_float(s1[2 * c]) : 0.f;
-              const float y1 = (vis >> (33 + 2 * c)) & 1ull ? __uint_as_float(s1[2 * c + 1]) : 0.f;
-              p[16 + c] = silu_pair<HALVE>(y0, y1);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              p[c] = silu_pair<HALVE>(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1]));
-              p[16 + c] = silu_pair<HALVE>(__uint_as_float(s1[2 * c]), __uint_as_float(s1[2 * c + 1]));
-            }
-          }
-          if (half == 0) {  // P buffer free once the previous P V of this buffer is done
-            if (!warp_wait(&p_free[gb], (r & 1) ^ 1)) { timed_out = true; break; }
-            tc_fence_after();
-          }
-          tmem_st32(tmem + lane_base + p_col(gb) + half * 32, p);
         }
-        if (timed_out) break;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[gb]);
       }
+      g0 += nnz;
     }
   } else {
     // ---------------------------------------------------- epilogue warps --
@@ -368,11 +393,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int et = (warp - 2 - NUM_SILU_WARPS) * 32 + lane;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     int32_t g = 0, li = 0;
-    for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += gridDim.x, ++li) {
-      const Item it = load_item(a, w);
+    Item nxt;
+    if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
+    for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
+      const Item it = nxt;
+      if (w + stride < n_items) nxt = load_item(a, w + stride);
       if (IN_BF16) {
         // convert this item's V tiles to f16 in place as they land
-        for (int32_t e = it.e0; e < it.e1; ++e, ++g) {
+        for (int32_t e = it.w.e0; e < it.w.e1; ++e, ++g) {
           const int st = g % KV_STAGES;
           if (!warp_wait(&kv_full[st], (g / KV_STAGES) & 1)) { timed_out = true; break; }
           uint4* v4 = reinterpret_cast<uint4*>(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
@@ -401,11 +429,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[ob]);
-      const int32_t i = it.qt * TM + quarter * 32 + lane;
-      if (i < it.n) {
-        const bool empty = it.e1 <= it.e0;
-        const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.b] : (float)it.n);
-        const int64_t row = it.us + i;
+      const int32_t i = it.w.qt * TM + quarter * 32 + lane;
+      if (i < it.w.n) {
+        const bool empty = it.w.e1 <= it.w.e0;
+        const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.w.b] : (float)it.w.n);
+        const int64_t row = it.w.us + i;
         const uint4* up = reinterpret_cast<const uint4*>(a.qkvu + row * 4 * d + 3 * d + it.h * DH);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // columns [8k, 8k + 8) of the head
@@ -440,7 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!IN_BF16) g += it.e1 - it.e0;
+      if (!IN_BF16) g += it.w.e1 - it.w.e0;
     }
   }
   if (timed_out) set_status(a.status, MTGR_ERR_TIMEOUT);
@@ -470,9 +498,8 @@ int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype,
   CUtensorMap tm;
   int rc = make_tmap_2d_16b(&tm, qkvu, (uint64_t)4 * d, (uint64_t)bt->T, (uint64_t)8 * d, DH, TM);
   if (rc != MTGR_OK) return rc;
-  AttnArgs a{d, H, static_cast<const uint16_t*>(qkvu), bt->seg_off, bt->ts, bt->qtile_desc,
-             bt->row_ptr, bt->entries, bt->order, bt->counts, bt->rt_cnt, bt->rt_off,
-             bt->rt_mask, bt->norm, bt->q_capacity, out, bt->status};
+  AttnArgs a{d, H, static_cast<const uint16_t*>(qkvu), bt->entries, bt->work, bt->counts,
+             bt->rt_cnt, bt->rt_mask, bt->norm, bt->q_capacity, out, bt->status};
   const int64_t items = (int64_t)bt->q_capacity * H;
   const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
   const bool f32 = out_dtype == MTGR_F32;

@@ -8,7 +8,9 @@
 // k-blocks staged by TMA (128-byte swizzle) through a 4-stage mbarrier
 // pipeline. Warp 0 issues TMA loads, one thread of warp 1 issues
 // tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM), warps 2-5 drain
-// the accumulator (tcgen05.ld), apply the epilogue and store. The 512 TMEM
+// the accumulator (tcgen05.ld), apply the epilogue, stage 32x32 blocks in
+// swizzled shared memory and write them with TMA tensor stores (the residual
+// of the last projection arrives the same way, by TMA load). The 512 TMEM
 // columns hold two accumulators so the epilogue of tile i overlaps the main
 // loop of tile i+1.
 #include <cuda.h>
@@ -32,7 +34,10 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int NUM_THREADS = 192;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+constexpr int EPI_WARPS = 4;
+constexpr int STG_BYTES = 4096;  // one 32x32 staging block (fp32; 16-bit uses half)
+constexpr size_t SMEM_BYTES =
+    1024 + (size_t)STAGES * STAGE_BYTES + (size_t)EPI_WARPS * 2 * STG_BYTES + 256;
 
 struct GemmArgs {
   int M, N, K;
@@ -45,13 +50,23 @@ struct GemmArgs {
 
 __device__ __forceinline__ float u32_as_f(uint32_t v) { return __uint_as_float(v); }
 
-// Epilogue of 32 consecutive columns [col0, col0+32) of one row.
+// Byte offset of 16-byte chunk c of row r in a staging block laid out as the
+// TMA 64-byte (16-bit rows of 32) or 128-byte (fp32 rows of 32) swizzle.
+template <int OUT>
+__device__ __forceinline__ uint32_t stg_off(int r, int c) {
+  return OUT == MTGR_F32 ? (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4))
+                         : (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
+
+// Epilogue math of 32 consecutive columns [col0, col0+32) of one row; the
+// result goes to row `r` of the staging block `stg` (holding the residual
+// block on entry for EPI_RESID).
 template <int EPI, int OUT>
-__device__ __forceinline__ void epilogue_store(const GemmArgs& a, int row, int col0,
-                                               const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
+                                               uint8_t* stg, int r) {
   float v[32];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) v[c] = u32_as_f(r[c]);
+  for (int c = 0; c < 32; ++c) v[c] = u32_as_f(acc[c]);
   if (a.bias != nullptr) {
 #pragma unroll
     for (int c = 0; c < 32; c += 4) {
@@ -67,45 +82,49 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int row, int c
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] = silu_fast(v[c]);
   }
-  const int64_t off = (int64_t)row * a.N + col0;
-  if (EPI == MTGR_EPI_RESID) {
-    const float4* rp = reinterpret_cast<const float4*>(a.resid + off);
+  if (OUT == MTGR_F32) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const float4 x = __ldg(rp + c);
-      v[4 * c] += x.x; v[4 * c + 1] += x.y; v[4 * c + 2] += x.z; v[4 * c + 3] += x.w;
+      float4* p = reinterpret_cast<float4*>(stg + stg_off<OUT>(r, c));
+      float4 x = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      if (EPI == MTGR_EPI_RESID) {
+        const float4 y = *p;
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      *p = x;
     }
-  }
-  if (OUT == MTGR_F32) {
-    float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + off);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) op[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
   } else {
-    uint32_t w[16];
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-      w[c] = OUT == MTGR_F16 ? cvt_f16x2(v[2 * c], v[2 * c + 1]) : cvt_bf16x2(v[2 * c], v[2 * c + 1]);
-    uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + off);
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) op[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      for (int k = 0; k < 4; ++k) {
+        const float lo = v[8 * c + 2 * k], hi = v[8 * c + 2 * k + 1];
+        w[k] = OUT == MTGR_F16 ? cvt_f16x2(lo, hi) : cvt_bf16x2(lo, hi);
+      }
+      *reinterpret_cast<uint4*>(stg + stg_off<OUT>(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
 template <int EPI, int OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* sStg = sB + STAGES * B_BYTES;  // [EPI_WARPS][2][STG_BYTES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + EPI_WARPS * 2 * STG_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* acc_empty = bars + 2 * STAGES + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  uint64_t* rbar = bars + 2 * STAGES + 4;  // [EPI_WARPS][2] residual block landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 2 * EPI_WARPS);
 
   const int warp = warp_id(), lane = lane_id();
   const int M = args.M, N = args.N, K = args.K;
@@ -116,6 +135,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmO);
+    if (EPI == MTGR_EPI_RESID) tma_prefetch_desc(&tmR);
+    for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&rbar[i], 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -179,29 +201,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
+    // epilogue warp ew drains accumulator rows [32 quarter, 32 quarter + 32)
     const int quarter = warp & 3;
+    const int ew = warp - 2;
+    uint8_t* stg = sStg + ew * 2 * STG_BYTES;
     int acc = 0;
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase = 0, chunk = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile / n_tiles, nb = tile % n_tiles;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
       if (!ok) { timed_out = true; break; }
       tc_fence_after();
-      const int row = mb * BM + quarter * 32 + lane;
+      const int row0 = mb * BM + quarter * 32;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c, ++chunk) {
         const int col0 = nb * BN + c * 32;
+        if (col0 >= N) break;
+        const int buf = chunk & 1;
+        uint8_t* sb = stg + buf * STG_BYTES;
+        // the TMA store that last read this buffer (two blocks ago) must be done
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        if (EPI == MTGR_EPI_RESID && lane == 0) {
+          mbar_arrive_expect_tx(&rbar[2 * ew + buf], STG_BYTES);
+          tma_load_2d(&tmR, &rbar[2 * ew + buf], sb, col0, row0);
+        }
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        if (row < M && col0 < N) epilogue_store<EPI, OUT>(args, row, col0, r);
+        if (EPI == MTGR_EPI_RESID &&
+            !__all_sync(0xffffffffu, mbar_wait(&rbar[2 * ew + buf], (chunk >> 1) & 1))) {
+          timed_out = true;
+          break;
+        }
+        epilogue_chunk<EPI, OUT>(args, col0, r, sb, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmO, sb, col0, row0);
+          bulk_commit_group();
+        }
       }
+      if (timed_out) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait_group<0>();  // stores complete before the CTA retires
   }
   if (timed_out) set_status(args.status, MTGR_ERR_TIMEOUT);
   __syncthreads();
@@ -212,14 +260,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int EPI, int OUT>
-int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, cudaStream_t s) {
+int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+             const CUtensorMap& tr, const GemmArgs& args, cudaStream_t s) {
   auto kern = gemm_tc_kernel<EPI, OUT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
       cudaSuccess)
     return MTGR_ERR_CUDA;
   const int tiles = ((args.M + BM - 1) / BM) * ((args.N + BN - 1) / BN);
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, args);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
   return launch_status();
 }
 
@@ -230,18 +279,32 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
                    const float* resid, int q_cols, int32_t out_dtype, void* out, int32_t* status,
                    cudaStream_t s) {
   if (M == 0 || N == 0) return MTGR_OK;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to, tr;
   int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
   if (rc != MTGR_OK) return rc;
   rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
   if (rc != MTGR_OK) return rc;
+  if (out_dtype == MTGR_F32) {
+    rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)M,
+                      (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N, (uint64_t)M,
+                      (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  if (rc != MTGR_OK) return rc;
+  tr = to;
+  if (epi == MTGR_EPI_RESID) {
+    rc = make_tmap_2d(&tr, resid, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)M,
+                      (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MTGR_OK) return rc;
+  }
   GemmArgs args{M, N, K, bias, resid, out, q_cols, status};
-  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_NONE, MTGR_F16>(ta, tb, args, s);
-  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_NONE, MTGR_BF16>(ta, tb, args, s);
-  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_NONE, MTGR_F32>(ta, tb, args, s);
-  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_SILU, MTGR_BF16>(ta, tb, args, s);
-  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, args, s);
-  if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_NONE, MTGR_F16>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_NONE, MTGR_BF16>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_NONE, MTGR_F32>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_SILU, MTGR_BF16>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, to, tr, args, s);
   return MTGR_ERR_UNSUPPORTED;
 }
 

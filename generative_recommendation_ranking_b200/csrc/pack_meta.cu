@@ -332,13 +332,15 @@ __global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, 
 // Work order: users by descending length (ties by ascending index), each
 // user's q-tiles contiguous and by ascending qt, so that every item of a user
 // (all its q-tiles and heads) runs close in time and its keys and values stay
-// in L2. One thread per user ranks it against all users.
-__global__ void __launch_bounds__(kScanThreads) meta_order_kernel(int32_t B, const int32_t* seg_off,
-                                                                  int32_t q_cap, int32_t* order,
-                                                                  const int64_t* counts) {
+// in L2. One thread per user ranks it against all users and writes the
+// user's q-tiles into order[] and the work list (runs after the row_ptr scan).
+__global__ void __launch_bounds__(kScanThreads) meta_order_kernel(
+    int32_t B, const int32_t* seg_off, int32_t q_cap, const int32_t* row_ptr,
+    const int64_t* rt_off, int32_t* order, mtgr_work_item* work, const int64_t* counts) {
   if (counts[0] == 0) return;
   for (int32_t b = threadIdx.x; b < B; b += blockDim.x) {
-    const int32_t n = seg_off[4 * (int64_t)b + 4] - seg_off[4 * (int64_t)b];
+    const int32_t* so = seg_off + 4 * (int64_t)b;
+    const int32_t n = so[4] - so[0];
     int64_t pos = 0, qstart = 0;
     for (int32_t k = 0; k < B; ++k) {
       const int32_t nk = seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
@@ -347,8 +349,24 @@ __global__ void __launch_bounds__(kScanThreads) meta_order_kernel(int32_t B, con
       if (nk > n || (nk == n && k < b)) pos += nqk;
     }
     const int32_t nq = (n + MTGR_TILE_M - 1) / MTGR_TILE_M;
-    for (int32_t qt = 0; qt < nq; ++qt)
-      if (pos + qt < q_cap) order[pos + qt] = (int32_t)(qstart + qt);
+    for (int32_t qt = 0; qt < nq; ++qt) {
+      const int64_t slot = pos + qt, q = qstart + qt;
+      if (slot >= q_cap || q >= q_cap) continue;
+      order[slot] = (int32_t)q;
+      mtgr_work_item it;
+      it.us = so[0];
+      it.n = n;
+      it.n_u = so[1] - so[0];
+      it.n_us = so[2] - so[0];
+      it.c_lo = so[3] - so[0];
+      it.qt = qt;
+      it.b = b;
+      it.e0 = row_ptr[q];
+      it.e1 = row_ptr[q + 1];
+      it.reserved = 0;
+      it.rt_base = rt_off[b];
+      work[slot] = it;
+    }
   }
 }
 
@@ -391,8 +409,8 @@ size_t mask_meta_ws_bytes(int32_t q_cap, int32_t kt_cap) {
 int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32_t q_cap,
                      int32_t kt_cap, int32_t e_cap, int64_t rt_cap, int32_t* qtile_desc,
                      int32_t* row_ptr, int32_t* entries, int32_t* order, int64_t* counts,
-                     int32_t* rt_cnt, int64_t* rt_off, uint64_t* rt_mask, void* ws,
-                     int32_t* status, cudaStream_t s) {
+                     int32_t* rt_cnt, int64_t* rt_off, uint64_t* rt_mask, mtgr_work_item* work,
+                     void* ws, int32_t* status, cudaStream_t s) {
   uint8_t* codes = static_cast<uint8_t*>(ws);
   meta_qtiles_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, kt_cap, rt_cap, qtile_desc,
                                                row_ptr, rt_off, counts, status);
@@ -413,7 +431,8 @@ int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32
   }
   meta_scan_kernel<<<1, kScanThreads, 0, s>>>(q_cap, e_cap, row_ptr, counts, status);
   if ((rc = launch_status()) != MTGR_OK) return rc;
-  meta_order_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, order, counts);
+  meta_order_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, row_ptr, rt_off, order, work,
+                                              counts);
   if ((rc = launch_status()) != MTGR_OK) return rc;
   if (q_cap > 0) {
     meta_fill_kernel<<<(q_cap + 7) / 8, 256, 0, s>>>(q_cap, kt_cap, e_cap, codes, row_ptr,

@@ -29,8 +29,9 @@ constexpr int kMaxDevices = 64;
 
 }  // namespace
 
-int make_tmap_2d_16b(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+int make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (fn == nullptr) return MTGR_ERR_CUDA;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (row_bytes & 15) != 0)
@@ -39,10 +40,16 @@ int make_tmap_2d_16b(CUtensorMap* map, const void* base, uint64_t inner, uint64_
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MTGR_OK : MTGR_ERR_CUDA;
+}
+
+int make_tmap_2d_16b(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  return make_tmap_2d(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT16, inner, outer, row_bytes,
+                      box_inner, box_outer, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 int device_sm_count() {

@@ -89,6 +89,20 @@ MTGR_API int mtgr_pack_offsets(int32_t B, const int32_t* d_lens, int32_t T, int3
 /* Bytes of device workspace mtgr_build_mask_meta needs. */
 MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_capacity);
 
+/* One q-tile of the attention's work list (48 bytes). */
+typedef struct mtgr_work_item {
+  int32_t us;      /* first row of the user */
+  int32_t n;       /* user length N_b */
+  int32_t n_u;     /* N_U */
+  int32_t n_us;    /* N_U + N_S */
+  int32_t c_lo;    /* N_U + N_S + N_R */
+  int32_t qt;      /* q-tile index within the user */
+  int32_t b;       /* user index */
+  int32_t e0, e1;  /* the q-tile's entries: [e0, e1) of the CSR */
+  int32_t reserved;
+  int64_t rt_base; /* the user's first rank-table entry */
+} mtgr_work_item;
+
 /*
  * Mask metadata: the canonical list of non-empty 128x128 tiles of every
  * user's mask M (fun-rec 7.3.4 Rules 1-3; summary page, Method, mask rules).
@@ -123,6 +137,8 @@ MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_ca
  *                within the user-relative 64-column group N_U+N_S rounded down
  *                to 64, plus g) of the R keys ranked below r. R key j != i is
  *                visible to query i iff its bit is set in the entry at r = cnt_i.
+ *   d_work       [q_capacity] mtgr_work_item: the q-tiles in work order, each
+ *                with its user's offsets and CSR range (one load per item)
  *   d_ws, ws_bytes  workspace of mtgr_mask_meta_workspace_bytes() bytes
  *   d_status     device status word (MTGR_ERR_CAPACITY if Q, E, the rank
  *                tables or a user's tile count exceed the capacities, or a
@@ -133,8 +149,8 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
                                   int64_t rt_capacity, int32_t* d_qtile_desc, int32_t* d_row_ptr,
                                   int32_t* d_entries, int32_t* d_order, int64_t* d_counts,
                                   int32_t* d_rt_cnt, int64_t* d_rt_off, uint64_t* d_rt_mask,
-                                  void* d_ws, size_t ws_bytes, int32_t* d_status,
-                                  mtgr_stream_t stream);
+                                  mtgr_work_item* d_work, void* d_ws, size_t ws_bytes,
+                                  int32_t* d_status, mtgr_stream_t stream);
 
 /*
  * Group-Layer Normalization (fun-rec 7.3.3, the GLN formula):
@@ -170,6 +186,7 @@ typedef struct mtgr_batch {
   const int32_t* rt_cnt;      /* [T] rank-table index of each token */
   const int64_t* rt_off;      /* [B+1] */
   const uint64_t* rt_mask;    /* rank tables of rule 2 */
+  const mtgr_work_item* work; /* [q_capacity] work list */
   const float* norm;          /* optional [B] normaliser override; NULL = user length */
   int32_t* status;            /* device status word */
 } mtgr_batch;

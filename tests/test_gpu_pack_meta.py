@@ -17,7 +17,7 @@ def _check_batch(lens, ts):
     b.check()
     # rebuild over dirty buffers: nothing may depend on pre-cleared memory
     for t in (b.meta_ws, b.qtile_desc, b.row_ptr, b.entries, b.order, b.counts, b.seg_off,
-              b.user_off, b.group_id, b.rt_cnt, b.rt_off, b.rt_mask):
+              b.user_off, b.group_id, b.rt_cnt, b.rt_off, b.rt_mask, b.work):
         t.view(torch.uint8).fill_(0xA7)
     b.pack()
     b.build_meta()
@@ -34,7 +34,22 @@ def _check_batch(lens, ts):
     np.testing.assert_array_equal(m["order"], ref["order"])
     assert m["visible_pairs"] == ref["visible_pairs"]
     _check_rank_tables(lens, ts, m)
+    _check_work_list(lens, m, ref)
     return b
+
+
+def _check_work_list(lens, m, ref):
+    """The work list restates, in work order, each q-tile's user offsets and CSR range."""
+    seg_off, _, _ = oracle.pack_offsets(lens)
+    w = m["work"]
+    assert w.shape[0] == len(ref["order"])
+    for slot, q in enumerate(ref["order"]):
+        b, qt = ref["qtile_desc"][q]
+        so = seg_off[4 * b:4 * b + 5].astype(np.int64)
+        want = [so[0], so[4] - so[0], so[1] - so[0], so[2] - so[0], so[3] - so[0], qt, b,
+                ref["row_ptr"][q], ref["row_ptr"][q + 1], 0]
+        np.testing.assert_array_equal(w[slot, :10], want)
+        assert int(w[slot, 10]) | (int(w[slot, 11]) << 32) == int(m["rt_off"][b])
 
 
 def _check_rank_tables(lens, ts, m):
@@ -140,6 +155,7 @@ def test_capacity_overflow_sets_device_status():
     mt.mtgr_build_mask_meta(1, b.seg_off, b.d_ts, 3, 3, 2, b.rt_cap, torch.empty(3, 2, **i32),
                             torch.empty(4, **i32), torch.empty(2, **i32), torch.empty(3, **i32),
                             torch.zeros(3, **i64), torch.empty(b.T, **i32), torch.empty(2, **i64),
-                            torch.empty(max(b.rt_cap, 1), **i64), ws, st)
+                            torch.empty(max(b.rt_cap, 1), **i64),
+                            torch.empty(3 * 48, dtype=torch.uint8, device=dev), ws, st)
     torch.cuda.synchronize()
     assert int(st.item()) == mt._lib.MTGR_ERR_CAPACITY

@@ -26,6 +26,34 @@ def lib():
     return _lib.load()
 
 
+def test_struct_layouts_match_header(tmp_path):
+    # the ctypes mirrors must match the C layouts field for field: compile the
+    # header with the host C compiler and compare every offset and size
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "mtgr.h"', 'int main(void) {']
+    for cname, cls in (("mtgr_batch", _lib.MtgrBatch), ("mtgr_block_params", _lib.MtgrBlockParams)):
+        lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append('printf("mtgr_work_item %zu\\n", sizeof(mtgr_work_item));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                  check=True).stdout.splitlines())
+    for cname, cls in (("mtgr_batch", _lib.MtgrBatch), ("mtgr_block_params", _lib.MtgrBlockParams)):
+        assert int(got[cname]) == ctypes.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(cls, f).offset, f"{cname}.{f}"
+    assert int(got["mtgr_work_item"]) == _lib.WORK_ITEM_BYTES
+
+
 def test_every_declared_symbol_is_exported(lib):
     names = _declared()
     assert len(names) >= 12
@@ -46,7 +74,7 @@ def test_host_validation_without_device(lib):
     assert lib.mtgr_pack_offsets(-1, None, 0, None, None, None, None, None) == E
     assert lib.mtgr_pack_offsets(2, None, 10, None, None, None, None, None) == E
     assert lib.mtgr_build_mask_meta(1, None, None, 1, 1, 1, 1, None, None, None, None, None, None,
-                                    None, None, None, 0, None, None) == E
+                                    None, None, None, None, 0, None, None) == E
     assert lib.mtgr_group_layernorm(4, 12, 0, None, None, 4, None, None, 1e-5, 0, None, None) == E
     assert lib.mtgr_hstu_attention_fwd(None, 64, 2, 0, None, 0, None, None) == E
     assert lib.mtgr_stack_fwd(None, 0, None, None, None, None, 0, None) == E
