@@ -73,6 +73,9 @@ _SIGNATURES = {
     "mtgr_build_mask_meta": (ctypes.c_int, [c_i32, c_vp, c_vp, c_i32, c_i32, c_i32, c_i64, c_vp,
                                             c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                             c_size, c_vp, c_vp]),
+    "mtgr_build_mask_meta_static": (ctypes.c_int, [c_i32, c_vp, c_vp, c_i32, c_i32, c_i32, c_i64,
+                                                   c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                                   c_vp, c_vp, c_vp, c_vp]),
     "mtgr_group_layernorm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp,
                                             c_float, c_i32, c_vp, c_vp]),
     "mtgr_hstu_attention_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_i32, c_i32, c_i32,
@@ -162,6 +165,20 @@ def mtgr_build_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity
         _ptr(d_qtile_desc), _ptr(d_row_ptr), _ptr(d_entries), _ptr(d_order), _ptr(d_counts),
         _ptr(d_rt_cnt), _ptr(d_rt_off), _ptr(d_rt_mask), _ptr(d_work), _ptr(d_ws), ws_bytes,
         _ptr(d_status), _stream(stream)))
+
+
+STATIC_META_SCRATCH_BYTES = 4 << 20
+
+
+def mtgr_build_mask_meta_static(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity,
+                                rt_capacity, d_qtile_desc, d_row_ptr, d_entries, d_order, d_counts,
+                                d_rt_cnt, d_rt_off, d_rt_mask, d_work, d_status, stream=None):
+    """mtgr_build_mask_meta with the library's fixed scratch instead of a workspace."""
+    _check("mtgr_build_mask_meta_static", load().mtgr_build_mask_meta_static(
+        B, _ptr(d_seg_off), _ptr(d_ts), q_capacity, kt_capacity, e_capacity, rt_capacity,
+        _ptr(d_qtile_desc), _ptr(d_row_ptr), _ptr(d_entries), _ptr(d_order), _ptr(d_counts),
+        _ptr(d_rt_cnt), _ptr(d_rt_off), _ptr(d_rt_mask), _ptr(d_work), _ptr(d_status),
+        _stream(stream)))
 
 
 def mtgr_group_layernorm(T, d, d_x, d_group_id, G, d_gamma, d_beta, eps, d_y, stream=None):

@@ -153,6 +153,41 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
                                   int32_t* d_status, mtgr_stream_t stream);
 
 /*
+ * mtgr_build_mask_meta without a caller-provided workspace, for callers that
+ * cannot allocate device memory when they build a batch: for example a serving
+ * process that hands all of its device memory to its own pool at start-up and
+ * forbids later allocations (cudaMalloc/cudaFree can synchronise the device and
+ * take unpredictable time), or a plain C host program that wants a fixed device
+ * footprint. The paper has no counterpart; this is a deployment convenience.
+ *
+ * Same arguments and results as mtgr_build_mask_meta minus d_ws / ws_bytes.
+ * The scratch (one byte per q-tile and k-tile) lives in a fixed array of
+ * MTGR_STATIC_META_SCRATCH_BYTES (4 MiB) inside the library's own device
+ * memory, which every GPU that loads the library holds until the process
+ * exits. Limits and behaviour:
+ *  - q_capacity * kt_capacity must not exceed MTGR_STATIC_META_SCRATCH_BYTES;
+ *    larger batches return MTGR_ERR_CAPACITY without touching the device (use
+ *    mtgr_build_mask_meta with your own workspace for those).
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - It never calls cudaMalloc, cudaFree or any allocating routine.
+ *  - All calls share the one array per device and it keeps the last call's
+ *    contents (every call overwrites what it reads, so nothing needs
+ *    clearing). Calls whose work overlaps on the GPU — on different streams or
+ *    from different host threads without ordering — race on it: order them.
+ */
+#define MTGR_STATIC_META_SCRATCH_BYTES (4u << 20)
+MTGR_API int mtgr_build_mask_meta_static(int32_t B, const int32_t* d_seg_off, const int64_t* d_ts,
+                                         int32_t q_capacity, int32_t kt_capacity,
+                                         int32_t e_capacity, int64_t rt_capacity,
+                                         int32_t* d_qtile_desc, int32_t* d_row_ptr,
+                                         int32_t* d_entries, int32_t* d_order, int64_t* d_counts,
+                                         int32_t* d_rt_cnt, int64_t* d_rt_off,
+                                         uint64_t* d_rt_mask, mtgr_work_item* d_work,
+                                         int32_t* d_status, mtgr_stream_t stream);
+
+/*
  * Group-Layer Normalization (fun-rec 7.3.3, the GLN formula):
  *   y_i = (x_i - mean_i) / sqrt(var_i + eps) * gamma[g(i)] + beta[g(i)]
  * with mean and biased variance of token i over its d features and g(i) the
