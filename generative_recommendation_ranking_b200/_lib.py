@@ -55,7 +55,7 @@ class MtgrBatch(ctypes.Structure):
                 ("counts", c_vp), ("rt_cnt", c_vp), ("rt_off", c_vp), ("rt_mask", c_vp),
                 ("work", c_vp), ("norm", c_vp), ("status", c_vp)]
 
-WORK_ITEM_BYTES = 48  # sizeof(mtgr_work_item)
+WORK_ITEM_BYTES = 64  # sizeof(mtgr_work_item)
 
 
 class MtgrBlockParams(ctypes.Structure):

@@ -61,7 +61,7 @@ class PackedBatch:
         self.row_ptr = torch.empty(self.q_cap + 1, **i32)
         self.entries = torch.empty(max(self.e_cap, 1), **i32)
         self.order = torch.empty(max(self.q_cap, 1), **i32)
-        self.counts = torch.zeros(3, dtype=torch.int64, device=dev)
+        self.counts = torch.zeros(4, dtype=torch.int64, device=dev)
         self.rt_cnt = torch.empty(max(self.T, 1), **i32)
         self.rt_off = torch.empty(self.B + 1, dtype=torch.int64, device=dev)
         self.rt_mask = torch.empty(max(self.rt_cap, 1), dtype=torch.int64, device=dev)
@@ -109,7 +109,7 @@ class PackedBatch:
     def meta(self) -> dict:
         """Mask metadata copied to the host (for inspection and tests)."""
         torch.cuda.synchronize(self.device)
-        Q, E, V = (int(v) for v in self.counts.cpu())
+        Q, E, V, P = (int(v) for v in self.counts.cpu())
         return dict(
             seg_off=self.seg_off.cpu().numpy(), user_off=self.user_off.cpu().numpy(),
             group_id=self.group_id[:self.T].cpu().numpy(),
@@ -118,7 +118,8 @@ class PackedBatch:
             order=self.order[:Q].cpu().numpy(), visible_pairs=V, Q=Q, E=E,
             rt_cnt=self.rt_cnt[:self.T].cpu().numpy(), rt_off=self.rt_off.cpu().numpy(),
             rt_mask=self.rt_mask[:self.rt_cap].cpu().numpy().view(np.uint64),
-            work=self.work[:Q * _lib.WORK_ITEM_BYTES].cpu().numpy().view(np.int32).reshape(Q, 12))
+            work=self.work[:P * _lib.WORK_ITEM_BYTES].cpu().numpy().view(np.int32).reshape(P, 16),
+            P=P)
 
 
 class BlockWeights:

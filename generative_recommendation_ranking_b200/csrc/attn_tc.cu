@@ -9,18 +9,23 @@
 // per-element test (only the user's column bound on the last tile), PARTIAL
 // tiles evaluate the rules per element.
 //
-// Work item = (q-tile, head), taken longest-first from the metadata's order.
-// Persistent CTAs, one per SM, 14 warps:
-//   warp 0      TMA producer: Q tile once per item, K and V tiles per k-tile
-//   warp 1      MMA issuer:  S = Q K^T (SS, M=128 N=128 K=16) into TMEM,
-//                            O += P V  (TS: P read from TMEM, M=128 N=64)
-//   warps 2-9   SiLU, two groups of 4 warps taking alternate k-tiles: S from
-//               TMEM -> mask -> P = silu(S) in f16 -> TMEM
+// Work item = (two consecutive q-tiles A, B of one user, head), from the
+// metadata's work list (users by descending length). The two q-tiles share
+// every key/value tile, so each 32 KB K/V load feeds 256 query rows; the
+// item walks the union of the two q-tiles' k-tile lists (a k-tile EMPTY for
+// one of them is fully masked for it). Persistent CTAs, one per SM, 14 warps:
+//   warp 0      TMA producer: Q_A, Q_B once per item, K and V per k-tile, the
+//               U tiles of the item at its end
+//   warp 1      MMA issuer:  S_A = Q_A K^T, S_B = Q_B K^T (SS, M=128 N=128
+//               K=16) into TMEM, then O_A += P_A V, O_B += P_B V (TS: P read
+//               from TMEM, M=128 N=64); S of k-tile j+1 is issued before P V
+//               of k-tile j
+//   warps 2-5   SiLU for q-tile A, warps 6-9 for q-tile B: S from TMEM ->
+//               mask -> P = silu(S) in f16 -> TMEM
 //   warps 10-13 epilogue: O from TMEM -> O / N (.) U -> global; and, for bf16
 //               inputs, the in-place bf16 -> f16 conversion of V tiles
-// TMEM (512 columns): S[2] (128 each), P[2] (64 each, f16 pairs), O[2] (64).
-// S and P are double-buffered, so S of tile j+1 is computed on the tensor
-// cores while the SiLU warps work on tile j.
+// TMEM (512 columns): S_A, S_B (128 each), P_A, P_B (64 each, f16 pairs),
+// O_A, O_B (64 each).
 //
 // P and V enter the second MMA as f16 (11-bit significand) rather than bf16:
 // the unnormalised silu weights span a wide range and bf16 rounding of P alone
@@ -43,18 +48,19 @@ namespace mtgr {
 namespace {
 
 constexpr int DH = 64;
-constexpr int TM = MTGR_TILE_M;  // 128 query rows per item
+constexpr int TM = MTGR_TILE_M;  // 128 query rows per q-tile
 constexpr int TN = MTGR_TILE_N;  // 128 keys per k-tile
-constexpr int KV_STAGES = 5;
-constexpr int TILE_BYTES = TM * DH * 2;  // 16 KB (Q, K or V tile)
+constexpr int KV_STAGES = 4;
+constexpr int TILE_BYTES = TM * DH * 2;  // 16 KB (one Q, K, V or U tile)
 constexpr int NUM_SILU_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_THREADS = 32 * (2 + NUM_SILU_WARPS + NUM_EPI_WARPS);  // 448
-__host__ __device__ constexpr uint32_t s_col(int b) { return 128u * b; }        // S[b]
-__host__ __device__ constexpr uint32_t p_col(int b) { return 256u + 64u * b; }  // P[b]
-__host__ __device__ constexpr uint32_t o_col(int b) { return 384u + 64u * b; }  // O[b]
+__host__ __device__ constexpr uint32_t s_col(int q) { return 128u * q; }        // S_A, S_B
+__host__ __device__ constexpr uint32_t p_col(int q) { return 256u + 64u * q; }  // P_A, P_B
+__host__ __device__ constexpr uint32_t o_col(int q) { return 384u + 64u * q; }  // O_A, O_B
 constexpr uint32_t TMEM_COLS = 512;
-constexpr size_t SMEM_BYTES = 1024 + 2 * TILE_BYTES + KV_STAGES * 2 * TILE_BYTES + 512;
+constexpr size_t SMEM_BYTES =
+    1024 + 4 * TILE_BYTES + KV_STAGES * 2 * TILE_BYTES + 2 * TILE_BYTES + 512;
 
 struct AttnArgs {
   int32_t d, H;
@@ -75,25 +81,50 @@ struct Item {
   int32_t h;
 };
 
-// Item w = (work-list slot w / H, head w % H): a single 48-byte record, so
-// the load has no dependent chain and can be issued one item ahead.
+// Item w = (work-list slot w / H, head w % H): one 64-byte record with no
+// dependent loads, so every role can issue it one item ahead.
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int32_t w) {
   Item it;
   const int32_t slot = w / a.H;
   it.h = w - slot * a.H;
   const int4* p = reinterpret_cast<const int4*>(a.work + slot);
-  const int4 x0 = __ldg(p), x1 = __ldg(p + 1), x2 = __ldg(p + 2);
+  const int4 x0 = __ldg(p), x1 = __ldg(p + 1), x2 = __ldg(p + 2), x3 = __ldg(p + 3);
   it.w.us = x0.x; it.w.n = x0.y; it.w.n_u = x0.z; it.w.n_us = x0.w;
-  it.w.c_lo = x1.x; it.w.qt = x1.y; it.w.b = x1.z; it.w.e0 = x1.w;
-  it.w.e1 = x2.x; it.w.reserved = x2.y;
-  it.w.rt_base = (int64_t)(uint32_t)x2.z | ((int64_t)x2.w << 32);
+  it.w.c_lo = x1.x; it.w.qt0 = x1.y; it.w.b = x1.z; it.w.nq = x1.w;
+  it.w.e0a = x2.x; it.w.e1a = x2.y; it.w.e0b = x2.z; it.w.e1b = x2.w;
+  it.w.n_union = x3.x; it.w.reserved = x3.y;
+  it.w.rt_base = (int64_t)(uint32_t)x3.z | ((int64_t)x3.w << 32);
   return it;
 }
 
 __device__ __forceinline__ int32_t num_items(const AttnArgs& a) {
-  const int64_t Q = a.counts[0] < a.q_cap ? a.counts[0] : a.q_cap;
-  return (int32_t)(Q * a.H);
+  const int64_t P = a.counts[3] < a.q_cap ? a.counts[3] : a.q_cap;
+  return (int32_t)(P * a.H);
 }
+
+// Walks the union of the two sorted k-tile lists of an item, in ascending kt.
+struct UnionCursor {
+  const int32_t* entries;
+  int32_t ia, e1a, ib, e1b, enta, entb;
+  __device__ __forceinline__ void init(const int32_t* ent, const mtgr_work_item& w) {
+    entries = ent;
+    ia = w.e0a; e1a = w.e1a; ib = w.e0b; e1b = w.e1b;
+    enta = ia < e1a ? __ldg(entries + ia) : 0;
+    entb = ib < e1b ? __ldg(entries + ib) : 0;
+  }
+  // Next k-tile: its index and each q-tile's entry code (-1 = EMPTY there,
+  // else (kt << 1) | partial).
+  __device__ __forceinline__ int32_t next(int32_t& code_a, int32_t& code_b) {
+    const int32_t ka = ia < e1a ? (enta >> 1) : 0x7fffffff;
+    const int32_t kb = ib < e1b ? (entb >> 1) : 0x7fffffff;
+    const int32_t kt = ka < kb ? ka : kb;
+    code_a = ka == kt ? enta : -1;
+    code_b = kb == kt ? entb : -1;
+    if (ka == kt && ++ia < e1a) enta = __ldg(entries + ia);
+    if (kb == kt && ++ib < e1b) entb = __ldg(entries + ib);
+    return kt;
+  }
+};
 
 // bits [lo, hi) of a 64-bit mask, clipped to [0, 64)
 __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
@@ -116,6 +147,8 @@ __device__ __forceinline__ uint32_t silu_pair(float a, float b) {
 
 // Visibility of keys [j0, j0 + 64) (user-relative, j0 a multiple of 64) to
 // query row i, whose rank-table index is cnt_i (rule 2 as a table lookup).
+// Evaluated from the rules alone, so it is exact for FULL, PARTIAL and EMPTY
+// tiles alike.
 __device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, const uint64_t* rt_mask,
                                                  int32_t i, int32_t cnt_i, int32_t j0) {
   uint64_t vis = range_bits(0, it.n_us - j0);  // rule 1: U and S keys
@@ -129,7 +162,7 @@ __device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, const
   return vis & range_bits(0, it.n - j0);  // keys past the user's end
 }
 
-// P for 32 consecutive keys [j0, j0 + 32) of one query row: 16 f16 pairs.
+// P for 32 consecutive keys of one query row: 16 f16 pairs.
 template <bool HALVE>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p)[16], bool masked,
                                            uint32_t vis) {
@@ -147,7 +180,6 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p
   }
 }
 
-
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
@@ -161,21 +193,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                       // [2][16 KB]
-  uint8_t* sKV = smem + 2 * TILE_BYTES;     // [stage][K 16 KB | V 16 KB]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + KV_STAGES * 2 * TILE_BYTES);
-  uint64_t* q_full = bars;                  // [2]
-  uint64_t* q_empty = bars + 2;             // [2]
-  uint64_t* kv_full = bars + 4;             // [KV_STAGES]
-  uint64_t* kv_empty = kv_full + KV_STAGES; // [KV_STAGES]
-  uint64_t* v_ready = kv_empty + KV_STAGES; // [KV_STAGES]
-  uint64_t* s_full = v_ready + KV_STAGES;   // [2]
-  uint64_t* s_free = s_full + 2;            // [2]
-  uint64_t* p_full = s_free + 2;            // [2]
-  uint64_t* p_free = p_full + 2;            // [2]
-  uint64_t* o_full = p_free + 2;            // [2]
-  uint64_t* o_free = o_full + 2;            // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 2);
+  uint8_t* sQ = smem;                        // [2 buffers][A | B][16 KB]
+  uint8_t* sKV = smem + 4 * TILE_BYTES;      // [stage][K 16 KB | V 16 KB]
+  uint8_t* sU = sKV + KV_STAGES * 2 * TILE_BYTES;  // [A | B][16 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sU + 2 * TILE_BYTES);
+  uint64_t* q_full = bars;                   // [2]
+  uint64_t* q_empty = bars + 2;              // [2]
+  uint64_t* kv_full = bars + 4;              // [KV_STAGES]
+  uint64_t* kv_empty = kv_full + KV_STAGES;  // [KV_STAGES]
+  uint64_t* v_ready = kv_empty + KV_STAGES;  // [KV_STAGES]
+  uint64_t* s_full = v_ready + KV_STAGES;    // [A, B]
+  uint64_t* s_free = s_full + 2;             // [A, B]
+  uint64_t* p_full = s_free + 2;             // [A, B]
+  uint64_t* p_free = p_full + 2;             // [A, B]
+  uint64_t* o_full = p_free + 2;
+  uint64_t* o_free = o_full + 1;
+  uint64_t* u_full = o_free + 1;
+  uint64_t* u_empty = u_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(u_empty + 1);
 
   const int warp = warp_id(), lane = lane_id();
   if (warp == 0 && lane == 0) {
@@ -187,14 +222,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&s_free[i], NUM_SILU_WARPS / 2);
       mbar_init(&p_full[i], NUM_SILU_WARPS / 2);
       mbar_init(&p_free[i], 1);
-      mbar_init(&o_full[i], 1);
-      mbar_init(&o_free[i], NUM_EPI_WARPS);
     }
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&v_ready[s], NUM_EPI_WARPS);
     }
+    mbar_init(o_full, 1);
+    mbar_init(o_free, NUM_EPI_WARPS);
+    mbar_init(u_full, 1);
+    mbar_init(u_empty, NUM_EPI_WARPS);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -220,14 +257,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const Item it = nxt;
         if (w + stride < n_items) nxt = load_item(a, w + stride);
         const int qb = li & 1;
-        const int32_t row_q = it.w.us + it.w.qt * TM;
+        const int32_t row_a = it.w.us + it.w.qt0 * TM;
         if (!mbar_wait(&q_empty[qb], ((li >> 1) & 1) ^ 1)) { timed_out = true; break; }
-        mbar_arrive_expect_tx(&q_full[qb], TILE_BYTES);
-        tma_load_2d(&tm, &q_full[qb], sQ + qb * TILE_BYTES, it.h * DH, row_q);
-        int32_t ent = it.w.e0 < it.w.e1 ? __ldg(a.entries + it.w.e0) : 0;
-        for (int32_t e = it.w.e0; e < it.w.e1; ++e, ++g) {
-          const int32_t kt = ent >> 1;
-          if (e + 1 < it.w.e1) ent = __ldg(a.entries + e + 1);
+        mbar_arrive_expect_tx(&q_full[qb], it.w.nq * TILE_BYTES);
+        tma_load_2d(&tm, &q_full[qb], sQ + (2 * qb) * TILE_BYTES, it.h * DH, row_a);
+        if (it.w.nq == 2)
+          tma_load_2d(&tm, &q_full[qb], sQ + (2 * qb + 1) * TILE_BYTES, it.h * DH, row_a + TM);
+        UnionCursor cur;
+        cur.init(a.entries, it.w);
+        for (int32_t t = 0; t < it.w.n_union; ++t, ++g) {
+          int32_t ca, cb;
+          const int32_t kt = cur.next(ca, cb);
           const int st = g % KV_STAGES;
           if (!mbar_wait(&kv_empty[st], ((g / KV_STAGES) & 1) ^ 1)) { timed_out = true; break; }
           uint8_t* sk = sKV + st * 2 * TILE_BYTES;
@@ -235,6 +275,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d(&tm, &kv_full[st], sk, d + it.h * DH, it.w.us + kt * TN);
           tma_load_2d(&tm, &kv_full[st], sk + TILE_BYTES, 2 * d + it.h * DH, it.w.us + kt * TN);
         }
+        if (timed_out) break;
+        // U of this item, needed only by its epilogue
+        if (!mbar_wait(u_empty, (li & 1) ^ 1)) { timed_out = true; break; }
+        mbar_arrive_expect_tx(u_full, it.w.nq * TILE_BYTES);
+        tma_load_2d(&tm, u_full, sU, 3 * d + it.h * DH, row_a);
+        if (it.w.nq == 2) tma_load_2d(&tm, u_full, sU + TILE_BYTES, 3 * d + it.h * DH, row_a + TM);
       }
     }
   } else if (warp == 1) {
@@ -242,91 +288,93 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
       constexpr uint32_t idesc_o = idesc_f16(TM, DH, 0u, false, true);
-      struct Pend { int32_t g, li, st; bool first, last; };
+      struct Pend { int32_t g, gb, st, li; bool first, last, two; };
       auto issue_pv = [&](const Pend& p) -> bool {
-        const int pb = p.g & 1, ob = p.li & 1;
-        if (p.first && !mbar_wait(&o_free[ob], ((p.li >> 1) & 1) ^ 1)) return false;
-        if (!mbar_wait(&p_full[pb], (p.g >> 1) & 1)) return false;
+        if (p.first && !mbar_wait(o_free, (p.li & 1) ^ 1)) return false;
         if (IN_BF16 && !mbar_wait(&v_ready[p.st], (p.g / KV_STAGES) & 1)) return false;
-        tc_fence_after();
         const uint32_t v_addr = smem_u32(sKV + p.st * 2 * TILE_BYTES + TILE_BYTES);
+        for (int q = 0; q < (p.two ? 2 : 1); ++q) {
+          const int32_t r = q == 0 ? p.g : p.gb;
+          if (!mbar_wait(&p_full[q], r & 1)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < TN / 16; ++k) {
-          tc_mma_ts(tmem + o_col(ob), tmem + p_col(pb) + 8 * k,
-                    sdesc_sw128(v_addr + 2048 * k, 16384, 1024), idesc_o,
-                    (!p.first || k > 0) ? 1u : 0u);
+          for (int k = 0; k < TN / 16; ++k) {
+            tc_mma_ts(tmem + o_col(q), tmem + p_col(q) + 8 * k,
+                      sdesc_sw128(v_addr + 2048 * k, 16384, 1024), idesc_o,
+                      (!p.first || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&p_free[q]);
         }
         tc_commit(&kv_empty[p.st]);
-        tc_commit(&p_free[pb]);
-        if (p.last) tc_commit(&o_full[ob]);
+        if (p.last) tc_commit(o_full);
         return true;
       };
-      // Issue order S_0, S_1, S_2, PV_0, S_3, PV_1, ...: S runs two k-tiles ahead
-      // of P V, so each SiLU group finds its next S computed when it finishes.
-      constexpr int LAG = 2;
-      Pend ring[LAG + 1];
-      int n_pend = 0, head = 0;
-      auto pop = [&]() -> bool {
-        const bool ok = issue_pv(ring[head]);
-        head = (head + 1) % (LAG + 1);
-        --n_pend;
-        return ok;
-      };
-      int32_t g = 0, li = 0;
+      // S of k-tile j+1 (both q-tiles) is issued before P V of k-tile j.
+      Pend pend{};
+      bool have_pend = false;
+      int32_t g = 0, gb = 0, li = 0;
       Item nxt;
       if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
       for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
         const Item it = nxt;
         if (w + stride < n_items) nxt = load_item(a, w + stride);
-        const int qb = li & 1, ob = li & 1;
-        const int32_t nnz = it.w.e1 - it.w.e0;
-        if (nnz <= 0) {  // cannot happen for valid metadata (the diagonal tile)
-          while (n_pend > 0 && !timed_out)
-            if (!pop()) timed_out = true;
-          if (timed_out) break;
+        const int qb = li & 1;
+        const bool two = it.w.nq == 2;
+        const int32_t nu = it.w.n_union;
+        if (nu <= 0) {  // cannot happen for valid metadata (the diagonal tile)
+          if (have_pend && !issue_pv(pend)) { timed_out = true; break; }
+          have_pend = false;
           if (!mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
           tc_commit(&q_empty[qb]);
-          if (!mbar_wait(&o_free[ob], ((li >> 1) & 1) ^ 1)) { timed_out = true; break; }
-          tc_commit(&o_full[ob]);
+          if (!mbar_wait(o_free, (li & 1) ^ 1)) { timed_out = true; break; }
+          tc_commit(o_full);
           continue;
         }
-        for (int32_t t = 0; t < nnz; ++t, ++g) {
-          const int st = g % KV_STAGES, sb = g & 1;
+        for (int32_t t = 0; t < nu; ++t, ++g) {
+          const int st = g % KV_STAGES;
           if (t == 0 && !mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
           if (!mbar_wait(&kv_full[st], (g / KV_STAGES) & 1)) { timed_out = true; break; }
-          if (!mbar_wait(&s_free[sb], ((g >> 1) & 1) ^ 1)) { timed_out = true; break; }
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(sQ + qb * TILE_BYTES);
           const uint32_t k_addr = smem_u32(sKV + st * 2 * TILE_BYTES);
+          bool ok = true;
+          for (int q = 0; q < (two ? 2 : 1); ++q) {
+            const int32_t r = q == 0 ? g : gb;
+            if (!mbar_wait(&s_free[q], (r & 1) ^ 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(sQ + (2 * qb + q) * TILE_BYTES);
 #pragma unroll
-          for (int k = 0; k < DH / 16; ++k) {
-            tc_mma_ss(tmem + s_col(sb), sdesc_sw128(q_addr + 32 * k, 16, 1024),
-                      sdesc_sw128(k_addr + 32 * k, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
+            for (int k = 0; k < DH / 16; ++k) {
+              tc_mma_ss(tmem + s_col(q), sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                        sdesc_sw128(k_addr + 32 * k, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
+            }
+            tc_commit(&s_full[q]);
           }
-          tc_commit(&s_full[sb]);
-          if (t == nnz - 1) tc_commit(&q_empty[qb]);
-          ring[(head + n_pend) % (LAG + 1)] = Pend{g, li, st, t == 0, t == nnz - 1};
-          if (++n_pend > LAG && !pop()) { timed_out = true; break; }
+          if (!ok) { timed_out = true; break; }
+          if (t == nu - 1) tc_commit(&q_empty[qb]);
+          if (have_pend && !issue_pv(pend)) { timed_out = true; break; }
+          pend = Pend{g, gb, st, li, t == 0, t == nu - 1, two};
+          have_pend = true;
+          if (two) ++gb;
         }
       }
-      while (!timed_out && n_pend > 0)
-        if (!pop()) timed_out = true;
+      if (!timed_out && have_pend && !issue_pv(pend)) timed_out = true;
     }
   } else if (warp < 2 + NUM_SILU_WARPS) {
     // -------------------------------------------------------- SiLU warps --
-    // Group gb takes the k-tiles g with g % 2 == gb (S and P buffer gb); each
-    // warp covers its 32 query rows across all 128 keys, in four 32-key
+    // warps 2-5 take q-tile A of every item, warps 6-9 q-tile B; each warp
+    // covers 32 query rows across all 128 keys of a k-tile, in four 32-key
     // chunks with the TMEM load of chunk k+1 in flight while chunk k is
     // computed.
     const int quarter = warp & 3;
-    const int gb = (warp - 2) >> 2;
+    const int q = (warp - 2) >> 2;  // 0: q-tile A, 1: q-tile B
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int32_t g0 = 0;  // CTA-wide index of the current item's first k-tile
+    const uint32_t s_addr = tmem + lane_base + s_col(q);
+    const uint32_t p_addr = tmem + lane_base + p_col(q);
+    int32_t gq = 0;  // this q-tile slot's k-tile counter (barrier rounds)
     Item nxt;
     int32_t cnt_nxt = 0;
     auto cnt_of = [&](const Item& x) -> int32_t {
-      const int32_t i = x.w.qt * TM + quarter * 32 + lane;
-      return i < x.w.n ? __ldg(a.rt_cnt + x.w.us + i) : 0;
+      const int32_t i = (x.w.qt0 + q) * TM + quarter * 32 + lane;
+      return (q < x.w.nq && i < x.w.n) ? __ldg(a.rt_cnt + x.w.us + i) : 0;
     };
     if ((int32_t)blockIdx.x < n_items) {
       nxt = load_item(a, blockIdx.x);
@@ -339,59 +387,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         nxt = load_item(a, w + stride);
         cnt_nxt = cnt_of(nxt);
       }
-      const int32_t i = it.w.qt * TM + quarter * 32 + lane;  // user-relative query row
-      const int32_t nnz = it.w.e1 - it.w.e0;
-      int32_t t = ((g0 & 1) == gb) ? 0 : 1;  // this group's first k-tile of the item
-      int32_t ent = t < nnz ? __ldg(a.entries + it.w.e0 + t) : 0;
-      for (; t < nnz; t += 2) {
-        const int32_t g = g0 + t;
-        const int32_t kt = ent >> 1;
-        const bool partial = ent & 1;
-        if (t + 2 < nnz) ent = __ldg(a.entries + it.w.e0 + t + 2);
-        const uint32_t r = static_cast<uint32_t>(g >> 1);
-        const bool masked = partial || kt * TN + TN > it.w.n;
+      if (q >= it.w.nq) continue;  // this item has no q-tile B
+      const int32_t i = (it.w.qt0 + q) * TM + quarter * 32 + lane;  // user-relative row
+      UnionCursor cur;
+      cur.init(a.entries, it.w);
+      for (int32_t t = 0; t < it.w.n_union; ++t, ++gq) {
+        int32_t ca, cb;
+        const int32_t kt = cur.next(ca, cb);
+        const int32_t code = q == 0 ? ca : cb;  // -1: EMPTY for this q-tile
+        const bool masked = code < 0 || (code & 1) || kt * TN + TN > it.w.n;
+        const uint32_t r = static_cast<uint32_t>(gq);
         uint64_t vis_lo = 0, vis_hi = 0;
         if (masked) {
           vis_lo = visible_bits(it.w, a.rt_mask, i, cnt_i, kt * TN);
           vis_hi = visible_bits(it.w, a.rt_mask, i, cnt_i, kt * TN + 64);
         }
-        if (!warp_wait(&s_full[gb], r & 1)) { timed_out = true; break; }
+        if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-        const uint32_t s_addr = tmem + lane_base + s_col(gb);
-        const uint32_t p_addr = tmem + lane_base + p_col(gb);
         uint32_t sa[32], sbuf[32];
         tmem_ld32(s_addr, sa);
         tmem_ld_wait();
-        if (!warp_wait(&p_free[gb], (r & 1) ^ 1)) { timed_out = true; break; }
+        if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          uint32_t (&cur)[32] = (k & 1) ? sbuf : sa;
+          uint32_t (&curv)[32] = (k & 1) ? sbuf : sa;
           uint32_t (&ahead)[32] = (k & 1) ? sa : sbuf;
           if (k < 3) tmem_ld32(s_addr + 32 * (k + 1), ahead);
           const uint64_t vv = k < 2 ? vis_lo : vis_hi;
           uint32_t p[16];
-          silu_chunk<HALVE>(cur, p, masked, (uint32_t)(vv >> (32 * (k & 1))));
+          silu_chunk<HALVE>(curv, p, masked, (uint32_t)(vv >> (32 * (k & 1))));
           tmem_st16(p_addr + 16 * k, p);
           if (k < 3) tmem_ld_wait();
           if (k == 2) {  // all of S is in registers: the MMA may overwrite it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[gb]);
+            if (lane == 0) mbar_arrive(&s_free[q]);
           }
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[gb]);
+        if (lane == 0) mbar_arrive(&p_full[q]);
       }
-      g0 += nnz;
     }
   } else {
     // ---------------------------------------------------- epilogue warps --
     const int quarter = warp & 3;
     const int et = (warp - 2 - NUM_SILU_WARPS) * 32 + lane;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int rr = quarter * 32 + lane;  // row within each q-tile
     int32_t g = 0, li = 0;
     Item nxt;
     if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
@@ -400,7 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (w + stride < n_items) nxt = load_item(a, w + stride);
       if (IN_BF16) {
         // convert this item's V tiles to f16 in place as they land
-        for (int32_t e = it.w.e0; e < it.w.e1; ++e, ++g) {
+        for (int32_t t = 0; t < it.w.n_union; ++t, ++g) {
           const int st = g % KV_STAGES;
           if (!warp_wait(&kv_full[st], (g / KV_STAGES) & 1)) { timed_out = true; break; }
           uint4* v4 = reinterpret_cast<uint4*>(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
@@ -419,56 +464,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (timed_out) break;
       }
-      const int ob = li & 1;
-      if (!warp_wait(&o_full[ob], (li >> 1) & 1)) { timed_out = true; break; }
+      if (!warp_wait(o_full, li & 1)) { timed_out = true; break; }
+      if (!warp_wait(u_full, li & 1)) { timed_out = true; break; }
       tc_fence_after();
-      uint32_t o0[32], o1[32];
-      tmem_ld32(tmem + lane_base + o_col(ob), o0);
-      tmem_ld32(tmem + lane_base + o_col(ob) + 32, o1);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[ob]);
-      const int32_t i = it.w.qt * TM + quarter * 32 + lane;
-      if (i < it.w.n) {
-        const bool empty = it.w.e1 <= it.w.e0;
-        const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.w.b] : (float)it.w.n);
-        const int64_t row = it.w.us + i;
-        const uint4* up = reinterpret_cast<const uint4*>(a.qkvu + row * 4 * d + 3 * d + it.h * DH);
+      const bool empty = it.w.n_union <= 0;
+      const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.w.b] : (float)it.w.n);
+      for (int q = 0; q < it.w.nq; ++q) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tmem + lane_base + o_col(q), o0);
+        tmem_ld32(tmem + lane_base + o_col(q) + 32, o1);
+        tmem_ld_wait();
+        if (q == it.w.nq - 1) {  // all of O read: the next item may accumulate
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
+        const int32_t i = (it.w.qt0 + q) * TM + rr;
+        if (i < it.w.n) {
+          const int64_t row = it.w.us + i;
+          const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {  // columns [8k, 8k + 8) of the head
-          const uint4 x = __ldg(up + k);
-          const uint32_t uw[4] = {x.x, x.y, x.z, x.w};
-          float ov[8];
+          for (int k = 0; k < 8; ++k) {  // columns [8k, 8k + 8) of the head
+            const uint4 x = *reinterpret_cast<const uint4*>(urow + ((k ^ (rr & 7)) << 4));
+            const uint32_t uw[4] = {x.x, x.y, x.z, x.w};
+            float ov[8];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float u0, u1;
-            if (IN_BF16) {
-              u0 = __uint_as_float(uw[c] << 16);
-              u1 = __uint_as_float(uw[c] & 0xffff0000u);
-            } else {
-              const __half2 hh = *reinterpret_cast<const __half2*>(&uw[c]);
-              u0 = __low2float(hh);
-              u1 = __high2float(hh);
+            for (int c = 0; c < 4; ++c) {
+              float u0, u1;
+              if (IN_BF16) {
+                u0 = __uint_as_float(uw[c] << 16);
+                u1 = __uint_as_float(uw[c] & 0xffff0000u);
+              } else {
+                const __half2 hh = *reinterpret_cast<const __half2*>(&uw[c]);
+                u0 = __low2float(hh);
+                u1 = __high2float(hh);
+              }
+              const int col = 8 * k + 2 * c;
+              const uint32_t r0 = col < 32 ? o0[col] : o1[col - 32];
+              const uint32_t r1 = col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32];
+              ov[2 * c] = __uint_as_float(r0) * inv_n * u0;
+              ov[2 * c + 1] = __uint_as_float(r1) * inv_n * u1;
             }
-            const int col = 8 * k + 2 * c;
-            const uint32_t r0 = col < 32 ? o0[col] : o1[col - 32];
-            const uint32_t r1 = col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32];
-            ov[2 * c] = __uint_as_float(r0) * inv_n * u0;
-            ov[2 * c + 1] = __uint_as_float(r1) * inv_n * u1;
-          }
-          if (OUT_F32) {
-            float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * d + it.h * DH + 8 * k);
-            op[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
-            op[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
-          } else {
-            uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * d + it.h * DH + 8 * k);
-            *op = make_uint4(cvt_bf16x2(ov[0], ov[1]), cvt_bf16x2(ov[2], ov[3]),
-                             cvt_bf16x2(ov[4], ov[5]), cvt_bf16x2(ov[6], ov[7]));
+            if (OUT_F32) {
+              float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * d + it.h * DH + 8 * k);
+              op[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
+              op[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+            } else {
+              uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * d + it.h * DH + 8 * k);
+              *op = make_uint4(cvt_bf16x2(ov[0], ov[1]), cvt_bf16x2(ov[2], ov[3]),
+                               cvt_bf16x2(ov[4], ov[5]), cvt_bf16x2(ov[6], ov[7]));
+            }
           }
         }
       }
-      if (!IN_BF16) g += it.w.e1 - it.w.e0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(u_empty);  // U of this item consumed
+      if (!IN_BF16) g += it.w.n_union;
     }
   }
   if (timed_out) set_status(a.status, MTGR_ERR_TIMEOUT);

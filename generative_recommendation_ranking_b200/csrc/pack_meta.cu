@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kScanThreads) meta_qtiles_kernel(
     int32_t B, const int32_t* seg_off, int32_t q_cap, int32_t kt_cap, int64_t rt_cap,
     int32_t* qtile_desc, int32_t* row_ptr, int64_t* rt_off, int64_t* counts, int32_t* status) {
   __shared__ int64_t warp_tot[32];
-  int64_t carry = 0, rt_carry = 0;
+  int64_t carry = 0, rt_carry = 0, pair_carry = 0;
   bool over = false;
   for (int32_t base = 0; base < B; base += kScanThreads) {
     const int32_t b = base + threadIdx.x;
@@ -155,9 +155,10 @@ __global__ void __launch_bounds__(kScanThreads) meta_qtiles_kernel(
       if (n_r > kMaxRt) over = true;
       rt = (int64_t)rt_groups(so[2] - so[0], so[3] - so[0]) * (n_r + 1);
     }
-    int64_t excl, rt_excl;
+    int64_t excl, rt_excl, pair_excl;
     const int64_t chunk = block_exclusive_scan(nq, warp_tot, excl);
     const int64_t rt_chunk = block_exclusive_scan(rt, warp_tot, rt_excl);
+    pair_carry += block_exclusive_scan((nq + 1) / 2, warp_tot, pair_excl);
     if (b < B) {
       rt_off[b] = rt_carry + rt_excl;
       for (int32_t qt = 0; qt < nq; ++qt) {
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(kScanThreads) meta_qtiles_kernel(
     counts[0] = any_over ? 0 : carry;
     counts[1] = 0;
     counts[2] = 0;
+    counts[3] = any_over ? 0 : pair_carry;
     row_ptr[0] = 0;
     if (any_over) set_status(status, MTGR_ERR_CAPACITY);
   }
@@ -322,6 +324,7 @@ __global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, 
     if (threadIdx.x == 0) {
       counts[0] = 0;
       counts[1] = 0;
+      counts[3] = 0;
       set_status(status, MTGR_ERR_CAPACITY);
     }
     return;
@@ -336,33 +339,64 @@ __global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, 
 // user's q-tiles into order[] and the work list (runs after the row_ptr scan).
 __global__ void __launch_bounds__(kScanThreads) meta_order_kernel(
     int32_t B, const int32_t* seg_off, int32_t q_cap, const int32_t* row_ptr,
-    const int64_t* rt_off, int32_t* order, mtgr_work_item* work, const int64_t* counts) {
+    const int32_t* entries, const int64_t* rt_off, int32_t* order, mtgr_work_item* work,
+    const int64_t* counts) {
+  constexpr int32_t kSmemUsers = 8192;
+  __shared__ int32_t n_sh[kSmemUsers];  // user lengths, when they fit
   if (counts[0] == 0) return;
+  const bool in_smem = B <= kSmemUsers;
+  if (in_smem) {
+    for (int32_t k = threadIdx.x; k < B; k += blockDim.x)
+      n_sh[k] = seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
+  }
+  __syncthreads();
   for (int32_t b = threadIdx.x; b < B; b += blockDim.x) {
     const int32_t* so = seg_off + 4 * (int64_t)b;
     const int32_t n = so[4] - so[0];
-    int64_t pos = 0, qstart = 0;
+    int64_t pos = 0, qstart = 0, ppos = 0;
     for (int32_t k = 0; k < B; ++k) {
-      const int32_t nk = seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
+      const int32_t nk =
+          in_smem ? n_sh[k] : seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
       const int32_t nqk = (nk + MTGR_TILE_M - 1) / MTGR_TILE_M;
       if (k < b) qstart += nqk;
-      if (nk > n || (nk == n && k < b)) pos += nqk;
+      if (nk > n || (nk == n && k < b)) {
+        pos += nqk;
+        ppos += (nqk + 1) / 2;
+      }
     }
     const int32_t nq = (n + MTGR_TILE_M - 1) / MTGR_TILE_M;
     for (int32_t qt = 0; qt < nq; ++qt) {
       const int64_t slot = pos + qt, q = qstart + qt;
-      if (slot >= q_cap || q >= q_cap) continue;
-      order[slot] = (int32_t)q;
+      if (slot < q_cap && q < q_cap) order[slot] = (int32_t)q;
+    }
+    for (int32_t pp = 0; 2 * pp < nq; ++pp) {
+      const int64_t slot = ppos + pp, qa = qstart + 2 * pp;
+      const bool two = 2 * pp + 1 < nq;
+      if (slot >= q_cap || qa + (two ? 1 : 0) >= q_cap) continue;
       mtgr_work_item it;
       it.us = so[0];
       it.n = n;
       it.n_u = so[1] - so[0];
       it.n_us = so[2] - so[0];
       it.c_lo = so[3] - so[0];
-      it.qt = qt;
+      it.qt0 = 2 * pp;
       it.b = b;
-      it.e0 = row_ptr[q];
-      it.e1 = row_ptr[q + 1];
+      it.nq = two ? 2 : 1;
+      it.e0a = row_ptr[qa];
+      it.e1a = row_ptr[qa + 1];
+      it.e0b = two ? row_ptr[qa + 1] : it.e1a;
+      it.e1b = two ? row_ptr[qa + 2] : it.e1a;
+      // size of the union of the two sorted k-tile lists
+      int32_t ia = it.e0a, ib = it.e0b, u = 0;
+      while (ia < it.e1a || ib < it.e1b) {
+        const int32_t ka = ia < it.e1a ? (entries[ia] >> 1) : 0x7fffffff;
+        const int32_t kb = ib < it.e1b ? (entries[ib] >> 1) : 0x7fffffff;
+        const int32_t kt = ka < kb ? ka : kb;
+        ia += ka == kt ? 1 : 0;
+        ib += kb == kt ? 1 : 0;
+        ++u;
+      }
+      it.n_union = u;
       it.reserved = 0;
       it.rt_base = rt_off[b];
       work[slot] = it;
@@ -431,14 +465,13 @@ int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32
   }
   meta_scan_kernel<<<1, kScanThreads, 0, s>>>(q_cap, e_cap, row_ptr, counts, status);
   if ((rc = launch_status()) != MTGR_OK) return rc;
-  meta_order_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, row_ptr, rt_off, order, work,
-                                              counts);
-  if ((rc = launch_status()) != MTGR_OK) return rc;
   if (q_cap > 0) {
     meta_fill_kernel<<<(q_cap + 7) / 8, 256, 0, s>>>(q_cap, kt_cap, e_cap, codes, row_ptr,
                                                      entries, counts);
-    rc = launch_status();
+    if ((rc = launch_status()) != MTGR_OK) return rc;
   }
-  return rc;
+  meta_order_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, row_ptr, entries, rt_off, order,
+                                              work, counts);
+  return launch_status();
 }
 }  // namespace mtgr

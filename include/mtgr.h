@@ -89,18 +89,22 @@ MTGR_API int mtgr_pack_offsets(int32_t B, const int32_t* d_lens, int32_t T, int3
 /* Bytes of device workspace mtgr_build_mask_meta needs. */
 MTGR_API size_t mtgr_mask_meta_workspace_bytes(int32_t q_capacity, int32_t kt_capacity);
 
-/* One q-tile of the attention's work list (48 bytes). */
+/* One item of the attention's work list (64 bytes): up to two consecutive
+ * q-tiles (qt0, qt0 + 1) of one user, which share every key/value tile load. */
 typedef struct mtgr_work_item {
-  int32_t us;      /* first row of the user */
-  int32_t n;       /* user length N_b */
-  int32_t n_u;     /* N_U */
-  int32_t n_us;    /* N_U + N_S */
-  int32_t c_lo;    /* N_U + N_S + N_R */
-  int32_t qt;      /* q-tile index within the user */
-  int32_t b;       /* user index */
-  int32_t e0, e1;  /* the q-tile's entries: [e0, e1) of the CSR */
+  int32_t us;       /* first row of the user */
+  int32_t n;        /* user length N_b */
+  int32_t n_u;      /* N_U */
+  int32_t n_us;     /* N_U + N_S */
+  int32_t c_lo;     /* N_U + N_S + N_R */
+  int32_t qt0;      /* first q-tile of the pair (within the user) */
+  int32_t b;        /* user index */
+  int32_t nq;       /* q-tiles in the item: 1 or 2 */
+  int32_t e0a, e1a; /* entries of q-tile qt0: [e0a, e1a) of the CSR */
+  int32_t e0b, e1b; /* entries of q-tile qt0 + 1 (empty range when nq == 1) */
+  int32_t n_union;  /* k-tiles non-empty for at least one of the two q-tiles */
   int32_t reserved;
-  int64_t rt_base; /* the user's first rank-table entry */
+  int64_t rt_base;  /* the user's first rank-table entry */
 } mtgr_work_item;
 
 /*
@@ -124,7 +128,8 @@ typedef struct mtgr_work_item {
  *   d_order      [q_capacity] int32: the attention's work order: q-tiles user
  *                by user, users by descending length (ties by ascending user
  *                index), each user's q-tiles by ascending qt
- *   d_counts     [3] int64: Q (q-tiles), E (entries), visible (query,key) pairs
+ *   d_counts     [4] int64: Q (q-tiles), E (entries), visible (query,key) pairs,
+ *                P (work items: q-tile pairs)
  *   rt_capacity  entries available in d_rt_mask (>= sum over users of
  *                G_b (N_R,b + 1), G_b = number of 64-column groups of the
  *                user's key range [N_U+N_S, N_U+N_S+N_R) that hold R keys)
@@ -137,8 +142,9 @@ typedef struct mtgr_work_item {
  *                within the user-relative 64-column group N_U+N_S rounded down
  *                to 64, plus g) of the R keys ranked below r. R key j != i is
  *                visible to query i iff its bit is set in the entry at r = cnt_i.
- *   d_work       [q_capacity] mtgr_work_item: the q-tiles in work order, each
- *                with its user's offsets and CSR range (one load per item)
+ *   d_work       [q_capacity] mtgr_work_item: the work list, in work order:
+ *                each user's q-tiles in pairs (qt 0-1, 2-3, ...), with the
+ *                user's offsets and both CSR ranges (one load per item)
  *   d_ws, ws_bytes  workspace of mtgr_mask_meta_workspace_bytes() bytes
  *   d_status     device status word (MTGR_ERR_CAPACITY if Q, E, the rank
  *                tables or a user's tile count exceed the capacities, or a
@@ -217,7 +223,7 @@ typedef struct mtgr_batch {
   const int32_t* row_ptr;     /* [q_capacity+1] */
   const int32_t* entries;     /* [E] */
   const int32_t* order;       /* [q_capacity] */
-  const int64_t* counts;      /* [3] Q, E, visible pairs */
+  const int64_t* counts;      /* [4] Q, E, visible pairs, P */
   const int32_t* rt_cnt;      /* [T] rank-table index of each token */
   const int64_t* rt_off;      /* [B+1] */
   const uint64_t* rt_mask;    /* rank tables of rule 2 */

@@ -150,11 +150,18 @@ def _xavier(rng: np.random.Generator, fan_out: int, fan_in: int) -> np.ndarray:
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bfloat16 (ties to even), kept as float32."""
-    a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return (r & 0xFFFFFFFF).astype(np.uint32).view(np.float32).reshape(a.shape)
+    """Round float32 values to the nearest bfloat16 (ties to even), kept as float32.
+
+    Works on the 32-bit patterns in place: add 0x7FFF plus the lowest kept bit,
+    then clear the low 16 bits (exact for every finite input)."""
+    a = np.array(a, dtype=np.float32, copy=True, order="C")
+    u = a.view(np.uint32)
+    lsb = u >> np.uint32(16)
+    lsb &= np.uint32(1)
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u &= np.uint32(0xFFFF0000)
+    return a
 
 
 def make_block_params(d: int, d_ff: int, rng: np.random.Generator, dtype: str = "bf16") -> dict:

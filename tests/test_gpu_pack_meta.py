@@ -38,20 +38,6 @@ def _check_batch(lens, ts):
     return b
 
 
-def _check_work_list(lens, m, ref):
-    """The work list restates, in work order, each q-tile's user offsets and CSR range."""
-    seg_off, _, _ = oracle.pack_offsets(lens)
-    w = m["work"]
-    assert w.shape[0] == len(ref["order"])
-    for slot, q in enumerate(ref["order"]):
-        b, qt = ref["qtile_desc"][q]
-        so = seg_off[4 * b:4 * b + 5].astype(np.int64)
-        want = [so[0], so[4] - so[0], so[1] - so[0], so[2] - so[0], so[3] - so[0], qt, b,
-                ref["row_ptr"][q], ref["row_ptr"][q + 1], 0]
-        np.testing.assert_array_equal(w[slot, :10], want)
-        assert int(w[slot, 10]) | (int(w[slot, 11]) << 32) == int(m["rt_off"][b])
-
-
 def _check_rank_tables(lens, ts, m):
     """Rule 2 as tables: for every query row i and every 64-column group g
     holding R keys, the table entry at cnt_i must equal the R columns of that
@@ -75,6 +61,33 @@ def _check_rank_tables(lens, ts, m):
             weights = np.left_shift(np.uint64(1), np.arange(64, dtype=np.uint64))
             want = (sub.astype(np.uint64) * weights[None, :]).sum(axis=1, dtype=np.uint64)
             np.testing.assert_array_equal(tab[cnt], want)
+
+
+def _check_work_list(lens, m, ref):
+    """The work list restates, in work order, each user's q-tiles in pairs
+    (qt 0-1, 2-3, ...) with the user offsets, both CSR ranges and the size of
+    the union of the two k-tile lists."""
+    seg_off, _, _ = oracle.pack_offsets(lens)
+    order, desc, rp, ent = ref["order"], ref["qtile_desc"], ref["row_ptr"], ref["entries"]
+    want = []
+    i = 0
+    while i < len(order):
+        qa = order[i]
+        b, qt = desc[qa]
+        two = i + 1 < len(order) and desc[order[i + 1]][0] == b and qt % 2 == 0
+        qb = order[i + 1] if two else None
+        so = seg_off[4 * b:4 * b + 5].astype(np.int64)
+        ka = set((ent[rp[qa]:rp[qa + 1]] >> 1).tolist())
+        kb = set((ent[rp[qb]:rp[qb + 1]] >> 1).tolist()) if two else set()
+        want.append([so[0], so[4] - so[0], so[1] - so[0], so[2] - so[0], so[3] - so[0], qt, b,
+                     2 if two else 1, rp[qa], rp[qa + 1], rp[qb] if two else rp[qa + 1],
+                     rp[qb + 1] if two else rp[qa + 1], len(ka | kb), 0, int(m["rt_off"][b])])
+        i += 2 if two else 1
+    w = m["work"]
+    assert m["P"] == len(want) == w.shape[0]
+    for got, exp in zip(w, want):
+        np.testing.assert_array_equal(got[:14], exp[:14])
+        assert int(got[14]) | (int(got[15]) << 32) == exp[14]
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2, 3])
@@ -154,8 +167,8 @@ def test_capacity_overflow_sets_device_status():
     # e_capacity 2 < the 9 tiles this user has
     mt.mtgr_build_mask_meta(1, b.seg_off, b.d_ts, 3, 3, 2, b.rt_cap, torch.empty(3, 2, **i32),
                             torch.empty(4, **i32), torch.empty(2, **i32), torch.empty(3, **i32),
-                            torch.zeros(3, **i64), torch.empty(b.T, **i32), torch.empty(2, **i64),
+                            torch.zeros(4, **i64), torch.empty(b.T, **i32), torch.empty(2, **i64),
                             torch.empty(max(b.rt_cap, 1), **i64),
-                            torch.empty(3 * 48, dtype=torch.uint8, device=dev), ws, st)
+                            torch.empty(3 * 64, dtype=torch.uint8, device=dev), ws, st)
     torch.cuda.synchronize()
     assert int(st.item()) == mt._lib.MTGR_ERR_CAPACITY

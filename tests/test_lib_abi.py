@@ -40,6 +40,7 @@ def test_struct_layouts_match_header(tmp_path):
         for f, _ in cls._fields_:
             lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
     lines.append('printf("mtgr_work_item %zu\\n", sizeof(mtgr_work_item));')
+    lines.append('printf("mtgr_work_item.rt_base %zu\\n", offsetof(mtgr_work_item, rt_base));')
     lines.append("return 0; }")
     src = tmp_path / "layout.c"
     src.write_text("\n".join(lines))
@@ -52,6 +53,7 @@ def test_struct_layouts_match_header(tmp_path):
         for f, _ in cls._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(cls, f).offset, f"{cname}.{f}"
     assert int(got["mtgr_work_item"]) == _lib.WORK_ITEM_BYTES
+    assert int(got["mtgr_work_item.rt_base"]) == 56
 
 
 def test_every_declared_symbol_is_exported(lib):

@@ -16,10 +16,12 @@ def test_bf16_round_matches_torch():
 
 def test_workloads_deterministic_and_shaped():
     for idx in (0, 1):
-        a = synth.make_workload(idx, seed=3)
-        b = synth.make_workload(idx, seed=3)
+        a = synth.make_workload(idx, seed=3, B=8)
+        b = synth.make_workload(idx, seed=3, B=8)
         np.testing.assert_array_equal(a["lens"], b["lens"])
         np.testing.assert_array_equal(a["ts"], b["ts"])
+        feats = "x" if idx == 0 else "qkvu"
+        np.testing.assert_array_equal(a[feats], b[feats])
     w0 = synth.make_workload(0)
     assert w0["lens"].tolist() == [[4, 32, 8, 8]] * 4
     assert w0["x"].shape == (208, 64) and len(w0["layers"]) == 1

@@ -27,7 +27,7 @@ def _buffers(lens, dev):
         row_ptr=torch.full((q_cap + 1,), -7, **i32),
         entries=torch.full((max(e_cap, 1),), -7, **i32),
         order=torch.full((max(q_cap, 1),), -7, **i32),
-        counts=torch.full((3,), -7, **i64),
+        counts=torch.full((4,), -7, **i64),
         rt_cnt=torch.full((max(T, 1),), -7, **i32),
         rt_off=torch.full((B + 1,), -7, **i64),
         rt_mask=torch.full((max(rt_cap, 1),), -7, **i64),
@@ -37,13 +37,13 @@ def _buffers(lens, dev):
 
 def _results(bf):
     torch.cuda.synchronize()
-    Q, E = int(bf["counts"][0]), int(bf["counts"][1])
+    Q, E, P = int(bf["counts"][0]), int(bf["counts"][1]), int(bf["counts"][3])
     return dict(
         counts=bf["counts"].cpu().numpy(), qtile_desc=bf["qtile_desc"][:Q].cpu().numpy(),
         row_ptr=bf["row_ptr"][:Q + 1].cpu().numpy(), entries=bf["entries"][:E].cpu().numpy(),
         order=bf["order"][:Q].cpu().numpy(), rt_cnt=bf["rt_cnt"].cpu().numpy(),
         rt_off=bf["rt_off"].cpu().numpy(), rt_mask=bf["rt_mask"][:bf["rt_cap"]].cpu().numpy(),
-        work=bf["work"][:Q * _lib.WORK_ITEM_BYTES].cpu().numpy(),
+        work=bf["work"][:P * _lib.WORK_ITEM_BYTES].cpu().numpy(),
         status=int(bf["status"].item()))
 
 
