@@ -52,7 +52,9 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, help="workload index (0-3)")
+    ap.add_argument("--config", type=int, default=2,
+                    help="workload: 0 fp32 block, 1 attention only, 2 block (default), "
+                         "3 8-layer stack, 4 candidate sweep")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -241,34 +243,125 @@ def ncu_traffic(cls: str):
     return e.get("bytes_per_launch")
 
 
+class Workspace:
+    """Device-side state of one workload: inputs, batch metadata, weights and
+    workspace; ``step`` runs one pass of the hot path through the C ABI."""
+
+    def __init__(self, wl, dev, stream):
+        import generative_recommendation_ranking_b200 as mt
+        from generative_recommendation_ranking_b200 import _lib
+        self.wl, self.dev, self.stream, self._lib = wl, dev, stream, _lib
+        self.kind = wl["kind"]
+        self.d, self.H = wl["d"], wl["H"]
+        if self.kind == "attention":
+            self.x = torch.from_numpy(wl["qkvu"]).to(dev).to(torch.bfloat16)
+            self.out = torch.empty(int(wl["lens"].sum()), self.d, dtype=torch.float32, device=dev)
+        else:
+            self.x = torch.from_numpy(wl["x"]).to(dev)
+            self.out = torch.empty_like(self.x)
+        self.batch = mt.PackedBatch(wl["lens"], wl["ts"], device=dev, norm=wl.get("norm"))
+        self.layers = [mt.BlockWeights(p, self.H, dtype=wl["dtype"], device=dev)
+                       for p in wl["layers"]]
+        self.ws = mt.stack_workspace(self.layers, self.batch) if self.layers else None
+        self.batch.check()
+
+    def step(self, lens_d=None, ts_d=None, x_d=None, out_d=None, stream=None):
+        s = self.stream if stream is None else stream
+        b = self.batch
+        b.pack(s, d_lens=b.d_lens if lens_d is None else lens_d)
+        b.build_meta(s, d_ts=b.d_ts if ts_d is None else ts_d)
+        x_d = self.x if x_d is None else x_d
+        out_d = self.out if out_d is None else out_d
+        if self.kind == "attention":
+            self._lib.mtgr_hstu_attention_fwd(b.c, self.d, self.H, x_d, out_d, s)
+        else:
+            self._lib.mtgr_stack_fwd([l.c for l in self.layers], b.c, x_d, out_d, self.ws, s)
+
+
+def time_steps(fn, n, stream) -> float:
+    """Device milliseconds of n calls of fn on `stream` (CUDA events)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_e2e(wsp: Workspace, steps: int, world: int, dev):
+    """The same step end to end through the C ABI with pinned host buffers:
+    every step copies its inputs host->device and its whole output back. Copies
+    in, compute and copies out run on three streams with two buffer sets, so
+    step k's output copy overlaps step k+1's input copy (PCIe is full duplex)."""
+    wl = wsp.wl
+    hx = torch.from_numpy(np.ascontiguousarray(wl["qkvu"] if wsp.kind == "attention" else wl["x"]))
+    hx = (hx.to(torch.bfloat16) if wsp.kind == "attention" else hx).pin_memory()
+    hl = torch.from_numpy(np.ascontiguousarray(wl["lens"])).pin_memory()
+    ht = torch.from_numpy(np.ascontiguousarray(wl["ts"])).pin_memory()
+    hout = [torch.empty(wsp.out.shape, dtype=wsp.out.dtype).pin_memory() for _ in range(2)]
+    dx = [torch.empty_like(wsp.x) for _ in range(2)]
+    dl = [torch.empty_like(wsp.batch.d_lens) for _ in range(2)]
+    dts = [torch.empty_like(wsp.batch.d_ts) for _ in range(2)]
+    dout = [torch.empty_like(wsp.out) for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "cmp", "out")}
+    h2d = hx.numel() * hx.element_size() + hl.numel() * 4 + ht.numel() * 8
+    d2h = hout[0].numel() * hout[0].element_size()
+
+    def run(n):
+        for k in range(n):
+            i = k & 1
+            s_in.wait_event(ev["cmp"][i])   # step k-2 has finished reading these inputs
+            with torch.cuda.stream(s_in):
+                dx[i].copy_(hx, non_blocking=True)
+                dl[i].copy_(hl, non_blocking=True)
+                dts[i].copy_(ht, non_blocking=True)
+            ev["in"][i].record(s_in)
+            s_cmp.wait_event(ev["in"][i])
+            s_cmp.wait_event(ev["out"][i])  # step k-2's output has been copied out
+            wsp.step(dl[i], dts[i], dx[i], dout[i], stream=s_cmp)
+            ev["cmp"][i].record(s_cmp)
+            s_out.wait_event(ev["cmp"][i])
+            with torch.cuda.stream(s_out):
+                hout[i].copy_(dout[i], non_blocking=True)
+            ev["out"][i].record(s_out)
+
+    run(2)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    run(steps)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
+    torch.cuda.synchronize(dev)
+    ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    wsp.batch.check()
+    wsp.step()
+    torch.cuda.synchronize(dev)
+    assert torch.equal(hout[(steps - 1) & 1], wsp.out.cpu()), "e2e output mismatch"
+    B = int(wl["lens"].shape[0])
+    return {"value": B * world * steps / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ems / steps,
+            "pipelining": "3 streams (copy in / compute / copy out), 2 buffer sets"}
+
+
 def run_ours(args, world, rank, local):
-    import generative_recommendation_ranking_b200 as mt
     from generative_recommendation_ranking_b200 import _lib
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     wl = synth.make_workload(args.config, seed=args.seed + rank)
-    if wl["kind"] not in ("block", "stack"):
-        raise SystemExit("bench.py times the block/stack workloads (configs 0, 2, 3)")
+    if wl["kind"] == "sweep":
+        raise SystemExit("use --config 4 through run_sweep")
     B, T, d, H, dff, L = (int(wl["lens"].shape[0]), int(wl["lens"].sum()), wl["d"], wl["H"],
                           wl["d_ff"], wl["L"])
     stream = torch.cuda.current_stream(dev)
-
-    # inputs resident in HBM
-    x = torch.from_numpy(wl["x"]).to(dev)
-    batch = mt.PackedBatch(wl["lens"], wl["ts"], device=dev)
-    layers = [mt.BlockWeights(p, H, dtype=wl["dtype"], device=dev) for p in wl["layers"]]
-    ws = mt.stack_workspace(layers, batch)
-    out = torch.empty_like(x)
-    batch.check()
-
-    def step(lens_d, ts_d, x_d, out_d):
-        batch.pack(stream, d_lens=lens_d)
-        batch.build_meta(stream, d_ts=ts_d)
-        _lib.mtgr_stack_fwd([l.c for l in layers], batch.c, x_d, out_d, ws, stream)
-
+    wsp = Workspace(wl, dev, stream)
+    batch = wsp.batch
     for _ in range(args.warmup):
-        step(batch.d_lens, batch.d_ts, x, out)
+        wsp.step()
     batch.check()
 
     timer = _lib.Timer()
@@ -277,69 +370,29 @@ def run_ours(args, world, rank, local):
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize(dev)
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     timer.attach()
-    t_start.record(stream)
-    for _ in range(args.steps):
-        step(batch.d_lens, batch.d_ts, x, out)
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
+    ms = time_steps(wsp.step, args.steps, stream)
     timer.detach()
     barrier(world)
     clk = clocks.stop()
-    ms = t_start.elapsed_time(t_end)
     ms_max = max_over_ranks(ms, world, dev)
     batch.check()
     per_class = timer.read()
-    Q, E, V = (int(v) for v in batch.counts.cpu())
-
-    # e2e: host (pinned) inputs -> device -> step -> host output, through the C ABI
-    e2e = None
-    if not args.no_e2e:
-        hx = torch.from_numpy(wl["x"]).pin_memory()
-        hl = torch.from_numpy(np.ascontiguousarray(wl["lens"])).pin_memory()
-        ht = torch.from_numpy(np.ascontiguousarray(wl["ts"])).pin_memory()
-        hout = torch.empty(T, d, dtype=torch.float32).pin_memory()
-        dx, dl, dts = torch.empty_like(x), torch.empty_like(batch.d_lens), torch.empty_like(batch.d_ts)
-        h2d = hx.numel() * 4 + hl.numel() * 4 + ht.numel() * 8
-        d2h = hout.numel() * 4
-
-        def e2e_step():
-            dx.copy_(hx, non_blocking=True)
-            dl.copy_(hl, non_blocking=True)
-            dts.copy_(ht, non_blocking=True)
-            step(dl, dts, dx, out)
-            hout.copy_(out, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        batch.check()
-        assert torch.equal(hout, out.cpu()), "e2e output mismatch"
-        e2e = {"value": B * world * args.e2e_steps / (ems / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": ems / args.e2e_steps}
+    Q, E, V, P = (int(v) for v in batch.counts.cpu())
+    e2e = None if args.no_e2e else run_e2e(wsp, args.e2e_steps, world, dev)
 
     if rank != 0:
         return
     peaks, peak_src = load_peaks()
+    f32 = wl["dtype"] == "f32"
     # algorithmic work per launch of each class
+    gln_bytes = (8.0 if f32 else 5.0) * d * T  # bf16 path: GroupLN_1 6d, GroupLN_2 4d bytes/token
     work = {
         "gemm_qkvu": ("tensor", 2.0 * T * 4 * d * d),
         "attention": ("tensor", 4.0 * d * V),
         "gemm_mlp1": ("tensor", 2.0 * T * dff * d),
         "gemm_mlp2": ("tensor", 2.0 * T * d * dff),
-        # GroupLN_1 reads f32 and writes bf16 (6d bytes/token); GroupLN_2 reads and
-        # writes bf16 (4d bytes/token): 5d bytes/token per launch on average
-        "gln": ("hbm", 5.0 * d * T),
+        "gln": ("hbm", gln_bytes),
     }
     kernels = {}
     for cls, (bound, w) in work.items():
@@ -379,14 +432,49 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": wl["dtype"], "data": "synthetic",
         "config": workload_config(wl, world),
         "masked_attn": {"tflops": att.get("achieved"),
                         "frac_of_bf16_peak": att.get("frac"),
-                        "visible_pairs_per_gpu": V, "q_tiles": Q, "tile_entries": E},
+                        "visible_pairs_per_gpu": V, "q_tiles": Q, "tile_entries": E,
+                        "work_items": P},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": launches, "kernels": kernels,
     }
+    print(json.dumps(line), flush=True)
+
+
+def run_sweep(args, local):
+    """Candidate scaling for one user (d_model 512, 8 heads, one block): the
+    aggregated sample [U, S, R, c_1..c_K] against K expanded rows [U, S, R, c_i]
+    at the same normaliser, for K in 1, 8, 64, 512."""
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for K in synth.WORKLOADS[4].sweep_k:
+        agg = synth.make_workload(4, seed=args.seed, k_override=K)
+        res = {"K": K}
+        for name, wl in (("aggregated", agg), ("expanded", synth.sweep_expanded(agg))):
+            wsp = Workspace(wl, dev, stream)
+            for _ in range(max(3, args.warmup)):
+                wsp.step()
+            wsp.batch.check()
+            n = max(5, min(args.steps, 50))
+            ms = time_steps(wsp.step, n, stream) / n
+            wsp.batch.check()
+            res[f"{name}_ms"] = ms
+            res[f"{name}_ms_per_candidate"] = ms / K
+            del wsp
+            torch.cuda.empty_cache()
+        rows.append(res)
+    marginal = (rows[-1]["aggregated_ms"] - rows[0]["aggregated_ms"]) / (rows[-1]["K"] - rows[0]["K"])
+    line = {"metric": "candidate sweep: HSTU-block fwd ms per candidate, aggregated vs expanded rows",
+            "unit": "ms", "higher_is_better": False, "data": "synthetic", "dtype": "bf16",
+            "config": {"workload": "sweep_b1_d512", "d_model": 512, "heads": 8, "d_ff": 2048,
+                       "n_u": 24, "s": 1000, "r": 64},
+            "sweep": rows, "aggregated_marginal_ms_per_added_candidate": marginal,
+            "expanded_ms_per_row_at_k512": rows[-1]["expanded_ms_per_candidate"]}
     print(json.dumps(line), flush=True)
 
 
@@ -397,6 +485,9 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif synth.WORKLOADS[args.config].kind == "sweep":
+            if rank == 0:
+                run_sweep(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:
