@@ -13,16 +13,22 @@
 // metadata's work list (users by descending length). The two q-tiles share
 // every key/value tile, so each 32 KB K/V load feeds 256 query rows; the
 // item walks the union of the two q-tiles' k-tile lists (a k-tile EMPTY for
-// one of them is fully masked for it). Persistent CTAs, one per SM, 14 warps:
+// one of them is fully masked for it). Persistent CTAs, one per SM, 15 warps:
 //   warp 0      TMA producer: Q_A, Q_B once per item, K and V per k-tile, the
 //               U tiles of the item at its end
-//   warp 1      MMA issuer:  S_A = Q_A K^T, S_B = Q_B K^T (SS, M=128 N=128
-//               K=16) into TMEM, then O_A += P_A V, O_B += P_B V (TS: P read
-//               from TMEM, M=128 N=64); S of k-tile j+1 is issued before P V
-//               of k-tile j
-//   warps 2-5   SiLU for q-tile A, warps 6-9 for q-tile B: S from TMEM ->
-//               mask -> P = silu(S) in f16 -> TMEM
-//   warps 10-13 epilogue: O from TMEM -> O / N (.) U -> global; and, for bf16
+//   warp 1      S issuer:  S_A = Q_A K^T, S_B = Q_B K^T (SS, M=128 N=128 K=16)
+//               into TMEM
+//   warp 2      PV issuer: O_A += P_A V, O_B += P_B V (TS: P read from TMEM,
+//               M=128 N=64 K=16)
+//               A tcgen05.mma issue returns only once the tensor pipe takes
+//               the instruction, so an issuing thread that stops to wait on a
+//               barrier leaves the pipe idle; with two issuers each one's
+//               barrier waits overlap the other's MMAs.
+//   warps 3-6   SiLU for q-tile A, warps 7-10 for q-tile B: S from TMEM to
+//               registers (S released at once, so the next k-tile's scores
+//               can be computed meanwhile) -> mask -> P = silu(S) in f16 ->
+//               TMEM once the previous P V has read P
+//   warps 11-14 epilogue: O from TMEM -> O / N (.) U -> global; and, for bf16
 //               inputs, the in-place bf16 -> f16 conversion of V tiles
 // TMEM (512 columns): S_A, S_B (128 each), P_A, P_B (64 each, f16 pairs),
 // O_A, O_B (64 each).
@@ -54,7 +60,9 @@ constexpr int KV_STAGES = 4;
 constexpr int TILE_BYTES = TM * DH * 2;  // 16 KB (one Q, K, V or U tile)
 constexpr int NUM_SILU_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
-constexpr int NUM_THREADS = 32 * (2 + NUM_SILU_WARPS + NUM_EPI_WARPS);  // 448
+constexpr int SILU_WARP0 = 3;  // warps 0-2: TMA producer, S issuer, PV issuer
+constexpr int EPI_WARP0 = SILU_WARP0 + NUM_SILU_WARPS;
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);  // 480
 __host__ __device__ constexpr uint32_t s_col(int q) { return 128u * q; }        // S_A, S_B
 __host__ __device__ constexpr uint32_t p_col(int q) { return 256u + 64u * q; }  // P_A, P_B
 __host__ __device__ constexpr uint32_t o_col(int q) { return 384u + 64u * q; }  // O_A, O_B
@@ -135,16 +143,6 @@ __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
   return m << lo;
 }
 
-template <bool HALVE>
-__device__ __forceinline__ uint32_t silu_pair(float a, float b) {
-  if (HALVE) {
-    a *= 0.5f;
-    b *= 0.5f;
-  }
-  const uint32_t h = cvt_f16x2(a, b);
-  return fma_f16x2(h, tanh_f16x2(h), h);
-}
-
 // Visibility of keys [j0, j0 + 64) (user-relative, j0 a multiple of 64) to
 // query row i, whose rank-table index is cnt_i (rule 2 as a table lookup).
 // Evaluated from the rules alone, so it is exact for FULL, PARTIAL and EMPTY
@@ -162,21 +160,23 @@ __device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, const
   return vis & range_bits(0, it.n - j0);  // keys past the user's end
 }
 
-// P for 32 consecutive keys of one query row: 16 f16 pairs.
+// h = s / 2 (or s, when the scores arrive halved) for 16 consecutive keys of
+// one query row as 8 f16 pairs, masked keys set to 0 (silu(0) = 0).
 template <bool HALVE>
-__device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p)[16], bool masked,
-                                           uint32_t vis) {
-  if (masked) {
+__device__ __forceinline__ void scores_to_h(const uint32_t (&s)[16], uint32_t* h, bool masked,
+                                            uint32_t vis) {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const float x0 = (vis >> (2 * c)) & 1u ? __uint_as_float(s[2 * c]) : 0.f;
-      const float x1 = (vis >> (2 * c + 1)) & 1u ? __uint_as_float(s[2 * c + 1]) : 0.f;
-      p[c] = silu_pair<HALVE>(x0, x1);
+  for (int c = 0; c < 8; ++c) {
+    float x0 = __uint_as_float(s[2 * c]), x1 = __uint_as_float(s[2 * c + 1]);
+    if (masked) {
+      x0 = (vis >> (2 * c)) & 1u ? x0 : 0.f;
+      x1 = (vis >> (2 * c + 1)) & 1u ? x1 : 0.f;
     }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 16; ++c)
-      p[c] = silu_pair<HALVE>(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
+    if (HALVE) {
+      x0 *= 0.5f;
+      x1 *= 0.5f;
+    }
+    h[c] = cvt_f16x2(x0, x1);
   }
 }
 
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);  // K read by the S MMAs, V by the P V MMAs
       mbar_init(&v_ready[s], NUM_EPI_WARPS);
     }
     mbar_init(o_full, 1);
@@ -284,34 +284,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // -------------------------------------------------------- MMA issuer --
+    // --------------------------------------------------- S issuer (MMA) --
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
-      constexpr uint32_t idesc_o = idesc_f16(TM, DH, 0u, false, true);
-      struct Pend { int32_t g, gb, st, li; bool first, last, two; };
-      auto issue_pv = [&](const Pend& p) -> bool {
-        if (p.first && !mbar_wait(o_free, (p.li & 1) ^ 1)) return false;
-        if (IN_BF16 && !mbar_wait(&v_ready[p.st], (p.g / KV_STAGES) & 1)) return false;
-        const uint32_t v_addr = smem_u32(sKV + p.st * 2 * TILE_BYTES + TILE_BYTES);
-        for (int q = 0; q < (p.two ? 2 : 1); ++q) {
-          const int32_t r = q == 0 ? p.g : p.gb;
-          if (!mbar_wait(&p_full[q], r & 1)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < TN / 16; ++k) {
-            tc_mma_ts(tmem + o_col(q), tmem + p_col(q) + 8 * k,
-                      sdesc_sw128(v_addr + 2048 * k, 16384, 1024), idesc_o,
-                      (!p.first || k > 0) ? 1u : 0u);
-          }
-          tc_commit(&p_free[q]);
-        }
-        tc_commit(&kv_empty[p.st]);
-        if (p.last) tc_commit(o_full);
-        return true;
-      };
-      // S of k-tile j+1 (both q-tiles) is issued before P V of k-tile j.
-      Pend pend{};
-      bool have_pend = false;
       int32_t g = 0, gb = 0, li = 0;
       Item nxt;
       if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
@@ -320,25 +295,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (w + stride < n_items) nxt = load_item(a, w + stride);
         const int qb = li & 1;
         const bool two = it.w.nq == 2;
-        const int32_t nu = it.w.n_union;
-        if (nu <= 0) {  // cannot happen for valid metadata (the diagonal tile)
-          if (have_pend && !issue_pv(pend)) { timed_out = true; break; }
-          have_pend = false;
-          if (!mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
-          tc_commit(&q_empty[qb]);
-          if (!mbar_wait(o_free, (li & 1) ^ 1)) { timed_out = true; break; }
-          tc_commit(o_full);
-          continue;
-        }
-        for (int32_t t = 0; t < nu; ++t, ++g) {
+        if (!mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
+        for (int32_t t = 0; t < it.w.n_union && !timed_out; ++t, ++g) {
           const int st = g % KV_STAGES;
-          if (t == 0 && !mbar_wait(&q_full[qb], (li >> 1) & 1)) { timed_out = true; break; }
           if (!mbar_wait(&kv_full[st], (g / KV_STAGES) & 1)) { timed_out = true; break; }
           const uint32_t k_addr = smem_u32(sKV + st * 2 * TILE_BYTES);
-          bool ok = true;
           for (int q = 0; q < (two ? 2 : 1); ++q) {
             const int32_t r = q == 0 ? g : gb;
-            if (!mbar_wait(&s_free[q], (r & 1) ^ 1)) { ok = false; break; }
+            if (!mbar_wait(&s_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
             tc_fence_after();
             const uint32_t q_addr = smem_u32(sQ + (2 * qb + q) * TILE_BYTES);
 #pragma unroll
@@ -348,24 +312,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tc_commit(&s_full[q]);
           }
-          if (!ok) { timed_out = true; break; }
-          if (t == nu - 1) tc_commit(&q_empty[qb]);
-          if (have_pend && !issue_pv(pend)) { timed_out = true; break; }
-          pend = Pend{g, gb, st, li, t == 0, t == nu - 1, two};
-          have_pend = true;
           if (two) ++gb;
+          tc_commit(&kv_empty[st]);  // K read (V's reader commits separately)
         }
+        if (!timed_out) tc_commit(&q_empty[qb]);
       }
-      if (!timed_out && have_pend && !issue_pv(pend)) timed_out = true;
     }
-  } else if (warp < 2 + NUM_SILU_WARPS) {
+  } else if (warp == 2) {
+    // -------------------------------------------------- PV issuer (MMA) --
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_f16(TM, DH, 0u, false, true);
+      int32_t g = 0, gb = 0, li = 0;
+      Item nxt;
+      if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
+      for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
+        const Item it = nxt;
+        if (w + stride < n_items) nxt = load_item(a, w + stride);
+        const bool two = it.w.nq == 2;
+        if (!mbar_wait(o_free, (li & 1) ^ 1)) { timed_out = true; break; }
+        for (int32_t t = 0; t < it.w.n_union && !timed_out; ++t, ++g) {
+          const int st = g % KV_STAGES;
+          // V landed (and, for bf16 inputs, was converted to f16)
+          if (!mbar_wait(IN_BF16 ? &v_ready[st] : &kv_full[st], (g / KV_STAGES) & 1)) {
+            timed_out = true;
+            break;
+          }
+          const uint32_t v_addr = smem_u32(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
+          for (int q = 0; q < (two ? 2 : 1); ++q) {
+            const int32_t r = q == 0 ? g : gb;
+            if (!mbar_wait(&p_full[q], r & 1)) { timed_out = true; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < TN / 16; ++k) {
+              tc_mma_ts(tmem + o_col(q), tmem + p_col(q) + 8 * k,
+                        sdesc_sw128(v_addr + 2048 * k, 16384, 1024), idesc_o,
+                        (t > 0 || k > 0) ? 1u : 0u);
+            }
+            tc_commit(&p_free[q]);
+          }
+          if (two) ++gb;
+          tc_commit(&kv_empty[st]);
+        }
+        if (!timed_out) tc_commit(o_full);  // O complete (an item with no k-tiles: O unused)
+      }
+    }
+  } else if (warp < EPI_WARP0) {
     // -------------------------------------------------------- SiLU warps --
     // warps 2-5 take q-tile A of every item, warps 6-9 q-tile B; each warp
     // covers 32 query rows across all 128 keys of a k-tile, in four 32-key
     // chunks with the TMEM load of chunk k+1 in flight while chunk k is
     // computed.
     const int quarter = warp & 3;
-    const int q = (warp - 2) >> 2;  // 0: q-tile A, 1: q-tile B
+    const int q = (warp - SILU_WARP0) >> 2;  // 0: q-tile A, 1: q-tile B
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + s_col(q);
     const uint32_t p_addr = tmem + lane_base + p_col(q);
@@ -404,27 +402,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-        uint32_t sa[32], sbuf[32];
-        tmem_ld32(s_addr, sa);
+        // S -> h in 16-column steps, the load of step k + 1 in flight while
+        // step k is converted; S is released as soon as it is in registers,
+        // so the MMA can compute the next k-tile's scores meanwhile.
+        uint32_t h[64], sa[16], sb[16];
+        tmem_ld16(s_addr, sa);
         tmem_ld_wait();
-        if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
-        tc_fence_after();
+        reg_fence(sa);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t (&curv)[32] = (k & 1) ? sbuf : sa;
-          uint32_t (&ahead)[32] = (k & 1) ? sa : sbuf;
-          if (k < 3) tmem_ld32(s_addr + 32 * (k + 1), ahead);
-          const uint64_t vv = k < 2 ? vis_lo : vis_hi;
-          uint32_t p[16];
-          silu_chunk<HALVE>(curv, p, masked, (uint32_t)(vv >> (32 * (k & 1))));
-          tmem_st16(p_addr + 16 * k, p);
-          if (k < 3) tmem_ld_wait();
-          if (k == 2) {  // all of S is in registers: the MMA may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[q]);
+        for (int k = 0; k < 8; ++k) {
+          uint32_t (&cur)[16] = (k & 1) ? sb : sa;
+          uint32_t (&ahead)[16] = (k & 1) ? sa : sb;
+          if (k < 7) tmem_ld16(s_addr + 16 * (k + 1), ahead);
+          const uint64_t vv = k < 4 ? vis_lo : vis_hi;
+          scores_to_h<HALVE>(cur, h + 8 * k, masked, (uint32_t)(vv >> (16 * (k & 3))));
+          if (k < 7) {
+            tmem_ld_wait();
+            reg_fence(ahead);
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[q]);
+        // P = h + h tanh(h) = silu(s), in place
+#pragma unroll
+        for (int c = 0; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
+        // P of the previous k-tile must have been consumed by its P V
+        if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
+        tc_fence_after();
+        tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(h));
+        tmem_st32(p_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(h + 32));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -434,7 +441,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------------------------------------------- epilogue warps --
     const int quarter = warp & 3;
-    const int et = (warp - 2 - NUM_SILU_WARPS) * 32 + lane;  // 0..127
+    const int et = (warp - EPI_WARP0) * 32 + lane;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int rr = quarter * 32 + lane;  // row within each q-tile
     int32_t g = 0, li = 0;
