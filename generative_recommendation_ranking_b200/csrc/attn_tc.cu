@@ -13,7 +13,7 @@
 // metadata's work list (users by descending length). The two q-tiles share
 // every key/value tile, so each 32 KB K/V load feeds 256 query rows; the
 // item walks the union of the two q-tiles' k-tile lists (a k-tile EMPTY for
-// one of them is fully masked for it). Persistent CTAs, one per SM, 15 warps:
+// one of them is fully masked for it). Persistent CTAs, one per SM, 16 warps:
 //   warp 0      TMA producer: Q_A, Q_B once per item, K and V per k-tile, the
 //               U tiles of the item at its end
 //   warp 1      S issuer:  S_A = Q_A K^T, S_B = Q_B K^T (SS, M=128 N=128 K=16)
@@ -24,11 +24,12 @@
 //               the instruction, so an issuing thread that stops to wait on a
 //               barrier leaves the pipe idle; with two issuers each one's
 //               barrier waits overlap the other's MMAs.
-//   warps 3-6   SiLU for q-tile A, warps 7-10 for q-tile B: S from TMEM to
+//   warp 3      idle (it completes warpgroup 0 for the register re-split)
+//   warps 4-7   SiLU for q-tile A, warps 8-11 for q-tile B: S from TMEM to
 //               registers (S released at once, so the next k-tile's scores
 //               can be computed meanwhile) -> mask -> P = silu(S) in f16 ->
 //               TMEM once the previous P V has read P
-//   warps 11-14 epilogue: O from TMEM -> O / N (.) U -> global; and, for bf16
+//   warps 12-15 epilogue: O from TMEM -> O / N (.) U -> global; and, for bf16
 //               inputs, the in-place bf16 -> f16 conversion of V tiles
 // TMEM (512 columns): S_A, S_B (128 each), P_A, P_B (64 each, f16 pairs),
 // O_A, O_B (64 each).
@@ -60,9 +61,16 @@ constexpr int KV_STAGES = 4;
 constexpr int TILE_BYTES = TM * DH * 2;  // 16 KB (one Q, K, V or U tile)
 constexpr int NUM_SILU_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
-constexpr int SILU_WARP0 = 3;  // warps 0-2: TMA producer, S issuer, PV issuer
+// Four warpgroups: 0 = TMA producer, S issuer, PV issuer (warp 3 idle);
+// 1 = SiLU of q-tile A; 2 = SiLU of q-tile B; 3 = epilogue.
+constexpr int SILU_WARP0 = 4;
 constexpr int EPI_WARP0 = SILU_WARP0 + NUM_SILU_WARPS;
-constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);  // 480
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);  // 512
+// Registers per thread after the split (launched with 65536 / 512 = 128):
+// the single-thread roles need few, the SiLU warps hold a row's 64 packed
+// scores. 128 x (80 + 152 + 152 + 128) = 65536.
+constexpr uint32_t REGS_CTRL = 80, REGS_SILU = 152;
+static_assert(128u * (REGS_CTRL + 2 * REGS_SILU + 128u) <= 65536u, "register split over budget");
 __host__ __device__ constexpr uint32_t s_col(int q) { return 128u * q; }        // S_A, S_B
 __host__ __device__ constexpr uint32_t p_col(int q) { return 256u + 64u * q; }  // P_A, P_B
 __host__ __device__ constexpr uint32_t o_col(int q) { return 384u + 64u * q; }  // O_A, O_B
@@ -143,21 +151,33 @@ __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
   return m << lo;
 }
 
-// Visibility of keys [j0, j0 + 64) (user-relative, j0 a multiple of 64) to
-// query row i, whose rank-table index is cnt_i (rule 2 as a table lookup).
-// Evaluated from the rules alone, so it is exact for FULL, PARTIAL and EMPTY
-// tiles alike.
-__device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, const uint64_t* rt_mask,
-                                                 int32_t i, int32_t cnt_i, int32_t j0) {
-  uint64_t vis = range_bits(0, it.n_us - j0);  // rule 1: U and S keys
+// Rule 2 as a table lookup: the rank-table word of query row i (rank-table
+// index cnt_i) for keys [j0, j0 + 64) (user-relative, j0 a multiple of 64),
+// or 0 where that range holds no R key. Issued a k-tile ahead of its use.
+__device__ __forceinline__ uint64_t rt_word(const mtgr_work_item& it, const uint64_t* rt_mask,
+                                            int32_t cnt_i, int32_t j0) {
   const int32_t n_r = it.c_lo - it.n_us;
-  if (n_r > 0 && j0 + 64 > it.n_us && j0 < it.c_lo) {  // rule 2: R keys earlier than t_i
+  if (n_r > 0 && j0 + 64 > it.n_us && j0 < it.c_lo) {
     const int32_t gidx = j0 / 64 - it.n_us / 64;
-    vis |= __ldg(rt_mask + it.rt_base + (int64_t)gidx * (n_r + 1) + cnt_i);
+    return __ldg(rt_mask + it.rt_base + (int64_t)gidx * (n_r + 1) + cnt_i);
   }
+  return 0ull;
+}
+
+// Visibility of keys [j0, j0 + 64) to query row i from the three rules, rule
+// 2 given by its rank-table word rt. Exact for FULL, PARTIAL and EMPTY tiles
+// alike.
+__device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, uint64_t rt, int32_t i,
+                                                 int32_t j0) {
+  uint64_t vis = range_bits(0, it.n_us - j0) | rt;  // rule 1: U and S keys; rule 2
   const int dc = i - j0;  // the diagonal: every token sees itself (rules 1-3)
   if (dc >= 0 && dc < 64) vis |= 1ull << dc;
   return vis & range_bits(0, it.n - j0);  // keys past the user's end
+}
+
+// Keep-mask of one f16 pair from its two visibility bits (bit 0: low half).
+__device__ __forceinline__ uint32_t pair_mask(uint32_t bits) {
+  return ((bits & 1u) ? 0x0000ffffu : 0u) | ((bits & 2u) ? 0xffff0000u : 0u);
 }
 
 // h = s / 2 (or s, when the scores arrive halved) for 16 consecutive keys of
@@ -210,7 +230,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* o_free = o_full + 1;
   uint64_t* u_full = o_free + 1;
   uint64_t* u_empty = u_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(u_empty + 1);
+  uint64_t* turn_b = u_empty + 1;  // [2] A's tanh of a k-tile done: B's turn
+  uint64_t* turn_a = turn_b + 2;   // [2] B's tanh of a k-tile done: A's turn
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn_a + 2);
 
   const int warp = warp_id(), lane = lane_id();
   if (warp == 0 && lane == 0) {
@@ -232,6 +254,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(o_free, NUM_EPI_WARPS);
     mbar_init(u_full, 1);
     mbar_init(u_empty, NUM_EPI_WARPS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&turn_b[i], NUM_SILU_WARPS / 2);
+      mbar_init(&turn_a[i], NUM_SILU_WARPS / 2);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -246,7 +272,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int32_t d = a.d;
   const int32_t stride = gridDim.x;
   bool timed_out = false;
+  // Each warpgroup re-splits the registers and finishes on its own branch, so
+  // no code after the split is shared between register budgets.
+  auto finish = [&]() {
+    if (timed_out) set_status(a.status, MTGR_ERR_TIMEOUT);
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, TMEM_COLS);
+    }
+  };
 
+  if (warp < SILU_WARP0) {
+  setmaxnreg_dec<REGS_CTRL>();
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
@@ -286,7 +324,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // --------------------------------------------------- S issuer (MMA) --
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
+      // f16 operands: f16 scores (the SiLU works in f16 anyway); bf16: f32
+      constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false, !IN_BF16);
       int32_t g = 0, gb = 0, li = 0;
       Item nxt;
       if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
@@ -356,77 +395,131 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!timed_out) tc_commit(o_full);  // O complete (an item with no k-tiles: O unused)
       }
     }
+  }
+  finish();
   } else if (warp < EPI_WARP0) {
+    setmaxnreg_inc<REGS_SILU>();
     // -------------------------------------------------------- SiLU warps --
-    // warps 2-5 take q-tile A of every item, warps 6-9 q-tile B; each warp
-    // covers 32 query rows across all 128 keys of a k-tile, in four 32-key
-    // chunks with the TMEM load of chunk k+1 in flight while chunk k is
-    // computed.
+    // Warps 4-7 take q-tile A of every item, warps 8-11 q-tile B; each warp
+    // covers 32 query rows (its TMEM lane quarter) across all 128 keys of a
+    // k-tile. S goes to registers in one step and is released at once; the
+    // next k-tile's entry and rule-2 words are fetched while this one's
+    // tanh runs.
     const int quarter = warp & 3;
     const int q = (warp - SILU_WARP0) >> 2;  // 0: q-tile A, 1: q-tile B
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + s_col(q);
     const uint32_t p_addr = tmem + lane_base + p_col(q);
     int32_t gq = 0;  // this q-tile slot's k-tile counter (barrier rounds)
-    Item nxt;
-    int32_t cnt_nxt = 0;
-    auto cnt_of = [&](const Item& x) -> int32_t {
-      const int32_t i = (x.w.qt0 + q) * TM + quarter * 32 + lane;
-      return (q < x.w.nq && i < x.w.n) ? __ldg(a.rt_cnt + x.w.us + i) : 0;
-    };
-    if ((int32_t)blockIdx.x < n_items) {
-      nxt = load_item(a, blockIdx.x);
-      cnt_nxt = cnt_of(nxt);
-    }
+    int32_t gt = 0;  // k-tiles of two-q-tile items (rounds of the turn barriers)
     for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride) {
-      const Item it = nxt;
-      const int32_t cnt_i = cnt_nxt;
-      if (w + stride < n_items) {
-        nxt = load_item(a, w + stride);
-        cnt_nxt = cnt_of(nxt);
-      }
+      // no look-ahead copy of the next item here: the 64 registers of a
+      // row's scores leave no room for one
+      const Item it = load_item(a, w);
       if (q >= it.w.nq) continue;  // this item has no q-tile B
+      const bool two = it.w.nq == 2;
       const int32_t i = (it.w.qt0 + q) * TM + quarter * 32 + lane;  // user-relative row
+      const int32_t cnt_i = i < it.w.n ? __ldg(a.rt_cnt + it.w.us + i) : 0;
       UnionCursor cur;
       cur.init(a.entries, it.w);
-      for (int32_t t = 0; t < it.w.n_union; ++t, ++gq) {
+      // the upcoming k-tile: index, whether it needs the per-element rules,
+      // and its two rule-2 words
+      int32_t kt_n = 0;
+      bool masked_n = false;
+      uint64_t rt_lo_n = 0, rt_hi_n = 0;
+      auto fetch = [&]() {
         int32_t ca, cb;
-        const int32_t kt = cur.next(ca, cb);
+        kt_n = cur.next(ca, cb);
         const int32_t code = q == 0 ? ca : cb;  // -1: EMPTY for this q-tile
-        const bool masked = code < 0 || (code & 1) || kt * TN + TN > it.w.n;
-        const uint32_t r = static_cast<uint32_t>(gq);
-        uint64_t vis_lo = 0, vis_hi = 0;
-        if (masked) {
-          vis_lo = visible_bits(it.w, a.rt_mask, i, cnt_i, kt * TN);
-          vis_hi = visible_bits(it.w, a.rt_mask, i, cnt_i, kt * TN + 64);
+        masked_n = code < 0 || (code & 1) || kt_n * TN + TN > it.w.n;
+        if (masked_n) {
+          rt_lo_n = rt_word(it.w, a.rt_mask, cnt_i, kt_n * TN);
+          rt_hi_n = rt_word(it.w, a.rt_mask, cnt_i, kt_n * TN + 64);
         }
+      };
+      fetch();
+      for (int32_t t = 0; t < it.w.n_union; ++t, ++gq) {
+        const int32_t kt = kt_n;
+        const bool masked = masked_n;
+        const uint64_t rt_lo = rt_lo_n, rt_hi = rt_hi_n;
+        const uint32_t r = static_cast<uint32_t>(gq);
         if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-        // S -> h in 16-column steps, the load of step k + 1 in flight while
-        // step k is converted; S is released as soon as it is in registers,
-        // so the MMA can compute the next k-tile's scores meanwhile.
-        uint32_t h[64], sa[16], sb[16];
-        tmem_ld16(s_addr, sa);
-        tmem_ld_wait();
-        reg_fence(sa);
+        uint32_t h[64];
+        if (!IN_BF16) {
+          // f16 scores (f16 accumulator, one per column): one packed load
+          tmem_ld64_pack16(s_addr, h);
+          tmem_ld_wait();
+          reg_fence(h);
+        } else {
+          // f32 scores: 16-column steps, the load of step k + 1 in flight
+          // while step k is converted and masked
+          uint64_t vis_lo = 0, vis_hi = 0;
+          if (masked) {
+            vis_lo = visible_bits(it.w, rt_lo, i, kt * TN);
+            vis_hi = visible_bits(it.w, rt_hi, i, kt * TN + 64);
+          }
+          uint32_t sa[16], sb[16];
+          tmem_ld16(s_addr, sa);
+          tmem_ld_wait();
+          reg_fence(sa);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          uint32_t (&cur)[16] = (k & 1) ? sb : sa;
-          uint32_t (&ahead)[16] = (k & 1) ? sa : sb;
-          if (k < 7) tmem_ld16(s_addr + 16 * (k + 1), ahead);
-          const uint64_t vv = k < 4 ? vis_lo : vis_hi;
-          scores_to_h<HALVE>(cur, h + 8 * k, masked, (uint32_t)(vv >> (16 * (k & 3))));
-          if (k < 7) {
-            tmem_ld_wait();
-            reg_fence(ahead);
+          for (int k = 0; k < 8; ++k) {
+            uint32_t (&cur_s)[16] = (k & 1) ? sb : sa;
+            uint32_t (&ahead)[16] = (k & 1) ? sa : sb;
+            if (k < 7) tmem_ld16(s_addr + 16 * (k + 1), ahead);
+            const uint64_t vv = k < 4 ? vis_lo : vis_hi;
+            scores_to_h<HALVE>(cur_s, h + 8 * k, masked, (uint32_t)(vv >> (16 * (k & 3))));
+            if (k < 7) {
+              tmem_ld_wait();
+              reg_fence(ahead);
+            }
           }
         }
+        // S is in registers: the S issuer may overwrite it
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
+        uint64_t vis_lo = 0, vis_hi = 0;
+        if (!IN_BF16 && masked) {
+          vis_lo = visible_bits(it.w, rt_lo, i, kt * TN);
+          vis_hi = visible_bits(it.w, rt_hi, i, kt * TN + 64);
+        }
+        if (t + 1 < it.w.n_union) fetch();
+        if (!IN_BF16) {
+          if (masked) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              h[c] &= pair_mask(static_cast<uint32_t>((c < 32 ? vis_lo : vis_hi) >> (2 * (c & 31))));
+          }
+          if (HALVE) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) h[c] = mul_f16x2(h[c], 0x38003800u);  // x 0.5, exact
+          }
+        }
+        // The tanh of both q-tiles runs on the SM's one MUFU pipe (16 values
+        // per clock), the bound of this kernel. Within a two-q-tile item the
+        // groups take turns, A(0) B(0) A(1) B(1) ...: each group's loads,
+        // stores and waits then overlap the other's tanh instead of
+        // coinciding with it, and each tanh phase has the pipe to itself.
+        // Every wait is on a phase the other group reaches without waiting
+        // on this one (its previous turn), so the turns cannot deadlock, and
+        // the two-slot rings keep each parity wait unambiguous.
+        if (two && (q == 1 || gt > 0)) {
+          uint64_t* bar = q == 0 ? &turn_a[(gt - 1) & 1] : &turn_b[gt & 1];
+          const uint32_t par = q == 0 ? (((gt - 1) >> 1) & 1) : ((gt >> 1) & 1);
+          if (!warp_wait(bar, par)) { timed_out = true; break; }
+          reg_fence(h);  // the arithmetic below may not move above the wait
+        }
         // P = h + h tanh(h) = silu(s), in place
 #pragma unroll
         for (int c = 0; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
+        if (two) {
+          reg_fence(h);  // hand over the turn only once this tile's tanh is done
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[gt & 1] : &turn_a[gt & 1]);
+          ++gt;
+        }
         // P of the previous k-tile must have been consumed by its P V
         if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
         tc_fence_after();
@@ -438,6 +531,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[q]);
       }
     }
+    finish();
   } else {
     // ---------------------------------------------------- epilogue warps --
     const int quarter = warp & 3;
@@ -528,12 +622,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(u_empty);  // U of this item consumed
       if (!IN_BF16) g += it.w.n_union;
     }
-  }
-  if (timed_out) set_status(a.status, MTGR_ERR_TIMEOUT);
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    finish();
   }
 }
 
