@@ -230,9 +230,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* o_free = o_full + 1;
   uint64_t* u_full = o_free + 1;
   uint64_t* u_empty = u_full + 1;
-  uint64_t* turn_b = u_empty + 1;  // [2] A's tanh of a k-tile done: B's turn
-  uint64_t* turn_a = turn_b + 2;   // [2] B's tanh of a k-tile done: A's turn
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn_a + 2);
+  // Turns on each SM sub-partition's MUFU pipe, one barrier pair per A/B
+  // warp pair sharing it: [sub-partition][slot]
+  uint64_t* turn_b = u_empty + 1;  // [4][2] A's tanh of a k-tile done: B's turn
+  uint64_t* turn_a = turn_b + 8;   // [4][2] B's tanh of a k-tile done: A's turn
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn_a + 8);
 
   const int warp = warp_id(), lane = lane_id();
   if (warp == 0 && lane == 0) {
@@ -254,9 +256,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(o_free, NUM_EPI_WARPS);
     mbar_init(u_full, 1);
     mbar_init(u_empty, NUM_EPI_WARPS);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&turn_b[i], NUM_SILU_WARPS / 2);
-      mbar_init(&turn_a[i], NUM_SILU_WARPS / 2);
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(&turn_b[i], 1);
+      mbar_init(&turn_a[i], 1);
     }
     fence_barrier_init();
   }
@@ -497,16 +499,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < 64; ++c) h[c] = mul_f16x2(h[c], 0x38003800u);  // x 0.5, exact
           }
         }
-        // The tanh of both q-tiles runs on the SM's one MUFU pipe (16 values
-        // per clock), the bound of this kernel. Within a two-q-tile item the
-        // groups take turns, A(0) B(0) A(1) B(1) ...: each group's loads,
-        // stores and waits then overlap the other's tanh instead of
-        // coinciding with it, and each tanh phase has the pipe to itself.
-        // Every wait is on a phase the other group reaches without waiting
-        // on this one (its previous turn), so the turns cannot deadlock, and
-        // the two-slot rings keep each parity wait unambiguous.
+        // The tanh of both q-tiles runs on the MUFU pipes (16 values per
+        // clock per SM, one pipe per sub-partition), the bound of this
+        // kernel. The A and B warps of one sub-partition (same lane quarter)
+        // share its pipe; within a two-q-tile item they take turns, A(0)
+        // B(0) A(1) B(1) ...: each one's loads, stores and waits then
+        // overlap the other's tanh instead of coinciding with it. The turns
+        // are per warp pair, so a slow warp elsewhere does not idle this
+        // pipe. Every wait is on a phase the other warp reaches without
+        // waiting on this one (its previous turn), so the turns cannot
+        // deadlock, and the two-slot rings keep each parity wait exact.
         if (two && (q == 1 || gt > 0)) {
-          uint64_t* bar = q == 0 ? &turn_a[(gt - 1) & 1] : &turn_b[gt & 1];
+          uint64_t* bar = q == 0 ? &turn_a[2 * quarter + ((gt - 1) & 1)] : &turn_b[2 * quarter + (gt & 1)];
           const uint32_t par = q == 0 ? (((gt - 1) >> 1) & 1) : ((gt >> 1) & 1);
           if (!warp_wait(bar, par)) { timed_out = true; break; }
           reg_fence(h);  // the arithmetic below may not move above the wait
@@ -517,7 +521,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (two) {
           reg_fence(h);  // hand over the turn only once this tile's tanh is done
           __syncwarp();
-          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[gt & 1] : &turn_a[gt & 1]);
+          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
           ++gt;
         }
         // P of the previous k-tile must have been consumed by its P V
