@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--users", type=int, default=None,
+                    help="run only the first N users of the workload (profiling a smaller case)")
     ap.add_argument("--config", type=int, default=2,
                     help="workload: 0 fp32 block, 1 attention only, 2 block (default), "
                          "3 8-layer stack, 4 candidate sweep")
@@ -182,7 +184,7 @@ def run_reference(args, world, rank):
     """The reference arm: the CPU oracle timed on bounded samples of the workload."""
     if rank != 0:
         return
-    wl = synth.make_workload(args.config, seed=args.seed)
+    wl = synth.make_workload(args.config, seed=args.seed, B=args.users)
     per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
     import oracle  # noqa: F401
     for _ in range(args.warmup):
@@ -352,7 +354,7 @@ def run_ours(args, world, rank, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = synth.make_workload(args.config, seed=args.seed + rank)
+    wl = synth.make_workload(args.config, seed=args.seed + rank, B=args.users)
     if wl["kind"] == "sweep":
         raise SystemExit("use --config 4 through run_sweep")
     B, T, d, H, dff, L = (int(wl["lens"].shape[0]), int(wl["lens"].sum()), wl["d"], wl["H"],
