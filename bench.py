@@ -280,6 +280,31 @@ class Workspace:
             self._lib.mtgr_stack_fwd([l.c for l in self.layers], b.c, x_d, out_d, self.ws, s)
 
 
+def graph_steps_ms(fn, n: int, warmup: int) -> float:
+    """Device milliseconds per replay of fn(stream) captured once into a CUDA
+    graph: the launch cost of a step made of short kernels drops out."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            fn(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        fn(side)
+    cur = torch.cuda.current_stream()
+    for _ in range(warmup):
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(n):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / n
+
+
 def time_steps(fn, n, stream) -> float:
     """Device milliseconds of n calls of fn on `stream` (CUDA events)."""
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -463,6 +488,52 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def incremental_leg(agg: dict, dev, stream, args) -> dict:
+    """The same user served with its context cached: the context pass (U, S,
+    R through the block, Q|K|V|U kept) timed once per request of new context,
+    and the candidate pass (all K candidates over the cached keys) timed as
+    the per-request work once the context is cached. Both include their
+    packing and mask metadata."""
+    import generative_recommendation_ranking_b200 as mt
+    from generative_recommendation_ranking_b200 import _lib
+    n_u, n_s, n_r, K = (int(v) for v in agg["lens"][0])
+    n_ctx = n_u + n_s + n_r
+    layers = [mt.BlockWeights(p, agg["H"], dtype="bf16", device=dev) for p in agg["layers"]]
+    x = torch.from_numpy(agg["x"]).to(dev)
+    xc, xk = x[:n_ctx], x[n_ctx:]
+    cc = mt.ContextCache(layers, n_u, n_s, n_r, agg["ts"][:n_ctx], xc, K, K, stream=stream)
+    cb = cc._ctx_batch
+    batch = cc.candidate_batch(agg["ts"][n_ctx:], stream)
+    ws = cc.workspace(K)
+    out = torch.empty(K, agg["d"], dtype=torch.float32, device=dev)
+
+    def ctx_step(s=stream):
+        cb.pack(s)
+        cb.build_meta(s)
+        _lib.mtgr_stack_fwd_rows(cc.c_layers, cb.c, 0, cc.cache, cc.cache_rows, xc, cc.out,
+                                 cc._ws, s)
+
+    def cand_step(s=stream):
+        batch.pack(s)
+        batch.build_meta(s)
+        _lib.mtgr_restrict_work(batch.c, cc.q_first, s)
+        cc.score(None, xk, out=out, ws=ws, batch=batch, stream=s)
+
+    res = {}
+    n = max(5, min(args.steps, 50))
+    for name, fn in (("context", ctx_step), ("incremental", cand_step)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        ms = time_steps(fn, n, stream) / n
+        batch.check()
+        res[f"{name}_ms"] = ms
+        res[f"{name}_graph_ms"] = graph_steps_ms(fn, n, max(3, args.warmup))
+        batch.check()
+    res["incremental_ms_per_candidate"] = res["incremental_ms"] / K
+    res["incremental_graph_ms_per_candidate"] = res["incremental_graph_ms"] / K
+    return res
+
+
 def run_sweep(args, local):
     """Candidate scaling for one user (d_model 512, 8 heads, one block): the
     aggregated sample [U, S, R, c_1..c_K] against K expanded rows [U, S, R, c_i]
@@ -484,15 +555,22 @@ def run_sweep(args, local):
             wsp.batch.check()
             res[f"{name}_ms"] = ms
             res[f"{name}_ms_per_candidate"] = ms / K
+            res[f"{name}_graph_ms"] = graph_steps_ms(lambda s: wsp.step(stream=s), n,
+                                                     max(3, args.warmup))
+            wsp.batch.check()
             del wsp
             torch.cuda.empty_cache()
+        res.update(incremental_leg(agg, dev, stream, args))
         rows.append(res)
     marginal = (rows[-1]["aggregated_ms"] - rows[0]["aggregated_ms"]) / (rows[-1]["K"] - rows[0]["K"])
-    line = {"metric": "candidate sweep: HSTU-block fwd ms per candidate, aggregated vs expanded rows",
+    line = {"metric": "candidate sweep: HSTU-block fwd ms per candidate, aggregated vs expanded rows vs cached context",
             "unit": "ms", "higher_is_better": False, "data": "synthetic", "dtype": "bf16",
             "config": {"workload": "sweep_b1_d512", "d_model": 512, "heads": 8, "d_ff": 2048,
                        "n_u": 24, "s": 1000, "r": 64},
+            "l2": "not flushed: one user's inputs and weights fit in L2",
             "sweep": rows, "aggregated_marginal_ms_per_added_candidate": marginal,
+            "incremental_ms_per_candidate_at_k512": rows[-1]["incremental_ms_per_candidate"],
+            "graph": "*_graph_ms: the same step captured once into a CUDA graph and replayed",
             "expanded_ms_per_row_at_k512": rows[-1]["expanded_ms_per_candidate"]}
     print(json.dumps(line), flush=True)
 

@@ -23,13 +23,17 @@ from ._lib import (  # noqa: F401
     mtgr_hstu_block_fwd,
     mtgr_mask_meta_workspace_bytes,
     mtgr_pack_offsets,
+    mtgr_restrict_work,
     mtgr_stack_fwd,
+    mtgr_stack_fwd_rows,
+    mtgr_stack_rows_workspace_bytes,
     mtgr_stack_workspace_bytes,
     mtgr_version,
     status_string,
 )
 from .api import (  # noqa: F401
     BlockWeights,
+    ContextCache,
     PackedBatch,
     capacities,
     gemm,

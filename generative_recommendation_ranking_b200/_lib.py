@@ -87,6 +87,12 @@ _SIGNATURES = {
     "mtgr_stack_workspace_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams), c_i32]),
     "mtgr_stack_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams), c_i32,
                                       ctypes.POINTER(MtgrBatch), c_vp, c_vp, c_vp, c_size, c_vp]),
+    "mtgr_restrict_work": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_vp, c_vp]),
+    "mtgr_stack_rows_workspace_bytes": (c_size, [c_i32, c_i32, ctypes.POINTER(MtgrBlockParams),
+                                                 c_i32]),
+    "mtgr_stack_fwd_rows": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams), c_i32,
+                                           ctypes.POINTER(MtgrBatch), c_i32, c_vp, c_i32, c_vp, c_vp,
+                                           c_vp, c_size, c_vp]),
     "mtgr_gemm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32,
                                  c_i32, c_vp, c_vp, c_vp]),
     "mtgr_timer_create": (c_vp, []),
@@ -213,6 +219,24 @@ def mtgr_stack_fwd(layers, batch: MtgrBatch, d_x_in, d_x_out, d_ws, stream=None)
     _check("mtgr_stack_fwd", load().mtgr_stack_fwd(
         arr, len(layers), ctypes.byref(batch), _ptr(d_x_in), _ptr(d_x_out), _ptr(d_ws),
         d_ws.numel() * d_ws.element_size(), _stream(stream)))
+
+
+def mtgr_restrict_work(batch: MtgrBatch, d_q_first, stream=None):
+    _check("mtgr_restrict_work", load().mtgr_restrict_work(
+        ctypes.byref(batch), _ptr(d_q_first), _stream(stream)))
+
+
+def mtgr_stack_rows_workspace_bytes(T: int, row0: int, layers) -> int:
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    return load().mtgr_stack_rows_workspace_bytes(T, row0, arr, len(layers))
+
+
+def mtgr_stack_fwd_rows(layers, batch: MtgrBatch, row0: int, d_cache, cache_rows: int, d_x_in,
+                        d_x_out, d_ws, stream=None):
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    _check("mtgr_stack_fwd_rows", load().mtgr_stack_fwd_rows(
+        arr, len(layers), ctypes.byref(batch), row0, _ptr(d_cache), cache_rows, _ptr(d_x_in),
+        _ptr(d_x_out), _ptr(d_ws), d_ws.numel() * d_ws.element_size(), _stream(stream)))
 
 
 TIMER_CLASSES = ("pack", "mask_meta", "gln", "gemm_qkvu", "attention", "gemm_mlp1", "gemm_mlp2")

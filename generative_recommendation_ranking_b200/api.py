@@ -207,3 +207,80 @@ def gemm(a: torch.Tensor, b: torch.Tensor, bias=None, epi: int = 0, resid=None, 
         status = torch.zeros(1, dtype=torch.int32, device=a.device)
     _lib.mtgr_gemm(a, b, bias, epi, resid, q_cols, out, status, stream)
     return out
+
+
+class ContextCache:
+    """One user's context tokens (U, S, R) run once through a bf16 stack, with
+    every layer's Q|K|V|U kept on the device, so that the user's candidates
+    can then be scored chunk by chunk over the cached keys.
+
+    The context never attends to a candidate and a candidate sees no other
+    candidate (fun-rec 7.3.4, mask rules 1-3), so the context rows of every
+    layer are the same whichever candidates follow; the MTGR practice
+    article (5.2, inference latency) caches the rarely changing User/Seq
+    tokens on that ground. ``k_total`` fixes the normaliser N = N_U + N_S +
+    N_R + k_total that the aggregated pass over all candidates would use;
+    ``max_chunk`` bounds the candidates of one ``score`` call.
+
+    ``x_ctx`` float32 [N_U + N_S + N_R, d] and ``ts_ctx`` int64 (host or
+    device) are the context features and timestamps (U tokens' stamps are
+    not read). ``out`` holds the stack's output on the context rows.
+    """
+
+    def __init__(self, layers, n_u: int, n_s: int, n_r: int, ts_ctx, x_ctx: torch.Tensor,
+                 k_total: int, max_chunk: int, stream=None):
+        self.layers = list(layers)
+        self.c_layers = [l.c for l in self.layers]
+        self.n_u, self.n_s, self.n_r = int(n_u), int(n_s), int(n_r)
+        self.n_ctx = self.n_u + self.n_s + self.n_r
+        self.max_chunk = int(max_chunk)
+        self.norm = float(self.n_ctx + int(k_total))
+        dev = x_ctx.device
+        d = self.layers[0].d
+        self.cache_rows = self.n_ctx + self.max_chunk
+        self.cache = torch.empty(len(self.layers), self.cache_rows, 4 * d, dtype=torch.float16,
+                                 device=dev)
+        self.ts_ctx = (ts_ctx if isinstance(ts_ctx, torch.Tensor) else torch.from_numpy(
+            np.ascontiguousarray(ts_ctx, dtype=np.int64))).to(dev, dtype=torch.int64)
+        self.q_first = torch.tensor([self.n_ctx], dtype=torch.int32, device=dev)
+        batch = PackedBatch([[self.n_u, self.n_s, self.n_r, 0]], self.ts_ctx, device=dev,
+                            norm=[self.norm], stream=stream)
+        self.out = torch.empty_like(x_ctx)
+        ws = _ws(_lib.mtgr_stack_rows_workspace_bytes(self.n_ctx, 0, self.c_layers), dev)
+        _lib.mtgr_stack_fwd_rows(self.c_layers, batch.c, 0, self.cache, self.cache_rows, x_ctx,
+                                 self.out, ws, stream)
+        self._ctx_batch = batch  # keeps its buffers alive until the stream has run
+        self._ws = ws
+
+    def candidate_batch(self, ts_cand, stream=None) -> PackedBatch:
+        """The virtual batch of one chunk: the context followed by the
+        chunk's candidates, with the work list cut to the candidate rows."""
+        ts_c = (ts_cand if isinstance(ts_cand, torch.Tensor) else torch.from_numpy(
+            np.ascontiguousarray(ts_cand, dtype=np.int64))).to(self.cache.device, dtype=torch.int64)
+        k = int(ts_c.shape[0])
+        if k < 1 or k > self.max_chunk:
+            raise ValueError(f"chunk of {k} candidates, 1..{self.max_chunk} allowed")
+        batch = PackedBatch([[self.n_u, self.n_s, self.n_r, k]], torch.cat([self.ts_ctx, ts_c]),
+                            device=self.cache.device, norm=[self.norm], stream=stream)
+        _lib.mtgr_restrict_work(batch.c, self.q_first, stream)
+        return batch
+
+    def workspace(self, k: int) -> torch.Tensor:
+        return _ws(_lib.mtgr_stack_rows_workspace_bytes(self.n_ctx + k, self.n_ctx, self.c_layers),
+                   self.cache.device)
+
+    def score(self, ts_cand, x_cand: torch.Tensor, out=None, ws=None, batch=None,
+              stream=None) -> torch.Tensor:
+        """Stack output [k, d] float32 of k candidates (features ``x_cand``
+        float32 [k, d], timestamps ``ts_cand``), equal to their rows of the
+        aggregated pass over the context and all k_total candidates."""
+        if batch is None:
+            batch = self.candidate_batch(ts_cand, stream)
+        k = batch.T - self.n_ctx
+        if out is None:
+            out = torch.empty(k, x_cand.shape[1], dtype=torch.float32, device=x_cand.device)
+        if ws is None:
+            ws = self.workspace(k)
+        _lib.mtgr_stack_fwd_rows(self.c_layers, batch.c, self.n_ctx, self.cache, self.cache_rows,
+                                 x_cand, out, ws, stream)
+        return out

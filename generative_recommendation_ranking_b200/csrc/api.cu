@@ -23,6 +23,8 @@ int launch_gemm_f32(int M, int N, int K, const float* a, const float* b, const f
 int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
                    const float* resid, int q_cols, int32_t out_dtype, void* out, int32_t* status,
                    cudaStream_t s);
+int launch_restrict_work(const int32_t* q_first, int32_t q_cap, mtgr_work_item* work, int64_t* counts,
+                         cudaStream_t s);
 int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu, float* g,
                     cudaStream_t s);
 int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
@@ -95,6 +97,75 @@ BlockWs block_ws_layout(int32_t T, const mtgr_block_params* p, void* base) {
   w.h = b + off;    off += align_up(t * p->d_ff * e, 256);
   w.bytes = off;
   return w;
+}
+
+// Workspace of the bf16 block computing rows [row0, T) only: the GroupLN
+// output, MLP hidden and (unless the caller provides it) Q|K|V|U cover those
+// rows; the attention output covers all T rows (whole q-tiles are written).
+struct PartWs {
+  void* xt;
+  void* qkvu;
+  void* g;
+  void* h;
+  size_t bytes;
+};
+
+PartWs part_ws_layout(int32_t T, int32_t row0, const mtgr_block_params* p, bool own_qkvu, void* base) {
+  const size_t k = (size_t)(T - row0), t = (size_t)T;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  PartWs w;
+  size_t off = 0;
+  w.xt = b + off;   off += align_up(k * p->d * 2, 256);
+  w.qkvu = own_qkvu ? b + off : nullptr;
+  if (own_qkvu) off += align_up(t * 4 * p->d * 2, 256);
+  w.g = b + off;    off += align_up(t * p->d * 2, 256);
+  w.h = b + off;    off += align_up(k * p->d_ff * 2, 256);
+  w.bytes = off;
+  return w;
+}
+
+// The bf16 block on rows [row0, T) of the batch: x_in / x_out hold those rows;
+// qkvu ([T][4d] f16) is the caller's when given — rows [row0, T) are written,
+// earlier rows must already hold the Q|K|V|U of those tokens — and the
+// attention computes the work items of the batch's (restricted) work list.
+int block_fwd_rows(const mtgr_block_params* p, const mtgr_batch* bt, int32_t row0,
+                   const float* x_in, float* x_out, void* qkvu_ext, void* ws, cudaStream_t s) {
+  const int32_t T = bt->T, d = p->d, H = p->H, dff = p->d_ff, k = T - row0;
+  if (k <= 0) return MTGR_OK;
+  PartWs w = part_ws_layout(T, row0, p, qkvu_ext == nullptr, ws);
+  uint16_t* qkvu = static_cast<uint16_t*>(qkvu_ext != nullptr ? qkvu_ext : w.qkvu);
+  int rc;
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(k, d, MTGR_F32, x_in, bt->group_id + row0, 4, p->gln1_gamma,
+                         p->gln1_beta, p->eps, MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
+  }
+  {
+    // Q|K|V|U in f16 with the Q columns halved (silu's tanh form takes s/2)
+    TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
+    if ((rc = launch_gemm_tc(k, 4 * d, d, w.xt, p->w_qkvu, p->b_qkvu, MTGR_EPI_NONE, nullptr, d,
+                             MTGR_F16, qkvu + (size_t)row0 * 4 * d, bt->status, s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
+    if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, qkvu, MTGR_BF16, w.g, s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(k, d, MTGR_BF16, static_cast<uint16_t*>(w.g) + (size_t)row0 * d,
+                         bt->group_id + row0, 4, p->gln2_gamma, p->gln2_beta, p->eps, MTGR_BF16,
+                         w.xt, s)) != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
+    if ((rc = launch_gemm_tc(k, dff, d, w.xt, p->w1, p->b1, MTGR_EPI_SILU, nullptr, 0, MTGR_BF16,
+                             w.h, bt->status, s)) != MTGR_OK) return rc;
+  }
+  TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
+  return launch_gemm_tc(k, d, dff, w.h, p->w2, p->b2, MTGR_EPI_RESID, x_in, 0, MTGR_F32, x_out,
+                        bt->status, s);
 }
 
 int block_fwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_in, float* x_out,
@@ -335,6 +406,89 @@ MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mt
     in = out;
   }
   return MTGR_OK;
+}
+
+MTGR_API int mtgr_restrict_work(const mtgr_batch* batch, const int32_t* d_q_first,
+                                mtgr_stream_t stream) {
+  if (!batch_ok(batch) || (batch->B > 0 && d_q_first == nullptr)) return MTGR_ERR_INVALID_ARG;
+  if (batch->q_capacity == 0) return MTGR_OK;
+  return launch_restrict_work(d_q_first, batch->q_capacity, const_cast<mtgr_work_item*>(batch->work),
+                              const_cast<int64_t*>(batch->counts), as_stream(stream));
+}
+
+namespace {
+// Checks shared by the cached-context and candidate stack entries.
+int serve_check(const mtgr_block_params* layers, int32_t L, const mtgr_batch* batch) {
+  if (layers == nullptr || L <= 0) return MTGR_ERR_INVALID_ARG;
+  for (int32_t l = 0; l < L; ++l) {
+    const int rc = params_check(&layers[l]);
+    if (rc != MTGR_OK) return rc;
+    if (layers[l].d != layers[0].d || layers[l].H != layers[0].H) return MTGR_ERR_INVALID_ARG;
+    if (layers[l].dtype != MTGR_BF16) return MTGR_ERR_UNSUPPORTED;
+  }
+  if (!batch_ok(batch)) return MTGR_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  return MTGR_OK;
+}
+
+size_t part_stack_bytes(int32_t T, int32_t row0, const mtgr_block_params* layers, int32_t L,
+                        bool own_qkvu) {
+  size_t m = 0;
+  for (int32_t l = 0; l < L; ++l) {
+    const size_t b = part_ws_layout(T, row0, &layers[l], own_qkvu, nullptr).bytes;
+    m = b > m ? b : m;
+  }
+  return m;
+}
+
+// Layers 0..L-1 on rows [row0, T): layer l reads and writes the Q|K|V|U of
+// cache + l * cache_rows * 4d; the spare x buffer follows the block workspace.
+int stack_rows(const mtgr_block_params* layers, int32_t L, const mtgr_batch* batch, int32_t row0,
+               uint16_t* cache, int32_t cache_rows, const float* x_in, float* x_out, void* ws,
+               cudaStream_t s) {
+  const int32_t k = batch->T - row0;
+  if (k <= 0) return MTGR_OK;
+  const size_t block_bytes = part_stack_bytes(batch->T, row0, layers, L, false);
+  float* spare = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + block_bytes);
+  const float* in = x_in;
+  for (int32_t l = 0; l < L; ++l) {
+    float* out = ((L - 1 - l) % 2 == 0) ? x_out : spare;
+    uint16_t* qkvu = cache + (size_t)l * cache_rows * 4 * layers[0].d;
+    const int rc = block_fwd_rows(&layers[l], batch, row0, in, out, qkvu, ws, s);
+    if (rc != MTGR_OK) return rc;
+    in = out;
+  }
+  return MTGR_OK;
+}
+}  // namespace
+
+MTGR_API size_t mtgr_stack_rows_workspace_bytes(int32_t T, int32_t row0,
+                                                const mtgr_block_params* layers, int32_t L) {
+  if (T < 0 || row0 < 0 || row0 > T || L <= 0 || layers == nullptr) return 0;
+  for (int32_t l = 0; l < L; ++l)
+    if (params_check(&layers[l]) != MTGR_OK || layers[l].dtype != MTGR_BF16) return 0;
+  return part_stack_bytes(T, row0, layers, L, false) +
+         (L > 1 ? align_up((size_t)(T - row0) * layers[0].d * sizeof(float), 256) : 0);
+}
+
+MTGR_API int mtgr_stack_fwd_rows(const mtgr_block_params* layers, int32_t L,
+                                 const mtgr_batch* batch, int32_t row0, void* d_qkvu_cache,
+                                 int32_t cache_rows, const float* d_x_in, float* d_x_out,
+                                 void* d_ws, size_t ws_bytes, mtgr_stream_t stream) {
+  int rc = serve_check(layers, L, batch);
+  if (rc != MTGR_OK) return rc;
+  if (row0 < 0 || row0 > batch->T || cache_rows < batch->T) return MTGR_ERR_INVALID_ARG;
+  if (row0 > 0 && batch->B != 1) return MTGR_ERR_UNSUPPORTED;  // rows [row0, T) must be one user's
+  const int32_t k = batch->T - row0;
+  if (k == 0) return MTGR_OK;
+  if (batch->group_id == nullptr || d_qkvu_cache == nullptr || d_x_in == nullptr ||
+      d_x_out == nullptr || d_ws == nullptr || d_x_in == d_x_out)
+    return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_qkvu_cache) || !aligned16(d_x_in) || !aligned16(d_x_out) || !aligned16(d_ws))
+    return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < mtgr_stack_rows_workspace_bytes(batch->T, row0, layers, L)) return MTGR_ERR_CAPACITY;
+  return stack_rows(layers, L, batch, row0, static_cast<uint16_t*>(d_qkvu_cache), cache_rows,
+                    d_x_in, d_x_out, d_ws, as_stream(stream));
 }
 
 MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const void* d_a,

@@ -425,6 +425,70 @@ __global__ void meta_fill_kernel(int32_t q_cap, int32_t kt_cap, int32_t e_cap,
   }
 }
 
+
+// Keeps the work items with a query row at or after q_first[b] (user-relative)
+// in place and in order; a pair whose first q-tile lies wholly before it
+// becomes a single-q-tile item of the second. One block, the list in chunks
+// of kScanThreads: every thread reads its item before any is written, and an
+// item only moves to a lower index, so no unread item is overwritten.
+__global__ void restrict_work_kernel(const int32_t* __restrict__ q_first, int32_t q_cap,
+                                     mtgr_work_item* work, int64_t* counts) {
+  __shared__ int32_t warp_sums[kScanThreads / 32];
+  __shared__ int32_t base_s;
+  const int64_t P64 = counts[3] < q_cap ? counts[3] : q_cap;
+  const int32_t P = P64 > 0 ? static_cast<int32_t>(P64) : 0;
+  if (threadIdx.x == 0) base_s = 0;
+  __syncthreads();
+  for (int32_t c0 = 0; c0 < P; c0 += kScanThreads) {
+    const int32_t i = c0 + static_cast<int32_t>(threadIdx.x);
+    mtgr_work_item it;
+    int32_t keep = 0;
+    if (i < P) {
+      it = work[i];
+      const int32_t qf = q_first[it.b];
+      const int32_t row_end = (it.qt0 + it.nq) * MTGR_TILE_M;  // one past the item's last row
+      if (row_end > qf && it.n > qf) {
+        keep = 1;
+        if (it.nq == 2 && (it.qt0 + 1) * MTGR_TILE_M <= qf) {  // only q-tile B is needed
+          it.qt0 += 1;
+          it.nq = 1;
+          it.e0a = it.e0b;
+          it.e1a = it.e1b;
+          it.e0b = it.e1b;
+          it.n_union = it.e1a - it.e0a;
+        }
+      }
+    }
+    // block-wide exclusive scan of keep
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int32_t incl = keep;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      int32_t v = lane < kScanThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (lane < kScanThreads / 32) warp_sums[lane] = v;  // inclusive over warps
+    }
+    __syncthreads();
+    const int32_t before = (wid > 0 ? warp_sums[wid - 1] : 0) + incl - keep;
+    const int32_t base = base_s;
+    if (keep) work[base + before] = it;
+    __syncthreads();
+    if (threadIdx.x == kScanThreads - 1) base_s = base + warp_sums[kScanThreads / 32 - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) counts[3] = base_s;
+}
+
 }  // namespace
 
 int launch_pack(int32_t B, const int32_t* lens, int32_t T, int32_t* seg_off, int32_t* user_off,
@@ -474,4 +538,10 @@ int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32
                                               work, counts);
   return launch_status();
 }
+int launch_restrict_work(const int32_t* q_first, int32_t q_cap, mtgr_work_item* work, int64_t* counts,
+                         cudaStream_t s) {
+  restrict_work_kernel<<<1, kScanThreads, 0, s>>>(q_first, q_cap, work, counts);
+  return launch_status();
+}
+
 }  // namespace mtgr

@@ -298,6 +298,51 @@ MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mt
                             mtgr_stream_t stream);
 
 /*
+ * Candidate-incremental scoring (serving). A user's U, S and R tokens never
+ * attend to candidates (mask rules 1-3), so the context side of every layer
+ * is computed once and candidates are scored against it afterwards, in one
+ * or more chunks (fun-rec 7.3.4: at inference the candidates of a request
+ * are independent of one another; the MTGR practice article, 5.2 on
+ * inference latency: cache the User/Seq tokens, which change rarely).
+ *
+ * mtgr_restrict_work: rewrites batch->work and counts[3] in place so that
+ * the attention computes only the work items holding a query row at or
+ * after d_q_first[b] (user-relative, int32 [B], device); a q-tile pair whose
+ * first q-tile lies wholly before it becomes a single-q-tile item. Order is
+ * kept. Call after mtgr_build_mask_meta on the same stream.
+ */
+MTGR_API int mtgr_restrict_work(const mtgr_batch* batch, const int32_t* d_q_first,
+                                mtgr_stream_t stream);
+
+/* Workspace bytes of mtgr_stack_fwd_rows (0 on invalid params; bf16 only). */
+MTGR_API size_t mtgr_stack_rows_workspace_bytes(int32_t T, int32_t row0,
+                                                const mtgr_block_params* layers, int32_t L);
+
+/*
+ * L bf16 blocks on rows [row0, T) of the batch, with every layer's Q|K|V|U
+ * kept in a caller-owned cache: layer l uses rows [0, T) of
+ * d_qkvu_cache + l * cache_rows * 4d (f16, [cache_rows][4d] per layer,
+ * cache_rows >= T, Q columns halved). Rows [row0, T) of each layer's slot
+ * are written; rows before row0 must already hold that layer's Q|K|V|U.
+ * d_x_in, d_x_out: [T - row0][d] float32, distinct.
+ *   Context pass: the user's U, S, R tokens as the batch (lens (N_U, N_S,
+ *     N_R, 0), normaliser override N = N_U + N_S + N_R + K for the K
+ *     candidates to come), row0 = 0.
+ *   Candidate pass: one user (B = 1) holding the same U, S, R tokens and a
+ *     chunk of candidates (lens (N_U, N_S, N_R, k), same timestamps and
+ *     normaliser N), row0 = N_U + N_S + N_R, work list restricted with
+ *     mtgr_restrict_work to rows >= row0; writes the k candidates' outputs.
+ *     Rows [row0, T) of the cache are overwritten, so chunks run one after
+ *     another. The result equals the candidate rows of the aggregated pass
+ *     over [U, S, R, all candidates] with the same N, up to the rounding
+ *     order of each candidate's self term.
+ */
+MTGR_API int mtgr_stack_fwd_rows(const mtgr_block_params* layers, int32_t L,
+                                 const mtgr_batch* batch, int32_t row0, void* d_qkvu_cache,
+                                 int32_t cache_rows, const float* d_x_in, float* d_x_out,
+                                 void* d_ws, size_t ws_bytes, mtgr_stream_t stream);
+
+/*
  * Dense GEMM with the block's epilogues, exposed for testing:
  *   out[m][n] = epi( sum_k a[m][k] * b[n][k] + bias[n] )
  *   epi = MTGR_EPI_NONE (out dtype MTGR_F16/MTGR_BF16/MTGR_F32),

@@ -81,6 +81,8 @@ def test_host_validation_without_device(lib):
     assert lib.mtgr_hstu_attention_fwd(None, 64, 2, 0, None, 0, None, None) == E
     assert lib.mtgr_stack_fwd(None, 0, None, None, None, None, 0, None) == E
     assert lib.mtgr_gemm(-1, 2, 64, 1, None, None, None, 0, None, 0, 0, None, None, None) == E
+    assert lib.mtgr_restrict_work(None, None, None) == E
+    assert lib.mtgr_stack_fwd_rows(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
 
 
 def _params(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16):
@@ -103,6 +105,24 @@ def test_workspace_sizes(lib):
     assert two == want + -(-T * 512 * 4 // 256) * 256
     assert _lib.mtgr_stack_workspace_bytes(T, [p]) == want
     assert _lib.mtgr_mask_meta_workspace_bytes(100, 8) == 1024
+
+
+def test_rows_workspace_sizes(lib):
+    # rows [row0, T) of a bf16 stack: GroupLN output and MLP hidden over the
+    # k = T - row0 rows, attention output over all T rows, Q|K|V|U in the
+    # caller's cache; a spare x buffer of k rows when L > 1
+    T, row0 = 1000, 900
+    p = _params()
+    k = T - row0
+    up = lambda n: -(-n // 256) * 256  # noqa: E731
+    one = up(k * 512 * 2) + up(T * 512 * 2) + up(k * 2048 * 2)
+    assert _lib.mtgr_stack_rows_workspace_bytes(T, row0, [p]) == one
+    assert _lib.mtgr_stack_rows_workspace_bytes(T, row0, [p, p, p]) == one + up(k * 512 * 4)
+    assert _lib.mtgr_stack_rows_workspace_bytes(T, 0, [p]) == up(T * 512 * 2) * 2 + up(T * 2048 * 2)
+    assert _lib.mtgr_stack_rows_workspace_bytes(T, T + 1, [p]) == 0
+    assert _lib.mtgr_stack_rows_workspace_bytes(T, -1, [p]) == 0
+    f = _params(d=64, H=2, d_ff=256, dtype=_lib.MTGR_F32)
+    assert _lib.mtgr_stack_rows_workspace_bytes(T, row0, [f]) == 0  # bf16 only
 
 
 def test_capacities_host_logic():
