@@ -5,7 +5,8 @@ user-aggregated sample D = [U, S, R, [C,I]_1..K], Group-Layer Normalization, the
 three-rule dynamic mask, pointwise SiLU attention normalised by the user's token
 count, the U gate, the second GroupLN and the MLP with residual (MTGR paper,
 "Method", the block update equations; fun-rec chapter 7.3, sections 7.3.3
-"Group Layer Normalization" and 7.3.4 "Dynamic Masking").
+"Group Layer Normalization" and 7.3.4 "Dynamic Masking"); and, on either side
+of the stack, the per-domain token MLPs and the CTR/CTCVR heads (``tokens.py``).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
 reference legs may import this package. The CUDA library never links, imports or
@@ -31,4 +32,9 @@ from .mtgr import (  # noqa: F401
     hstu_stack,
     mask_meta,
     visible_pairs,
+)
+from .tokens import (  # noqa: F401
+    token_mlp,
+    tokenize,
+    candidate_heads,
 )
