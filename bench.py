@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--pipeline", action="store_true",
+                    help="time token MLPs -> block -> CTR/CTCVR heads on the 512-user block "
+                         "workload, each part with its roofline (one JSON line)")
     return ap.parse_args()
 
 
@@ -575,6 +578,91 @@ def run_sweep(args, local):
     print(json.dumps(line), flush=True)
 
 
+def run_pipeline(args, local):
+    """The ranking forward around the block on the 512-user block workload:
+    the per-domain token MLPs build X, the HSTU block runs, the task heads
+    score the candidates. Each part is timed with the library's event timer;
+    the step is the three calls back to back (pack and mask metadata once)."""
+    import generative_recommendation_ranking_b200 as mt
+    from generative_recommendation_ranking_b200 import _lib
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    wl = synth.make_workload(2, seed=args.seed, B=args.users)
+    lens, d = wl["lens"], wl["d"]
+    rng = np.random.default_rng(args.seed + 1)
+    e = [torch.from_numpy(a).to(dev).to(torch.bfloat16) for a in synth.make_token_inputs(lens, d, rng)]
+    mlps = mt.TokenMLPs(synth.make_token_params(d, rng), device=dev)
+    heads = mt.CandidateHeads(synth.make_head_params(d, rng), device=dev)
+    batch = mt.PackedBatch(lens, wl["ts"], device=dev)
+    layers = [mt.BlockWeights(p, wl["H"], device=dev) for p in wl["layers"]]
+    T = batch.T
+    n_rows = [int(lens[:, g].sum()) for g in range(4)]
+    K = n_rows[3]
+    x = torch.empty(T, d, dtype=torch.float32, device=dev)
+    y = torch.empty_like(x)
+    logits = torch.empty(K, heads.n_tasks, dtype=torch.float32, device=dev)
+    tws = torch.empty(_lib.mtgr_tokenize_workspace_bytes(batch.B, d, n_rows), dtype=torch.uint8,
+                      device=dev)
+    hws = torch.empty(_lib.mtgr_heads_workspace_bytes(batch.B, K, heads.c), dtype=torch.uint8,
+                      device=dev)
+    sws = mt.stack_workspace(layers, batch)
+
+    def step():
+        _lib.mtgr_tokenize(batch.c, d, n_rows, e, mlps.c, x, tws, stream)
+        _lib.mtgr_stack_fwd([l.c for l in layers], batch.c, x, y, sws, stream)
+        _lib.mtgr_candidate_heads(heads.c, batch.c, K, y, logits, hws, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    batch.check()
+    n = max(5, min(args.steps, 100))
+    timer = _lib.Timer()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    timer.attach()
+    ms = time_steps(step, n, stream) / n
+    timer.detach()
+    clk = clocks.stop()
+    batch.check()
+    per = timer.read()
+    peaks, _ = load_peaks()
+    f = synth.TOKEN_F
+    tok_flop = 2.0 * sum(n_rows[g] * (f[g - 1] * d + d * d) for g in (1, 2, 3))
+    head_flop = 2.0 * K * d * heads.n_tasks * synth.HEAD_DH
+    parts = {}
+    for cls, flop in (("token_mlp", tok_flop), ("head_mlp", head_flop)):
+        t_ms, cnt = per[cls]
+        avg = t_ms / n
+        ach = flop / (avg * 1e-3) / 1e12
+        parts[cls] = {"bound": "tensor", "ms_per_step": avg, "launches_per_step": cnt / n,
+                      "achieved": ach, "unit": "TFLOP/s", "peak": peaks["bf16_tflops_sustained"],
+                      "frac": ach / peaks["bf16_tflops_sustained"]}
+    block_ms = sum(per[c][0] for c in ("pack", "mask_meta", "gln", "gemm_qkvu", "attention",
+                                       "gemm_mlp1", "gemm_mlp2")) / n
+    parts["block"] = {"ms_per_step": block_ms}
+    rows_ms = per["rows"][0] / n
+    # row bookkeeping: U rows bf16 in -> fp32 out; candidate rows fp32 in -> bf16
+    # out; the heads' last layer reads the hidden rows (bf16) once
+    rows_bytes = (n_rows[0] * d * 6 + K * d * 6 + K * heads.n_tasks * synth.HEAD_DH * 2
+                  + 4 * (T + K))
+    parts["rows"] = {"bound": "hbm", "ms_per_step": rows_ms, "launches_per_step": per["rows"][1] / n,
+                     "achieved": rows_bytes / (rows_ms * 1e-3) / 1e9, "unit": "GB/s",
+                     "peak": peaks["hbm_gbs"]}
+    parts["rows"]["frac"] = parts["rows"]["achieved"] / parts["rows"]["peak"]
+    line = {"metric": "ranking forward: token MLPs -> HSTU block -> CTR/CTCVR heads",
+            "value": batch.B / (ms * 1e-3), "unit": "user-samples/s", "ms_per_step": ms,
+            "steps": n, "warmup": max(3, args.warmup), "higher_is_better": True, "n_gpus": 1,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl["name"], "users": batch.B, "tokens": T, "candidates": K,
+                       "token_f": list(f), "head_dh": synth.HEAD_DH, "tasks": heads.n_tasks,
+                       "l2": "inputs 0.9 GB > L2"},
+            "parts": parts, "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args) if args.impl == "ours" else (
@@ -582,6 +670,9 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.pipeline:
+            if rank == 0:
+                run_pipeline(args, local)
         elif synth.WORKLOADS[args.config].kind == "sweep":
             if rank == 0:
                 run_sweep(args, local)

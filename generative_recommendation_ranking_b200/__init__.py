@@ -17,6 +17,8 @@ from ._lib import (  # noqa: F401
     load,
     mtgr_block_workspace_bytes,
     mtgr_build_mask_meta,
+    mtgr_candidate_heads,
+    mtgr_heads_workspace_bytes,
     mtgr_gemm,
     mtgr_group_layernorm,
     mtgr_hstu_attention_fwd,
@@ -28,12 +30,18 @@ from ._lib import (  # noqa: F401
     mtgr_stack_fwd_rows,
     mtgr_stack_rows_workspace_bytes,
     mtgr_stack_workspace_bytes,
+    mtgr_tokenize,
+    mtgr_tokenize_workspace_bytes,
     mtgr_version,
     status_string,
 )
 from .api import (  # noqa: F401
     BlockWeights,
+    CandidateHeads,
     ContextCache,
+    TokenMLPs,
+    candidate_heads,
+    tokenize,
     PackedBatch,
     capacities,
     gemm,

@@ -65,6 +65,16 @@ class MtgrBlockParams(ctypes.Structure):
                 ("w2", c_vp), ("b_qkvu", c_vp), ("b1", c_vp), ("b2", c_vp)]
 
 
+class MtgrTokenMlp(ctypes.Structure):
+    _fields_ = [("f", c_i32), ("reserved", c_i32), ("w1", c_vp), ("b1", c_vp), ("w2", c_vp),
+                ("b2", c_vp)]
+
+
+class MtgrHeadParams(ctypes.Structure):
+    _fields_ = [("d", c_i32), ("d_h", c_i32), ("n_tasks", c_i32), ("reserved", c_i32),
+                ("w1", c_vp), ("b1", c_vp), ("w2", c_vp), ("b2", c_vp)]
+
+
 _SIGNATURES = {
     "mtgr_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mtgr_version": (ctypes.c_int, []),
@@ -93,6 +103,13 @@ _SIGNATURES = {
     "mtgr_stack_fwd_rows": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams), c_i32,
                                            ctypes.POINTER(MtgrBatch), c_i32, c_vp, c_i32, c_vp, c_vp,
                                            c_vp, c_size, c_vp]),
+    "mtgr_tokenize_workspace_bytes": (c_size, [c_i32, c_i32, ctypes.POINTER(c_i32)]),
+    "mtgr_tokenize": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_i32, ctypes.POINTER(c_i32),
+                                     ctypes.POINTER(c_vp), ctypes.POINTER(MtgrTokenMlp), c_vp, c_vp,
+                                     c_size, c_vp]),
+    "mtgr_heads_workspace_bytes": (c_size, [c_i32, c_i32, ctypes.POINTER(MtgrHeadParams)]),
+    "mtgr_candidate_heads": (ctypes.c_int, [ctypes.POINTER(MtgrHeadParams), ctypes.POINTER(MtgrBatch),
+                                            c_i32, c_vp, c_vp, c_vp, c_size, c_vp]),
     "mtgr_gemm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32,
                                  c_i32, c_vp, c_vp, c_vp]),
     "mtgr_timer_create": (c_vp, []),
@@ -239,7 +256,32 @@ def mtgr_stack_fwd_rows(layers, batch: MtgrBatch, row0: int, d_cache, cache_rows
         _ptr(d_x_out), _ptr(d_ws), d_ws.numel() * d_ws.element_size(), _stream(stream)))
 
 
-TIMER_CLASSES = ("pack", "mask_meta", "gln", "gemm_qkvu", "attention", "gemm_mlp1", "gemm_mlp2")
+def mtgr_tokenize_workspace_bytes(B: int, d: int, n_rows) -> int:
+    return load().mtgr_tokenize_workspace_bytes(B, d, (c_i32 * 4)(*n_rows))
+
+
+def mtgr_tokenize(batch: MtgrBatch, d: int, n_rows, d_e, mlps, d_x, d_ws, stream=None):
+    """d_e: four device tensors (U, S, R, C inputs; None where a domain has no
+    rows); mlps: three MtgrTokenMlp (S, R, C)."""
+    _check("mtgr_tokenize", load().mtgr_tokenize(
+        ctypes.byref(batch), d, (c_i32 * 4)(*n_rows), (c_vp * 4)(*[_ptr(e) for e in d_e]),
+        (MtgrTokenMlp * 3)(*mlps), _ptr(d_x), _ptr(d_ws), d_ws.numel() * d_ws.element_size(),
+        _stream(stream)))
+
+
+def mtgr_heads_workspace_bytes(B: int, k_total: int, p: MtgrHeadParams) -> int:
+    return load().mtgr_heads_workspace_bytes(B, k_total, ctypes.byref(p))
+
+
+def mtgr_candidate_heads(p: MtgrHeadParams, batch: MtgrBatch, k_total: int, d_x, d_out, d_ws,
+                         stream=None):
+    _check("mtgr_candidate_heads", load().mtgr_candidate_heads(
+        ctypes.byref(p), ctypes.byref(batch), k_total, _ptr(d_x), _ptr(d_out), _ptr(d_ws),
+        d_ws.numel() * d_ws.element_size(), _stream(stream)))
+
+
+TIMER_CLASSES = ("pack", "mask_meta", "gln", "gemm_qkvu", "attention", "gemm_mlp1", "gemm_mlp2",
+                 "token_mlp", "head_mlp", "rows")
 
 
 class Timer:

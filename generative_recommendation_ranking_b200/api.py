@@ -284,3 +284,81 @@ class ContextCache:
         _lib.mtgr_stack_fwd_rows(self.c_layers, batch.c, self.n_ctx, self.cache, self.cache_rows,
                                  x_cand, out, ws, stream)
         return out
+
+
+class TokenMLPs:
+    """The S, R and candidate token MLPs on the device: Linear(F_g, d) ->
+    SiLU -> Linear(d, d) per domain, bf16 weights ([out, in]), fp32 biases.
+    ``p`` holds ``w1_g``, ``b1_g``, ``w2_g``, ``b2_g`` for g in s, r, c
+    (biases may be None)."""
+
+    def __init__(self, p: dict, device="cuda"):
+        dev = torch.device(device)
+        self.t = {}
+        mlps = []
+        for g in ("s", "r", "c"):
+            w1 = torch.as_tensor(np.asarray(p["w1_" + g], np.float32)).to(dev).to(torch.bfloat16).contiguous()
+            w2 = torch.as_tensor(np.asarray(p["w2_" + g], np.float32)).to(dev).to(torch.bfloat16).contiguous()
+            b1 = p.get("b1_" + g)
+            b2 = p.get("b2_" + g)
+            b1 = None if b1 is None else torch.as_tensor(np.asarray(b1, np.float32)).to(dev)
+            b2 = None if b2 is None else torch.as_tensor(np.asarray(b2, np.float32)).to(dev)
+            self.t[g] = (w1, b1, w2, b2)
+            mlps.append(_lib.MtgrTokenMlp(f=w1.shape[1], reserved=0, w1=w1.data_ptr(),
+                                          b1=None if b1 is None else b1.data_ptr(), w2=w2.data_ptr(),
+                                          b2=None if b2 is None else b2.data_ptr()))
+        self.c = mlps
+        self.d = self.t["s"][2].shape[0]
+
+
+def tokenize(mlps: TokenMLPs, batch: PackedBatch, e: list, out=None, ws=None,
+             stream=None) -> torch.Tensor:
+    """Block input X [T, d] float32 from the per-domain inputs ``e`` = [E_U,
+    E_S, E_R, E_C] (bf16 device tensors, each domain's tokens user by user)."""
+    d = mlps.d
+    n_rows = [int(batch.lens[:, g].sum()) for g in range(4)]
+    if out is None:
+        out = torch.empty(batch.T, d, dtype=torch.float32, device=batch.device)
+    need = _lib.mtgr_tokenize_workspace_bytes(batch.B, d, n_rows)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, batch.device)
+    _lib.mtgr_tokenize(batch.c, d, n_rows, [t if t is not None and t.numel() else None for t in e],
+                       mlps.c, out, ws, stream)
+    return out
+
+
+class CandidateHeads:
+    """Task heads (CTR, CTCVR, ...) on the device: per task Linear(d, d_h) ->
+    SiLU -> Linear(d_h, 1). ``p``: ``w1`` [n_tasks, d_h, d], ``b1``
+    [n_tasks, d_h] or None, ``w2`` [n_tasks, d_h], ``b2`` [n_tasks] or None."""
+
+    def __init__(self, p: dict, device="cuda"):
+        dev = torch.device(device)
+        w1 = np.asarray(p["w1"], np.float32)
+        n_tasks, d_h, d = w1.shape
+        self.w1 = torch.as_tensor(w1.reshape(n_tasks * d_h, d)).to(dev).to(torch.bfloat16).contiguous()
+        self.b1 = (None if p.get("b1") is None else
+                   torch.as_tensor(np.asarray(p["b1"], np.float32).reshape(-1)).to(dev))
+        self.w2 = torch.as_tensor(np.asarray(p["w2"], np.float32).reshape(n_tasks, d_h)).to(dev).contiguous()
+        self.b2 = (None if p.get("b2") is None else
+                   torch.as_tensor(np.asarray(p["b2"], np.float32).reshape(-1)).to(dev))
+        self.c = _lib.MtgrHeadParams(d=d, d_h=d_h, n_tasks=n_tasks, reserved=0,
+                                     w1=self.w1.data_ptr(),
+                                     b1=None if self.b1 is None else self.b1.data_ptr(),
+                                     w2=self.w2.data_ptr(),
+                                     b2=None if self.b2 is None else self.b2.data_ptr())
+        self.n_tasks = n_tasks
+
+
+def candidate_heads(heads: CandidateHeads, batch: PackedBatch, x: torch.Tensor, out=None, ws=None,
+                    stream=None) -> torch.Tensor:
+    """Logits [K_total, n_tasks] float32 of the batch's candidates (user by
+    user) from the stack output x [T, d] float32."""
+    k_total = int(batch.lens[:, 3].sum())
+    if out is None:
+        out = torch.empty(k_total, heads.n_tasks, dtype=torch.float32, device=x.device)
+    need = _lib.mtgr_heads_workspace_bytes(batch.B, k_total, heads.c)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x.device)
+    _lib.mtgr_candidate_heads(heads.c, batch.c, k_total, x, out, ws, stream)
+    return out

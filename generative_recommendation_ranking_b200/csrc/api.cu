@@ -25,6 +25,19 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
                    cudaStream_t s);
 int launch_restrict_work(const int32_t* q_first, int32_t q_cap, mtgr_work_item* work, int64_t* counts,
                          cudaStream_t s);
+int launch_gemm_tc_rowmap(int M, int N, int K, const void* a, const void* b, const float* bias,
+                          const int32_t* row_map, float* out, int out_rows, int32_t* status,
+                          cudaStream_t s);
+int launch_dom_scan(int32_t B, const int32_t* seg_off, const int32_t n_rows[4], uint32_t check_mask,
+                    int32_t* dom_off, int32_t* status, cudaStream_t s);
+int launch_row_map(int32_t B, const int32_t* seg_off, const int32_t* dom_off, const int32_t base[4],
+                   const int32_t n_rows[4], uint32_t dom_mask, int32_t* map, cudaStream_t s);
+int launch_scatter_rows(int32_t n, int32_t d, const void* src, const int32_t* map, int32_t dst_rows,
+                        float* dst, cudaStream_t s);
+int launch_gather_rows(int32_t n, int32_t d, const float* src, int32_t src_rows, const int32_t* map,
+                       void* dst, cudaStream_t s);
+int launch_head_dot(int32_t n, int32_t n_tasks, int32_t d_h, const void* h, const float* w2,
+                    const float* b2, float* out, cudaStream_t s);
 int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu, float* g,
                     cudaStream_t s);
 int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
@@ -489,6 +502,172 @@ MTGR_API int mtgr_stack_fwd_rows(const mtgr_block_params* layers, int32_t L,
   if (ws_bytes < mtgr_stack_rows_workspace_bytes(batch->T, row0, layers, L)) return MTGR_ERR_CAPACITY;
   return stack_rows(layers, L, batch, row0, static_cast<uint16_t*>(d_qkvu_cache), cache_rows,
                     d_x_in, d_x_out, d_ws, as_stream(stream));
+}
+
+namespace {
+// Workspace of mtgr_tokenize: per-domain user offsets, the domain-major row
+// map, and the hidden rows of the largest domain (domains run one by one).
+struct TokWs {
+  int32_t* dom_off;
+  int32_t* map;
+  void* h;
+  size_t bytes;
+};
+
+TokWs tok_ws_layout(int32_t B, int32_t d, const int32_t n_rows[4], void* base) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  int64_t T = 0, hmax = 0;
+  for (int g = 0; g < 4; ++g) T += n_rows[g];
+  for (int g = 1; g < 4; ++g) hmax = n_rows[g] > hmax ? n_rows[g] : hmax;
+  TokWs w;
+  size_t off = 0;
+  w.dom_off = reinterpret_cast<int32_t*>(p + off); off += align_up(4 * ((size_t)B + 1) * 4, 256);
+  w.map = reinterpret_cast<int32_t*>(p + off);     off += align_up((size_t)T * 4, 256);
+  w.h = p + off;                                   off += align_up((size_t)hmax * d * 2, 256);
+  w.bytes = off;
+  return w;
+}
+
+struct HeadWs {
+  int32_t* dom_off;
+  int32_t* map;
+  void* xc;
+  void* h;
+  size_t bytes;
+};
+
+HeadWs head_ws_layout(int32_t B, int32_t k_total, const mtgr_head_params* p, void* base) {
+  uint8_t* b = static_cast<uint8_t*>(base);
+  HeadWs w;
+  size_t off = 0;
+  w.dom_off = reinterpret_cast<int32_t*>(b + off); off += align_up(4 * ((size_t)B + 1) * 4, 256);
+  w.map = reinterpret_cast<int32_t*>(b + off);     off += align_up((size_t)k_total * 4, 256);
+  w.xc = b + off;  off += align_up((size_t)k_total * p->d * 2, 256);
+  w.h = b + off;   off += align_up((size_t)k_total * p->n_tasks * p->d_h * 2, 256);
+  w.bytes = off;
+  return w;
+}
+
+bool tok_sizes_ok(int32_t B, int32_t d, const int32_t n_rows[4]) {
+  if (B < 0 || d <= 0 || d % 64 != 0 || d > kMaxD || n_rows == nullptr) return false;
+  int64_t T = 0;
+  for (int g = 0; g < 4; ++g) {
+    if (n_rows[g] < 0) return false;
+    T += n_rows[g];
+  }
+  return T <= INT32_MAX;
+}
+
+int heads_check(const mtgr_head_params* p) {
+  if (p == nullptr || p->d <= 0 || p->d % 64 != 0 || p->d > kMaxD || p->d_h <= 0 ||
+      p->d_h % 32 != 0 || p->n_tasks <= 0 || p->w1 == nullptr || p->w2 == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  if ((int64_t)p->n_tasks * p->d_h > (1 << 16)) return MTGR_ERR_UNSUPPORTED;
+  if (!aligned16(p->w1) || !aligned16(p->w2) || (p->b1 && !aligned16(p->b1)))
+    return MTGR_ERR_INVALID_ARG;
+  return MTGR_OK;
+}
+}  // namespace
+
+MTGR_API size_t mtgr_tokenize_workspace_bytes(int32_t B, int32_t d, const int32_t n_rows[4]) {
+  if (!tok_sizes_ok(B, d, n_rows)) return 0;
+  return tok_ws_layout(B, d, n_rows, nullptr).bytes;
+}
+
+MTGR_API int mtgr_tokenize(const mtgr_batch* batch, int32_t d, const int32_t n_rows[4],
+                           const void* const d_e[4], const mtgr_token_mlp mlp[3], float* d_x,
+                           void* d_ws, size_t ws_bytes, mtgr_stream_t stream) {
+  if (!batch_ok(batch) || !tok_sizes_ok(batch->B, d, n_rows) || d_e == nullptr || mlp == nullptr ||
+      d_x == nullptr || d_ws == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  int64_t T = 0;
+  for (int g = 0; g < 4; ++g) T += n_rows[g];
+  if (T != batch->T) return MTGR_ERR_INVALID_ARG;
+  for (int g = 0; g < 4; ++g)
+    if (n_rows[g] > 0 && (d_e[g] == nullptr || !aligned16(d_e[g]))) return MTGR_ERR_INVALID_ARG;
+  for (int g = 0; g < 3; ++g) {
+    const mtgr_token_mlp& m = mlp[g];
+    if (m.f <= 0 || m.f % 64 != 0 || m.w1 == nullptr || m.w2 == nullptr || !aligned16(m.w1) ||
+        !aligned16(m.w2) || (m.b1 && !aligned16(m.b1)) || (m.b2 && !aligned16(m.b2)))
+      return MTGR_ERR_INVALID_ARG;
+  }
+  if (!aligned16(d_x) || !aligned16(d_ws)) return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < mtgr_tokenize_workspace_bytes(batch->B, d, n_rows)) return MTGR_ERR_CAPACITY;
+  if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  if (T == 0) return MTGR_OK;
+  const cudaStream_t s = as_stream(stream);
+  TokWs w = tok_ws_layout(batch->B, d, n_rows, d_ws);
+  const int32_t base[4] = {0, n_rows[0], n_rows[0] + n_rows[1], n_rows[0] + n_rows[1] + n_rows[2]};
+  int rc;
+  {
+    TimedScope tsc(MTGR_TIMER_ROWS, s, n_rows[0] > 0 ? 3 : 2);
+    if (cudaMemsetAsync(w.map, 0xFF, (size_t)T * 4, s) != cudaSuccess) return MTGR_ERR_CUDA;
+    if ((rc = launch_dom_scan(batch->B, batch->seg_off, n_rows, 0xFu, w.dom_off, batch->status, s)) !=
+        MTGR_OK)
+      return rc;
+    if ((rc = launch_row_map(batch->B, batch->seg_off, w.dom_off, base, n_rows, 0xFu, w.map, s)) !=
+        MTGR_OK)
+      return rc;
+    if ((rc = launch_scatter_rows(n_rows[0], d, d_e[0], w.map, batch->T, d_x, s)) != MTGR_OK)
+      return rc;
+  }
+  int launches = 0;
+  for (int g = 1; g < 4; ++g) launches += n_rows[g] > 0 ? 2 : 0;
+  TimedScope tsc(MTGR_TIMER_TOKEN_MLP, s, launches);
+  for (int g = 1; g < 4; ++g) {
+    if (n_rows[g] == 0) continue;
+    const mtgr_token_mlp& m = mlp[g - 1];
+    if ((rc = launch_gemm_tc(n_rows[g], d, m.f, d_e[g], m.w1, m.b1, MTGR_EPI_SILU, nullptr, 0,
+                             MTGR_BF16, w.h, batch->status, s)) != MTGR_OK)
+      return rc;
+    if ((rc = launch_gemm_tc_rowmap(n_rows[g], d, d, w.h, m.w2, m.b2, w.map + base[g], d_x,
+                                    batch->T, batch->status, s)) != MTGR_OK)
+      return rc;
+  }
+  return MTGR_OK;
+}
+
+MTGR_API size_t mtgr_heads_workspace_bytes(int32_t B, int32_t k_total, const mtgr_head_params* p) {
+  if (B < 0 || k_total < 0 || heads_check(p) != MTGR_OK) return 0;
+  return head_ws_layout(B, k_total, p, nullptr).bytes;
+}
+
+MTGR_API int mtgr_candidate_heads(const mtgr_head_params* p, const mtgr_batch* batch,
+                                  int32_t k_total, const float* d_x, float* d_out, void* d_ws,
+                                  size_t ws_bytes, mtgr_stream_t stream) {
+  int rc = heads_check(p);
+  if (rc != MTGR_OK) return rc;
+  if (!batch_ok(batch) || k_total < 0 || k_total > batch->T || d_x == nullptr || d_out == nullptr ||
+      d_ws == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x) || !aligned16(d_ws) || !aligned16(d_out)) return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < mtgr_heads_workspace_bytes(batch->B, k_total, p)) return MTGR_ERR_CAPACITY;
+  if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  const cudaStream_t s = as_stream(stream);
+  HeadWs w = head_ws_layout(batch->B, k_total, p, d_ws);
+  const int32_t n_rows[4] = {0, 0, 0, k_total};
+  const int32_t base[4] = {0, 0, 0, 0};
+  {
+    TimedScope tsc(MTGR_TIMER_ROWS, s, k_total > 0 ? 3 : 1);
+    if (k_total > 0 && cudaMemsetAsync(w.map, 0xFF, (size_t)k_total * 4, s) != cudaSuccess)
+      return MTGR_ERR_CUDA;
+    if ((rc = launch_dom_scan(batch->B, batch->seg_off, n_rows, 0x8u, w.dom_off, batch->status, s)) !=
+        MTGR_OK)
+      return rc;
+    if (k_total == 0) return MTGR_OK;
+    if ((rc = launch_row_map(batch->B, batch->seg_off, w.dom_off, base, n_rows, 0x8u, w.map, s)) !=
+        MTGR_OK)
+      return rc;
+    if ((rc = launch_gather_rows(k_total, p->d, d_x, batch->T, w.map, w.xc, s)) != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_HEAD_MLP, s, 1);
+    if ((rc = launch_gemm_tc(k_total, p->n_tasks * p->d_h, p->d, w.xc, p->w1, p->b1, MTGR_EPI_SILU,
+                             nullptr, 0, MTGR_BF16, w.h, batch->status, s)) != MTGR_OK)
+      return rc;
+  }
+  TimedScope tsc(MTGR_TIMER_ROWS, s, 1);
+  return launch_head_dot(k_total, p->n_tasks, p->d_h, w.h, p->w2, p->b2, d_out, s);
 }
 
 MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const void* d_a,

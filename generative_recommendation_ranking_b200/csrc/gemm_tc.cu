@@ -46,6 +46,8 @@ struct GemmArgs {
   void* out;
   int q_cols;
   int32_t* status;
+  const int32_t* row_map;  // row-map form: output row of each a row (-1: dropped)
+  int out_rows;            // row-map form: rows of out
 };
 
 __device__ __forceinline__ float u32_as_f(uint32_t v) { return __uint_as_float(v); }
@@ -61,10 +63,9 @@ __device__ __forceinline__ uint32_t stg_off(int r, int c) {
 // Epilogue math of 32 consecutive columns [col0, col0+32) of one row; the
 // result goes to row `r` of the staging block `stg` (holding the residual
 // block on entry for EPI_RESID).
-template <int EPI, int OUT>
-__device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
-                                               uint8_t* stg, int r) {
-  float v[32];
+template <int EPI>
+__device__ __forceinline__ void epilogue_math(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
+                                              float (&v)[32]) {
 #pragma unroll
   for (int c = 0; c < 32; ++c) v[c] = u32_as_f(acc[c]);
   if (a.bias != nullptr) {
@@ -82,6 +83,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, cons
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] = silu_fast(v[c]);
   }
+}
+
+template <int EPI, int OUT>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
+                                               uint8_t* stg, int r) {
+  float v[32];
+  epilogue_math<EPI>(a, col0, acc, v);
   if (OUT == MTGR_F32) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -107,7 +115,24 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, cons
   }
 }
 
-template <int EPI, int OUT>
+// Row-map form, rows that do not form one run: each lane holds the
+// destination of its row; the values wait in the warp's staging block (as
+// written by epilogue_chunk), and every store instruction writes four whole
+// 128-byte row pieces.
+__device__ __forceinline__ void rowmap_scatter(const GemmArgs& a, int col0, const uint8_t* stg,
+                                               int my_dst, int lane) {
+  const int q = lane & 7;
+#pragma unroll
+  for (int r0 = 0; r0 < 32; r0 += 4) {
+    const int r = r0 + (lane >> 3);
+    const int dst = __shfl_sync(0xffffffffu, my_dst, r);
+    const float4 x = *reinterpret_cast<const float4*>(stg + stg_off<MTGR_F32>(r, q));
+    if (dst >= 0 && dst < a.out_rows)
+      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)dst * a.N + col0 + 4 * q) = x;
+  }
+}
+
+template <int EPI, int OUT, bool ROWMAP>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
@@ -207,6 +232,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* stg = sStg + ew * 2 * STG_BYTES;
     int acc = 0;
     uint32_t acc_phase = 0, chunk = 0;
+    bool prev_scatter = false;  // row-map form: the last chunk left row by row
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile / n_tiles, nb = tile % n_tiles;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
@@ -219,6 +245,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int col0 = nb * BN + c * 32;
         if (col0 >= N) break;
         const int buf = chunk & 1;
+        if (ROWMAP) {
+          // 32 rows whose destinations are 32 consecutive rows leave by one
+          // TMA store, like the plain form; any other group row by row
+          uint8_t* sb = stg + buf * STG_BYTES;
+          if (lane == 0) {
+            if (prev_scatter) bulk_wait_group_read<0>();  // chunk - 1 committed no store
+            else bulk_wait_group_read<1>();
+          }
+          __syncwarp();
+          uint32_t r[32];
+          tmem_ld32(t_row + c * 32, r);
+          tmem_ld_wait();
+          epilogue_chunk<EPI, OUT>(args, col0, r, sb, lane);
+          const int m = row0 + lane;
+          const int my_dst = m < M ? __ldg(args.row_map + m) : -1;
+          const int dst0 = __shfl_sync(0xffffffffu, my_dst, 0);
+          const bool run = __all_sync(0xffffffffu, my_dst == dst0 + lane) && dst0 >= 0 &&
+                           dst0 + 32 <= args.out_rows;
+          if (run) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmO, sb, col0, dst0);
+              bulk_commit_group();
+            }
+          } else {
+            __syncwarp();
+            rowmap_scatter(args, col0, sb, my_dst, lane);
+          }
+          prev_scatter = !run;
+          continue;
+        }
         uint8_t* sb = stg + buf * STG_BYTES;
         // the TMA store that last read this buffer (two blocks ago) must be done
         if (lane == 0) bulk_wait_group_read<1>();
@@ -259,10 +317,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EPI, int OUT>
+template <int EPI, int OUT, bool ROWMAP = false>
 int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
              const CUtensorMap& tr, const GemmArgs& args, cudaStream_t s) {
-  auto kern = gemm_tc_kernel<EPI, OUT>;
+  auto kern = gemm_tc_kernel<EPI, OUT, ROWMAP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
       cudaSuccess)
     return MTGR_ERR_CUDA;
@@ -298,7 +356,7 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
                       (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MTGR_OK) return rc;
   }
-  GemmArgs args{M, N, K, bias, resid, out, q_cols, status};
+  GemmArgs args{M, N, K, bias, resid, out, q_cols, status, nullptr, 0};
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_NONE, MTGR_F16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_NONE, MTGR_BF16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_NONE, MTGR_F32>(ta, tb, to, tr, args, s);
@@ -306,6 +364,27 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
   if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, to, tr, args, s);
   return MTGR_ERR_UNSUPPORTED;
+}
+
+// out[row_map[m]][n] = sum_k a[m][k] b[n][k] + bias[n] (fp32 out with out_rows
+// rows; a row whose map entry is negative or past out_rows is dropped).
+int launch_gemm_tc_rowmap(int M, int N, int K, const void* a, const void* b, const float* bias,
+                          const int32_t* row_map, float* out, int out_rows, int32_t* status,
+                          cudaStream_t s) {
+  if (M == 0 || N == 0) return MTGR_OK;
+  CUtensorMap ta, tb;
+  int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
+  if (rc != MTGR_OK) return rc;
+  if (out_rows <= 0) return MTGR_OK;
+  CUtensorMap to;
+  rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)out_rows,
+                    (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != MTGR_OK) return rc;
+  GemmArgs args{M, N, K, bias, nullptr, out, 0, status, row_map, out_rows};
+  // the residual map is not read in this form
+  return launch_t<MTGR_EPI_NONE, MTGR_F32, true>(ta, tb, to, to, args, s);
 }
 
 }  // namespace mtgr

@@ -343,6 +343,67 @@ MTGR_API int mtgr_stack_fwd_rows(const mtgr_block_params* layers, int32_t L,
                                  void* d_ws, size_t ws_bytes, mtgr_stream_t stream);
 
 /*
+ * Token MLPs and candidate heads: the steps on either side of the stack
+ * (blog posts "generative recommendation 18: MTGR", "Converting
+ * heterogeneous features into tokens"; summary page, "Method"; fun-rec
+ * 7.3.3: CandidateToken_i = MLP(Concat(Emb(Item_i), Emb(Cross_i)))).
+ *
+ * One domain's token MLP: Linear(f, d) -> SiLU -> Linear(d, d).
+ */
+typedef struct mtgr_token_mlp {
+  int32_t f;          /* input width (concatenated field embeddings), % 64 == 0 */
+  int32_t reserved;
+  const void* w1;     /* [d][f] bf16 */
+  const float* b1;    /* [d] or NULL */
+  const void* w2;     /* [d][d] bf16 */
+  const float* b2;    /* [d] or NULL */
+} mtgr_token_mlp;
+
+/* Workspace bytes of mtgr_tokenize (0 on invalid sizes). */
+MTGR_API size_t mtgr_tokenize_workspace_bytes(int32_t B, int32_t d, const int32_t n_rows[4]);
+
+/*
+ * Builds the block input X of a packed batch from per-domain inputs:
+ *   d_e[0]: U tokens, bf16 [n_rows[0]][d] (the feature embeddings; no MLP);
+ *   d_e[g], g = 1, 2, 3 (S, R, C): bf16 [n_rows[g]][mlp[g-1].f], the
+ *     concatenated field embeddings, through mlp[g-1].
+ * Each input lists its domain's tokens user by user, each user's in sequence
+ * order; X row seg_off[4b + g] + j (float32 [T][d]) gets user b's j-th token
+ * of domain g. n_rows (host) must equal the batch's per-domain totals; a
+ * mismatch is a device error (MTGR_ERR_DEVICE_VALIDATION in the batch status)
+ * and X is then undefined. d % 64 == 0; all pointers 16-byte aligned.
+ */
+MTGR_API int mtgr_tokenize(const mtgr_batch* batch, int32_t d, const int32_t n_rows[4],
+                           const void* const d_e[4], const mtgr_token_mlp mlp[3], float* d_x,
+                           void* d_ws, size_t ws_bytes, mtgr_stream_t stream);
+
+/* Task heads on the candidates' rows: per task t, Linear(d, d_h) -> SiLU ->
+ * Linear(d_h, 1), giving a logit (CTR, CTCVR, ...). */
+typedef struct mtgr_head_params {
+  int32_t d;          /* d_model, % 64 == 0 */
+  int32_t d_h;        /* hidden width per task, % 32 == 0 */
+  int32_t n_tasks;    /* >= 1 */
+  int32_t reserved;
+  const void* w1;     /* [n_tasks * d_h][d] bf16 (task t: rows [t d_h, (t+1) d_h)) */
+  const float* b1;    /* [n_tasks * d_h] or NULL */
+  const float* w2;    /* [n_tasks][d_h] float32 */
+  const float* b2;    /* [n_tasks] or NULL */
+} mtgr_head_params;
+
+/* Workspace bytes of mtgr_candidate_heads (0 on invalid params). */
+MTGR_API size_t mtgr_heads_workspace_bytes(int32_t B, int32_t k_total, const mtgr_head_params* p);
+
+/*
+ * Logits d_out float32 [k_total][n_tasks] of the candidates of the batch,
+ * user by user, each user's in sequence order, from its output rows d_x
+ * float32 [T][d]. k_total (host) must equal the batch's candidate count; a
+ * mismatch is a device error as for mtgr_tokenize.
+ */
+MTGR_API int mtgr_candidate_heads(const mtgr_head_params* p, const mtgr_batch* batch,
+                                  int32_t k_total, const float* d_x, float* d_out, void* d_ws,
+                                  size_t ws_bytes, mtgr_stream_t stream);
+
+/*
  * Dense GEMM with the block's epilogues, exposed for testing:
  *   out[m][n] = epi( sum_k a[m][k] * b[n][k] + bias[n] )
  *   epi = MTGR_EPI_NONE (out dtype MTGR_F16/MTGR_BF16/MTGR_F32),
@@ -367,7 +428,9 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
  * them, per class: MTGR_TIMER_PACK (2 kernels per call), MTGR_TIMER_MASK_META
  * (6), MTGR_TIMER_GLN, MTGR_TIMER_GEMM_QKVU, MTGR_TIMER_ATTENTION,
  * MTGR_TIMER_GEMM_MLP1, MTGR_TIMER_GEMM_MLP2 (1 each; mtgr_gemm counts as
- * MTGR_TIMER_GEMM_QKVU). mtgr_timer_read synchronises on the recorded events,
+ * MTGR_TIMER_GEMM_QKVU); MTGR_TIMER_TOKEN_MLP (the token MLPs' GEMMs, 2 per
+ * domain with tokens), MTGR_TIMER_HEAD_MLP (the heads' first layer, 1) and
+ * MTGR_TIMER_ROWS (the row bookkeeping of tokenize and heads: 3 and 4). mtgr_timer_read synchronises on the recorded events,
  * writes the summed milliseconds and launch counts per class into
  * ms[MTGR_TIMER_CLASSES] and launches[MTGR_TIMER_CLASSES] (host arrays) and
  * clears the records. Attaching NULL detaches. Not for use during CUDA graph
@@ -380,7 +443,10 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
 #define MTGR_TIMER_ATTENTION 4
 #define MTGR_TIMER_GEMM_MLP1 5
 #define MTGR_TIMER_GEMM_MLP2 6
-#define MTGR_TIMER_CLASSES 7
+#define MTGR_TIMER_TOKEN_MLP 7
+#define MTGR_TIMER_HEAD_MLP 8
+#define MTGR_TIMER_ROWS 9
+#define MTGR_TIMER_CLASSES 10
 typedef struct mtgr_timer mtgr_timer;
 MTGR_API mtgr_timer* mtgr_timer_create(void);
 MTGR_API void mtgr_timer_destroy(mtgr_timer* timer);

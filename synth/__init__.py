@@ -18,4 +18,10 @@ from .workloads import (  # noqa: F401
     bf16_round,
     group_scales,
     sweep_expanded,
+    TOKEN_F,
+    HEAD_DH,
+    N_TASKS,
+    make_token_inputs,
+    make_token_params,
+    make_head_params,
 )

@@ -19,6 +19,11 @@ Random-draw recipe (numpy ``default_rng(seed)``, always in this order):
      then GroupLN-2 the same way, then W_qkvu as four stacked d x d
      Xavier-uniform blocks, then W1 [d_ff, d] and W2 [d, d_ff] Xavier-uniform.
 
+Inputs of the steps around the stack, drawn on their own generator: per-domain
+token inputs (E_U [sum N_U, d], E_S, E_R, E_C at the TOKEN_F widths, N(0, 1)),
+then the token MLPs (per domain: W1 Xavier, b1, W2 Xavier, b2 N(0, var 0.01)),
+then the task heads (W1 Xavier, b1, w2 Xavier, b2).
+
 "N(0, x)" in the workload descriptions is read as variance x (the candidate
 features of the sweep are written N(0, 10^2), i.e. standard deviation 10).
 
@@ -235,3 +240,48 @@ def sweep_expanded(wl: dict) -> dict:
     out["norm"] = np.full(K, float(n_ctx + K), dtype=np.float32)
     out["kind"] = "sweep_expanded"
     return out
+
+
+# Input widths of the token MLPs (S, R, candidate): an S or R item is four
+# 64-wide field embeddings; a candidate is four item fields and four cross
+# fields. The pages give no widths; these are the assumed sizes.
+TOKEN_F = (256, 256, 512)
+# Hidden width of each task head and the number of tasks (CTR, CTCVR).
+HEAD_DH = 256
+N_TASKS = 2
+
+
+def make_token_inputs(lens: np.ndarray, d: int, rng: np.random.Generator,
+                      f: tuple = TOKEN_F) -> list:
+    """Per-domain inputs [E_U, E_S, E_R, E_C] (float32, bf16-representable):
+    E_U [sum N_U, d] and E_g [sum N_g, F_g], N(0, 1), each domain's tokens user
+    by user."""
+    lens = np.asarray(lens, np.int64).reshape(-1, 4)
+    widths = (d,) + tuple(f)
+    return [bf16_round(rng.standard_normal((int(lens[:, g].sum()), widths[g]), dtype=np.float32))
+            for g in range(4)]
+
+
+def make_token_params(d: int, rng: np.random.Generator, f: tuple = TOKEN_F) -> dict:
+    """Token MLP weights per domain s, r, c: W1 [d, F_g] and W2 [d, d]
+    Xavier-uniform (bf16-representable), biases N(0, var 0.01)."""
+    p = {}
+    for g, fin in zip(("s", "r", "c"), f):
+        p["w1_" + g] = bf16_round(_xavier(rng, d, fin))
+        p["b1_" + g] = (0.1 * rng.standard_normal(d, dtype=np.float32)).astype(np.float32)
+        p["w2_" + g] = bf16_round(_xavier(rng, d, d))
+        p["b2_" + g] = (0.1 * rng.standard_normal(d, dtype=np.float32)).astype(np.float32)
+    return p
+
+
+def make_head_params(d: int, rng: np.random.Generator, d_h: int = HEAD_DH,
+                     n_tasks: int = N_TASKS) -> dict:
+    """Task heads: W1 [n_tasks, d_h, d] Xavier-uniform (bf16-representable),
+    b1 N(0, var 0.01), w2 [n_tasks, d_h] Xavier-uniform (fan_out 1), b2
+    N(0, var 0.01)."""
+    w1 = np.stack([bf16_round(_xavier(rng, d_h, d)) for _ in range(n_tasks)])
+    b1 = (0.1 * rng.standard_normal((n_tasks, d_h), dtype=np.float32)).astype(np.float32)
+    w2 = np.stack([_xavier(rng, 1, d_h)[0] for _ in range(n_tasks)])
+    b2 = (0.1 * rng.standard_normal(n_tasks, dtype=np.float32)).astype(np.float32)
+    return dict(w1=w1, b1=b1, w2=w2, b2=b2)
+

@@ -35,7 +35,9 @@ def test_struct_layouts_match_header(tmp_path):
     if cc is None:
         pytest.skip("no C compiler")
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "mtgr.h"', 'int main(void) {']
-    for cname, cls in (("mtgr_batch", _lib.MtgrBatch), ("mtgr_block_params", _lib.MtgrBlockParams)):
+    structs = (("mtgr_batch", _lib.MtgrBatch), ("mtgr_block_params", _lib.MtgrBlockParams),
+               ("mtgr_token_mlp", _lib.MtgrTokenMlp), ("mtgr_head_params", _lib.MtgrHeadParams))
+    for cname, cls in structs:
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
         for f, _ in cls._fields_:
             lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
@@ -48,7 +50,7 @@ def test_struct_layouts_match_header(tmp_path):
     subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True,
                                                   check=True).stdout.splitlines())
-    for cname, cls in (("mtgr_batch", _lib.MtgrBatch), ("mtgr_block_params", _lib.MtgrBlockParams)):
+    for cname, cls in structs:
         assert int(got[cname]) == ctypes.sizeof(cls), cname
         for f, _ in cls._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(cls, f).offset, f"{cname}.{f}"
@@ -82,6 +84,8 @@ def test_host_validation_without_device(lib):
     assert lib.mtgr_stack_fwd(None, 0, None, None, None, None, 0, None) == E
     assert lib.mtgr_gemm(-1, 2, 64, 1, None, None, None, 0, None, 0, 0, None, None, None) == E
     assert lib.mtgr_restrict_work(None, None, None) == E
+    assert lib.mtgr_tokenize(None, 512, None, None, None, None, None, 0, None) == E
+    assert lib.mtgr_candidate_heads(None, None, 0, None, None, None, 0, None) == E
     assert lib.mtgr_stack_fwd_rows(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
 
 
@@ -132,3 +136,22 @@ def test_capacities_host_logic():
     # R groups: user 0 cols [36, 44) -> 1 group; user 1 [316, 366) -> groups 4, 5;
     # user 3 [60, 70) -> groups 0, 1
     assert rt == 1 * 9 + 2 * 51 + 0 + 2 * 11
+
+
+def test_token_and_head_workspace_sizes(lib):
+    # tokenize: per-domain user offsets 4 (B + 1) int32, the row map T int32,
+    # the hidden rows of the largest of S, R, C (d bf16 each)
+    up = lambda n: -(-n // 256) * 256  # noqa: E731
+    n_rows = [48, 1000, 130, 300]
+    B, d = 2, 512
+    want = up(4 * (B + 1) * 4) + up(sum(n_rows) * 4) + up(1000 * d * 2)
+    assert _lib.mtgr_tokenize_workspace_bytes(B, d, n_rows) == want
+    assert _lib.mtgr_tokenize_workspace_bytes(B, 100, n_rows) == 0          # d % 64
+    assert _lib.mtgr_tokenize_workspace_bytes(B, d, [1, -1, 0, 0]) == 0    # negative rows
+    # heads: offsets, the candidate map, gathered rows (d bf16), hidden rows
+    fake = 0x100000
+    p = _lib.MtgrHeadParams(d=512, d_h=256, n_tasks=2, reserved=0, w1=fake, b1=None, w2=fake, b2=None)
+    want = up(4 * (B + 1) * 4) + up(300 * 4) + up(300 * 512 * 2) + up(300 * 512 * 2)
+    assert _lib.mtgr_heads_workspace_bytes(B, 300, p) == want
+    p.d_h = 100  # % 32
+    assert _lib.mtgr_heads_workspace_bytes(B, 300, p) == 0
