@@ -31,6 +31,36 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
     v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
   }
 }
+// 8 consecutive elements as loaded (fp32: two float4; bf16: one uint4), so
+// that a lane's share of a row costs as few registers as its bytes
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void unpack(float (&v)[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 a;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { a = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void unpack(float (&v)[8]) const {
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __uint_as_float(w[k] << 16);
+      v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  }
+};
+
 __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
   reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
   reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -51,58 +81,82 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// VPL = 8-element vectors per lane (ceil(d / 256)); the row stays in registers.
-template <typename Tin, typename Tout, int VPL>
-__global__ void __launch_bounds__(256) gln_reg_kernel(int32_t T, int32_t d, const Tin* __restrict__ x,
+// VPL = 8-element vectors per lane (ceil(d / 256)); TPW tokens per warp, all
+// of their loads issued before any reduction so that each lane keeps about
+// 128 bytes of the input in flight; the rows stay in registers.
+template <typename Tin, typename Tout, int VPL, int TPW>
+__global__ void __launch_bounds__(256, 4) gln_reg_kernel(int32_t T, int32_t d, const Tin* __restrict__ x,
                                                       const int8_t* __restrict__ gid, int32_t G,
                                                       const float* __restrict__ gamma,
                                                       const float* __restrict__ beta, float eps,
                                                       Tout* __restrict__ y) {
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t t0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * TPW;
   const int lane = threadIdx.x & 31;
-  if (t >= T) return;
+  if (t0 >= T) return;
   const int nv = d >> 3;
-  const Tin* xr = x + t * d;
-  float v[VPL][8];
-  float s = 0.f;
+  Raw8<Tin> raw[TPW][VPL];
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    const int vi = lane + 32 * k;
-    if (vi < nv) {
-      load8(xr + 8 * vi, v[k]);
+  for (int j = 0; j < TPW; ++j) {
+    const int64_t t = t0 + j;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[k][e];
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = lane + 32 * k;
+      if (t < T && vi < nv) raw[j][k].load(x + t * d + 8 * vi);
     }
   }
-  const float mean = warp_sum(s) / (float)d;
-  float q = 0.f;
+  float mean[TPW], rstd[TPW];
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    if (lane + 32 * k < nv) {
+  for (int j = 0; j < TPW; ++j) {
+    float s = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float c = v[k][e] - mean;
-        q += c * c;
+    for (int k = 0; k < VPL; ++k) {
+      if (t0 + j < T && lane + 32 * k < nv) {
+        float v[8];
+        raw[j][k].unpack(v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += v[e];
       }
     }
+    mean[j] = warp_sum(s) / (float)d;
   }
-  const float var = warp_sum(q) / (float)d;
-  const float rstd = 1.0f / sqrtf(var + eps);
-  int g = gid[t];
-  g = g < 0 ? 0 : (g >= G ? G - 1 : g);
-  const float* ga = gamma + (int64_t)g * d;
-  const float* be = beta + (int64_t)g * d;
-  Tout* yr = y + t * d;
 #pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    const int vi = lane + 32 * k;
-    if (vi < nv) {
-      float gm[8], bt[8], o[8];
-      load8(ga + 8 * vi, gm);
-      load8(be + 8 * vi, bt);
+  for (int j = 0; j < TPW; ++j) {
+    float q = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (v[k][e] - mean) * rstd * gm[e] + bt[e];
-      store8(yr + 8 * vi, o);
+    for (int k = 0; k < VPL; ++k) {
+      if (t0 + j < T && lane + 32 * k < nv) {
+        float v[8];
+        raw[j][k].unpack(v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float c = v[e] - mean[j];
+          q += c * c;
+        }
+      }
+    }
+    rstd[j] = 1.0f / sqrtf(warp_sum(q) / (float)d + eps);
+  }
+#pragma unroll
+  for (int j = 0; j < TPW; ++j) {
+    const int64_t t = t0 + j;
+    if (t >= T) break;
+    int g = gid[t];
+    g = g < 0 ? 0 : (g >= G ? G - 1 : g);
+    const float* ga = gamma + (int64_t)g * d;
+    const float* be = beta + (int64_t)g * d;
+    Tout* yr = y + t * d;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = lane + 32 * k;
+      if (vi < nv) {
+        float v[8], gm[8], bt[8], o[8];
+        raw[j][k].unpack(v);
+        load8(ga + 8 * vi, gm);
+        load8(be + 8 * vi, bt);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = (v[e] - mean[j]) * rstd[j] * gm[e] + bt[e];
+        store8(yr + 8 * vi, o);
+      }
     }
   }
 }
@@ -158,16 +212,18 @@ __global__ void __launch_bounds__(256) gln_loop_kernel(int32_t T, int32_t d, con
 template <typename Tin, typename Tout>
 int launch_gln_t(int32_t T, int32_t d, const void* x, const int8_t* gid, int32_t G,
                  const float* gamma, const float* beta, float eps, void* y, cudaStream_t s) {
-  const unsigned grid = (unsigned)((T + 7) / 8);
   const Tin* xi = static_cast<const Tin*>(x);
   Tout* yo = static_cast<Tout*>(y);
   const int vpl = (d + 255) / 256;
+  // tokens per warp: about 128 bytes of input per lane in flight
+  constexpr int B1 = 128 / (8 * (int)sizeof(Tin));
+  auto grid = [T](int tpw) { return (unsigned)((T + 8 * tpw - 1) / (8 * tpw)); };
   switch (vpl) {
-    case 1: gln_reg_kernel<Tin, Tout, 1><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
-    case 2: gln_reg_kernel<Tin, Tout, 2><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
-    case 3: gln_reg_kernel<Tin, Tout, 3><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
-    case 4: gln_reg_kernel<Tin, Tout, 4><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
-    default: gln_loop_kernel<Tin, Tout><<<grid, 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 1: gln_reg_kernel<Tin, Tout, 1, 4><<<grid(4), 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 2: gln_reg_kernel<Tin, Tout, 2, B1 / 2><<<grid(B1 / 2), 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 3: gln_reg_kernel<Tin, Tout, 3, 1><<<grid(1), 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    case 4: gln_reg_kernel<Tin, Tout, 4, 1><<<grid(1), 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
+    default: gln_loop_kernel<Tin, Tout><<<grid(1), 256, 0, s>>>(T, d, xi, gid, G, gamma, beta, eps, yo); break;
   }
   return launch_status();
 }
