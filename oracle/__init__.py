@@ -27,6 +27,9 @@ from .mtgr import (  # noqa: F401
     pack_offsets,
     user_mask,
     group_layernorm,
+    group_layernorm_pooled,
+    VARIANT_POOLED_GLN,
+    VARIANT_SILU_QKVU,
     hstu_attention,
     hstu_block,
     hstu_stack,

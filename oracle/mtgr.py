@@ -116,6 +116,38 @@ def group_layernorm(x: np.ndarray, group_id: np.ndarray, gamma: np.ndarray,
     return xhat * np.asarray(gamma, np.float64)[g] + np.asarray(beta, np.float64)[g]
 
 
+# Block variants the pages leave open (bit flags, combinable):
+#   VARIANT_POOLED_GLN: GroupLN statistics pooled over all tokens and features
+#     of one group of one user, the reading of the practice article's 3.1 GLN
+#     pseudocode (group_mean = mean(group_hidden_states), group_std likewise);
+#   VARIANT_SILU_QKVU: Q, K, V, U = silu(X~ W_qkvu^T + b), HSTU's pointwise
+#     SiLU on the projections, one reading of the blog posts' "HSTU-style SiLU
+#     attention and gating" (it also puts SiLU on U before the gate).
+VARIANT_POOLED_GLN = 1
+VARIANT_SILU_QKVU = 2
+
+
+def group_layernorm_pooled(x: np.ndarray, lens: np.ndarray, gamma: np.ndarray,
+                           beta: np.ndarray, eps: float = EPS) -> np.ndarray:
+    """GroupLN with pooled statistics: for every user b and group g, mu and
+    var are the mean and the biased variance of all N_{b,g} x d values of that
+    group's tokens; y = (x - mu) / sqrt(var + eps) * gamma_g + beta_g."""
+    x = np.asarray(x, dtype=np.float64)
+    seg_off, _, _ = pack_offsets(lens)
+    y = np.zeros_like(x)
+    for b in range(np.asarray(lens).reshape(-1, 4).shape[0]):
+        for g in range(4):
+            s, e = int(seg_off[4 * b + g]), int(seg_off[4 * b + g + 1])
+            if e == s:
+                continue
+            blk = x[s:e]
+            mu = blk.mean()
+            var = ((blk - mu) ** 2).mean()
+            y[s:e] = (blk - mu) / np.sqrt(var + eps) * np.asarray(gamma, np.float64)[g] \
+                + np.asarray(beta, np.float64)[g]
+    return y
+
+
 def hstu_attention(qkvu: np.ndarray, lens: np.ndarray, ts: np.ndarray, H: int,
                    norm: np.ndarray | None = None) -> np.ndarray:
     """G = (silu(Q K^T) * M / N) V, gated by U, per user and head.
@@ -149,22 +181,31 @@ def hstu_attention(qkvu: np.ndarray, lens: np.ndarray, ts: np.ndarray, H: int,
 
 
 def hstu_block(x: np.ndarray, lens: np.ndarray, ts: np.ndarray, p: dict, H: int,
-               norm: np.ndarray | None = None, eps: float = EPS) -> np.ndarray:
+               norm: np.ndarray | None = None, eps: float = EPS, variant: int = 0) -> np.ndarray:
     """One HSTU block of MTGR (summary page, Method):
 
       X~ = GroupLN_1(X);  Q,K,V,U = X~ W_qkvu^T
       G  = (silu(Q K^T) M / N) V (.) U
       X  <- MLP(GroupLN_2(G)) + X,  MLP = Linear -> SiLU -> Linear
     Optional biases ``b_qkvu``, ``b1``, ``b2`` are added when present in ``p``.
+    ``variant`` selects the VARIANT_* readings above (0: the block as written).
     """
     x = np.asarray(x, dtype=np.float64)
     _, _, gid = pack_offsets(lens)
-    xt = group_layernorm(x, gid, p["gln1_gamma"], p["gln1_beta"], eps)
+
+    def gln(z, gamma, beta):
+        if variant & VARIANT_POOLED_GLN:
+            return group_layernorm_pooled(z, lens, gamma, beta, eps)
+        return group_layernorm(z, gid, gamma, beta, eps)
+
+    xt = gln(x, p["gln1_gamma"], p["gln1_beta"])
     qkvu = xt @ np.asarray(p["w_qkvu"], np.float64).T
     if p.get("b_qkvu") is not None:
         qkvu = qkvu + np.asarray(p["b_qkvu"], np.float64)
+    if variant & VARIANT_SILU_QKVU:
+        qkvu = silu(qkvu)
     g = hstu_attention(qkvu, lens, ts, H, norm)
-    gt = group_layernorm(g, gid, p["gln2_gamma"], p["gln2_beta"], eps)
+    gt = gln(g, p["gln2_gamma"], p["gln2_beta"])
     h = gt @ np.asarray(p["w1"], np.float64).T
     if p.get("b1") is not None:
         h = h + np.asarray(p["b1"], np.float64)
@@ -176,11 +217,11 @@ def hstu_block(x: np.ndarray, lens: np.ndarray, ts: np.ndarray, p: dict, H: int,
 
 
 def hstu_stack(x: np.ndarray, lens: np.ndarray, ts: np.ndarray, layers: list, H: int,
-               norm: np.ndarray | None = None, eps: float = EPS) -> np.ndarray:
+               norm: np.ndarray | None = None, eps: float = EPS, variant: int = 0) -> np.ndarray:
     """L stacked HSTU blocks (summary page, Method: "L stacked HSTU blocks")."""
     y = np.asarray(x, dtype=np.float64)
     for p in layers:
-        y = hstu_block(y, lens, ts, p, H, norm, eps)
+        y = hstu_block(y, lens, ts, p, H, norm, eps, variant)
     return y
 
 

@@ -1,0 +1,150 @@
+"""Pins of the oracle's block variants: GroupLN with statistics pooled over
+a user's group (the practice article's 3.1 GLN pseudocode) and SiLU on the
+Q|K|V|U projections (HSTU's pointwise SiLU, one reading of the blog posts'
+"HSTU-style SiLU attention and gating"). Checked against PyTorch's
+layer_norm over whole segments and closed forms in which the attention
+reduces to a masked sum."""
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synth
+
+T64 = torch.float64
+
+
+def _t(a):
+    return torch.as_tensor(np.asarray(a, np.float64), dtype=T64)
+
+
+def _pooled_torch(x, lens, gamma, beta, eps):
+    """layer_norm over each (user, group) segment as one [n, d] block."""
+    seg_off, _, _ = oracle.pack_offsets(lens)
+    y = torch.zeros(x.shape, dtype=T64)
+    xt = _t(x)
+    for b in range(lens.shape[0]):
+        for g in range(4):
+            s, e = int(seg_off[4 * b + g]), int(seg_off[4 * b + g + 1])
+            if e > s:
+                y[s:e] = F.layer_norm(xt[s:e], (e - s, x.shape[1]), eps=eps) * _t(gamma[g]) + _t(beta[g])
+    return y.numpy()
+
+
+def _case(seed, d=16):
+    rng = np.random.default_rng(seed)
+    lens = np.array([[2, 6, 4, 5], [3, 4, 0, 3], [1, 0, 2, 1]], np.int64)
+    x = synth.make_tokens(lens, d, rng).astype(np.float64)
+    gamma = 1.0 + 0.3 * rng.standard_normal((4, d))
+    beta = 0.3 * rng.standard_normal((4, d))
+    return rng, lens, x, gamma, beta
+
+
+def test_pooled_gln_matches_torch_layer_norm_over_segments():
+    _, lens, x, gamma, beta = _case(0)
+    y = oracle.group_layernorm_pooled(x, lens, gamma, beta, 1e-5)
+    np.testing.assert_allclose(y, _pooled_torch(x, lens, gamma, beta, 1e-5), rtol=1e-12, atol=1e-12)
+
+
+def test_pooled_gln_one_token_per_group_is_per_token_gln():
+    rng = np.random.default_rng(1)
+    lens = np.array([[1, 1, 1, 1], [1, 1, 0, 1]], np.int64)
+    d = 8
+    x = rng.standard_normal((int(lens.sum()), d)) * 3 + 1
+    gamma, beta = rng.standard_normal((4, d)), rng.standard_normal((4, d))
+    _, _, gid = oracle.pack_offsets(lens)
+    np.testing.assert_allclose(oracle.group_layernorm_pooled(x, lens, gamma, beta),
+                               oracle.group_layernorm(x, gid, gamma, beta), rtol=1e-12, atol=1e-12)
+
+
+def test_pooled_gln_segment_scale_invariance():
+    # with eps = 0, scaling and shifting one segment leaves the output unchanged
+    _, lens, x, gamma, beta = _case(2)
+    seg_off, _, _ = oracle.pack_offsets(lens)
+    y = oracle.group_layernorm_pooled(x, lens, gamma, beta, 0.0)
+    x2 = x.copy()
+    s, e = int(seg_off[1]), int(seg_off[2])  # user 0's S tokens
+    x2[s:e] = 7.5 * x2[s:e] - 3.0
+    y2 = oracle.group_layernorm_pooled(x2, lens, gamma, beta, 0.0)
+    np.testing.assert_allclose(y2, y, rtol=1e-10, atol=1e-10)
+    # a per-token GLN would not see the other tokens of the segment; the
+    # pooled one does: changing one token moves the others
+    x3 = x.copy()
+    x3[s] += 10.0
+    y3 = oracle.group_layernorm_pooled(x3, lens, gamma, beta, 0.0)
+    assert not np.allclose(y3[s + 1], y[s + 1])
+
+
+def _mlp(z, p):
+    h = F.silu(F.linear(_t(z), _t(p["w1"])))
+    return F.linear(h, _t(p["w2"])).numpy()
+
+
+def _ln_tok(z, gid, gamma, beta, eps=1e-5):
+    return (F.layer_norm(_t(z), (z.shape[1],), eps=eps) * _t(gamma)[gid] + _t(beta)[gid]).numpy()
+
+
+def test_silu_qkvu_closed_form():
+    # W_qkvu = 0, b_qkvu = c: every projection is silu(c). Per head h the
+    # score is s_h = silu(c_q) . silu(c_k) for every pair, so
+    # G_i = silu(s_h) * rowsum(M_i) / N_b * silu(c_v) (.) silu(c_u)
+    rng, lens, x, _, _ = _case(3)
+    d, H = 16, 2
+    dh = d // H
+    p = synth.make_block_params(d, 40, rng, dtype="f32")
+    p = {k: np.asarray(v, np.float64) for k, v in p.items()}
+    p["w_qkvu"] = np.zeros((4 * d, d))
+    c = 0.7 * rng.standard_normal(4 * d)
+    p["b_qkvu"] = c
+    ts = synth.make_timestamps(lens, rng)
+    y = oracle.hstu_block(x, lens, ts, p, H, variant=oracle.VARIANT_SILU_QKVU)
+    sc = F.silu(_t(c)).numpy()
+    q, k, v, u = sc[:d], sc[d:2 * d], sc[2 * d:3 * d], sc[3 * d:]
+    _, user_off, gid = oracle.pack_offsets(lens)
+    g = np.zeros_like(x)
+    for b in range(lens.shape[0]):
+        s_, e_ = int(user_off[b]), int(user_off[b + 1])
+        M = oracle.user_mask(*(int(t) for t in lens[b]), ts[s_:e_])
+        rs = M.sum(axis=1)
+        for h in range(H):
+            cs = slice(h * dh, (h + 1) * dh)
+            sh = float(q[cs] @ k[cs])
+            silu_s = float(F.silu(torch.tensor(sh, dtype=T64)))
+            g[s_:e_, cs] = silu_s * rs[:, None] / (e_ - s_) * (v[cs] * u[cs])[None, :]
+    ref = x + _mlp(_ln_tok(g, gid, p["gln2_gamma"], p["gln2_beta"]), p)
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-10)
+
+
+def test_pooled_block_constant_scores_reduce_to_masked_sum():
+    # W_q = W_k = 0 with biases c_q, c_k: the score of every pair of head h
+    # is s_h = c_q . c_k, so the attention is silu(s_h)/N_b times M @ V.
+    # Both GroupLNs pooled: checked against layer_norm over whole segments.
+    rng, lens, x, _, _ = _case(4)
+    d, H = 16, 2
+    dh = d // H
+    p = synth.make_block_params(d, 40, rng, dtype="f32")
+    p = {k: np.asarray(v, np.float64) for k, v in p.items()}
+    p["w_qkvu"] = p["w_qkvu"].copy()
+    p["w_qkvu"][:2 * d] = 0.0
+    c = np.zeros(4 * d)
+    c[:2 * d] = 0.5 * rng.standard_normal(2 * d)
+    p["b_qkvu"] = c
+    ts = synth.make_timestamps(lens, rng)
+    y = oracle.hstu_block(x, lens, ts, p, H, variant=oracle.VARIANT_POOLED_GLN)
+    xt = _pooled_torch(x, lens, p["gln1_gamma"], p["gln1_beta"], 1e-5)
+    V = F.linear(_t(xt), _t(p["w_qkvu"][2 * d:3 * d])).numpy()
+    U = F.linear(_t(xt), _t(p["w_qkvu"][3 * d:])).numpy()
+    _, user_off, _ = oracle.pack_offsets(lens)
+    g = np.zeros_like(x)
+    for b in range(lens.shape[0]):
+        s_, e_ = int(user_off[b]), int(user_off[b + 1])
+        M = oracle.user_mask(*(int(t) for t in lens[b]), ts[s_:e_]).astype(np.float64)
+        for h in range(H):
+            cs = slice(h * dh, (h + 1) * dh)
+            sh = float(c[:d][cs] @ c[d:2 * d][cs])
+            silu_s = float(F.silu(torch.tensor(sh, dtype=T64)))
+            g[s_:e_, cs] = silu_s / (e_ - s_) * (M @ V[s_:e_, cs]) * U[s_:e_, cs]
+    gt = _pooled_torch(g, lens, p["gln2_gamma"], p["gln2_beta"], 1e-5)
+    ref = x + _mlp(gt, p)
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-10)
