@@ -13,6 +13,8 @@ from ._lib import (  # noqa: F401
     MTGR_EPI_SILU,
     MTGR_F16,
     MTGR_F32,
+    MTGR_VARIANT_POOLED_GLN,
+    MTGR_VARIANT_SILU_QKVU,
     MTGRError,
     load,
     mtgr_block_workspace_bytes,
@@ -21,6 +23,7 @@ from ._lib import (  # noqa: F401
     mtgr_heads_workspace_bytes,
     mtgr_gemm,
     mtgr_group_layernorm,
+    mtgr_group_layernorm_pooled,
     mtgr_hstu_attention_fwd,
     mtgr_hstu_block_fwd,
     mtgr_mask_meta_workspace_bytes,
@@ -45,6 +48,7 @@ from .api import (  # noqa: F401
     PackedBatch,
     capacities,
     gemm,
+    group_layernorm_pooled,
     group_layernorm,
     hstu_attention,
     hstu_block_forward,

@@ -19,6 +19,8 @@ MTGR_OK = 0
 MTGR_ERR_INVALID_ARG = 1
 MTGR_ERR_CUDA = 2
 MTGR_ERR_UNSUPPORTED = 3
+MTGR_VARIANT_POOLED_GLN = 1
+MTGR_VARIANT_SILU_QKVU = 2
 MTGR_ERR_CAPACITY = 4
 MTGR_ERR_TIMEOUT = 5
 MTGR_ERR_DEVICE_VALIDATION = 6
@@ -60,7 +62,7 @@ WORK_ITEM_BYTES = 64  # sizeof(mtgr_work_item)
 
 class MtgrBlockParams(ctypes.Structure):
     _fields_ = [("d", c_i32), ("H", c_i32), ("d_ff", c_i32), ("dtype", c_i32), ("eps", c_float),
-                ("reserved", c_i32), ("gln1_gamma", c_vp), ("gln1_beta", c_vp),
+                ("variant", c_i32), ("gln1_gamma", c_vp), ("gln1_beta", c_vp),
                 ("gln2_gamma", c_vp), ("gln2_beta", c_vp), ("w_qkvu", c_vp), ("w1", c_vp),
                 ("w2", c_vp), ("b_qkvu", c_vp), ("b1", c_vp), ("b2", c_vp)]
 
@@ -88,6 +90,8 @@ _SIGNATURES = {
                                                    c_vp, c_vp, c_vp, c_vp]),
     "mtgr_group_layernorm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp,
                                             c_float, c_i32, c_vp, c_vp]),
+    "mtgr_group_layernorm_pooled": (ctypes.c_int, [c_i32, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp,
+                                                   c_float, c_i32, c_vp, c_vp]),
     "mtgr_hstu_attention_fwd": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_i32, c_i32, c_i32,
                                                c_vp, c_i32, c_vp, c_vp]),
     "mtgr_block_workspace_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams)]),
@@ -208,6 +212,12 @@ def mtgr_group_layernorm(T, d, d_x, d_group_id, G, d_gamma, d_beta, eps, d_y, st
     _check("mtgr_group_layernorm", load().mtgr_group_layernorm(
         T, d, dtype_code(d_x.dtype), _ptr(d_x), _ptr(d_group_id), G, _ptr(d_gamma), _ptr(d_beta),
         float(eps), dtype_code(d_y.dtype), _ptr(d_y), _stream(stream)))
+
+
+def mtgr_group_layernorm_pooled(B, d_seg_off, d, d_x, d_gamma, d_beta, eps, d_y, stream=None):
+    _check("mtgr_group_layernorm_pooled", load().mtgr_group_layernorm_pooled(
+        B, _ptr(d_seg_off), d, dtype_code(d_x.dtype), _ptr(d_x), _ptr(d_gamma), _ptr(d_beta), eps,
+        dtype_code(d_y.dtype), _ptr(d_y), _stream(stream)))
 
 
 def mtgr_hstu_attention_fwd(batch: MtgrBatch, d, H, d_qkvu, d_g, stream=None):

@@ -127,9 +127,12 @@ class BlockWeights:
 
     ``dtype`` "bf16" keeps W_qkvu, W1, W2 in bf16 (tensor-core path); "f32"
     keeps everything in fp32 (CUDA-core path). GroupLN parameters are fp32.
+    ``variant``: 0, or MTGR_VARIANT_* flags (bf16 only): pooled GroupLN
+    statistics, SiLU on the Q|K|V|U projections.
     """
 
-    def __init__(self, p: dict, H: int, dtype: str = "bf16", device="cuda", eps: float = EPS):
+    def __init__(self, p: dict, H: int, dtype: str = "bf16", device="cuda", eps: float = EPS,
+                 variant: int = 0):
         dev = torch.device(device)
         wdt = torch.bfloat16 if dtype == "bf16" else torch.float32
 
@@ -148,7 +151,7 @@ class BlockWeights:
         ptr = {k: (None if v is None else v.data_ptr()) for k, v in self.t.items()}
         self.c = MtgrBlockParams(d=d, H=H, d_ff=d_ff,
                                  dtype=MTGR_BF16 if dtype == "bf16" else MTGR_F32, eps=eps,
-                                 reserved=0, **ptr)
+                                 variant=variant, **ptr)
         self.d, self.H, self.d_ff, self.dtype = d, H, d_ff, dtype
 
 
@@ -181,6 +184,15 @@ def hstu_stack_forward(layers, batch: PackedBatch, x: torch.Tensor, out=None, ws
         ws = stack_workspace(layers, batch)
     _lib.mtgr_stack_fwd([l.c for l in layers], batch.c, x, out, ws, stream)
     return out
+
+
+def group_layernorm_pooled(batch: PackedBatch, x: torch.Tensor, gamma: torch.Tensor,
+                           beta: torch.Tensor, eps: float = EPS, out_dtype=None, stream=None):
+    """GroupLN with one mean and variance per (user, group) segment."""
+    y = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _lib.mtgr_group_layernorm_pooled(batch.B, batch.seg_off, x.shape[1], x, gamma, beta, eps, y,
+                                     stream)
+    return y
 
 
 def hstu_attention(batch: PackedBatch, qkvu: torch.Tensor, d: int, H: int,

@@ -25,6 +25,9 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
                    cudaStream_t s);
 int launch_restrict_work(const int32_t* q_first, int32_t q_cap, mtgr_work_item* work, int64_t* counts,
                          cudaStream_t s);
+int launch_gln_pooled(int32_t B, const int32_t* seg_off, int32_t d, int32_t x_dtype, const void* x,
+                      const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
+                      cudaStream_t s);
 int launch_gemm_tc_rowmap(int M, int N, int K, const void* a, const void* b, const float* bias,
                           const int32_t* row_map, float* out, int out_rows, int32_t* status,
                           cudaStream_t s);
@@ -74,6 +77,8 @@ int params_check(const mtgr_block_params* p) {
   if (p->d <= 0 || p->H <= 0 || p->d_ff <= 0 || p->d > kMaxD || p->d % p->H != 0)
     return MTGR_ERR_INVALID_ARG;
   if (!(p->eps >= 0.0f)) return MTGR_ERR_INVALID_ARG;
+  if (p->variant & ~(MTGR_VARIANT_POOLED_GLN | MTGR_VARIANT_SILU_QKVU)) return MTGR_ERR_INVALID_ARG;
+  if (p->variant != 0 && p->dtype != MTGR_BF16) return MTGR_ERR_UNSUPPORTED;
   if (p->gln1_gamma == nullptr || p->gln1_beta == nullptr || p->gln2_gamma == nullptr ||
       p->gln2_beta == nullptr || p->w_qkvu == nullptr || p->w1 == nullptr || p->w2 == nullptr)
     return MTGR_ERR_INVALID_ARG;
@@ -148,15 +153,23 @@ int block_fwd_rows(const mtgr_block_params* p, const mtgr_batch* bt, int32_t row
   PartWs w = part_ws_layout(T, row0, p, qkvu_ext == nullptr, ws);
   uint16_t* qkvu = static_cast<uint16_t*>(qkvu_ext != nullptr ? qkvu_ext : w.qkvu);
   int rc;
+  // pooled GroupLN statistics span whole (user, group) segments: only with row0 == 0
+  const bool pooled = (p->variant & MTGR_VARIANT_POOLED_GLN) != 0;
+  if (pooled && row0 != 0) return MTGR_ERR_UNSUPPORTED;
   {
     TimedScope tsc(MTGR_TIMER_GLN, s, 1);
-    if ((rc = launch_gln(k, d, MTGR_F32, x_in, bt->group_id + row0, 4, p->gln1_gamma,
-                         p->gln1_beta, p->eps, MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
+    rc = pooled ? launch_gln_pooled(bt->B, bt->seg_off, d, MTGR_F32, x_in, p->gln1_gamma,
+                                    p->gln1_beta, p->eps, MTGR_BF16, w.xt, s)
+                : launch_gln(k, d, MTGR_F32, x_in, bt->group_id + row0, 4, p->gln1_gamma,
+                             p->gln1_beta, p->eps, MTGR_BF16, w.xt, s);
+    if (rc != MTGR_OK) return rc;
   }
   {
-    // Q|K|V|U in f16 with the Q columns halved (silu's tanh form takes s/2)
+    // Q|K|V|U in f16 with the Q columns halved (silu's tanh form takes s/2);
+    // the SiLU variant applies silu before the halving
     TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
-    if ((rc = launch_gemm_tc(k, 4 * d, d, w.xt, p->w_qkvu, p->b_qkvu, MTGR_EPI_NONE, nullptr, d,
+    const int epi = (p->variant & MTGR_VARIANT_SILU_QKVU) ? MTGR_EPI_SILU : MTGR_EPI_NONE;
+    if ((rc = launch_gemm_tc(k, 4 * d, d, w.xt, p->w_qkvu, p->b_qkvu, epi, nullptr, d,
                              MTGR_F16, qkvu + (size_t)row0 * 4 * d, bt->status, s)) != MTGR_OK)
       return rc;
   }
@@ -167,9 +180,12 @@ int block_fwd_rows(const mtgr_block_params* p, const mtgr_batch* bt, int32_t row
   }
   {
     TimedScope tsc(MTGR_TIMER_GLN, s, 1);
-    if ((rc = launch_gln(k, d, MTGR_BF16, static_cast<uint16_t*>(w.g) + (size_t)row0 * d,
-                         bt->group_id + row0, 4, p->gln2_gamma, p->gln2_beta, p->eps, MTGR_BF16,
-                         w.xt, s)) != MTGR_OK) return rc;
+    rc = pooled ? launch_gln_pooled(bt->B, bt->seg_off, d, MTGR_BF16, w.g, p->gln2_gamma,
+                                    p->gln2_beta, p->eps, MTGR_BF16, w.xt, s)
+                : launch_gln(k, d, MTGR_BF16, static_cast<uint16_t*>(w.g) + (size_t)row0 * d,
+                             bt->group_id + row0, 4, p->gln2_gamma, p->gln2_beta, p->eps,
+                             MTGR_BF16, w.xt, s);
+    if (rc != MTGR_OK) return rc;
   }
   {
     TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
@@ -187,37 +203,9 @@ int block_fwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
   if (T == 0) return MTGR_OK;
   BlockWs w = block_ws_layout(T, p, ws);
   int rc;
-  if (p->dtype == MTGR_BF16) {
-    {
-      TimedScope tsc(MTGR_TIMER_GLN, s, 1);
-      if ((rc = launch_gln(T, d, MTGR_F32, x_in, bt->group_id, 4, p->gln1_gamma, p->gln1_beta,
-                           p->eps, MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
-    }
-    {
-      // Q|K|V|U in f16 with the Q columns halved (silu's tanh form takes s/2)
-      TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
-      if ((rc = launch_gemm_tc(T, 4 * d, d, w.xt, p->w_qkvu, p->b_qkvu, MTGR_EPI_NONE, nullptr, d,
-                               MTGR_F16, w.qkvu, bt->status, s)) != MTGR_OK) return rc;
-    }
-    {
-      TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
-      if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, w.qkvu, MTGR_BF16, w.g, s)) != MTGR_OK)
-        return rc;
-    }
-    {
-      TimedScope tsc(MTGR_TIMER_GLN, s, 1);
-      if ((rc = launch_gln(T, d, MTGR_BF16, w.g, bt->group_id, 4, p->gln2_gamma, p->gln2_beta,
-                           p->eps, MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
-    }
-    {
-      TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
-      if ((rc = launch_gemm_tc(T, dff, d, w.xt, p->w1, p->b1, MTGR_EPI_SILU, nullptr, 0, MTGR_BF16,
-                               w.h, bt->status, s)) != MTGR_OK) return rc;
-    }
-    TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
-    return launch_gemm_tc(T, d, dff, w.h, p->w2, p->b2, MTGR_EPI_RESID, x_in, 0, MTGR_F32, x_out,
-                          bt->status, s);
-  }
+  // bf16: the rows form over all rows, with the workspace laid out as
+  // block_ws_layout lays it out (GroupLN output, Q|K|V|U, G, MLP hidden)
+  if (p->dtype == MTGR_BF16) return block_fwd_rows(p, bt, 0, x_in, x_out, nullptr, ws, s);
   {
     TimedScope tsc(MTGR_TIMER_GLN, s, 1);
     if ((rc = launch_gln(T, d, MTGR_F32, x_in, bt->group_id, 4, p->gln1_gamma, p->gln1_beta, p->eps,
@@ -329,6 +317,21 @@ MTGR_API int mtgr_group_layernorm(int32_t T, int32_t d, int32_t x_dtype, const v
   TimedScope tsc(MTGR_TIMER_GLN, as_stream(stream), T > 0 ? 1 : 0);
   return launch_gln(T, d, x_dtype, d_x, d_group_id, G, d_gamma, d_beta, eps, y_dtype, d_y,
                     as_stream(stream));
+}
+
+MTGR_API int mtgr_group_layernorm_pooled(int32_t B, const int32_t* d_seg_off, int32_t d,
+                                         int32_t x_dtype, const void* d_x, const float* d_gamma,
+                                         const float* d_beta, float eps, int32_t y_dtype, void* d_y,
+                                         mtgr_stream_t stream) {
+  if (B < 0 || d <= 0 || d % 8 != 0 || d > kMaxD || !(eps >= 0.0f)) return MTGR_ERR_INVALID_ARG;
+  if (B > 0 && (d_seg_off == nullptr || d_x == nullptr || d_gamma == nullptr || d_beta == nullptr ||
+                d_y == nullptr))
+    return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x) || !aligned16(d_y) || !aligned16(d_gamma) || !aligned16(d_beta))
+    return MTGR_ERR_INVALID_ARG;
+  TimedScope tsc(MTGR_TIMER_GLN, as_stream(stream), B > 0 ? 1 : 0);
+  return launch_gln_pooled(B, d_seg_off, d, x_dtype, d_x, d_gamma, d_beta, eps, y_dtype, d_y,
+                           as_stream(stream));
 }
 
 MTGR_API int mtgr_hstu_attention_fwd(const mtgr_batch* batch, int32_t d, int32_t H,

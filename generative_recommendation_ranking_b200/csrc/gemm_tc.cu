@@ -63,7 +63,7 @@ __device__ __forceinline__ uint32_t stg_off(int r, int c) {
 // Epilogue math of 32 consecutive columns [col0, col0+32) of one row; the
 // result goes to row `r` of the staging block `stg` (holding the residual
 // block on entry for EPI_RESID).
-template <int EPI>
+template <int EPI, int OUT>
 __device__ __forceinline__ void epilogue_math(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
                                               float (&v)[32]) {
 #pragma unroll
@@ -75,11 +75,18 @@ __device__ __forceinline__ void epilogue_math(const GemmArgs& a, int col0, const
       v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
     }
   }
+  // the f16 SiLU form (SiLU on the Q|K|V|U projections) halves Q after the
+  // SiLU; the other forms never combine the two
+  constexpr bool kSiluFirst = EPI == MTGR_EPI_SILU && OUT == MTGR_F16;
+  if (kSiluFirst) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = silu_fast(v[c]);
+  }
   if (col0 < a.q_cols) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] *= 0.5f;
   }
-  if (EPI == MTGR_EPI_SILU) {
+  if (EPI == MTGR_EPI_SILU && !kSiluFirst) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] = silu_fast(v[c]);
   }
@@ -89,7 +96,7 @@ template <int EPI, int OUT>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
                                                uint8_t* stg, int r) {
   float v[32];
-  epilogue_math<EPI>(a, col0, acc, v);
+  epilogue_math<EPI, OUT>(a, col0, acc, v);
   if (OUT == MTGR_F32) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -360,6 +367,7 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_NONE, MTGR_F16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_NONE, MTGR_BF16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_NONE, MTGR_F32>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_SILU, MTGR_F16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_SILU, MTGR_BF16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, to, tr, args, s);

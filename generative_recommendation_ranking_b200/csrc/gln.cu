@@ -209,6 +209,95 @@ __global__ void __launch_bounds__(256) gln_loop_kernel(int32_t T, int32_t d, con
   }
 }
 
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Pooled statistics (the practice article's 3.1 GLN pseudocode read as one
+// mean and one standard deviation per group of a user): a block per (user,
+// group) segment of rows [seg_off[sg], seg_off[sg + 1]); the sum and the sum
+// of squares of all its values in fp64 (fp32 within each 8-value load), then
+// y = (x - mean) * rstd * gamma_g + beta_g over the segment.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(512) gln_pooled_kernel(int32_t nseg, int32_t d,
+                                                         const int32_t* __restrict__ seg_off,
+                                                         const Tin* __restrict__ x,
+                                                         const float* __restrict__ gamma,
+                                                         const float* __restrict__ beta, float eps,
+                                                         Tout* __restrict__ y) {
+  __shared__ double red[2][16];
+  __shared__ float stat[2];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int32_t sg = blockIdx.x; sg < nseg; sg += gridDim.x) {
+    const int32_t r0 = seg_off[sg], r1 = seg_off[sg + 1];
+    if (r1 <= r0) continue;  // the same for every thread of the block
+    const int g = sg & 3;
+    const int64_t n8 = (int64_t)(r1 - r0) * d / 8;
+    const Tin* xs = x + (int64_t)r0 * d;
+    double s = 0.0, q = 0.0;
+    for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
+      float v[8];
+      load8(xs + 8 * i, v);
+      float fs = 0.f, fq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        fs += v[e];
+        fq = fmaf(v[e], v[e], fq);
+      }
+      s += fs;
+      q += fq;
+    }
+    s = warp_sum_d(s);
+    q = warp_sum_d(q);
+    if (lane == 0) {
+      red[0][wid] = s;
+      red[1][wid] = q;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double S = 0.0, Q = 0.0;
+      for (int w = 0; w < nw; ++w) {
+        S += red[0][w];
+        Q += red[1][w];
+      }
+      const double cnt = (double)(r1 - r0) * d;
+      const double mean = S / cnt;
+      double var = Q / cnt - mean * mean;
+      var = var < 0.0 ? 0.0 : var;
+      stat[0] = (float)mean;
+      stat[1] = (float)(1.0 / sqrt(var + (double)eps));
+    }
+    __syncthreads();
+    const float mean = stat[0], rstd = stat[1];
+    const float* ga = gamma + (int64_t)g * d;
+    const float* be = beta + (int64_t)g * d;
+    Tout* ys = y + (int64_t)r0 * d;
+    for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
+      const int c = (int)((8 * i) % d);
+      float v[8], gm[8], bt[8], o[8];
+      load8(xs + 8 * i, v);
+      load8(ga + c, gm);
+      load8(be + c, bt);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (v[e] - mean) * rstd * gm[e] + bt[e];
+      store8(ys + 8 * i, o);
+    }
+    __syncthreads();  // red and stat are reused by the next segment
+  }
+}
+
+template <typename Tin, typename Tout>
+int launch_gln_pooled_t(int32_t nseg, int32_t d, const int32_t* seg_off, const void* x,
+                        const float* gamma, const float* beta, float eps, void* y, cudaStream_t s) {
+  const int cap = device_sm_count() * 4;
+  const int grid = nseg < cap ? nseg : cap;
+  gln_pooled_kernel<Tin, Tout><<<grid, 512, 0, s>>>(nseg, d, seg_off, static_cast<const Tin*>(x),
+                                                    gamma, beta, eps, static_cast<Tout*>(y));
+  return launch_status();
+}
+
 template <typename Tin, typename Tout>
 int launch_gln_t(int32_t T, int32_t d, const void* x, const int8_t* gid, int32_t G,
                  const float* gamma, const float* beta, float eps, void* y, cudaStream_t s) {
@@ -240,6 +329,22 @@ int launch_gln(int32_t T, int32_t d, int32_t x_dtype, const void* x, const int8_
     return launch_gln_t<float, __nv_bfloat16>(T, d, x, gid, G, gamma, beta, eps, y, s);
   if (x_dtype == MTGR_BF16 && y_dtype == MTGR_BF16)
     return launch_gln_t<__nv_bfloat16, __nv_bfloat16>(T, d, x, gid, G, gamma, beta, eps, y, s);
+  return MTGR_ERR_UNSUPPORTED;
+}
+
+// GroupLN with statistics pooled over each (user, group) segment of the
+// packed batch (B users, seg_off [4B + 1]; gamma, beta [4][d]).
+int launch_gln_pooled(int32_t B, const int32_t* seg_off, int32_t d, int32_t x_dtype, const void* x,
+                      const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
+                      cudaStream_t s) {
+  if (B == 0) return MTGR_OK;
+  const int32_t nseg = 4 * B;
+  if (x_dtype == MTGR_F32 && y_dtype == MTGR_F32)
+    return launch_gln_pooled_t<float, float>(nseg, d, seg_off, x, gamma, beta, eps, y, s);
+  if (x_dtype == MTGR_F32 && y_dtype == MTGR_BF16)
+    return launch_gln_pooled_t<float, __nv_bfloat16>(nseg, d, seg_off, x, gamma, beta, eps, y, s);
+  if (x_dtype == MTGR_BF16 && y_dtype == MTGR_BF16)
+    return launch_gln_pooled_t<__nv_bfloat16, __nv_bfloat16>(nseg, d, seg_off, x, gamma, beta, eps, y, s);
   return MTGR_ERR_UNSUPPORTED;
 }
 

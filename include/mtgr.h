@@ -209,6 +209,19 @@ MTGR_API int mtgr_group_layernorm(int32_t T, int32_t d, int32_t x_dtype, const v
                                   const float* d_beta, float eps, int32_t y_dtype, void* d_y,
                                   mtgr_stream_t stream);
 
+/*
+ * GroupLN with pooled statistics (MTGR_VARIANT_POOLED_GLN): for every user b
+ * and group g, one mean and one biased variance over all N_{b,g} x d values of
+ * rows [d_seg_off[4b+g], d_seg_off[4b+g+1]) (d_seg_off from
+ * mtgr_pack_offsets, [4B+1], device); y = (x - mean) / sqrt(var + eps) *
+ * gamma[g] + beta[g]. gamma, beta [4][d] float32; x, y [T][d] of x_dtype,
+ * y_dtype (F32 -> F32, F32 -> BF16, BF16 -> BF16); d % 8 == 0.
+ */
+MTGR_API int mtgr_group_layernorm_pooled(int32_t B, const int32_t* d_seg_off, int32_t d,
+                                         int32_t x_dtype, const void* d_x, const float* d_gamma,
+                                         const float* d_beta, float eps, int32_t y_dtype, void* d_y,
+                                         mtgr_stream_t stream);
+
 /* A packed batch plus its mask metadata (all device pointers). */
 typedef struct mtgr_batch {
   int32_t B;                  /* users */
@@ -250,6 +263,21 @@ MTGR_API int mtgr_hstu_attention_fwd(const mtgr_batch* batch, int32_t d, int32_t
                                      int32_t qkvu_dtype, const void* d_qkvu, int32_t out_dtype,
                                      void* d_g, mtgr_stream_t stream);
 
+/*
+ * Block variants, readings the pages leave open (flags of
+ * mtgr_block_params.variant, bf16 blocks only; 0 is the block as the
+ * summary page's Method writes it):
+ *   MTGR_VARIANT_POOLED_GLN: both GroupLNs take one mean and one variance
+ *     over all values of each (user, group) segment (the practice article's
+ *     3.1 GLN pseudocode, group_mean = mean(group_hidden_states)). Not with
+ *     mtgr_stack_fwd_rows on rows after 0 (MTGR_ERR_UNSUPPORTED).
+ *   MTGR_VARIANT_SILU_QKVU: Q, K, V, U = silu(X~ W_qkvu^T + b), HSTU's
+ *     pointwise SiLU on the projections (one reading of the blog posts'
+ *     "HSTU-style SiLU attention and gating"; it also gates with silu(U)).
+ */
+#define MTGR_VARIANT_POOLED_GLN 1
+#define MTGR_VARIANT_SILU_QKVU 2
+
 /* Parameters of one HSTU block (device pointers; PyTorch Linear [out][in] layout). */
 typedef struct mtgr_block_params {
   int32_t d;                  /* d_model */
@@ -257,7 +285,7 @@ typedef struct mtgr_block_params {
   int32_t d_ff;               /* MLP hidden width */
   int32_t dtype;              /* MTGR_BF16: bf16 weights, tensor cores; MTGR_F32: f32 SIMT */
   float eps;                  /* GroupLN epsilon */
-  int32_t reserved;
+  int32_t variant;            /* 0, or MTGR_VARIANT_* flags (bf16 only) */
   const float* gln1_gamma;    /* [4][d] */
   const float* gln1_beta;     /* [4][d] */
   const float* gln2_gamma;    /* [4][d] */
@@ -407,12 +435,12 @@ MTGR_API int mtgr_candidate_heads(const mtgr_head_params* p, const mtgr_batch* b
  * Dense GEMM with the block's epilogues, exposed for testing:
  *   out[m][n] = epi( sum_k a[m][k] * b[n][k] + bias[n] )
  *   epi = MTGR_EPI_NONE (out dtype MTGR_F16/MTGR_BF16/MTGR_F32),
- *         MTGR_EPI_SILU (out MTGR_BF16/MTGR_F32),
+ *         MTGR_EPI_SILU (out MTGR_F16/MTGR_BF16/MTGR_F32),
  *         MTGR_EPI_RESID (adds d_resid[m][n] float32; out MTGR_F32)
  *   ab_dtype MTGR_BF16: tcgen05 tensor cores (K % 64 == 0, N % 32 == 0);
  *   ab_dtype MTGR_F32: CUDA cores. a [M][K], b [N][K] row-major; bias may
- *   be NULL. q_cols > 0 multiplies output columns [0, q_cols) by 0.5 before
- *   the epilogue conversion (used to pre-halve Q for the attention).
+ *   be NULL. q_cols > 0 multiplies output columns [0, q_cols) by 0.5 after
+ *   the SiLU and before the conversion (used to pre-halve Q for the attention).
  */
 #define MTGR_EPI_NONE 0
 #define MTGR_EPI_SILU 1

@@ -84,6 +84,7 @@ def test_host_validation_without_device(lib):
     assert lib.mtgr_stack_fwd(None, 0, None, None, None, None, 0, None) == E
     assert lib.mtgr_gemm(-1, 2, 64, 1, None, None, None, 0, None, 0, 0, None, None, None) == E
     assert lib.mtgr_restrict_work(None, None, None) == E
+    assert lib.mtgr_group_layernorm_pooled(2, None, 64, 0, None, None, None, 1e-5, 0, None, None) == E
     assert lib.mtgr_tokenize(None, 512, None, None, None, None, None, 0, None) == E
     assert lib.mtgr_candidate_heads(None, None, 0, None, None, None, 0, None) == E
     assert lib.mtgr_stack_fwd_rows(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
@@ -91,7 +92,7 @@ def test_host_validation_without_device(lib):
 
 def _params(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16):
     fake = 0x100000  # 16-byte aligned stand-in addresses; never dereferenced
-    return _lib.MtgrBlockParams(d=d, H=H, d_ff=d_ff, dtype=dtype, eps=1e-5, reserved=0,
+    return _lib.MtgrBlockParams(d=d, H=H, d_ff=d_ff, dtype=dtype, eps=1e-5, variant=0,
                                 gln1_gamma=fake, gln1_beta=fake, gln2_gamma=fake, gln2_beta=fake,
                                 w_qkvu=fake, w1=fake, w2=fake, b_qkvu=None, b1=None, b2=None)
 
@@ -103,6 +104,14 @@ def test_workspace_sizes(lib):
     assert _lib.mtgr_block_workspace_bytes(T, p) == want
     assert _lib.mtgr_block_workspace_bytes(T, _params(H=4)) == 0        # dh = 128 unsupported
     assert _lib.mtgr_block_workspace_bytes(T, _params(d=100, H=2)) == 0  # d % 64 != 0
+    v = _params()
+    v.variant = _lib.MTGR_VARIANT_POOLED_GLN | _lib.MTGR_VARIANT_SILU_QKVU
+    assert _lib.mtgr_block_workspace_bytes(T, v) == want
+    v.variant = 4  # no such flag
+    assert _lib.mtgr_block_workspace_bytes(T, v) == 0
+    fv = _params(d=64, H=2, d_ff=256, dtype=_lib.MTGR_F32)
+    fv.variant = _lib.MTGR_VARIANT_SILU_QKVU  # variants are bf16 only
+    assert _lib.mtgr_block_workspace_bytes(T, fv) == 0
     f = _params(d=64, H=2, d_ff=256, dtype=_lib.MTGR_F32)
     assert _lib.mtgr_block_workspace_bytes(T, f) > 0
     two = _lib.mtgr_stack_workspace_bytes(T, [p, p])
