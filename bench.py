@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--serving", action="store_true",
+                    help="cached-context candidate scoring on the 512-user block workload: the "
+                         "candidate pass against the aggregated pass (one JSON line)")
     ap.add_argument("--pipeline", action="store_true",
                     help="time token MLPs -> block -> CTR/CTCVR heads on the 512-user block "
                          "workload, each part with its roofline (one JSON line)")
@@ -578,6 +581,72 @@ def run_sweep(args, local):
     print(json.dumps(line), flush=True)
 
 
+def run_serving(args, local):
+    """Serving with cached contexts on the 512-user block workload: the
+    contexts (U, S, R) of all users run once with every layer's Q|K|V|U kept;
+    each candidate request then recomputes the candidate rows only. Timed:
+    the aggregated pass (pack + metadata + block over every row), the context
+    pass, and the candidate pass (pack + metadata + the candidate rows)."""
+    import generative_recommendation_ranking_b200 as mt
+    from generative_recommendation_ranking_b200 import _lib
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    wl = synth.make_workload(2, seed=args.seed, B=args.users)
+    lens = wl["lens"]
+    wsp = Workspace(wl, dev, stream)
+    layers = wsp.layers
+    x = wsp.x
+    gid = torch.from_numpy(np.repeat(np.tile(np.arange(4), lens.shape[0]),
+                                     lens.reshape(-1).astype(np.int64)).astype(np.int64)).to(dev)
+    cand = gid == 3
+    x_cand = x[cand].contiguous()
+    cc = mt.BatchContextCache(layers, lens, wl["ts"], x, stream=stream)
+    cb = cc.batch
+    cws = cc._ws
+    batch = cc.candidate_batch(wl["ts"], stream)
+    ws = cc.workspace()
+    out = torch.empty(cc.k_total, wl["d"], dtype=torch.float32, device=dev)
+    c_layers = [l.c for l in layers]
+
+    def ctx_step():
+        cb.pack(stream)
+        cb.build_meta(stream)
+        _lib.mtgr_stack_fwd_rows(c_layers, cb.c, 0, cc.cache, cc.T, x, cc.out, cws, stream)
+
+    def cand_step():
+        batch.pack(stream)
+        batch.build_meta(stream)
+        _lib.mtgr_stack_fwd_candidates(c_layers, batch.c, cc.k_total, cc.cache, cc.T, x_cand, out, ws,
+                                       stream)
+
+    n = max(5, min(args.steps, 100))
+    res = {}
+    for name, fn in (("aggregated", wsp.step), ("context", ctx_step), ("candidates", cand_step)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        timer = _lib.Timer()
+        timer.attach()
+        ms = time_steps(fn, n, stream) / n
+        timer.detach()
+        batch.check()
+        per = timer.read()
+        res[name] = {"ms_per_step": ms,
+                     "kernels_ms": {c: round(t / n, 4) for c, (t, k) in per.items() if k}}
+    K = cc.k_total
+    line = {"metric": "cached-context candidate scoring: candidate pass vs aggregated pass",
+            "value": lens.shape[0] / (res["candidates"]["ms_per_step"] * 1e-3),
+            "unit": "user-samples/s", "ms_per_step": res["candidates"]["ms_per_step"],
+            "steps": n, "higher_is_better": True, "n_gpus": 1, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl["name"], "users": int(lens.shape[0]), "tokens": cc.T,
+                       "candidates": K, "l2": "inputs 0.9 GB > L2"},
+            "candidates_per_s": K / (res["candidates"]["ms_per_step"] * 1e-3),
+            "speedup_vs_aggregated": res["aggregated"]["ms_per_step"] / res["candidates"]["ms_per_step"],
+            "parts": res}
+    print(json.dumps(line), flush=True)
+
+
 def run_pipeline(args, local):
     """The ranking forward around the block on the 512-user block workload:
     the per-domain token MLPs build X, the HSTU block runs, the task heads
@@ -670,6 +739,9 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.serving:
+            if rank == 0:
+                run_serving(args, local)
         elif args.pipeline:
             if rank == 0:
                 run_pipeline(args, local)

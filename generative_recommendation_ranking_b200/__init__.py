@@ -30,6 +30,8 @@ from ._lib import (  # noqa: F401
     mtgr_pack_offsets,
     mtgr_restrict_work,
     mtgr_stack_fwd,
+    mtgr_stack_candidates_workspace_bytes,
+    mtgr_stack_fwd_candidates,
     mtgr_stack_fwd_rows,
     mtgr_stack_rows_workspace_bytes,
     mtgr_stack_workspace_bytes,
@@ -39,6 +41,7 @@ from ._lib import (  # noqa: F401
     status_string,
 )
 from .api import (  # noqa: F401
+    BatchContextCache,
     BlockWeights,
     CandidateHeads,
     ContextCache,

@@ -107,6 +107,11 @@ _SIGNATURES = {
     "mtgr_stack_fwd_rows": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams), c_i32,
                                            ctypes.POINTER(MtgrBatch), c_i32, c_vp, c_i32, c_vp, c_vp,
                                            c_vp, c_size, c_vp]),
+    "mtgr_stack_candidates_workspace_bytes": (c_size, [c_i32, c_i32, c_i32,
+                                                       ctypes.POINTER(MtgrBlockParams), c_i32]),
+    "mtgr_stack_fwd_candidates": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams), c_i32,
+                                                 ctypes.POINTER(MtgrBatch), c_i32, c_vp, c_i32, c_vp,
+                                                 c_vp, c_vp, c_size, c_vp]),
     "mtgr_tokenize_workspace_bytes": (c_size, [c_i32, c_i32, ctypes.POINTER(c_i32)]),
     "mtgr_tokenize": (ctypes.c_int, [ctypes.POINTER(MtgrBatch), c_i32, ctypes.POINTER(c_i32),
                                      ctypes.POINTER(c_vp), ctypes.POINTER(MtgrTokenMlp), c_vp, c_vp,
@@ -263,6 +268,19 @@ def mtgr_stack_fwd_rows(layers, batch: MtgrBatch, row0: int, d_cache, cache_rows
     arr = (MtgrBlockParams * len(layers))(*layers)
     _check("mtgr_stack_fwd_rows", load().mtgr_stack_fwd_rows(
         arr, len(layers), ctypes.byref(batch), row0, _ptr(d_cache), cache_rows, _ptr(d_x_in),
+        _ptr(d_x_out), _ptr(d_ws), d_ws.numel() * d_ws.element_size(), _stream(stream)))
+
+
+def mtgr_stack_candidates_workspace_bytes(B: int, T: int, k_total: int, layers) -> int:
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    return load().mtgr_stack_candidates_workspace_bytes(B, T, k_total, arr, len(layers))
+
+
+def mtgr_stack_fwd_candidates(layers, batch: MtgrBatch, k_total: int, d_cache, cache_rows: int,
+                              d_x_cand, d_x_out, d_ws, stream=None):
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    _check("mtgr_stack_fwd_candidates", load().mtgr_stack_fwd_candidates(
+        arr, len(layers), ctypes.byref(batch), k_total, _ptr(d_cache), cache_rows, _ptr(d_x_cand),
         _ptr(d_x_out), _ptr(d_ws), d_ws.numel() * d_ws.element_size(), _stream(stream)))
 
 

@@ -298,6 +298,63 @@ class ContextCache:
         return out
 
 
+class BatchContextCache:
+    """The contexts (U, S, R) of a whole batch of users run once through a
+    bf16 stack, every layer's Q|K|V|U kept, so that each user's candidates
+    can then be scored for the whole batch in one call that computes the
+    candidate rows only.
+
+    ``lens`` [B, 4] = (N_U, N_S, N_R, K_b): K_b candidate slots per user, the
+    same in every later ``score``; ``ts`` and ``x`` [T, d] float32 are the
+    packed timestamps and features of the batch. Their candidate rows may
+    hold anything: no context token sees a candidate (fun-rec 7.3.4, mask
+    rules 1-3). Each user's normaliser is its length N_U + N_S + N_R + K_b
+    (or ``norm``), as in the aggregated pass over the batch. ``out`` holds
+    the stack's output on all rows of this context pass.
+    """
+
+    def __init__(self, layers, lens, ts, x: torch.Tensor, norm=None, stream=None):
+        self.layers = list(layers)
+        self.c_layers = [l.c for l in self.layers]
+        self.lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(-1, 4))
+        self.norm = norm
+        dev = x.device
+        self.batch = PackedBatch(self.lens, ts, device=dev, norm=norm, stream=stream)
+        T, d = self.batch.T, self.layers[0].d
+        self.T = T
+        self.k_total = int(self.lens[:, 3].sum())
+        self.cache = torch.empty(len(self.layers), max(T, 1), 4 * d, dtype=torch.float16, device=dev)
+        self.out = torch.empty_like(x)
+        ws = _ws(_lib.mtgr_stack_rows_workspace_bytes(T, 0, self.c_layers), dev)
+        _lib.mtgr_stack_fwd_rows(self.c_layers, self.batch.c, 0, self.cache, T, x, self.out, ws,
+                                 stream)
+        self._ws = ws  # alive until the stream has run
+
+    def candidate_batch(self, ts, stream=None) -> PackedBatch:
+        """The batch of one candidate request: the same lens, with the packed
+        timestamps ``ts`` holding the candidates' exposure times."""
+        return PackedBatch(self.lens, ts, device=self.cache.device, norm=self.norm, stream=stream)
+
+    def workspace(self) -> torch.Tensor:
+        return _ws(_lib.mtgr_stack_candidates_workspace_bytes(self.batch.B, self.T, self.k_total,
+                                                              self.c_layers), self.cache.device)
+
+    def score(self, ts, x_cand: torch.Tensor, out=None, ws=None, batch=None,
+              stream=None) -> torch.Tensor:
+        """Stack output [K_total, d] float32 of the candidates (features
+        ``x_cand`` [K_total, d] float32, user by user), equal to their rows
+        of the aggregated pass over the batch."""
+        if batch is None:
+            batch = self.candidate_batch(ts, stream)
+        if out is None:
+            out = torch.empty(self.k_total, x_cand.shape[1], dtype=torch.float32, device=x_cand.device)
+        if ws is None:
+            ws = self.workspace()
+        _lib.mtgr_stack_fwd_candidates(self.c_layers, batch.c, self.k_total, self.cache, self.T,
+                                       x_cand, out, ws, stream)
+        return out
+
+
 class TokenMLPs:
     """The S, R and candidate token MLPs on the device: Linear(F_g, d) ->
     SiLU -> Linear(d, d) per domain, bf16 weights ([out, in]), fp32 biases.

@@ -29,8 +29,8 @@ int launch_gln_pooled(int32_t B, const int32_t* seg_off, int32_t d, int32_t x_dt
                       const float* gamma, const float* beta, float eps, int32_t y_dtype, void* y,
                       cudaStream_t s);
 int launch_gemm_tc_rowmap(int M, int N, int K, const void* a, const void* b, const float* bias,
-                          const int32_t* row_map, float* out, int out_rows, int32_t* status,
-                          cudaStream_t s);
+                          int epi, int q_cols, int32_t out_dtype, const int32_t* row_map, void* out,
+                          int out_rows, int32_t* status, cudaStream_t s);
 int launch_dom_scan(int32_t B, const int32_t* seg_off, const int32_t n_rows[4], uint32_t check_mask,
                     int32_t* dom_off, int32_t* status, cudaStream_t s);
 int launch_row_map(int32_t B, const int32_t* seg_off, const int32_t* dom_off, const int32_t base[4],
@@ -39,6 +39,8 @@ int launch_scatter_rows(int32_t n, int32_t d, const void* src, const int32_t* ma
                         float* dst, cudaStream_t s);
 int launch_gather_rows(int32_t n, int32_t d, const float* src, int32_t src_rows, const int32_t* map,
                        void* dst, cudaStream_t s);
+int launch_gather_rows16(int32_t n, int32_t d, const void* src, int32_t src_rows, const int32_t* map,
+                         void* dst, cudaStream_t s);
 int launch_head_dot(int32_t n, int32_t n_tasks, int32_t d_h, const void* h, const float* w2,
                     const float* b2, float* out, cudaStream_t s);
 int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu, float* g,
@@ -426,7 +428,7 @@ MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mt
 
 MTGR_API int mtgr_restrict_work(const mtgr_batch* batch, const int32_t* d_q_first,
                                 mtgr_stream_t stream) {
-  if (!batch_ok(batch) || (batch->B > 0 && d_q_first == nullptr)) return MTGR_ERR_INVALID_ARG;
+  if (!batch_ok(batch)) return MTGR_ERR_INVALID_ARG;
   if (batch->q_capacity == 0) return MTGR_OK;
   return launch_restrict_work(d_q_first, batch->q_capacity, const_cast<mtgr_work_item*>(batch->work),
                               const_cast<int64_t*>(batch->counts), as_stream(stream));
@@ -623,8 +625,8 @@ MTGR_API int mtgr_tokenize(const mtgr_batch* batch, int32_t d, const int32_t n_r
     if ((rc = launch_gemm_tc(n_rows[g], d, m.f, d_e[g], m.w1, m.b1, MTGR_EPI_SILU, nullptr, 0,
                              MTGR_BF16, w.h, batch->status, s)) != MTGR_OK)
       return rc;
-    if ((rc = launch_gemm_tc_rowmap(n_rows[g], d, d, w.h, m.w2, m.b2, w.map + base[g], d_x,
-                                    batch->T, batch->status, s)) != MTGR_OK)
+    if ((rc = launch_gemm_tc_rowmap(n_rows[g], d, d, w.h, m.w2, m.b2, MTGR_EPI_NONE, 0, MTGR_F32,
+                                    w.map + base[g], d_x, batch->T, batch->status, s)) != MTGR_OK)
       return rc;
   }
   return MTGR_OK;
@@ -671,6 +673,148 @@ MTGR_API int mtgr_candidate_heads(const mtgr_head_params* p, const mtgr_batch* b
   }
   TimedScope tsc(MTGR_TIMER_ROWS, s, 1);
   return launch_head_dot(k_total, p->n_tasks, p->d_h, w.h, p->w2, p->b2, d_out, s);
+}
+
+namespace {
+// Workspace of the candidate rows of a batch (the cached-context candidate
+// pass): candidate row map and per-domain offsets, the candidates' group ids
+// (all 3), GroupLN output, attention output over all T rows, the candidates'
+// gathered attention rows, MLP hidden, and a spare x buffer between layers.
+struct CandWs {
+  int32_t* dom_off;
+  int32_t* map;
+  int8_t* gid;
+  void* xt;
+  void* g;
+  void* gc;
+  void* h;
+  float* spare;
+  size_t bytes;
+};
+
+CandWs cand_ws_layout(int32_t B, int32_t T, int32_t K, const mtgr_block_params* layers, int32_t L,
+                      void* base) {
+  const size_t d = (size_t)layers[0].d, k = (size_t)K;
+  size_t dff = 0;
+  for (int32_t l = 0; l < L; ++l) dff = (size_t)layers[l].d_ff > dff ? (size_t)layers[l].d_ff : dff;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  CandWs w;
+  size_t off = 0;
+  w.dom_off = reinterpret_cast<int32_t*>(b + off); off += align_up(4 * ((size_t)B + 1) * 4, 256);
+  w.map = reinterpret_cast<int32_t*>(b + off);     off += align_up(k * 4, 256);
+  w.gid = reinterpret_cast<int8_t*>(b + off);      off += align_up(k, 256);
+  w.xt = b + off;                                  off += align_up(k * d * 2, 256);
+  w.g = b + off;                                   off += align_up((size_t)T * d * 2, 256);
+  w.gc = b + off;                                  off += align_up(k * d * 2, 256);
+  w.h = b + off;                                   off += align_up(k * dff * 2, 256);
+  w.spare = reinterpret_cast<float*>(b + off);     off += L > 1 ? align_up(k * d * 4, 256) : 0;
+  w.bytes = off;
+  return w;
+}
+
+// One bf16 block on the candidate rows only: x_in / x_out are the K
+// candidates' rows (user by user); the Q|K|V|U of every row of the batch is
+// in qkvu ([T][4d], the candidates' rows written here), and the batch's work
+// list holds the candidates' q-tiles only.
+int block_fwd_cand(const mtgr_block_params* p, const mtgr_batch* bt, int32_t K, const float* x_in,
+                   float* x_out, uint16_t* qkvu, const CandWs& w, cudaStream_t s) {
+  const int32_t d = p->d, H = p->H, dff = p->d_ff;
+  if (p->variant & MTGR_VARIANT_POOLED_GLN) return MTGR_ERR_UNSUPPORTED;
+  int rc;
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(K, d, MTGR_F32, x_in, w.gid, 4, p->gln1_gamma, p->gln1_beta, p->eps,
+                         MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
+  }
+  {
+    // Q|K|V|U of the candidates into their rows of the cache (Q halved)
+    TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
+    const int epi = (p->variant & MTGR_VARIANT_SILU_QKVU) ? MTGR_EPI_SILU : MTGR_EPI_NONE;
+    if ((rc = launch_gemm_tc_rowmap(K, 4 * d, d, w.xt, p->w_qkvu, p->b_qkvu, epi, d, MTGR_F16, w.map,
+                                    qkvu, bt->T, bt->status, s)) != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
+    if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, qkvu, MTGR_BF16, w.g, s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_ROWS, s, 1);
+    if ((rc = launch_gather_rows16(K, d, w.g, bt->T, w.map, w.gc, s)) != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(K, d, MTGR_BF16, w.gc, w.gid, 4, p->gln2_gamma, p->gln2_beta, p->eps,
+                         MTGR_BF16, w.xt, s)) != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
+    if ((rc = launch_gemm_tc(K, dff, d, w.xt, p->w1, p->b1, MTGR_EPI_SILU, nullptr, 0, MTGR_BF16,
+                             w.h, bt->status, s)) != MTGR_OK) return rc;
+  }
+  TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
+  return launch_gemm_tc(K, d, dff, w.h, p->w2, p->b2, MTGR_EPI_RESID, x_in, 0, MTGR_F32, x_out,
+                        bt->status, s);
+}
+}  // namespace
+
+MTGR_API size_t mtgr_stack_candidates_workspace_bytes(int32_t B, int32_t T, int32_t k_total,
+                                                      const mtgr_block_params* layers, int32_t L) {
+  if (B < 0 || T < 0 || k_total < 0 || k_total > T || L <= 0 || layers == nullptr) return 0;
+  for (int32_t l = 0; l < L; ++l)
+    if (params_check(&layers[l]) != MTGR_OK || layers[l].dtype != MTGR_BF16) return 0;
+  return cand_ws_layout(B, T, k_total, layers, L, nullptr).bytes;
+}
+
+MTGR_API int mtgr_stack_fwd_candidates(const mtgr_block_params* layers, int32_t L,
+                                       const mtgr_batch* batch, int32_t k_total, void* d_qkvu_cache,
+                                       int32_t cache_rows, const float* d_x_cand, float* d_x_out,
+                                       void* d_ws, size_t ws_bytes, mtgr_stream_t stream) {
+  int rc = serve_check(layers, L, batch);
+  if (rc != MTGR_OK) return rc;
+  for (int32_t l = 0; l < L; ++l)
+    if (layers[l].variant & MTGR_VARIANT_POOLED_GLN) return MTGR_ERR_UNSUPPORTED;
+  if (k_total < 0 || k_total > batch->T || cache_rows < batch->T) return MTGR_ERR_INVALID_ARG;
+  if (k_total == 0) return MTGR_OK;
+  if (d_qkvu_cache == nullptr || d_x_cand == nullptr || d_x_out == nullptr || d_ws == nullptr ||
+      d_x_cand == d_x_out)
+    return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_qkvu_cache) || !aligned16(d_x_cand) || !aligned16(d_x_out) || !aligned16(d_ws))
+    return MTGR_ERR_INVALID_ARG;
+  if (ws_bytes < mtgr_stack_candidates_workspace_bytes(batch->B, batch->T, k_total, layers, L))
+    return MTGR_ERR_CAPACITY;
+  const cudaStream_t s = as_stream(stream);
+  CandWs w = cand_ws_layout(batch->B, batch->T, k_total, layers, L, d_ws);
+  const int32_t n_rows[4] = {0, 0, 0, k_total};
+  const int32_t base[4] = {0, 0, 0, 0};
+  {
+    TimedScope tsc(MTGR_TIMER_ROWS, s, batch->q_capacity > 0 ? 3 : 2);
+    if (cudaMemsetAsync(w.map, 0xFF, (size_t)k_total * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(w.gid, 3, (size_t)k_total, s) != cudaSuccess)
+      return MTGR_ERR_CUDA;
+    if ((rc = launch_dom_scan(batch->B, batch->seg_off, n_rows, 0x8u, w.dom_off, batch->status, s)) !=
+        MTGR_OK)
+      return rc;
+    if ((rc = launch_row_map(batch->B, batch->seg_off, w.dom_off, base, n_rows, 0x8u, w.map, s)) !=
+        MTGR_OK)
+      return rc;
+    // the attention computes the candidates' q-tiles only (idempotent)
+    if (batch->q_capacity > 0 &&
+        (rc = launch_restrict_work(nullptr, batch->q_capacity,
+                                   const_cast<mtgr_work_item*>(batch->work),
+                                   const_cast<int64_t*>(batch->counts), s)) != MTGR_OK)
+      return rc;
+  }
+  const float* in = d_x_cand;
+  uint16_t* cache = static_cast<uint16_t*>(d_qkvu_cache);
+  for (int32_t l = 0; l < L; ++l) {
+    float* out = ((L - 1 - l) % 2 == 0) ? d_x_out : w.spare;
+    rc = block_fwd_cand(&layers[l], batch, k_total, in, out,
+                        cache + (size_t)l * cache_rows * 4 * layers[0].d, w, s);
+    if (rc != MTGR_OK) return rc;
+    in = out;
+  }
+  return MTGR_OK;
 }
 
 MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const void* d_a,

@@ -124,18 +124,23 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, cons
 
 // Row-map form, rows that do not form one run: each lane holds the
 // destination of its row; the values wait in the warp's staging block (as
-// written by epilogue_chunk), and every store instruction writes four whole
-// 128-byte row pieces.
+// written by epilogue_chunk), and every store instruction writes whole row
+// pieces of 32 columns (128 bytes fp32, four rows; 64 bytes 16-bit, eight).
+template <int OUT>
 __device__ __forceinline__ void rowmap_scatter(const GemmArgs& a, int col0, const uint8_t* stg,
                                                int my_dst, int lane) {
-  const int q = lane & 7;
+  constexpr int CH = OUT == MTGR_F32 ? 8 : 4;  // 16-byte pieces per row
+  constexpr int RPI = 32 / CH;                 // rows per store instruction
+  constexpr int ESZ = OUT == MTGR_F32 ? 4 : 2;
+  const int q = lane % CH;
 #pragma unroll
-  for (int r0 = 0; r0 < 32; r0 += 4) {
-    const int r = r0 + (lane >> 3);
+  for (int r0 = 0; r0 < 32; r0 += RPI) {
+    const int r = r0 + lane / CH;
     const int dst = __shfl_sync(0xffffffffu, my_dst, r);
-    const float4 x = *reinterpret_cast<const float4*>(stg + stg_off<MTGR_F32>(r, q));
+    const uint4 x = *reinterpret_cast<const uint4*>(stg + stg_off<OUT>(r, q));
     if (dst >= 0 && dst < a.out_rows)
-      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)dst * a.N + col0 + 4 * q) = x;
+      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + ((size_t)dst * a.N + col0) * ESZ +
+                                16 * q) = x;
   }
 }
 
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           } else {
             __syncwarp();
-            rowmap_scatter(args, col0, sb, my_dst, lane);
+            rowmap_scatter<OUT>(args, col0, sb, my_dst, lane);
           }
           prev_scatter = !run;
           continue;
@@ -374,25 +379,36 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
   return MTGR_ERR_UNSUPPORTED;
 }
 
-// out[row_map[m]][n] = sum_k a[m][k] b[n][k] + bias[n] (fp32 out with out_rows
-// rows; a row whose map entry is negative or past out_rows is dropped).
+// out[row_map[m]][n] = epi(sum_k a[m][k] b[n][k] + bias[n]) into out with
+// out_rows rows; a row whose map entry is negative or past out_rows is
+// dropped. Forms: EPI_NONE to fp32 or f16, EPI_SILU to f16; q_cols halves the
+// first q_cols columns (after the SiLU).
 int launch_gemm_tc_rowmap(int M, int N, int K, const void* a, const void* b, const float* bias,
-                          const int32_t* row_map, float* out, int out_rows, int32_t* status,
-                          cudaStream_t s) {
-  if (M == 0 || N == 0) return MTGR_OK;
-  CUtensorMap ta, tb;
+                          int epi, int q_cols, int32_t out_dtype, const int32_t* row_map, void* out,
+                          int out_rows, int32_t* status, cudaStream_t s) {
+  if (M == 0 || N == 0 || out_rows <= 0) return MTGR_OK;
+  CUtensorMap ta, tb, to;
   int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
   if (rc != MTGR_OK) return rc;
   rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
   if (rc != MTGR_OK) return rc;
-  if (out_rows <= 0) return MTGR_OK;
-  CUtensorMap to;
-  rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)out_rows,
-                    (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (out_dtype == MTGR_F32) {
+    rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)out_rows,
+                      (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N, (uint64_t)out_rows,
+                      (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
   if (rc != MTGR_OK) return rc;
-  GemmArgs args{M, N, K, bias, nullptr, out, 0, status, row_map, out_rows};
+  GemmArgs args{M, N, K, bias, nullptr, out, q_cols, status, row_map, out_rows};
   // the residual map is not read in this form
-  return launch_t<MTGR_EPI_NONE, MTGR_F32, true>(ta, tb, to, to, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32)
+    return launch_t<MTGR_EPI_NONE, MTGR_F32, true>(ta, tb, to, to, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16)
+    return launch_t<MTGR_EPI_NONE, MTGR_F16, true>(ta, tb, to, to, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F16)
+    return launch_t<MTGR_EPI_SILU, MTGR_F16, true>(ta, tb, to, to, args, s);
+  return MTGR_ERR_UNSUPPORTED;
 }
 
 }  // namespace mtgr

@@ -426,7 +426,8 @@ __global__ void meta_fill_kernel(int32_t q_cap, int32_t kt_cap, int32_t e_cap,
 }
 
 
-// Keeps the work items with a query row at or after q_first[b] (user-relative)
+// Keeps the work items with a query row at or after q_first[b] (user-relative;
+// a NULL q_first means each user's first candidate row, N_U + N_S + N_R)
 // in place and in order; a pair whose first q-tile lies wholly before it
 // becomes a single-q-tile item of the second. One block, the list in chunks
 // of kScanThreads: every thread reads its item before any is written, and an
@@ -445,7 +446,7 @@ __global__ void restrict_work_kernel(const int32_t* __restrict__ q_first, int32_
     int32_t keep = 0;
     if (i < P) {
       it = work[i];
-      const int32_t qf = q_first[it.b];
+      const int32_t qf = q_first != nullptr ? q_first[it.b] : it.c_lo;  // NULL: first candidate row
       const int32_t row_end = (it.qt0 + it.nq) * MTGR_TILE_M;  // one past the item's last row
       if (row_end > qf && it.n > qf) {
         keep = 1;

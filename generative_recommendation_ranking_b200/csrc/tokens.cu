@@ -170,6 +170,22 @@ __global__ void gather_rows_kernel(int32_t n, int32_t d, const float* __restrict
   }
 }
 
+// dst[r][:] = src[map[r]][:] for r < n (16-bit rows of d, d % 8 == 0); a map
+// entry outside [0, src_rows) gives a zero row.
+__global__ void gather_rows16_kernel(int32_t n, int32_t d, const uint16_t* __restrict__ src,
+                                     int32_t src_rows, const int32_t* __restrict__ map,
+                                     uint16_t* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n; r += warps) {
+    const int32_t o = map[r];
+    const bool ok = o >= 0 && o < src_rows;
+    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(ok ? o : 0) * d);
+    uint4* t = reinterpret_cast<uint4*>(dst + (size_t)r * d);
+    for (int c = lane; c < d / 8; c += 32) t[c] = ok ? __ldg(s + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 // out[r][t] = sum_k h[r][t d_h + k] w2[t][k] + b2[t]: a warp per row, fp32
 // accumulation, the lanes' partial sums combined by shuffles.
 __global__ void head_dot_kernel(int32_t n, int32_t n_tasks, int32_t d_h,
@@ -241,6 +257,14 @@ int launch_gather_rows(int32_t n, int32_t d, const float* src, int32_t src_rows,
   if (n == 0) return MTGR_OK;
   gather_rows_kernel<<<rows_grid(n), 256, 0, s>>>(n, d, src, src_rows, map,
                                                   static_cast<uint16_t*>(dst));
+  return launch_status();
+}
+
+int launch_gather_rows16(int32_t n, int32_t d, const void* src, int32_t src_rows, const int32_t* map,
+                         void* dst, cudaStream_t s) {
+  if (n == 0) return MTGR_OK;
+  gather_rows16_kernel<<<rows_grid(n), 256, 0, s>>>(n, d, static_cast<const uint16_t*>(src), src_rows,
+                                                    map, static_cast<uint16_t*>(dst));
   return launch_status();
 }
 

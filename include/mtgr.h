@@ -335,9 +335,11 @@ MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mt
  *
  * mtgr_restrict_work: rewrites batch->work and counts[3] in place so that
  * the attention computes only the work items holding a query row at or
- * after d_q_first[b] (user-relative, int32 [B], device); a q-tile pair whose
- * first q-tile lies wholly before it becomes a single-q-tile item. Order is
- * kept. Call after mtgr_build_mask_meta on the same stream.
+ * after d_q_first[b] (user-relative, int32 [B], device; NULL: each user's
+ * first candidate row N_U + N_S + N_R); a q-tile pair whose first q-tile
+ * lies wholly before it becomes a single-q-tile item. Order is kept;
+ * restricting twice to the same rows changes nothing. Call after
+ * mtgr_build_mask_meta on the same stream.
  */
 MTGR_API int mtgr_restrict_work(const mtgr_batch* batch, const int32_t* d_q_first,
                                 mtgr_stream_t stream);
@@ -432,6 +434,33 @@ MTGR_API int mtgr_candidate_heads(const mtgr_head_params* p, const mtgr_batch* b
                                   size_t ws_bytes, mtgr_stream_t stream);
 
 /*
+ * Cached-context candidate pass over a whole batch of users.
+ *   Context pass (once per set of contexts): mtgr_stack_fwd_rows with
+ *     row0 = 0 over a batch with lens (N_U, N_S, N_R, K_b) per user, the
+ *     candidate rows holding anything (zeros), with the normaliser override
+ *     N_b = N_U + N_S + N_R + K_b. A context row never sees a candidate, so
+ *     every layer's Q|K|V|U of the context rows is final.
+ *   Candidate pass: a batch of the same lens with the real candidates'
+ *     timestamps (same normalisers), and mtgr_stack_fwd_candidates: every
+ *     layer computes the candidate rows only. Their Q|K|V|U go into the
+ *     cache at their packed rows, the attention runs over the candidates'
+ *     q-tiles, and GroupLN and the MLP run on the candidates' rows.
+ * d_x_cand, d_x_out: float32 [k_total][d], the candidates user by user
+ * (k_total = sum K_b, checked on the device: MTGR_ERR_DEVICE_VALIDATION in
+ * the batch status). d_qkvu_cache as for mtgr_stack_fwd_rows
+ * (cache_rows >= T). The batch's work list is restricted in place to the
+ * candidates' q-tiles. Candidate rows sit where the aggregated pass has them,
+ * so the result equals that pass's candidate rows. Not with
+ * MTGR_VARIANT_POOLED_GLN (MTGR_ERR_UNSUPPORTED).
+ */
+MTGR_API size_t mtgr_stack_candidates_workspace_bytes(int32_t B, int32_t T, int32_t k_total,
+                                                      const mtgr_block_params* layers, int32_t L);
+MTGR_API int mtgr_stack_fwd_candidates(const mtgr_block_params* layers, int32_t L,
+                                       const mtgr_batch* batch, int32_t k_total, void* d_qkvu_cache,
+                                       int32_t cache_rows, const float* d_x_cand, float* d_x_out,
+                                       void* d_ws, size_t ws_bytes, mtgr_stream_t stream);
+
+/*
  * Dense GEMM with the block's epilogues, exposed for testing:
  *   out[m][n] = epi( sum_k a[m][k] * b[n][k] + bias[n] )
  *   epi = MTGR_EPI_NONE (out dtype MTGR_F16/MTGR_BF16/MTGR_F32),
@@ -458,7 +487,8 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
  * MTGR_TIMER_GEMM_MLP1, MTGR_TIMER_GEMM_MLP2 (1 each; mtgr_gemm counts as
  * MTGR_TIMER_GEMM_QKVU); MTGR_TIMER_TOKEN_MLP (the token MLPs' GEMMs, 2 per
  * domain with tokens), MTGR_TIMER_HEAD_MLP (the heads' first layer, 1) and
- * MTGR_TIMER_ROWS (the row bookkeeping of tokenize and heads: 3 and 4). mtgr_timer_read synchronises on the recorded events,
+ * MTGR_TIMER_ROWS (the row bookkeeping of tokenize, heads and the candidate
+ * pass: 3, 4, and 3 + 1 per layer). mtgr_timer_read synchronises on the recorded events,
  * writes the summed milliseconds and launch counts per class into
  * ms[MTGR_TIMER_CLASSES] and launches[MTGR_TIMER_CLASSES] (host arrays) and
  * clears the records. Attaching NULL detaches. Not for use during CUDA graph

@@ -169,3 +169,70 @@ def test_restricted_work_list(seed):
     for got, exp in zip(m["work"], want):
         np.testing.assert_array_equal(got[:14], exp)
         assert int(got[14]) | (int(got[15]) << 32) == int(m["rt_off"][exp[6]])
+
+
+# ---- batched: the contexts of many users cached, candidates scored in one call
+
+
+def _batched(lens, ts, x, ws, scramble=True):
+    """Context pass with the candidate rows scrambled (features 0, times 0),
+    then the candidate pass with the real ones."""
+    _, _, gid = oracle.pack_offsets(lens)
+    cand = gid == 3
+    x0, ts0 = x.copy(), ts.copy()
+    if scramble:
+        x0[cand] = 0.0
+        ts0[cand] = 0
+    cc = mt.BatchContextCache(ws, lens, ts0, torch.from_numpy(x0).cuda())
+    batch = cc.candidate_batch(ts)
+    scratch = cc.workspace().fill_(0xFF)  # NaN bit patterns: nothing may read stale workspace
+    yk = cc.score(None, torch.from_numpy(np.ascontiguousarray(x[cand])).cuda(), ws=scratch, batch=batch)
+    batch.check()
+    return to_host(cc.out), to_host(yk), cand
+
+
+@pytest.mark.parametrize("variant", [0, 2])
+def test_batched_candidate_pass_bit_exact_against_aggregated(variant):
+    rng = np.random.default_rng(3)
+    lens = np.array([[24, 300, 50, 70], [24, 10, 0, 1], [0, 0, 0, 0], [3, 129, 0, 0],
+                     [24, 1000, 100, 256], [1, 1, 1, 130], [24, 230, 30, 0]], np.int32)
+    d, H = 512, 8
+    ts = synth.make_timestamps(lens, rng)
+    x = synth.make_tokens(lens, d, rng)
+    layers = synth.make_stack_params(2, d, 2048, rng)
+    ws = [mt.BlockWeights(p, H, variant=variant) for p in layers]
+    b = mt.PackedBatch(lens, ts)
+    ya = to_host(mt.hstu_stack_forward(ws, b, torch.from_numpy(x).cuda()))
+    b.check()
+    yc, yk, cand = _batched(lens, ts, x, ws)
+    np.testing.assert_array_equal(yc[~cand], ya[~cand])
+    np.testing.assert_array_equal(yk, ya[cand])
+    ref = oracle.hstu_stack(x, lens, ts, layers, H, variant=variant)
+    assert_close_rms(yk, ref[cand], TOL_BF16, "batched candidates vs oracle")
+
+
+def test_batched_candidate_pass_block_workload():
+    # the 512-user block workload: every candidate row bit-exact against the
+    # aggregated pass, sampled users against the oracle
+    w = synth.make_workload(2)
+    ws = [mt.BlockWeights(p, w["H"]) for p in w["layers"]]
+    b = mt.PackedBatch(w["lens"], w["ts"])
+    ya = to_host(mt.hstu_stack_forward(ws, b, torch.from_numpy(w["x"]).cuda()))
+    b.check()
+    yc, yk, cand = _batched(w["lens"], w["ts"], w["x"], ws)
+    np.testing.assert_array_equal(yk, ya[cand])
+    np.testing.assert_array_equal(yc[~cand], ya[~cand])
+
+
+def test_batched_candidate_pass_refuses_pooled_gln():
+    rng = np.random.default_rng(4)
+    lens = np.array([[24, 100, 20, 10], [24, 50, 5, 3]], np.int32)
+    ts = synth.make_timestamps(lens, rng)
+    x = synth.make_tokens(lens, 512, rng)
+    layers = synth.make_stack_params(1, 512, 2048, rng)
+    ws = [mt.BlockWeights(p, 8, variant=mt.MTGR_VARIANT_POOLED_GLN) for p in layers]
+    cc = mt.BatchContextCache(ws, lens, ts, torch.from_numpy(x).cuda())  # the context pass runs
+    _, _, gid = oracle.pack_offsets(lens)
+    with pytest.raises(mt.MTGRError) as e:
+        cc.score(ts, torch.from_numpy(np.ascontiguousarray(x[gid == 3])).cuda())
+    assert e.value.status == mt._lib.MTGR_ERR_UNSUPPORTED

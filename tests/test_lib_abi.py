@@ -86,6 +86,7 @@ def test_host_validation_without_device(lib):
     assert lib.mtgr_restrict_work(None, None, None) == E
     assert lib.mtgr_group_layernorm_pooled(2, None, 64, 0, None, None, None, 1e-5, 0, None, None) == E
     assert lib.mtgr_tokenize(None, 512, None, None, None, None, None, 0, None) == E
+    assert lib.mtgr_stack_fwd_candidates(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
     assert lib.mtgr_candidate_heads(None, None, 0, None, None, None, 0, None) == E
     assert lib.mtgr_stack_fwd_rows(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
 
@@ -164,3 +165,17 @@ def test_token_and_head_workspace_sizes(lib):
     assert _lib.mtgr_heads_workspace_bytes(B, 300, p) == want
     p.d_h = 100  # % 32
     assert _lib.mtgr_heads_workspace_bytes(B, 300, p) == 0
+
+
+def test_candidate_pass_workspace_sizes(lib):
+    # offsets 4 (B + 1) int32, candidate map K int32, group ids K int8,
+    # GroupLN output K x d bf16, attention output T x d bf16, gathered rows
+    # K x d bf16, MLP hidden K x d_ff bf16, spare x K x d fp32 when L > 1
+    up = lambda n: -(-n // 256) * 256  # noqa: E731
+    B, T, K = 3, 2000, 300
+    p = _params()
+    one = (up(4 * (B + 1) * 4) + up(K * 4) + up(K) + up(K * 512 * 2) + up(T * 512 * 2)
+           + up(K * 512 * 2) + up(K * 2048 * 2))
+    assert _lib.mtgr_stack_candidates_workspace_bytes(B, T, K, [p]) == one
+    assert _lib.mtgr_stack_candidates_workspace_bytes(B, T, K, [p, p]) == one + up(K * 512 * 4)
+    assert _lib.mtgr_stack_candidates_workspace_bytes(B, T, T + 1, [p]) == 0
