@@ -299,7 +299,8 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
     return MTGR_ERR_INVALID_ARG;
   if (ws_bytes < mask_meta_ws_bytes(q_capacity, kt_capacity)) return MTGR_ERR_CAPACITY;
   if (q_capacity > 0 && kt_capacity > 0 && d_ws == nullptr) return MTGR_ERR_INVALID_ARG;
-  TimedScope tsc(MTGR_TIMER_MASK_META, as_stream(stream), q_capacity > 0 ? 6 : 4);
+  TimedScope tsc(MTGR_TIMER_MASK_META, as_stream(stream),
+                 2 + (B > 0 ? 2 : 0) + (q_capacity > 0 ? 2 : 0));
   return launch_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity, rt_capacity,
                           d_qtile_desc, d_row_ptr, d_entries, d_order, d_counts, d_rt_cnt,
                           d_rt_off, d_rt_mask, d_work, d_ws, d_status, as_stream(stream));

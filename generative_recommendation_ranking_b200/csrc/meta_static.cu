@@ -80,7 +80,7 @@ extern "C" MTGR_API int mtgr_build_mask_meta_static(
   const int rc = scratch_address(&scratch);
   if (rc != MTGR_OK) return rc;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  mtgr::TimedScope tsc(MTGR_TIMER_MASK_META, s, q_capacity > 0 ? 6 : 4);
+  mtgr::TimedScope tsc(MTGR_TIMER_MASK_META, s, 2 + (B > 0 ? 2 : 0) + (q_capacity > 0 ? 2 : 0));
   return mtgr::launch_mask_meta(B, d_seg_off, d_ts, q_capacity, kt_capacity, e_capacity,
                                 rt_capacity, d_qtile_desc, d_row_ptr, d_entries, d_order, d_counts,
                                 d_rt_cnt, d_rt_off, d_rt_mask, d_work, scratch, d_status, s);

@@ -335,28 +335,22 @@ __global__ void __launch_bounds__(kScanThreads) meta_scan_kernel(int32_t q_cap, 
 // Work order: users by descending length (ties by ascending index), each
 // user's q-tiles contiguous and by ascending qt, so that every item of a user
 // (all its q-tiles and heads) runs close in time and its keys and values stay
-// in L2. One thread per user ranks it against all users and writes the
-// user's q-tiles into order[] and the work list (runs after the row_ptr scan).
-__global__ void __launch_bounds__(kScanThreads) meta_order_kernel(
+// in L2. A warp per user: its lanes rank the user against all users (a strided
+// count and a warp sum), then write the user's q-tiles into order[] and its
+// q-tile pairs into the work list, a lane per pair (runs after the entries are
+// filled).
+__global__ void __launch_bounds__(32) meta_order_kernel(
     int32_t B, const int32_t* seg_off, int32_t q_cap, const int32_t* row_ptr,
     const int32_t* entries, const int64_t* rt_off, int32_t* order, mtgr_work_item* work,
     const int64_t* counts) {
-  constexpr int32_t kSmemUsers = 8192;
-  __shared__ int32_t n_sh[kSmemUsers];  // user lengths, when they fit
   if (counts[0] == 0) return;
-  const bool in_smem = B <= kSmemUsers;
-  if (in_smem) {
-    for (int32_t k = threadIdx.x; k < B; k += blockDim.x)
-      n_sh[k] = seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
-  }
-  __syncthreads();
-  for (int32_t b = threadIdx.x; b < B; b += blockDim.x) {
+  const int lane = threadIdx.x;
+  for (int32_t b = blockIdx.x; b < B; b += gridDim.x) {
     const int32_t* so = seg_off + 4 * (int64_t)b;
     const int32_t n = so[4] - so[0];
-    int64_t pos = 0, qstart = 0, ppos = 0;
-    for (int32_t k = 0; k < B; ++k) {
-      const int32_t nk =
-          in_smem ? n_sh[k] : seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
+    long long pos = 0, qstart = 0, ppos = 0;
+    for (int32_t k = lane; k < B; k += 32) {
+      const int32_t nk = seg_off[4 * (int64_t)k + 4] - seg_off[4 * (int64_t)k];
       const int32_t nqk = (nk + MTGR_TILE_M - 1) / MTGR_TILE_M;
       if (k < b) qstart += nqk;
       if (nk > n || (nk == n && k < b)) {
@@ -364,12 +358,18 @@ __global__ void __launch_bounds__(kScanThreads) meta_order_kernel(
         ppos += (nqk + 1) / 2;
       }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      pos += __shfl_xor_sync(0xffffffffu, pos, o);
+      qstart += __shfl_xor_sync(0xffffffffu, qstart, o);
+      ppos += __shfl_xor_sync(0xffffffffu, ppos, o);
+    }
     const int32_t nq = (n + MTGR_TILE_M - 1) / MTGR_TILE_M;
-    for (int32_t qt = 0; qt < nq; ++qt) {
+    for (int32_t qt = lane; qt < nq; qt += 32) {
       const int64_t slot = pos + qt, q = qstart + qt;
       if (slot < q_cap && q < q_cap) order[slot] = (int32_t)q;
     }
-    for (int32_t pp = 0; 2 * pp < nq; ++pp) {
+    for (int32_t pp = lane; 2 * pp < nq; pp += 32) {
       const int64_t slot = ppos + pp, qa = qstart + 2 * pp;
       const bool two = 2 * pp + 1 < nq;
       if (slot >= q_cap || qa + (two ? 1 : 0) >= q_cap) continue;
@@ -535,8 +535,11 @@ int launch_mask_meta(int32_t B, const int32_t* seg_off, const int64_t* ts, int32
                                                      entries, counts);
     if ((rc = launch_status()) != MTGR_OK) return rc;
   }
-  meta_order_kernel<<<1, kScanThreads, 0, s>>>(B, seg_off, q_cap, row_ptr, entries, rt_off, order,
-                                              work, counts);
+  if (B > 0) {
+    const int cap = device_sm_count() * 32;
+    meta_order_kernel<<<B < cap ? B : cap, 32, 0, s>>>(B, seg_off, q_cap, row_ptr, entries, rt_off,
+                                                       order, work, counts);
+  }
   return launch_status();
 }
 int launch_restrict_work(const int32_t* q_first, int32_t q_cap, mtgr_work_item* work, int64_t* counts,
