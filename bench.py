@@ -508,7 +508,7 @@ def incremental_leg(agg: dict, dev, stream, args) -> dict:
     x = torch.from_numpy(agg["x"]).to(dev)
     xc, xk = x[:n_ctx], x[n_ctx:]
     cc = mt.ContextCache(layers, n_u, n_s, n_r, agg["ts"][:n_ctx], xc, K, K, stream=stream)
-    cb = cc._ctx_batch
+    cb = cc.ctx_batch
     batch = cc.candidate_batch(agg["ts"][n_ctx:], stream)
     ws = cc.workspace(K)
     out = torch.empty(K, agg["d"], dtype=torch.float32, device=dev)
@@ -517,7 +517,7 @@ def incremental_leg(agg: dict, dev, stream, args) -> dict:
         cb.pack(s)
         cb.build_meta(s)
         _lib.mtgr_stack_fwd_rows(cc.c_layers, cb.c, 0, cc.cache, cc.cache_rows, xc, cc.out,
-                                 cc._ws, s)
+                                 cc.ctx_ws, s)
 
     def cand_step(s=stream):
         batch.pack(s)
@@ -603,7 +603,7 @@ def run_serving(args, local):
     x_cand = x[cand].contiguous()
     cc = mt.BatchContextCache(layers, lens, wl["ts"], x, stream=stream)
     cb = cc.batch
-    cws = cc._ws
+    cws = cc.ctx_ws
     batch = cc.candidate_batch(wl["ts"], stream)
     ws = cc.workspace()
     out = torch.empty(cc.k_total, wl["d"], dtype=torch.float32, device=dev)

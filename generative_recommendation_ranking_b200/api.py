@@ -261,8 +261,10 @@ class ContextCache:
         ws = _ws(_lib.mtgr_stack_rows_workspace_bytes(self.n_ctx, 0, self.c_layers), dev)
         _lib.mtgr_stack_fwd_rows(self.c_layers, batch.c, 0, self.cache, self.cache_rows, x_ctx,
                                  self.out, ws, stream)
-        self._ctx_batch = batch  # keeps its buffers alive until the stream has run
-        self._ws = ws
+        # the context pass's batch and workspace, kept so that the pass can be
+        # run again in place (their buffers also stay alive for the stream)
+        self.ctx_batch = batch
+        self.ctx_ws = ws
 
     def candidate_batch(self, ts_cand, stream=None) -> PackedBatch:
         """The virtual batch of one chunk: the context followed by the
@@ -328,7 +330,7 @@ class BatchContextCache:
         ws = _ws(_lib.mtgr_stack_rows_workspace_bytes(T, 0, self.c_layers), dev)
         _lib.mtgr_stack_fwd_rows(self.c_layers, self.batch.c, 0, self.cache, T, x, self.out, ws,
                                  stream)
-        self._ws = ws  # alive until the stream has run
+        self.ctx_ws = ws  # kept for re-running the context pass in place
 
     def candidate_batch(self, ts, stream=None) -> PackedBatch:
         """The batch of one candidate request: the same lens, with the packed

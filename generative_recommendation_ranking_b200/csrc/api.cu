@@ -203,11 +203,12 @@ int block_fwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
               void* ws, cudaStream_t s) {
   const int32_t T = bt->T, d = p->d, H = p->H, dff = p->d_ff;
   if (T == 0) return MTGR_OK;
-  BlockWs w = block_ws_layout(T, p, ws);
-  int rc;
   // bf16: the rows form over all rows, with the workspace laid out as
   // block_ws_layout lays it out (GroupLN output, Q|K|V|U, G, MLP hidden)
   if (p->dtype == MTGR_BF16) return block_fwd_rows(p, bt, 0, x_in, x_out, nullptr, ws, s);
+  // fp32: CUDA cores throughout
+  BlockWs w = block_ws_layout(T, p, ws);
+  int rc;
   {
     TimedScope tsc(MTGR_TIMER_GLN, s, 1);
     if ((rc = launch_gln(T, d, MTGR_F32, x_in, bt->group_id, 4, p->gln1_gamma, p->gln1_beta, p->eps,
