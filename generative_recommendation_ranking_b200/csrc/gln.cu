@@ -85,7 +85,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // of their loads issued before any reduction so that each lane keeps about
 // 128 bytes of the input in flight; the rows stay in registers.
 template <typename Tin, typename Tout, int VPL, int TPW>
-__global__ void __launch_bounds__(256, 4) gln_reg_kernel(int32_t T, int32_t d, const Tin* __restrict__ x,
+__global__ void __launch_bounds__(256, 3) gln_reg_kernel(int32_t T, int32_t d, const Tin* __restrict__ x,
                                                       const int8_t* __restrict__ gid, int32_t G,
                                                       const float* __restrict__ gamma,
                                                       const float* __restrict__ beta, float eps,
@@ -136,27 +136,33 @@ __global__ void __launch_bounds__(256, 4) gln_reg_kernel(int32_t T, int32_t d, c
     }
     rstd[j] = 1.0f / sqrtf(warp_sum(q) / (float)d + eps);
   }
+  // gamma and beta rows are loaded once per vector and run of same-group
+  // tokens (the warp's tokens are consecutive, so nearly always one group):
+  // reloading them per token made the L1, not HBM, the bound
+  int g[TPW];
 #pragma unroll
   for (int j = 0; j < TPW; ++j) {
-    const int64_t t = t0 + j;
-    if (t >= T) break;
-    int g = gid[t];
-    g = g < 0 ? 0 : (g >= G ? G - 1 : g);
-    const float* ga = gamma + (int64_t)g * d;
-    const float* be = beta + (int64_t)g * d;
-    Tout* yr = y + t * d;
+    const int gi = t0 + j < T ? gid[t0 + j] : 0;
+    g[j] = gi < 0 ? 0 : (gi >= G ? G - 1 : gi);
+  }
 #pragma unroll
-    for (int k = 0; k < VPL; ++k) {
-      const int vi = lane + 32 * k;
-      if (vi < nv) {
-        float v[8], gm[8], bt[8], o[8];
-        raw[j][k].unpack(v);
-        load8(ga + 8 * vi, gm);
-        load8(be + 8 * vi, bt);
+  for (int k = 0; k < VPL; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi >= nv) continue;
+    float gm[8], bt[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = (v[e] - mean[j]) * rstd[j] * gm[e] + bt[e];
-        store8(yr + 8 * vi, o);
+    for (int j = 0; j < TPW; ++j) {
+      const int64_t t = t0 + j;
+      if (t >= T) break;
+      if (j == 0 || g[j] != g[j - 1]) {
+        load8(gamma + (int64_t)g[j] * d + 8 * vi, gm);
+        load8(beta + (int64_t)g[j] * d + 8 * vi, bt);
       }
+      float v[8], o[8];
+      raw[j][k].unpack(v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (v[e] - mean[j]) * rstd[j] * gm[e] + bt[e];
+      store8(y + t * d + 8 * vi, o);
     }
   }
 }
