@@ -36,6 +36,7 @@ from .mtgr import (  # noqa: F401
     mask_meta,
     visible_pairs,
 )
+from .backward import hstu_block_backward  # noqa: F401
 from .tokens import (  # noqa: F401
     token_mlp,
     tokenize,
