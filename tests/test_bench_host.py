@@ -1,0 +1,76 @@
+"""Host logic of bench.py on the CPU: the ncu traffic record is used only
+while the kernel source matches the capture, the peaks come from the measured
+file (else the fallback), the workload description, and the default flags."""
+
+import hashlib
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def _fake_root(tmp_path, src_text, recorded_sha):
+    csrc = tmp_path / "generative_recommendation_ranking_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "attn_tc.cu").write_text(src_text)
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(
+        {"attention": {"bytes_per_launch": 12345, "src_sha": recorded_sha}}))
+    return str(tmp_path)
+
+
+def test_traffic_only_while_the_source_matches(tmp_path, monkeypatch):
+    text = "// kernel source\n"
+    sha = hashlib.sha256(text.encode()).hexdigest()[:16]
+    monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path / "a", text, sha))
+    assert bench.ncu_traffic("attention") == 12345
+    monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path / "b", text + "// changed\n", sha))
+    assert bench.ncu_traffic("attention") is None
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "missing"))
+    assert bench.ncu_traffic("attention") is None
+
+
+def test_committed_traffic_record_names_a_kernel_class_with_a_source():
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        rec = json.load(f)
+    for cls, e in rec.items():
+        assert cls in bench.KERNEL_SRC, cls
+        assert e["bytes_per_launch"] > 0 and len(e["src_sha"]) == 16
+        assert os.path.exists(os.path.join(ROOT, "profiles", os.path.basename(e["source"])))
+
+
+def test_peaks_measured_else_fallback(tmp_path, monkeypatch):
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 7000.0, "bf16_tflops": 1700.0, "bf16_tflops_sustained": 1500.0, "other": 1}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "measured" and peaks == {"hbm_gbs": 7000.0, "bf16_tflops": 1700.0,
+                                           "bf16_tflops_sustained": 1500.0}
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "nowhere"))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
+
+
+def test_workload_config_describes_the_block_workload():
+    wl = synth.make_workload(2)
+    c = bench.workload_config(wl, 4)
+    assert c["workload"] == "block_bf16_b512_d512" and c["users_per_gpu"] == 512
+    assert c["tokens_per_gpu"] == int(np.asarray(wl["lens"]).sum())
+    assert (c["d_model"], c["heads"], c["d_ff"], c["layers"]) == (512, 8, 2048, 1)
+    assert c["parallelism"].startswith("dp4")
+    assert "larger than L2" in c["l2"]
+
+
+def test_default_flags(monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse_args()
+    assert (a.gpus, a.config, a.impl) == (1, 2, "ours")
+    assert a.warmup >= 3 and a.steps > 0
+    assert not (a.pipeline or a.serving or a.no_e2e or a.no_cpu_baseline)
