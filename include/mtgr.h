@@ -13,6 +13,15 @@
  *   X  <- MLP(GroupLN_2(G)) + X,   MLP = Linear -> SiLU -> Linear
  * with the three-rule mask M and N the user's total token count.
  *
+ * Around the stack:
+ *  - the per-domain token MLPs that build X (mtgr_tokenize);
+ *  - the CTR/CTCVR heads on the candidates' output rows
+ *    (mtgr_candidate_heads);
+ *  - serving with each layer's Q|K|V|U of the users' contexts cached, the
+ *    candidates then scored against it (mtgr_stack_fwd_rows,
+ *    mtgr_stack_fwd_candidates);
+ *  - two block variants the pages leave open (mtgr_block_params.variant).
+ *
  * Conventions shared by every entry point:
  *  - Pointers named d_* are DEVICE pointers (CUDA global memory) on the
  *    current device; the caller owns and frees all memory. The library never
