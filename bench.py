@@ -165,10 +165,16 @@ def max_over_ranks(v: float, world: int, device) -> float:
 
 
 # --------------------------------------------------------- CPU oracle --------
-def oracle_users_per_s(wl: dict, budget_s: float, min_users: int = 1) -> dict:
-    """Time the CPU oracle on the first n users of the workload (n sized to the budget)."""
+def oracle_users_per_s(wl: dict, budget_s: float, min_users: int = 1,
+                       max_threads: int | None = None) -> dict:
+    """Time the CPU oracle on the first n users of the workload (n sized to
+    the budget); ``max_threads`` caps the BLAS thread pools while it runs."""
     import oracle
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
+
+    if max_threads is not None:
+        with threadpool_limits(limits=max_threads):
+            return oracle_users_per_s(wl, budget_s, min_users)
 
     def run(n):
         rows = np.arange(int(wl["lens"][:n].sum()))
@@ -475,9 +481,12 @@ def run_ours(args, world, rank, local):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         r = oracle_users_per_s(wl, args.cpu_seconds)
+        r1 = oracle_users_per_s(wl, args.cpu_seconds / 3, max_threads=1)
         cpu = {"value": r["value"], "unit": UNIT, "cores": r["threads"], "kind": "oracle",
                "sample": f"first {r['users']} users of {wl['name']} (seed {args.seed}), "
-                         f"float64 NumPy, {r['seconds']:.1f} s"}
+                         f"float64 NumPy, {r['seconds']:.1f} s",
+               "single_thread": {"value": r1["value"], "unit": UNIT,
+                                 "sample": f"first {r1['users']} users, {r1['seconds']:.1f} s"}}
     launches = int(sum(n for _, n in per_class.values()))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

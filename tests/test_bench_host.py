@@ -74,3 +74,13 @@ def test_default_flags(monkeypatch):
     assert (a.gpus, a.config, a.impl) == (1, 2, "ours")
     assert a.warmup >= 3 and a.steps > 0
     assert not (a.pipeline or a.serving or a.no_e2e or a.no_cpu_baseline)
+
+
+def test_cpu_baseline_thread_cap():
+    # the oracle timing runs on the fp32 block workload and reports its
+    # threads; capped at one thread it reports one
+    wl = synth.make_workload(0)
+    r = bench.oracle_users_per_s(wl, 0.05)
+    assert r["users"] >= 1 and r["value"] > 0 and r["threads"] >= 1
+    r1 = bench.oracle_users_per_s(wl, 0.05, max_threads=1)
+    assert r1["threads"] == 1 and r1["value"] > 0
