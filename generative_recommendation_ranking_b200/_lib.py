@@ -24,6 +24,7 @@ MTGR_VARIANT_SILU_QKVU = 2
 MTGR_ERR_CAPACITY = 4
 MTGR_ERR_TIMEOUT = 5
 MTGR_ERR_DEVICE_VALIDATION = 6
+MTGR_ERR_RANGE = 7
 
 MTGR_F32 = 0
 MTGR_BF16 = 1
@@ -126,6 +127,7 @@ _SIGNATURES = {
     "mtgr_timer_attach": (ctypes.c_int, [c_vp]),
     "mtgr_timer_read": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_double),
                                        ctypes.POINTER(ctypes.c_int64)]),
+    "mtgr_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, c_vp, c_vp]),
 }
 
 _lib = None
@@ -346,3 +348,8 @@ def mtgr_gemm(d_a, d_b, d_bias, epi, d_resid, q_cols, d_out, d_status, stream=No
     _check("mtgr_gemm", load().mtgr_gemm(
         M, N, K, dtype_code(d_a.dtype), _ptr(d_a), _ptr(d_b), _ptr(d_bias), epi, _ptr(d_resid),
         q_cols, dtype_code(d_out.dtype), _ptr(d_out), _ptr(d_status), _stream(stream)))
+
+
+def mtgr_selftest_bounded_wait(limit_ns: int, d_status, stream=None) -> None:
+    _check("mtgr_selftest_bounded_wait",
+           load().mtgr_selftest_bounded_wait(int(limit_ns), _ptr(d_status), _stream(stream)))

@@ -53,7 +53,6 @@ using namespace mtgr;
 
 namespace {
 
-constexpr int32_t kMaxKtCapacity = 4096;  // users up to 4096 * 128 tokens
 constexpr int32_t kMaxD = 8192;
 
 inline cudaStream_t as_stream(mtgr_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -258,11 +257,12 @@ MTGR_API const char* mtgr_status_string(int status) {
     case MTGR_ERR_CAPACITY: return "capacity exceeded";
     case MTGR_ERR_TIMEOUT: return "device wait timed out";
     case MTGR_ERR_DEVICE_VALIDATION: return "device-side validation failed";
+    case MTGR_ERR_RANGE: return "value out of the f16 range of an intermediate";
     default: return "unknown status";
   }
 }
 
-MTGR_API int mtgr_version(void) { return 100; }
+MTGR_API int mtgr_version(void) { return 101; }
 
 MTGR_API int mtgr_pack_offsets(int32_t B, const int32_t* d_lens, int32_t T, int32_t* d_seg_off,
                                int32_t* d_user_off, int8_t* d_group_id, int32_t* d_status,

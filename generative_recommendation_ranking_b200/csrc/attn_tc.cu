@@ -34,12 +34,17 @@
 // TMEM (512 columns): S_A, S_B (128 each), P_A, P_B (64 each, f16 pairs),
 // O_A, O_B (64 each).
 //
-// P and V enter the second MMA as f16 (11-bit significand) rather than bf16:
-// the unnormalised silu weights span a wide range and bf16 rounding of P alone
+// Scores accumulate in fp32 in TMEM (for f16 and bf16 operands alike). P and
+// V enter the second MMA as f16 (11-bit significand) rather than bf16: the
+// unnormalised silu weights span a wide range and bf16 rounding of P alone
 // would put the max-abs error near the 2e-2 x RMS bound on heavy-tailed
 // outputs. silu(s) = h + h tanh(h), h = s/2, is computed on f16x2 pairs
 // (one MUFU tanh per two scores). When Q arrives pre-halved (block path, the
 // projection epilogue scales the Q columns by 0.5 exactly) h is the score.
+// A score whose silu leaves the f16 range (above 65504) makes P infinite; the
+// epilogue finds the non-finite O and records MTGR_ERR_RANGE, so such inputs
+// are reported, never silently wrong. (Very negative scores saturate at
+// -65504 and give P = 0, which is silu's value to f16 precision there.)
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -326,8 +331,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // --------------------------------------------------- S issuer (MMA) --
     if (lane == 0) {
-      // f16 operands: f16 scores (the SiLU works in f16 anyway); bf16: f32
-      constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false, !IN_BF16);
+      constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
       int32_t g = 0, gb = 0, li = 0;
       Item nxt;
       if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
@@ -447,15 +451,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t r = static_cast<uint32_t>(gq);
         if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
+        // f32 scores: 16-column steps, the load of step k + 1 in flight while
+        // step k is masked, scaled and converted to f16 pairs
         uint32_t h[64];
-        if (!IN_BF16) {
-          // f16 scores (f16 accumulator, one per column): one packed load
-          tmem_ld64_pack16(s_addr, h);
-          tmem_ld_wait();
-          reg_fence(h);
-        } else {
-          // f32 scores: 16-column steps, the load of step k + 1 in flight
-          // while step k is converted and masked
+        {
           uint64_t vis_lo = 0, vis_hi = 0;
           if (masked) {
             vis_lo = visible_bits(it.w, rt_lo, i, kt * TN);
@@ -482,23 +481,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
-        uint64_t vis_lo = 0, vis_hi = 0;
-        if (!IN_BF16 && masked) {
-          vis_lo = visible_bits(it.w, rt_lo, i, kt * TN);
-          vis_hi = visible_bits(it.w, rt_hi, i, kt * TN + 64);
-        }
         if (t + 1 < it.w.n_union) fetch();
-        if (!IN_BF16) {
-          if (masked) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              h[c] &= pair_mask(static_cast<uint32_t>((c < 32 ? vis_lo : vis_hi) >> (2 * (c & 31))));
-          }
-          if (HALVE) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) h[c] = mul_f16x2(h[c], 0x38003800u);  // x 0.5, exact
-          }
-        }
         // The tanh of both q-tiles runs on the MUFU pipes (16 values per
         // clock per SM, one pipe per sub-partition), the bound of this
         // kernel. The A and B warps of one sub-partition (same lane quarter)
@@ -585,6 +568,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) mbar_arrive(o_free);
         }
         const int32_t i = (it.w.qt0 + q) * TM + rr;
+        bool bad = false;  // a non-finite O: some P left the f16 range
         if (i < it.w.n) {
           const int64_t row = it.w.us + i;
           const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
@@ -607,6 +591,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const int col = 8 * k + 2 * c;
               const uint32_t r0 = col < 32 ? o0[col] : o1[col - 32];
               const uint32_t r1 = col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32];
+              const float f0 = __uint_as_float(r0), f1 = __uint_as_float(r1);
+              bad |= (f0 - f0) != 0.f || (f1 - f1) != 0.f;  // inf - inf, NaN - NaN: NaN
               ov[2 * c] = __uint_as_float(r0) * inv_n * u0;
               ov[2 * c + 1] = __uint_as_float(r1) * inv_n * u1;
             }
@@ -621,6 +607,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, MTGR_ERR_RANGE);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(u_empty);  // U of this item consumed

@@ -13,6 +13,10 @@ namespace mtgr {
 // records MTGR_ERR_TIMEOUT and returns. No legitimate wait is near this.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
+// Largest kt_capacity (k-tiles of the longest user) any metadata builder or
+// batch accepts: users of up to 4096 * 128 tokens.
+constexpr int32_t kMaxKtCapacity = 4096;
+
 // Record a device-side error; the first error wins.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);

@@ -97,6 +97,16 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, cons
                                                uint8_t* stg, int r) {
   float v[32];
   epilogue_math<EPI, OUT>(a, col0, acc, v);
+  if (OUT == MTGR_F16) {
+    // the f16 conversion saturates at +-65504: report a value beyond it
+    // (the Q|K|V|U projection of an out-of-range input) instead of clamping
+    // it silently
+    float m = 0.f;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) m = fmaxf(m, fabsf(v[c]));
+    if (__any_sync(0xffffffffu, m > 65504.f) && (threadIdx.x & 31) == 0)
+      set_status(a.status, MTGR_ERR_RANGE);
+  }
   if (OUT == MTGR_F32) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {

@@ -10,10 +10,13 @@
 // mtgr_build_mask_meta_static keeps that scratch in a fixed-size array in the
 // library's own device memory instead. The caller still passes every input and
 // output buffer.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "timer.h"
@@ -33,25 +36,66 @@ namespace {
 // library holds this array until the process exits.
 __device__ __align__(256) uint8_t g_meta_scratch[MTGR_STATIC_META_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+// The array's device address depends on the CUDA context that loaded the
+// module: a device reset, or a caller running the library under a context of
+// its own, loads the module again at another address. So the address is
+// cached per context, keyed by the context's unique id (cuCtxGetId; ids are
+// never reused within a process, unlike context handles), and looked up with
+// that context current the first time the entry point runs in it.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+std::vector<ScratchEntry> g_scratch_cache;
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current. The array's name in host code is only
-// a host-side stand-in, never a device address.
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_driver_once;
+
+void load_driver_entry_points() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  p = nullptr;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+}
+
+// Device address of the scratch array in the current context. The array's
+// name in host code is only a host-side stand-in, never a device address.
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MTGR_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MTGR_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_meta_scratch) != cudaSuccess || p == nullptr)
+  std::call_once(g_driver_once, load_driver_entry_points);
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr) return MTGR_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return MTGR_ERR_CUDA;
+  if (ctx == nullptr) {
+    // no context current on this thread yet: cudaSetDevice initialises the
+    // current device's primary context (it allocates nothing)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess)
       return MTGR_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MTGR_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  unsigned long long id = 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return MTGR_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  for (const ScratchEntry& e : g_scratch_cache) {
+    if (e.ctx_id == id) {
+      *out = e.ptr;
+      return MTGR_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_meta_scratch) != cudaSuccess || p == nullptr)
+    return MTGR_ERR_CUDA;
+  g_scratch_cache.push_back(ScratchEntry{id, p});
+  *out = p;
   return MTGR_OK;
 }
 
@@ -64,7 +108,7 @@ extern "C" MTGR_API int mtgr_build_mask_meta_static(
     int32_t* d_rt_cnt, int64_t* d_rt_off, uint64_t* d_rt_mask, mtgr_work_item* d_work,
     int32_t* d_status, mtgr_stream_t stream) {
   if (B < 0 || q_capacity < 0 || kt_capacity < 0 || e_capacity < 0 || rt_capacity < 0 ||
-      kt_capacity > 4096)
+      kt_capacity > mtgr::kMaxKtCapacity)
     return MTGR_ERR_INVALID_ARG;
   if ((int64_t)q_capacity * (int64_t)kt_capacity > (int64_t)MTGR_STATIC_META_SCRATCH_BYTES)
     return MTGR_ERR_CAPACITY;  // beyond the fixed scratch: use mtgr_build_mask_meta

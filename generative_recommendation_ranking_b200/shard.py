@@ -53,3 +53,19 @@ def imbalance(lens: np.ndarray, shards: list, d: int, d_ff: int) -> float:
     cost = user_cost(lens, d, d_ff)
     loads = np.array([cost[s].sum() for s in shards])
     return float(loads.max() / max(loads.mean(), 1e-300))
+
+
+def rank_shard(lens: np.ndarray, ts: np.ndarray, world: int, rank: int, d: int, d_ff: int):
+    """This rank's share of one global batch, as the data-parallel forward runs
+    it: the rank's users (ascending), their rows in the global packed layout,
+    and the sub-batch (lens [n, 4], ts [rows]) the rank packs and processes on
+    its own GPU. Every rank calls it with the same global ``lens`` and ``ts``,
+    so the shards are disjoint and cover the batch; a rank's output rows go
+    back to ``rows`` of the global output."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    lens = np.asarray(lens).reshape(-1, 4)
+    mine = balance_users(lens, world, d, d_ff)[rank]
+    rows = shard_rows(lens, mine)
+    return (mine, rows, np.ascontiguousarray(lens[mine], dtype=np.int32),
+            np.ascontiguousarray(np.asarray(ts)[rows], dtype=np.int64))

@@ -61,6 +61,9 @@ extern "C" {
 #define MTGR_ERR_CAPACITY 4           /* an output or workspace buffer is too small */
 #define MTGR_ERR_TIMEOUT 5            /* device: an internal wait exceeded its limit */
 #define MTGR_ERR_DEVICE_VALIDATION 6  /* device: lengths negative or not summing to T */
+#define MTGR_ERR_RANGE 7              /* device: a value left the range of an f16 intermediate
+                                         (the Q|K|V|U projection or the attention's silu
+                                         weights P, both above 65504 in magnitude) */
 
 /* element types */
 #define MTGR_F32 0
@@ -183,9 +186,14 @@ MTGR_API int mtgr_build_mask_meta(int32_t B, const int32_t* d_seg_off, const int
  *  - q_capacity * kt_capacity must not exceed MTGR_STATIC_META_SCRATCH_BYTES;
  *    larger batches return MTGR_ERR_CAPACITY without touching the device (use
  *    mtgr_build_mask_meta with your own workspace for those).
- *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any
- *    stream capture.
+ *  - The first call in a CUDA context looks up the array's device address
+ *    (once per context, with that context current) and, under CUDA's lazy
+ *    module loading, is also the point where the driver loads the library's
+ *    module and commits the 4 MiB array on that device. Make that first call
+ *    (B = 0 is enough) at start-up, before the caller's memory pool takes the
+ *    device's free memory and before any stream capture. A device reset or a
+ *    new context (e.g. one the caller creates with the driver API) gets its
+ *    own lookup on its first call.
  *  - It never calls cudaMalloc, cudaFree or any allocating routine.
  *  - All calls share the one array per device and it keeps the last call's
  *    contents (every call overwrites what it reads, so nothing needs
@@ -519,6 +527,22 @@ MTGR_API mtgr_timer* mtgr_timer_create(void);
 MTGR_API void mtgr_timer_destroy(mtgr_timer* timer);
 MTGR_API int mtgr_timer_attach(mtgr_timer* timer);
 MTGR_API int mtgr_timer_read(mtgr_timer* timer, double* ms, int64_t* launches);
+
+/*
+ * Self-test of the bounded waits (failure handling, not part of the method):
+ * every internal wait of the library's tensor-core kernels gives up after a
+ * limit, records MTGR_ERR_TIMEOUT in the caller's status word, frees the
+ * kernel's tensor memory and returns, so that a protocol fault can never hang
+ * the GPU. This entry point launches one block of that shape whose waits can
+ * never be satisfied, under the given limit, so the whole wind-down runs:
+ * after the stream is synchronised, *d_status holds MTGR_ERR_TIMEOUT (if it
+ * was 0) and the device stays usable for the next launch.
+ *   limit_ns  per-wait limit in nanoseconds, 1e3 <= limit_ns <= 1e9
+ *             (MTGR_ERR_INVALID_ARG otherwise)
+ *   d_status  device int32 status word
+ */
+MTGR_API int mtgr_selftest_bounded_wait(uint64_t limit_ns, int32_t* d_status,
+                                        mtgr_stream_t stream);
 
 #ifdef __cplusplus
 }

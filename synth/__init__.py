@@ -15,6 +15,7 @@ from .workloads import (  # noqa: F401
     make_stack_params,
     make_qkvu,
     make_workload,
+    assemble_workload,
     bf16_round,
     group_scales,
     sweep_expanded,

@@ -215,6 +215,28 @@ def make_workload(index: int, seed: int = 0, k_override: int | None = None,
     return out
 
 
+def assemble_workload(index: int, lens: np.ndarray, ts: np.ndarray, token_rng: np.random.Generator,
+                      weight_rng: np.random.Generator) -> dict:
+    """A workload of the shape of ``index`` over given lengths and timestamps:
+    token features (or Q|K|V|U) from ``token_rng`` and the layers' weights
+    from ``weight_rng``. Used for one rank's share of a global batch: every
+    rank passes the same weight generator seed, so the weights are identical
+    (replicated) across ranks."""
+    wl = WORKLOADS[index]
+    lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(-1, 4))
+    out = dict(name=wl.name, index=index, kind=wl.kind, seed=None, d=wl.d, H=wl.H,
+               d_ff=wl.d_ff, L=wl.L, dtype=wl.dtype, lens=lens,
+               ts=np.ascontiguousarray(ts, dtype=np.int64), norm=None)
+    if wl.kind == "attention":
+        q = make_qkvu(lens, wl.d, token_rng)
+        out["qkvu"] = bf16_round(q) if wl.dtype == "bf16" else q
+        out["layers"] = []
+    else:
+        out["x"] = make_tokens(lens, wl.d, token_rng)
+        out["layers"] = make_stack_params(wl.L, wl.d, wl.d_ff, weight_rng, wl.dtype)
+    return out
+
+
 def sweep_expanded(wl: dict) -> dict:
     """The K single-candidate rows [U, S, R, c_i] of a one-user workload.
 

@@ -53,3 +53,41 @@ def sample_users(lens, k=4, seed=0):
 
 def to_host(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
+
+
+def _oracle_stack_chunk(args):
+    import oracle
+    x, lens, ts, layers, H, variant = args
+    return oracle.hstu_stack(x, lens, ts, layers, H, variant=variant)
+
+
+def oracle_stack_all_users(w, procs=None, chunk=8, variant=0):
+    """The oracle's stack output for every user of workload ``w``, computed in
+    chunks of users by a pool of single-threaded worker processes. The pool is
+    started with ``spawn`` (a forked child of a process that has used the GPU
+    can hang), and users are independent, so the chunks concatenate to the
+    whole batch's output."""
+    import multiprocessing as mp
+    import os
+    lens = np.asarray(w["lens"]).reshape(-1, 4)
+    n = lens.sum(1)
+    off = np.concatenate([[0], np.cumsum(n)])
+    jobs = []
+    for u0 in range(0, lens.shape[0], chunk):
+        u1 = min(lens.shape[0], u0 + chunk)
+        r0, r1 = int(off[u0]), int(off[u1])
+        jobs.append((w["x"][r0:r1], lens[u0:u1], w["ts"][r0:r1], w["layers"], w["H"], variant))
+    procs = procs or max(1, len(os.sched_getaffinity(0)))
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"  # inherited by the spawned workers: one BLAS thread each
+    try:
+        with mp.get_context("spawn").Pool(procs) as pool:
+            parts = pool.map(_oracle_stack_chunk, jobs)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    return np.concatenate(parts, axis=0)

@@ -84,3 +84,13 @@ def test_cpu_baseline_thread_cap():
     assert r["users"] >= 1 and r["value"] > 0 and r["threads"] >= 1
     r1 = bench.oracle_users_per_s(wl, 0.05, max_threads=1)
     assert r1["threads"] == 1 and r1["value"] > 0
+
+
+def test_tensor_peak_follows_the_timed_region_length():
+    # a short timed region runs at the burst clock: divide by the burst peak;
+    # only seconds-long regions settle at the sustained (power-capped) figure
+    import bench
+    assert bench.tensor_peak_key(0.09) == "bf16_tflops"
+    assert bench.tensor_peak_key(bench.SUSTAINED_AFTER_S - 1e-3) == "bf16_tflops"
+    assert bench.tensor_peak_key(bench.SUSTAINED_AFTER_S) == "bf16_tflops_sustained"
+    assert bench.tensor_peak_key(30.0) == "bf16_tflops_sustained"

@@ -9,7 +9,8 @@ import torch
 
 import oracle
 import synth
-from _util import TOL_BF16, TOL_F32, assert_close_rms, sample_users, to_host, user_rows
+from _util import (TOL_BF16, TOL_F32, assert_close_rms, oracle_stack_all_users, sample_users,
+                   to_host, user_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +73,23 @@ def test_bf16_block_full_workload_sampled_users(block_workload):
     assert_close_rms(y[rows], ref, TOL_BF16, "bf16 block, 512 users")
 
 
+def test_bf16_block_full_workload_every_user(block_workload):
+    # every one of the 512 users (459k tokens) against the oracle, in the
+    # launch configuration the benchmark times: a scheduling fault on any
+    # work item of the persistent attention would show here
+    w = block_workload
+    y = _gpu_stack(w)
+    ref = oracle_stack_all_users(w)
+    assert_close_rms(y, ref, TOL_BF16, "bf16 block, all 512 users")
+    # per user as well: no user's error hides under the batch RMS of others
+    n = w["lens"].sum(1)
+    off = np.concatenate([[0], np.cumsum(n)])
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    worst = max(float(np.abs(y[off[u]:off[u + 1]] - ref[off[u]:off[u + 1]]).max())
+                for u in range(len(n)) if n[u] > 0)
+    assert worst <= TOL_BF16 * rms
+
+
 def test_bf16_stack8_full_workload_sampled_users():
     w = synth.make_workload(3)
     y = _gpu_stack(w)
@@ -82,7 +100,7 @@ def test_bf16_stack8_full_workload_sampled_users():
     assert_close_rms(y[rows], ref, TOL_BF16, "bf16 8-layer stack, 256 users")
 
 
-@pytest.mark.parametrize("K", [1, 8, 64])
+@pytest.mark.parametrize("K", [1, 8, 64, 512])
 def test_candidate_sweep_aggregated_vs_expanded(K):
     w = synth.make_workload(4, k_override=K)
     ex = synth.sweep_expanded(w)

@@ -54,7 +54,13 @@ def _build(batch, lens, static):
             bf["rt_cap"], bf["qtile_desc"], bf["row_ptr"], bf["entries"], bf["order"],
             bf["counts"], bf["rt_cnt"], bf["rt_off"], bf["rt_mask"], bf["work"])
     if static:
+        # every buffer exists before the call: the device's free memory must
+        # not move across it (the fixed array was committed by an earlier call)
+        torch.cuda.synchronize(dev)
+        free0 = torch.cuda.mem_get_info(dev)[0]
         _lib.mtgr_build_mask_meta_static(*args, bf["status"])
+        torch.cuda.synchronize(dev)
+        assert torch.cuda.mem_get_info(dev)[0] == free0, "the static builder changed free device memory"
     else:
         ws = torch.full((max(_lib.mtgr_mask_meta_workspace_bytes(bf["q_cap"], bf["kt_cap"]), 1),),
                         0x5A, dtype=torch.uint8, device=dev)
@@ -73,8 +79,8 @@ def test_static_builder_rejects_oversized_batches_on_the_host():
 
 @pytest.mark.gpu
 def test_static_builder_matches_workspace_builder_on_consecutive_calls():
-    # two calls in a row with different shapes: the second call must not see
-    # anything the first left in the shared scratch array
+    # calls in a row with different shapes: no call may see anything an
+    # earlier one left in the shared scratch array
     cases = []
     for idx, seed in ((3, 1), (2, 2)):
         rng = np.random.default_rng(seed)
@@ -84,6 +90,14 @@ def test_static_builder_matches_workspace_builder_on_consecutive_calls():
     rng = np.random.default_rng(9)
     lens = rng.integers(0, 300, size=(37, 4)).astype(np.int32)
     cases.append((lens, rng.integers(0, 40, size=int(lens.sum())).astype(np.int64)))
+    # a first call on a larger, different batch leaves the shared array dirty
+    # (and commits it on this device), so every compared call starts from
+    # another call's tile codes, never from zeros
+    rng = np.random.default_rng(11)
+    warm_lens = synth.make_lengths(synth.WORKLOADS[3], rng)
+    warm = api.PackedBatch(warm_lens, synth.make_timestamps(warm_lens, rng))
+    warm.check()
+    assert _build(warm, warm_lens, static=True)["status"] == 0
     for lens, ts in cases:
         batch = api.PackedBatch(lens, ts)
         batch.check()
