@@ -55,6 +55,8 @@ from .api import (  # noqa: F401
     group_layernorm,
     hstu_attention,
     hstu_block_forward,
+    hstu_block_forward_train,
+    hstu_block_backward,
     hstu_stack_forward,
     stack_workspace,
 )

@@ -68,6 +68,12 @@ class MtgrBlockParams(ctypes.Structure):
                 ("w2", c_vp), ("b_qkvu", c_vp), ("b1", c_vp), ("b2", c_vp)]
 
 
+class MtgrBlockGrads(ctypes.Structure):
+    _fields_ = [("gln1_gamma", c_vp), ("gln1_beta", c_vp), ("w_qkvu", c_vp), ("b_qkvu", c_vp),
+                ("gln2_gamma", c_vp), ("gln2_beta", c_vp), ("w1", c_vp), ("b1", c_vp),
+                ("w2", c_vp), ("b2", c_vp)]
+
+
 class MtgrTokenMlp(ctypes.Structure):
     _fields_ = [("f", c_i32), ("reserved", c_i32), ("w1", c_vp), ("b1", c_vp), ("w2", c_vp),
                 ("b2", c_vp)]
@@ -128,6 +134,15 @@ _SIGNATURES = {
     "mtgr_timer_read": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_double),
                                        ctypes.POINTER(ctypes.c_int64)]),
     "mtgr_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, c_vp, c_vp]),
+    "mtgr_block_saved_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams)]),
+    "mtgr_hstu_block_fwd_train": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams),
+                                                 ctypes.POINTER(MtgrBatch), c_vp, c_vp, c_vp,
+                                                 c_size, c_vp]),
+    "mtgr_block_bwd_workspace_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams),
+                                                ctypes.POINTER(MtgrBatch)]),
+    "mtgr_hstu_block_bwd": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams),
+                                           ctypes.POINTER(MtgrBatch), c_vp, c_vp, c_vp, c_vp,
+                                           ctypes.POINTER(MtgrBlockGrads), c_vp, c_size, c_vp]),
 }
 
 _lib = None
@@ -311,7 +326,8 @@ def mtgr_candidate_heads(p: MtgrHeadParams, batch: MtgrBatch, k_total: int, d_x,
 
 
 TIMER_CLASSES = ("pack", "mask_meta", "gln", "gemm_qkvu", "attention", "gemm_mlp1", "gemm_mlp2",
-                 "token_mlp", "head_mlp", "rows")
+                 "token_mlp", "head_mlp", "rows", "bwd_gemm", "bwd_wgrad", "bwd_attention",
+                 "bwd_gln", "bwd_rows")
 
 
 class Timer:
@@ -353,3 +369,25 @@ def mtgr_gemm(d_a, d_b, d_bias, epi, d_resid, q_cols, d_out, d_status, stream=No
 def mtgr_selftest_bounded_wait(limit_ns: int, d_status, stream=None) -> None:
     _check("mtgr_selftest_bounded_wait",
            load().mtgr_selftest_bounded_wait(int(limit_ns), _ptr(d_status), _stream(stream)))
+
+
+def mtgr_block_saved_bytes(T: int, p: MtgrBlockParams) -> int:
+    return load().mtgr_block_saved_bytes(T, ctypes.byref(p))
+
+
+def mtgr_hstu_block_fwd_train(p: MtgrBlockParams, batch: MtgrBatch, d_x_in, d_x_out, d_saved,
+                              stream=None) -> None:
+    _check("mtgr_hstu_block_fwd_train", load().mtgr_hstu_block_fwd_train(
+        ctypes.byref(p), ctypes.byref(batch), _ptr(d_x_in), _ptr(d_x_out), _ptr(d_saved),
+        d_saved.numel() * d_saved.element_size(), _stream(stream)))
+
+
+def mtgr_block_bwd_workspace_bytes(T: int, p: MtgrBlockParams, batch: MtgrBatch) -> int:
+    return load().mtgr_block_bwd_workspace_bytes(T, ctypes.byref(p), ctypes.byref(batch))
+
+
+def mtgr_hstu_block_bwd(p: MtgrBlockParams, batch: MtgrBatch, d_x_in, d_saved, d_dy, d_dx,
+                        grads: MtgrBlockGrads, d_ws, stream=None) -> None:
+    _check("mtgr_hstu_block_bwd", load().mtgr_hstu_block_bwd(
+        ctypes.byref(p), ctypes.byref(batch), _ptr(d_x_in), _ptr(d_saved), _ptr(d_dy), _ptr(d_dx),
+        ctypes.byref(grads), _ptr(d_ws), d_ws.numel() * d_ws.element_size(), _stream(stream)))

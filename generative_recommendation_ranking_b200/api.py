@@ -171,6 +171,45 @@ def hstu_block_forward(w: BlockWeights, batch: PackedBatch, x: torch.Tensor, out
     return out
 
 
+GRAD_NAMES = ("gln1_gamma", "gln1_beta", "w_qkvu", "b_qkvu", "gln2_gamma", "gln2_beta", "w1", "b1",
+              "w2", "b2")
+
+
+def hstu_block_forward_train(w: BlockWeights, batch: PackedBatch, x: torch.Tensor, out=None,
+                             saved=None, stream=None):
+    """One HSTU block forward that keeps what its backward reads. Returns
+    (x_out [T, d] float32, saved activations: a uint8 device buffer)."""
+    if out is None:
+        out = torch.empty_like(x)
+    need = _lib.mtgr_block_saved_bytes(batch.T, w.c)
+    if saved is None or saved.numel() < need:
+        saved = _ws(need, x.device)
+    _lib.mtgr_hstu_block_fwd_train(w.c, batch.c, x, out, saved, stream)
+    return out, saved
+
+
+def hstu_block_backward(w: BlockWeights, batch: PackedBatch, x: torch.Tensor, saved: torch.Tensor,
+                        dy: torch.Tensor, bias_grads: bool = True, ws=None, stream=None):
+    """Gradients of one HSTU block for the upstream gradient dy [T, d]
+    (float32): returns (dx [T, d], {parameter name: fp32 gradient}). The
+    bias gradients are computed when ``bias_grads`` (the block's biases may be
+    absent; their gradients are defined all the same)."""
+    dev = x.device
+    d, dff = w.d, w.d_ff
+    shapes = {"gln1_gamma": (4, d), "gln1_beta": (4, d), "w_qkvu": (4 * d, d), "b_qkvu": (4 * d,),
+              "gln2_gamma": (4, d), "gln2_beta": (4, d), "w1": (dff, d), "b1": (dff,),
+              "w2": (d, dff), "b2": (d,)}
+    grads = {k: torch.empty(v, dtype=torch.float32, device=dev) for k, v in shapes.items()
+             if bias_grads or not k.startswith("b")}
+    c = _lib.MtgrBlockGrads(**{k: (grads[k].data_ptr() if k in grads else None) for k in GRAD_NAMES})
+    dx = torch.empty_like(x)
+    need = _lib.mtgr_block_bwd_workspace_bytes(batch.T, w.c, batch.c)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, dev)
+    _lib.mtgr_hstu_block_bwd(w.c, batch.c, x, saved, dy, dx, c, ws, stream)
+    return dx, grads
+
+
 def stack_workspace(layers, batch: PackedBatch) -> torch.Tensor:
     return _ws(_lib.mtgr_stack_workspace_bytes(batch.T, [l.c for l in layers]), batch.device)
 

@@ -24,7 +24,8 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG_DIR, "libmtgr.so")
 
 SOURCES = ["api.cu", "pack_meta.cu", "gln.cu", "simt.cu", "gemm_tc.cu", "attn_tc.cu", "tmap.cu", "timer.cu",
-           "meta_static.cu", "tokens.cu", "selftest.cu"]
+           "meta_static.cu", "tokens.cu", "selftest.cu",
+           "backward.cu", "attn_bwd_tc.cu", "gemm_wgrad.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -44,9 +44,33 @@ int launch_gather_rows16(int32_t n, int32_t d, const void* src, int32_t src_rows
 int launch_head_dot(int32_t n, int32_t n_tasks, int32_t d_h, const void* h, const float* w2,
                     const float* b2, float* out, cudaStream_t s);
 int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu, float* g,
-                    cudaStream_t s);
+                    cudaStream_t s, float* obar = nullptr);
 int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
-                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s);
+                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s,
+                   void* obar = nullptr);
+int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
+                       void* aux, void* out, int32_t* status, cudaStream_t s);
+int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const void* b,
+                      int64_t ldb, float* out, bool accumulate, int32_t* status, cudaStream_t s);
+int launch_gln_bwd(int32_t T, int32_t d, bool bf16, const void* x, const float* dy,
+                   const int8_t* gid, int32_t G, const float* gamma, float eps, float* dgamma,
+                   float* dbeta, float* dx, const float* dres, const void* qkvu, const void* obar,
+                   void* dobar, void* dz, int32_t* status, cudaStream_t s);
+int launch_tile_csc(const mtgr_batch* bt, int32_t* csc_ptr, int32_t* csc, cudaStream_t s);
+int launch_cvt_bf16(int64_t n, const float* x, void* y, cudaStream_t s);
+int launch_cvt_cols_bf16(int32_t T, int32_t d, const float* x, int32_t ld_out, void* out,
+                         cudaStream_t s);
+int launch_transpose16(int32_t R, int32_t C, const void* in, void* out, cudaStream_t s);
+int launch_colsum(int32_t T, int32_t N, bool bf16, const void* x, int32_t ld, float* out,
+                  cudaStream_t s);
+int launch_gemm_f32_strided(int M, int N, int K, const float* a, int64_t sam, int64_t sak,
+                            const float* b, int64_t sbk, int64_t sbn, int epi, const float* aux,
+                            float* c, cudaStream_t s);
+int launch_attn_bwd_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu,
+                        const float* dobar, float* dz, cudaStream_t s);
+int launch_attn_bwd_tc(const mtgr_batch* bt, int32_t d, int32_t H, const void* qkvu,
+                       const void* dobar, const int32_t* csc_ptr, const int32_t* csc, float* dq,
+                       void* dz, cudaStream_t s);
 }  // namespace mtgr
 
 using namespace mtgr;
@@ -242,6 +266,289 @@ int block_fwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
   return launch_gemm_f32(T, d, dff, static_cast<const float*>(w.h),
                          static_cast<const float*>(p->w2), p->b2, MTGR_EPI_RESID, x_in, 0,
                          MTGR_F32, x_out, s);
+}
+
+// ------------------------------------------------------------- training --
+// Activations the backward reads, kept by the training forward.
+struct SavedAct {
+  void* xt;    // GroupLN_1 output [T][d]
+  void* qkvu;  // [T][4d] (bf16 blocks: f16, Q halved)
+  void* obar;  // O / N [T][d]
+  void* g;     // G = O / N (.) U [T][d]
+  void* gt;    // GroupLN_2 output [T][d]
+  void* z1;    // MLP pre-activation [T][d_ff]
+  void* h;     // silu(z1) [T][d_ff]
+  size_t bytes;
+};
+
+SavedAct saved_layout(int32_t T, const mtgr_block_params* p, void* base) {
+  const size_t e = p->dtype == MTGR_BF16 ? 2 : 4;
+  const size_t t = (size_t)T, d = (size_t)p->d, f = (size_t)p->d_ff;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  SavedAct w;
+  size_t off = 0;
+  w.xt = b + off;   off += align_up(t * d * e, 256);
+  w.qkvu = b + off; off += align_up(t * 4 * d * e, 256);
+  w.obar = b + off; off += align_up(t * d * e, 256);
+  w.g = b + off;    off += align_up(t * d * e, 256);
+  w.gt = b + off;   off += align_up(t * d * e, 256);
+  w.z1 = b + off;   off += align_up(t * f * e, 256);
+  w.h = b + off;    off += align_up(t * f * e, 256);
+  w.bytes = off;
+  return w;
+}
+
+// Backward workspace.
+struct BwdWs {
+  void* dyb;     // bf16 dY [T][d]
+  void* w2t;     // bf16 W2^T [d_ff][d]
+  void* w1t;     // bf16 W1^T [d][d_ff]
+  void* wt;      // bf16 W^T [d][4d]
+  void* dz1;     // dZ1 [T][d_ff] (bf16 or fp32)
+  float* dgt;    // dG~, then dX~ [T][d] fp32
+  void* dobar;   // dO~ [T][d] (f16 or fp32)
+  void* dz;      // dZ = [dQ|dK|dV|dU] [T][4d] (bf16 or fp32)
+  float* dq;     // fp32 dQ accumulator [T][d] (bf16 blocks)
+  int32_t* csc_ptr;  // [q_cap + 1]
+  int32_t* csc;      // [q_cap * kt_cap]
+  size_t bytes;
+};
+
+BwdWs bwd_layout(int32_t T, const mtgr_block_params* p, const mtgr_batch* bt, void* base) {
+  const bool bf = p->dtype == MTGR_BF16;
+  const size_t e = bf ? 2 : 4;
+  const size_t t = (size_t)T, d = (size_t)p->d, f = (size_t)p->d_ff;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  BwdWs w{};
+  size_t off = 0;
+  if (bf) {
+    w.dyb = b + off; off += align_up(t * d * 2, 256);
+    w.w2t = b + off; off += align_up(f * d * 2, 256);
+    w.w1t = b + off; off += align_up(d * f * 2, 256);
+    w.wt = b + off;  off += align_up(d * 4 * d * 2, 256);
+  }
+  w.dz1 = b + off;   off += align_up(t * f * e, 256);
+  w.dgt = reinterpret_cast<float*>(b + off); off += align_up(t * d * 4, 256);
+  w.dobar = b + off; off += align_up(t * d * e, 256);
+  w.dz = b + off;    off += align_up(t * 4 * d * e, 256);
+  if (bf) {
+    w.dq = reinterpret_cast<float*>(b + off); off += align_up(t * d * 4, 256);
+    const size_t q = bt ? (size_t)bt->q_capacity : 0, kt = bt ? (size_t)bt->kt_capacity : 0;
+    w.csc_ptr = reinterpret_cast<int32_t*>(b + off); off += align_up((q + 1) * 4, 256);
+    w.csc = reinterpret_cast<int32_t*>(b + off);     off += align_up((q * kt > 0 ? q * kt : 1) * 4, 256);
+  }
+  w.bytes = off;
+  return w;
+}
+
+int train_check(const mtgr_block_params* p, const mtgr_batch* bt) {
+  const int rc = params_check(p);
+  if (rc != MTGR_OK) return rc;
+  if (p->variant != 0) return MTGR_ERR_UNSUPPORTED;
+  if (p->d > 1024) return MTGR_ERR_UNSUPPORTED;  // GroupLN backward holds a row per warp
+  if (!batch_ok(bt)) return MTGR_ERR_INVALID_ARG;
+  if (p->dtype == MTGR_BF16 && bt->T > 0 && !device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  return MTGR_OK;
+}
+
+int block_fwd_train(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_in,
+                    float* x_out, const SavedAct& sv, cudaStream_t s) {
+  const int32_t T = bt->T, d = p->d, H = p->H, dff = p->d_ff;
+  if (T == 0) return MTGR_OK;
+  int rc;
+  const bool bf = p->dtype == MTGR_BF16;
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(T, d, MTGR_F32, x_in, bt->group_id, 4, p->gln1_gamma, p->gln1_beta,
+                         p->eps, bf ? MTGR_BF16 : MTGR_F32, sv.xt, s)) != MTGR_OK)
+      return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GEMM_QKVU, s, 1);
+    rc = bf ? launch_gemm_tc(T, 4 * d, d, sv.xt, p->w_qkvu, p->b_qkvu, MTGR_EPI_NONE, nullptr, d,
+                             MTGR_F16, sv.qkvu, bt->status, s)
+            : launch_gemm_f32(T, 4 * d, d, static_cast<const float*>(sv.xt),
+                              static_cast<const float*>(p->w_qkvu), p->b_qkvu, MTGR_EPI_NONE,
+                              nullptr, 0, MTGR_F32, sv.qkvu, s);
+    if (rc != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
+    rc = bf ? launch_attn_tc(bt, d, H, MTGR_F16, true, sv.qkvu, MTGR_BF16, sv.g, s, sv.obar)
+            : launch_attn_f32(bt, d, H, static_cast<const float*>(sv.qkvu),
+                              static_cast<float*>(sv.g), s, static_cast<float*>(sv.obar));
+    if (rc != MTGR_OK) return rc;
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GLN, s, 1);
+    if ((rc = launch_gln(T, d, bf ? MTGR_BF16 : MTGR_F32, sv.g, bt->group_id, 4, p->gln2_gamma,
+                         p->gln2_beta, p->eps, bf ? MTGR_BF16 : MTGR_F32, sv.gt, s)) != MTGR_OK)
+      return rc;
+  }
+  if (bf) {
+    {
+      TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 1);
+      if ((rc = launch_gemm_tc_aux(T, dff, d, sv.gt, p->w1, p->b1, kEpiSilu2, sv.z1, sv.h,
+                                   bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
+    return launch_gemm_tc(T, d, dff, sv.h, p->w2, p->b2, MTGR_EPI_RESID, x_in, 0, MTGR_F32, x_out,
+                          bt->status, s);
+  }
+  {
+    TimedScope tsc(MTGR_TIMER_GEMM_MLP1, s, 2);
+    const float* gt = static_cast<const float*>(sv.gt);
+    const float* w1 = static_cast<const float*>(p->w1);
+    if ((rc = launch_gemm_f32(T, dff, d, gt, w1, p->b1, MTGR_EPI_NONE, nullptr, 0, MTGR_F32, sv.z1,
+                              s)) != MTGR_OK ||
+        (rc = launch_gemm_f32(T, dff, d, gt, w1, p->b1, MTGR_EPI_SILU, nullptr, 0, MTGR_F32, sv.h,
+                              s)) != MTGR_OK)
+      return rc;
+  }
+  TimedScope tsc(MTGR_TIMER_GEMM_MLP2, s, 1);
+  return launch_gemm_f32(T, d, dff, static_cast<const float*>(sv.h),
+                         static_cast<const float*>(p->w2), p->b2, MTGR_EPI_RESID, x_in, 0, MTGR_F32,
+                         x_out, s);
+}
+
+int block_bwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_in,
+              const SavedAct& sv, const float* dy, float* dx, const mtgr_block_grads* gr,
+              const BwdWs& w, cudaStream_t s) {
+  const int32_t T = bt->T, d = p->d, H = p->H, dff = p->d_ff;
+  int rc;
+  if (p->dtype == MTGR_BF16) {
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_ROWS, s, 4);
+      if ((rc = launch_cvt_bf16((int64_t)T * d, dy, w.dyb, s)) != MTGR_OK ||
+          (rc = launch_transpose16(d, dff, p->w2, w.w2t, s)) != MTGR_OK ||
+          (rc = launch_transpose16(dff, d, p->w1, w.w1t, s)) != MTGR_OK ||
+          (rc = launch_transpose16(4 * d, d, p->w_qkvu, w.wt, s)) != MTGR_OK)
+        return rc;
+    }
+    {  // dW2 = dY^T H
+      TimedScope tsc(MTGR_TIMER_BWD_WGRAD, s, 1);
+      if ((rc = launch_gemm_wgrad(d, dff, T, w.dyb, d, sv.h, dff, gr->w2, false, bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    {  // dZ1 = (dY W2) (.) silu'(Z1)
+      TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);
+      if ((rc = launch_gemm_tc_aux(T, dff, d, w.dyb, w.w2t, nullptr, kEpiDSilu, sv.z1, w.dz1,
+                                   bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    {  // dW1 = dZ1^T G~
+      TimedScope tsc(MTGR_TIMER_BWD_WGRAD, s, 1);
+      if ((rc = launch_gemm_wgrad(dff, d, T, w.dz1, dff, sv.gt, d, gr->w1, false, bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    {  // dG~ = dZ1 W1
+      TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);
+      if ((rc = launch_gemm_tc(T, d, dff, w.dz1, w.w1t, nullptr, MTGR_EPI_NONE, nullptr, 0, MTGR_F32,
+                               w.dgt, bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    {  // GroupLN_2 and the gate: dO~ (f16), dU into dZ
+      TimedScope tsc(MTGR_TIMER_BWD_GLN, s, 1);
+      if ((rc = launch_gln_bwd(T, d, true, sv.g, w.dgt, bt->group_id, 4, p->gln2_gamma, p->eps,
+                               gr->gln2_gamma, gr->gln2_beta, nullptr, nullptr, sv.qkvu, sv.obar,
+                               w.dobar, w.dz, bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    {  // attention: dK, dV into dZ; dQ through the fp32 accumulator
+      TimedScope tsc(MTGR_TIMER_BWD_ATTENTION, s, 2);
+      if (cudaMemsetAsync(w.dq, 0, (size_t)T * d * sizeof(float), s) != cudaSuccess) return MTGR_ERR_CUDA;
+      if ((rc = launch_tile_csc(bt, w.csc_ptr, w.csc, s)) != MTGR_OK ||
+          (rc = launch_attn_bwd_tc(bt, d, H, sv.qkvu, w.dobar, w.csc_ptr, w.csc, w.dq, w.dz, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_ROWS, s, 1);
+      if ((rc = launch_cvt_cols_bf16(T, d, w.dq, 4 * d, w.dz, s)) != MTGR_OK) return rc;
+    }
+    {  // dW = dZ^T X~
+      TimedScope tsc(MTGR_TIMER_BWD_WGRAD, s, 1);
+      if ((rc = launch_gemm_wgrad(4 * d, d, T, w.dz, 4 * d, sv.xt, d, gr->w_qkvu, false, bt->status,
+                                  s)) != MTGR_OK)
+        return rc;
+    }
+    {  // dX~ = dZ W
+      TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);
+      if ((rc = launch_gemm_tc(T, d, 4 * d, w.dz, w.wt, nullptr, MTGR_EPI_NONE, nullptr, 0, MTGR_F32,
+                               w.dgt, bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+  } else {
+    const float* dzf = static_cast<const float*>(w.dz);
+    const float* dz1f = static_cast<const float*>(w.dz1);
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_WGRAD, s, 1);  // dW2 = dY^T H
+      if ((rc = launch_gemm_f32_strided(d, dff, T, dy, 1, d, static_cast<const float*>(sv.h), dff,
+                                        1, MTGR_EPI_NONE, nullptr, gr->w2, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);  // dZ1 = (dY W2) (.) silu'(Z1)
+      if ((rc = launch_gemm_f32_strided(T, dff, d, dy, d, 1, static_cast<const float*>(p->w2), dff, 1,
+                                        kEpiDSilu, static_cast<const float*>(sv.z1),
+                                        static_cast<float*>(w.dz1), s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_WGRAD, s, 1);  // dW1 = dZ1^T G~
+      if ((rc = launch_gemm_f32_strided(dff, d, T, dz1f, 1, dff, static_cast<const float*>(sv.gt), d,
+                                        1, MTGR_EPI_NONE, nullptr, gr->w1, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);  // dG~ = dZ1 W1
+      if ((rc = launch_gemm_f32_strided(T, d, dff, dz1f, dff, 1, static_cast<const float*>(p->w1), d,
+                                        1, MTGR_EPI_NONE, nullptr, w.dgt, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_GLN, s, 1);
+      if ((rc = launch_gln_bwd(T, d, false, sv.g, w.dgt, bt->group_id, 4, p->gln2_gamma, p->eps,
+                               gr->gln2_gamma, gr->gln2_beta, nullptr, nullptr, sv.qkvu, sv.obar,
+                               w.dobar, w.dz, bt->status, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_ATTENTION, s, 2);
+      if ((rc = launch_attn_bwd_f32(bt, d, H, static_cast<const float*>(sv.qkvu),
+                                    static_cast<const float*>(w.dobar), static_cast<float*>(w.dz),
+                                    s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_WGRAD, s, 1);  // dW = dZ^T X~
+      if ((rc = launch_gemm_f32_strided(4 * d, d, T, dzf, 1, 4 * d, static_cast<const float*>(sv.xt),
+                                        d, 1, MTGR_EPI_NONE, nullptr, gr->w_qkvu, s)) != MTGR_OK)
+        return rc;
+    }
+    {
+      TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);  // dX~ = dZ W
+      if ((rc = launch_gemm_f32_strided(T, d, 4 * d, dzf, 4 * d, 1,
+                                        static_cast<const float*>(p->w_qkvu), d, 1, MTGR_EPI_NONE,
+                                        nullptr, w.dgt, s)) != MTGR_OK)
+        return rc;
+    }
+  }
+  {  // GroupLN_1 and the residual: dX = GLN_1 backward of dX~ + dY
+    TimedScope tsc(MTGR_TIMER_BWD_GLN, s, 1);
+    if ((rc = launch_gln_bwd(T, d, false, x_in, w.dgt, bt->group_id, 4, p->gln1_gamma, p->eps,
+                             gr->gln1_gamma, gr->gln1_beta, dx, dy, nullptr, nullptr, nullptr,
+                             nullptr, bt->status, s)) != MTGR_OK)
+      return rc;
+  }
+  const bool bf = p->dtype == MTGR_BF16;
+  TimedScope tsc(MTGR_TIMER_BWD_ROWS, s,
+                 (gr->b2 != nullptr) + (gr->b1 != nullptr) + (gr->b_qkvu != nullptr));
+  if (gr->b2 != nullptr && (rc = launch_colsum(T, d, false, dy, d, gr->b2, s)) != MTGR_OK) return rc;
+  if (gr->b1 != nullptr && (rc = launch_colsum(T, dff, bf, w.dz1, dff, gr->b1, s)) != MTGR_OK) return rc;
+  if (gr->b_qkvu != nullptr && (rc = launch_colsum(T, 4 * d, bf, w.dz, 4 * d, gr->b_qkvu, s)) != MTGR_OK)
+    return rc;
+  return MTGR_OK;
 }
 
 }  // namespace
@@ -844,6 +1151,54 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
   if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
   return launch_gemm_tc(M, N, K, d_a, d_b, d_bias, epi, d_resid, q_cols, out_dtype, d_out,
                         d_status, as_stream(stream));
+}
+
+MTGR_API size_t mtgr_block_saved_bytes(int32_t T, const mtgr_block_params* p) {
+  if (T < 0 || params_check(p) != MTGR_OK) return 0;
+  return saved_layout(T, p, nullptr).bytes;
+}
+
+MTGR_API int mtgr_hstu_block_fwd_train(const mtgr_block_params* p, const mtgr_batch* batch,
+                                       const float* d_x_in, float* d_x_out, void* d_saved,
+                                       size_t saved_bytes, mtgr_stream_t stream) {
+  int rc = train_check(p, batch);
+  if (rc != MTGR_OK) return rc;
+  if (batch->T > 0 && (batch->group_id == nullptr || d_x_in == nullptr || d_x_out == nullptr ||
+                       d_saved == nullptr))
+    return MTGR_ERR_INVALID_ARG;
+  if (d_x_in == d_x_out && batch->T > 0) return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x_in) || !aligned16(d_x_out) || !aligned16(d_saved)) return MTGR_ERR_INVALID_ARG;
+  const SavedAct sv = saved_layout(batch->T, p, d_saved);
+  if (saved_bytes < sv.bytes) return MTGR_ERR_CAPACITY;
+  return block_fwd_train(p, batch, d_x_in, d_x_out, sv, as_stream(stream));
+}
+
+MTGR_API size_t mtgr_block_bwd_workspace_bytes(int32_t T, const mtgr_block_params* p,
+                                               const mtgr_batch* batch) {
+  if (T < 0 || params_check(p) != MTGR_OK) return 0;
+  return bwd_layout(T, p, batch, nullptr).bytes;
+}
+
+MTGR_API int mtgr_hstu_block_bwd(const mtgr_block_params* p, const mtgr_batch* batch,
+                                 const float* d_x_in, const void* d_saved, const float* d_dy,
+                                 float* d_dx, const mtgr_block_grads* grads, void* d_ws,
+                                 size_t ws_bytes, mtgr_stream_t stream) {
+  int rc = train_check(p, batch);
+  if (rc != MTGR_OK) return rc;
+  if (grads == nullptr || grads->gln1_gamma == nullptr || grads->gln1_beta == nullptr ||
+      grads->w_qkvu == nullptr || grads->gln2_gamma == nullptr || grads->gln2_beta == nullptr ||
+      grads->w1 == nullptr || grads->w2 == nullptr)
+    return MTGR_ERR_INVALID_ARG;
+  if (batch->T > 0 && (batch->group_id == nullptr || d_x_in == nullptr || d_saved == nullptr ||
+                       d_dy == nullptr || d_dx == nullptr || d_ws == nullptr))
+    return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_x_in) || !aligned16(d_saved) || !aligned16(d_dy) || !aligned16(d_dx) ||
+      !aligned16(d_ws))
+    return MTGR_ERR_INVALID_ARG;
+  const BwdWs w = bwd_layout(batch->T, p, batch, d_ws);
+  if (ws_bytes < w.bytes) return MTGR_ERR_CAPACITY;
+  return block_bwd(p, batch, d_x_in, saved_layout(batch->T, p, const_cast<void*>(d_saved)), d_dy,
+                   d_dx, grads, w, as_stream(stream));
 }
 
 }  // extern "C"

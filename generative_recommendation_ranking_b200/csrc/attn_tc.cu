@@ -52,6 +52,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "mask_tile.cuh"
 #include "ptx.cuh"
 #include "tmap.h"
 
@@ -95,6 +96,7 @@ struct AttnArgs {
   int32_t q_cap;
   void* out;  // [T][d] f32 or bf16
   int32_t* status;
+  uint16_t* obar;  // optional [T][d] bf16: O / N before the gate (training forward)
 };
 
 struct Item {
@@ -146,39 +148,6 @@ struct UnionCursor {
     return kt;
   }
 };
-
-// bits [lo, hi) of a 64-bit mask, clipped to [0, 64)
-__device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
-  lo = lo < 0 ? 0 : lo;
-  hi = hi > 64 ? 64 : hi;
-  if (hi <= lo) return 0ull;
-  const uint64_t m = (hi - lo == 64) ? ~0ull : ((1ull << (hi - lo)) - 1ull);
-  return m << lo;
-}
-
-// Rule 2 as a table lookup: the rank-table word of query row i (rank-table
-// index cnt_i) for keys [j0, j0 + 64) (user-relative, j0 a multiple of 64),
-// or 0 where that range holds no R key. Issued a k-tile ahead of its use.
-__device__ __forceinline__ uint64_t rt_word(const mtgr_work_item& it, const uint64_t* rt_mask,
-                                            int32_t cnt_i, int32_t j0) {
-  const int32_t n_r = it.c_lo - it.n_us;
-  if (n_r > 0 && j0 + 64 > it.n_us && j0 < it.c_lo) {
-    const int32_t gidx = j0 / 64 - it.n_us / 64;
-    return __ldg(rt_mask + it.rt_base + (int64_t)gidx * (n_r + 1) + cnt_i);
-  }
-  return 0ull;
-}
-
-// Visibility of keys [j0, j0 + 64) to query row i from the three rules, rule
-// 2 given by its rank-table word rt. Exact for FULL, PARTIAL and EMPTY tiles
-// alike.
-__device__ __forceinline__ uint64_t visible_bits(const mtgr_work_item& it, uint64_t rt, int32_t i,
-                                                 int32_t j0) {
-  uint64_t vis = range_bits(0, it.n_us - j0) | rt;  // rule 1: U and S keys; rule 2
-  const int dc = i - j0;  // the diagonal: every token sees itself (rules 1-3)
-  if (dc >= 0 && dc < 64) vis |= 1ull << dc;
-  return vis & range_bits(0, it.n - j0);  // keys past the user's end
-}
 
 // Keep-mask of one f16 pair from its two visibility bits (bit 0: low half).
 __device__ __forceinline__ uint32_t pair_mask(uint32_t bits) {
@@ -439,8 +408,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int32_t code = q == 0 ? ca : cb;  // -1: EMPTY for this q-tile
         masked_n = code < 0 || (code & 1) || kt_n * TN + TN > it.w.n;
         if (masked_n) {
-          rt_lo_n = rt_word(it.w, a.rt_mask, cnt_i, kt_n * TN);
-          rt_hi_n = rt_word(it.w, a.rt_mask, cnt_i, kt_n * TN + 64);
+          rt_lo_n = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN);
+          rt_hi_n = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN + 64);
         }
       };
       fetch();
@@ -457,8 +426,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         {
           uint64_t vis_lo = 0, vis_hi = 0;
           if (masked) {
-            vis_lo = visible_bits(it.w, rt_lo, i, kt * TN);
-            vis_hi = visible_bits(it.w, rt_hi, i, kt * TN + 64);
+            vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
+            vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
           }
           uint32_t sa[16], sb[16];
           tmem_ld16(s_addr, sa);
@@ -596,6 +565,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ov[2 * c] = __uint_as_float(r0) * inv_n * u0;
               ov[2 * c + 1] = __uint_as_float(r1) * inv_n * u1;
             }
+            if (a.obar != nullptr) {
+              uint32_t w[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int col = 8 * k + 2 * c;
+                const float x0 = __uint_as_float(col < 32 ? o0[col] : o1[col - 32]);
+                const float x1 = __uint_as_float(col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32]);
+                w[c] = cvt_bf16x2(x0 * inv_n, x1 * inv_n);
+              }
+              *reinterpret_cast<uint4*>(a.obar + row * d + it.h * DH + 8 * k) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
             if (OUT_F32) {
               float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * d + it.h * DH + 8 * k);
               op[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
@@ -631,13 +611,14 @@ int launch_t(const CUtensorMap& tm, const AttnArgs& a, int grid, cudaStream_t s)
 
 // qkvu [T][4d] of 16-bit elements (bf16 or f16), dh = 64.
 int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
-                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s) {
+                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s, void* obar) {
   if (bt->q_capacity == 0 || bt->T == 0) return MTGR_OK;
   CUtensorMap tm;
   int rc = make_tmap_2d_16b(&tm, qkvu, (uint64_t)4 * d, (uint64_t)bt->T, (uint64_t)8 * d, DH, TM);
   if (rc != MTGR_OK) return rc;
   AttnArgs a{d, H, static_cast<const uint16_t*>(qkvu), bt->entries, bt->work, bt->counts,
-             bt->rt_cnt, bt->rt_mask, bt->norm, bt->q_capacity, out, bt->status};
+             bt->rt_cnt, bt->rt_mask, bt->norm, bt->q_capacity, out, bt->status,
+             static_cast<uint16_t*>(obar)};
   const int64_t items = (int64_t)bt->q_capacity * H;
   const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
   const bool f32 = out_dtype == MTGR_F32;

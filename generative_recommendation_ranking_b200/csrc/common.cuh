@@ -17,6 +17,13 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;
 // batch accepts: users of up to 4096 * 128 tokens.
 constexpr int32_t kMaxKtCapacity = 4096;
 
+// Internal GEMM epilogue forms of the backward pass, beside the public
+// MTGR_EPI_* ones: out = acc (.) silu'(aux) with aux the saved pre-activation
+// (bf16), and the training forward's MLP1, which writes silu(z) to out and
+// z = acc + bias to aux.
+constexpr int kEpiDSilu = 16;
+constexpr int kEpiSilu2 = 17;
+
 // Record a device-side error; the first error wins.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);

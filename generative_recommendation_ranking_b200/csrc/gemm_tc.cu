@@ -92,9 +92,60 @@ __device__ __forceinline__ void epilogue_math(const GemmArgs& a, int col0, const
   }
 }
 
+// silu'(z) = s (1 + z (1 - s)), s = sigmoid(z) = (1 + tanh(z / 2)) / 2
+__device__ __forceinline__ float silu_grad_fast(float z) {
+  const float s = fmaf(0.5f, tanh_approx_f32(0.5f * z), 0.5f);
+  return s * fmaf(z, 1.0f - s, 1.0f);
+}
+
+// Backward of the MLP's SiLU: dZ1 = dH (.) silu'(Z1) for 32 columns of one
+// row, Z1 read from the staging block (bf16, as the TMA load left it) and
+// the result written over it.
+__device__ __forceinline__ void epilogue_dsilu(const uint32_t (&acc)[32], uint8_t* stg, int r) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4* p = reinterpret_cast<uint4*>(stg + stg_off<MTGR_BF16>(r, c));
+    const uint4 z4 = *p;
+    const uint32_t zw[4] = {z4.x, z4.y, z4.z, z4.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float z0 = __uint_as_float(zw[k] << 16), z1 = __uint_as_float(zw[k] & 0xffff0000u);
+      const float g0 = u32_as_f(acc[8 * c + 2 * k]) * silu_grad_fast(z0);
+      const float g1 = u32_as_f(acc[8 * c + 2 * k + 1]) * silu_grad_fast(z1);
+      w[k] = cvt_bf16x2(g0, g1);
+    }
+    *p = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Training forward's MLP1: z = acc + bias to the staging block `zst` and
+// silu(z) to `hst` (both bf16).
+__device__ __forceinline__ void epilogue_silu2(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
+                                               uint8_t* zst, uint8_t* hst, int r) {
+  float v[32];
+  epilogue_math<MTGR_EPI_NONE, MTGR_BF16>(a, col0, acc, v);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t wz[4], wh[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = v[8 * c + 2 * k], hi = v[8 * c + 2 * k + 1];
+      wz[k] = cvt_bf16x2(lo, hi);
+      wh[k] = cvt_bf16x2(silu_fast(lo), silu_fast(hi));
+    }
+    *reinterpret_cast<uint4*>(zst + stg_off<MTGR_BF16>(r, c)) = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+    *reinterpret_cast<uint4*>(hst + stg_off<MTGR_BF16>(r, c)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+  }
+}
+
 template <int EPI, int OUT>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
                                                uint8_t* stg, int r) {
+  if constexpr (EPI == kEpiDSilu) {
+    epilogue_dsilu(acc, stg, r);
+    return;
+  }
   float v[32];
   epilogue_math<EPI, OUT>(a, col0, acc, v);
   if (OUT == MTGR_F16) {
@@ -183,7 +234,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmO);
-    if (EPI == MTGR_EPI_RESID) tma_prefetch_desc(&tmR);
+    if (EPI == MTGR_EPI_RESID || EPI == kEpiDSilu || EPI == kEpiSilu2) tma_prefetch_desc(&tmR);
     for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&rbar[i], 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -299,19 +350,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           prev_scatter = !run;
           continue;
         }
+        if constexpr (EPI == kEpiSilu2) {
+          // two outputs per block: z through tmR from buffer 0, silu(z)
+          // through tmO from buffer 1, once both earlier stores have read them
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          uint32_t r[32];
+          tmem_ld32(t_row + c * 32, r);
+          tmem_ld_wait();
+          epilogue_silu2(args, col0, r, stg, stg + STG_BYTES, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmR, stg, col0, row0);
+            tma_store_2d(&tmO, stg + STG_BYTES, col0, row0);
+            bulk_commit_group();
+          }
+          continue;
+        }
         uint8_t* sb = stg + buf * STG_BYTES;
         // the TMA store that last read this buffer (two blocks ago) must be done
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
-        if (EPI == MTGR_EPI_RESID && lane == 0) {
-          mbar_arrive_expect_tx(&rbar[2 * ew + buf], STG_BYTES);
+        // a second input block arrives by TMA into the staging block: the
+        // fp32 residual, or the bf16 pre-activation of the SiLU backward
+        constexpr bool kAuxIn = EPI == MTGR_EPI_RESID || EPI == kEpiDSilu;
+        constexpr uint32_t kAuxBytes = EPI == MTGR_EPI_RESID ? STG_BYTES : STG_BYTES / 2;
+        if (kAuxIn && lane == 0) {
+          mbar_arrive_expect_tx(&rbar[2 * ew + buf], kAuxBytes);
           tma_load_2d(&tmR, &rbar[2 * ew + buf], sb, col0, row0);
         }
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        if (EPI == MTGR_EPI_RESID &&
-            !__all_sync(0xffffffffu, mbar_wait(&rbar[2 * ew + buf], (chunk >> 1) & 1))) {
+        if (kAuxIn && !__all_sync(0xffffffffu, mbar_wait(&rbar[2 * ew + buf], (chunk >> 1) & 1))) {
           timed_out = true;
           break;
         }
@@ -386,6 +458,29 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
   if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_SILU, MTGR_BF16>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, to, tr, args, s);
+  return MTGR_ERR_UNSUPPORTED;
+}
+
+// The backward pass's forms (bf16 a [M][K], b [N][K]; aux and out bf16 [M][N]):
+//   kEpiDSilu: out = (a b^T) (.) silu'(aux)
+//   kEpiSilu2: aux = a b^T + bias, out = silu(aux)
+int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
+                       void* aux, void* out, int32_t* status, cudaStream_t s) {
+  if (M == 0 || N == 0) return MTGR_OK;
+  CUtensorMap ta, tb, to, tr;
+  int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N, (uint64_t)M,
+                    (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d(&tr, aux, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N, (uint64_t)M,
+                    (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc != MTGR_OK) return rc;
+  GemmArgs args{M, N, K, bias, nullptr, out, 0, status, nullptr, 0};
+  if (epi == kEpiDSilu) return launch_t<kEpiDSilu, MTGR_BF16>(ta, tb, to, tr, args, s);
+  if (epi == kEpiSilu2) return launch_t<kEpiSilu2, MTGR_BF16>(ta, tb, to, tr, args, s);
   return MTGR_ERR_UNSUPPORTED;
 }
 

@@ -1,0 +1,264 @@
+// Weight-gradient GEMM of the HSTU block's backward pass on tcgen05 tensor
+// cores: a reduction over the tokens of two activation matrices,
+//
+//   out[m][n] (+)= sum_t a[t][m] b[t][n]      (a [T][M], b [T][N] bf16, out fp32)
+//
+// e.g. dW = dZ^T X~ for a Linear layer Z = X~ W^T (summary page, "Method": the
+// block's projections; their gradients by the chain rule). Both operands are
+// read as they lie in memory, token-major, so the UMMA takes them MN-major:
+// TMA boxes of 64 output columns x 64 tokens (128-byte swizzle) give each
+// operand in blocks of 64 contiguous m (or n) values, LBO = 8 KB apart, with
+// 8-token groups SBO = 1 KB apart.
+//
+// The reduction dimension (T, hundreds of thousands of tokens) is far longer
+// than the output has tiles (a 2048 x 512 gradient is 32 tiles of 128 x 256),
+// so the work is split "stream-K": the (tile, 64-token block) space is cut
+// into one contiguous range per CTA, and each CTA adds every partial tile it
+// finishes into the fp32 output with TMA reduce-add stores
+// (cp.reduce.async.bulk.tensor ... .add). The caller zeroes the output first
+// unless it accumulates. Roles as in the block's forward GEMM: warp 0 TMA
+// producer, one thread of warp 1 issues the MMAs, warps 2-5 drain the
+// double-buffered TMEM accumulator.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace mtgr {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BOX = 64;                     // MN values per TMA box (128 bytes)
+constexpr int BOX_BYTES = BOX * BK * 2;     // 8 KB
+constexpr int A_BYTES = BM * BK * 2;        // 2 boxes
+constexpr int B_BYTES = BN * BK * 2;        // 4 boxes
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 4;
+constexpr int STG_BYTES = 4096;  // one 32x32 fp32 staging block
+constexpr size_t SMEM_BYTES =
+    1024 + (size_t)STAGES * STAGE_BYTES + (size_t)EPI_WARPS * 2 * STG_BYTES + 256;
+
+struct WgradArgs {
+  int M, N;
+  int kblocks;        // ceil(T / BK)
+  int n_tiles;        // tiles along N
+  int64_t total;      // tiles * kblocks: the stream-K work space
+  int32_t* status;
+};
+
+// The CTA's range [g0, g1) of the work space, split into runs that stay
+// inside one output tile.
+struct Segment {
+  int tile, kb0, n;
+};
+struct SegCursor {
+  int64_t g, g1;
+  int kblocks;
+  __device__ __forceinline__ SegCursor(const WgradArgs& a) {
+    g = a.total * blockIdx.x / gridDim.x;
+    g1 = a.total * (blockIdx.x + 1) / gridDim.x;
+    kblocks = a.kblocks;
+  }
+  __device__ __forceinline__ bool next(Segment& s) {
+    if (g >= g1) return false;
+    s.tile = (int)(g / kblocks);
+    s.kb0 = (int)(g - (int64_t)s.tile * kblocks);
+    const int64_t left = g1 - g;
+    s.n = (int)((int64_t)(kblocks - s.kb0) < left ? (int64_t)(kblocks - s.kb0) : left);
+    g += s.n;
+    return true;
+  }
+};
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmO, WgradArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint8_t* sStg = sB + STAGES * B_BYTES;  // [EPI_WARPS][2][STG_BYTES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + EPI_WARPS * 2 * STG_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmO);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], EPI_WARPS);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool timed_out = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      SegCursor cur(args);
+      Segment sg;
+      while (!timed_out && cur.next(sg)) {
+        const int m0 = (sg.tile / args.n_tiles) * BM, n0 = (sg.tile % args.n_tiles) * BN;
+        for (int kb = sg.kb0; kb < sg.kb0 + sg.n; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { timed_out = true; break; }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t* a = sA + stage * A_BYTES;
+          uint8_t* b = sB + stage * B_BYTES;
+#pragma unroll
+          for (int j = 0; j < BM / BOX; ++j)
+            tma_load_2d(&tmA, &full[stage], a + j * BOX_BYTES, m0 + j * BOX, kb * BK);
+#pragma unroll
+          for (int j = 0; j < BN / BOX; ++j)
+            tma_load_2d(&tmB, &full[stage], b + j * BOX_BYTES, n0 + j * BOX, kb * BK);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // bf16 operands, both MN-major, fp32 accumulator
+      constexpr uint32_t idesc = idesc_f16(BM, BN, 1u, true, true);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      SegCursor cur(args);
+      Segment sg;
+      while (!timed_out && cur.next(sg)) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { timed_out = true; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        for (int i = 0; i < sg.n; ++i) {
+          if (!mbar_wait(&full[stage], phase)) { timed_out = true; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // 16 tokens = two 8-token groups of 1 KB each
+            tc_mma_ss(d_tmem, sdesc_sw128(a_addr + 2048 * k, BOX_BYTES, 1024),
+                      sdesc_sw128(b_addr + 2048 * k, BOX_BYTES, 1024), idesc, (i | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (timed_out) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    // epilogue warp ew adds accumulator rows [32 quarter, 32 quarter + 32)
+    const int quarter = warp & 3;
+    const int ew = warp - 2;
+    uint8_t* stg = sStg + ew * 2 * STG_BYTES;
+    int acc = 0;
+    uint32_t acc_phase = 0, chunk = 0;
+    SegCursor cur(args);
+    Segment sg;
+    while (cur.next(sg)) {
+      const int m0 = (sg.tile / args.n_tiles) * BM, n0 = (sg.tile % args.n_tiles) * BN;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase))) { timed_out = true; break; }
+      tc_fence_after();
+      const int row0 = m0 + quarter * 32;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c, ++chunk) {
+        const int col0 = n0 + c * 32;
+        if (col0 >= args.N) break;
+        uint8_t* sb = stg + (chunk & 1) * STG_BYTES;
+        if (lane == 0) bulk_wait_group_read<1>();  // the store two blocks ago has read sb
+        __syncwarp();
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4* p = reinterpret_cast<float4*>(sb + lane * 128 + ((q ^ (lane & 7)) << 4));
+          *p = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < args.M) {
+          tma_reduce_add_2d(&tmO, sb, col0, row0);
+          bulk_commit_group();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (lane == 0) bulk_wait_group<0>();  // reductions complete before the CTA retires
+  }
+  if (timed_out) set_status(args.status, MTGR_ERR_TIMEOUT);
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+// out [M][N] fp32 (+)= a^T b, a [T][M] and b [T][N] bf16 (row strides lda,
+// ldb elements, multiples of 8; M % 8 == 0 and N % 8 == 0 not required beyond
+// the strides). accumulate == 0 zeroes out first.
+int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const void* b,
+                      int64_t ldb, float* out, bool accumulate, int32_t* status, cudaStream_t s) {
+  if (M == 0 || N == 0) return MTGR_OK;
+  if (!accumulate && cudaMemsetAsync(out, 0, (size_t)M * N * sizeof(float), s) != cudaSuccess)
+    return MTGR_ERR_CUDA;
+  if (T == 0) return MTGR_OK;
+  CUtensorMap ta, tb, to;
+  int rc = make_tmap_2d_16b(&ta, a, (uint64_t)M, (uint64_t)T, (uint64_t)lda * 2, BOX, BK);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d_16b(&tb, b, (uint64_t)N, (uint64_t)T, (uint64_t)ldb * 2, BOX, BK);
+  if (rc != MTGR_OK) return rc;
+  rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)M,
+                    (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != MTGR_OK) return rc;
+  WgradArgs args;
+  args.M = M;
+  args.N = N;
+  args.kblocks = (int)((T + BK - 1) / BK);
+  args.n_tiles = (N + BN - 1) / BN;
+  const int64_t tiles = (int64_t)((M + BM - 1) / BM) * args.n_tiles;
+  args.total = tiles * args.kblocks;
+  args.status = status;
+  const int64_t sms = device_sm_count();
+  const int grid = (int)(args.total < sms ? args.total : sms);
+  if (cudaFuncSetAttribute(gemm_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_BYTES) != cudaSuccess)
+    return MTGR_ERR_CUDA;
+  gemm_wgrad_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, to, args);
+  return launch_status();
+}
+
+}  // namespace mtgr

@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(MTGR_TILE_M) attn_f32_kernel(
     const int64_t* __restrict__ ts, const int32_t* __restrict__ qtile_desc,
     const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ entries,
     const int32_t* __restrict__ order, const int64_t* __restrict__ counts,
-    const float* __restrict__ norm, int32_t q_cap, float* __restrict__ g_out) {
+    const float* __restrict__ norm, int32_t q_cap, float* __restrict__ g_out,
+    float* __restrict__ obar) {
   extern __shared__ float sm[];
   float* Ks = sm;                          // [128][DH]
   float* Vs = sm + MTGR_TILE_N * DH;       // [128][DH]
@@ -151,6 +152,11 @@ __global__ void __launch_bounds__(MTGR_TILE_M) attn_f32_kernel(
   float* g = g_out + (int64_t)(us + i) * d + h * DH;
 #pragma unroll
   for (int c = 0; c < DH; ++c) g[c] = o[c] * inv_n * u[c];
+  if (obar != nullptr) {  // O / N before the gate, for the backward pass
+    float* ob = obar + (int64_t)(us + i) * d + h * DH;
+#pragma unroll
+    for (int c = 0; c < DH; ++c) ob[c] = o[c] * inv_n;
+  }
 }
 
 }  // namespace
@@ -179,7 +185,7 @@ int launch_gemm_f32(int M, int N, int K, const float* a, const float* b, const f
 }
 
 int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkvu, float* g,
-                    cudaStream_t s) {
+                    cudaStream_t s, float* obar) {
   const int dh = d / H;
   if (bt->q_capacity == 0) return MTGR_OK;
   const unsigned grid = (unsigned)bt->q_capacity * (unsigned)H;
@@ -188,14 +194,14 @@ int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkv
     attn_f32_kernel<32><<<grid, MTGR_TILE_M, smem, s>>>(d, H, qkvu, bt->seg_off, bt->ts,
                                                         bt->qtile_desc, bt->row_ptr, bt->entries,
                                                         bt->order, bt->counts, bt->norm,
-                                                        bt->q_capacity, g);
+                                                        bt->q_capacity, g, obar);
   } else if (dh == 64) {
     cudaFuncSetAttribute(attn_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     attn_f32_kernel<64><<<grid, MTGR_TILE_M, smem, s>>>(d, H, qkvu, bt->seg_off, bt->ts,
                                                         bt->qtile_desc, bt->row_ptr, bt->entries,
                                                         bt->order, bt->counts, bt->norm,
-                                                        bt->q_capacity, g);
+                                                        bt->q_capacity, g, obar);
   } else {
     return MTGR_ERR_UNSUPPORTED;
   }

@@ -521,12 +521,71 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
 #define MTGR_TIMER_TOKEN_MLP 7
 #define MTGR_TIMER_HEAD_MLP 8
 #define MTGR_TIMER_ROWS 9
-#define MTGR_TIMER_CLASSES 10
+#define MTGR_TIMER_BWD_GEMM 10      /* backward: dH, dG~, dX~ GEMMs (3 per block) */
+#define MTGR_TIMER_BWD_WGRAD 11     /* backward: dW2, dW1, dW_qkvu GEMMs (3) */
+#define MTGR_TIMER_BWD_ATTENTION 12 /* backward: attention (1, plus its k-tile list) */
+#define MTGR_TIMER_BWD_GLN 13       /* backward: both GroupLNs (2) */
+#define MTGR_TIMER_BWD_ROWS 14      /* backward: conversions, transposes, column sums */
+#define MTGR_TIMER_CLASSES 15
 typedef struct mtgr_timer mtgr_timer;
 MTGR_API mtgr_timer* mtgr_timer_create(void);
 MTGR_API void mtgr_timer_destroy(mtgr_timer* timer);
 MTGR_API int mtgr_timer_attach(mtgr_timer* timer);
 MTGR_API int mtgr_timer_read(mtgr_timer* timer, double* ms, int64_t* launches);
+
+/*
+ * Training: the block's forward keeping what its backward reads, and the
+ * backward (the gradients of the summary page's Method update equations by
+ * the chain rule; the pages' system numbers are training throughput, in
+ * bf16 mixed precision: summary page, main contributions and Method, the
+ * training system). Variant 0 blocks only (MTGR_ERR_UNSUPPORTED otherwise).
+ *
+ * mtgr_hstu_block_fwd_train: as mtgr_hstu_block_fwd, and d_saved (caller
+ * owned, mtgr_block_saved_bytes(T, p) bytes) receives the activations the
+ * backward reads: GroupLN_1 output, Q|K|V|U, O/N (the attention before the
+ * gate), G, GroupLN_2 output, the MLP pre-activation and its SiLU (bf16
+ * blocks: bf16, Q|K|V|U f16 with Q halved; fp32 blocks: fp32). Same output
+ * x_out as mtgr_hstu_block_fwd.
+ */
+MTGR_API size_t mtgr_block_saved_bytes(int32_t T, const mtgr_block_params* p);
+MTGR_API int mtgr_hstu_block_fwd_train(const mtgr_block_params* p, const mtgr_batch* batch,
+                                       const float* d_x_in, float* d_x_out, void* d_saved,
+                                       size_t saved_bytes, mtgr_stream_t stream);
+
+/* Parameter gradients of one block (device, fp32, same shapes as the
+ * parameters; written, not accumulated). A NULL bias entry skips that bias's
+ * gradient; every other entry is required. */
+typedef struct mtgr_block_grads {
+  float* gln1_gamma;  /* [4][d] */
+  float* gln1_beta;   /* [4][d] */
+  float* w_qkvu;      /* [4d][d] */
+  float* b_qkvu;      /* [4d] or NULL */
+  float* gln2_gamma;  /* [4][d] */
+  float* gln2_beta;   /* [4][d] */
+  float* w1;          /* [d_ff][d] */
+  float* b1;          /* [d_ff] or NULL */
+  float* w2;          /* [d][d_ff] */
+  float* b2;          /* [d] or NULL */
+} mtgr_block_grads;
+
+/*
+ * Backward of one block: given d_dy = dL/dX_out [T][d] fp32, writes
+ * d_dx = dL/dX_in [T][d] fp32 and the parameter gradients. d_x_in and
+ * d_saved are the forward's input and saved activations (same batch,
+ * parameters and normaliser). Workspace: mtgr_block_bwd_workspace_bytes.
+ * bf16 blocks run the contractions on tcgen05 tensor cores (the attention's
+ * with f16 operands, its dO~ = dG (.) U in f16: values beyond 65504 set
+ * MTGR_ERR_RANGE in the batch status, values below 2^-14 lose precision as
+ * f16 subnormals, so scale the loss as usual for f16 training); fp32 blocks
+ * on CUDA cores. Weight gradients are sums over all tokens accumulated in
+ * fp32 in an order that varies from run to run.
+ */
+MTGR_API size_t mtgr_block_bwd_workspace_bytes(int32_t T, const mtgr_block_params* p,
+                                               const mtgr_batch* batch);
+MTGR_API int mtgr_hstu_block_bwd(const mtgr_block_params* p, const mtgr_batch* batch,
+                                 const float* d_x_in, const void* d_saved, const float* d_dy,
+                                 float* d_dx, const mtgr_block_grads* grads, void* d_ws,
+                                 size_t ws_bytes, mtgr_stream_t stream);
 
 /*
  * Self-test of the bounded waits (failure handling, not part of the method):

@@ -91,3 +91,43 @@ def oracle_stack_all_users(w, procs=None, chunk=8, variant=0):
             else:
                 os.environ[k] = v
     return np.concatenate(parts, axis=0)
+
+
+def _oracle_backward_chunk(args):
+    import oracle
+    x, lens, ts, p, H, dy = args
+    return oracle.hstu_block_backward(x, lens, ts, p, H, dy)
+
+
+def oracle_backward_all_users(w, dy, procs=None, chunk=8):
+    """The oracle's block backward over every user of workload ``w`` (one
+    block): per-user chunks on a spawned pool of single-threaded workers; the
+    input gradient rows concatenate and the parameter gradients, sums over
+    tokens, add up across chunks."""
+    import multiprocessing as mp
+    import os
+    lens = np.asarray(w["lens"]).reshape(-1, 4)
+    off = np.concatenate([[0], np.cumsum(lens.sum(1))])
+    jobs = []
+    for u0 in range(0, lens.shape[0], chunk):
+        u1 = min(lens.shape[0], u0 + chunk)
+        r0, r1 = int(off[u0]), int(off[u1])
+        jobs.append((w["x"][r0:r1], lens[u0:u1], w["ts"][r0:r1], w["layers"][0], w["H"], dy[r0:r1]))
+    procs = procs or max(1, len(os.sched_getaffinity(0)))
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"
+    try:
+        with mp.get_context("spawn").Pool(procs) as pool:
+            parts = pool.map(_oracle_backward_chunk, jobs)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    out = {"x": np.concatenate([p["x"] for p in parts], axis=0)}
+    for k in parts[0]:
+        if k != "x":
+            out[k] = sum(p[k] for p in parts)
+    return out

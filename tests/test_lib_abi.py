@@ -36,7 +36,8 @@ def test_struct_layouts_match_header(tmp_path):
         pytest.skip("no C compiler")
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "mtgr.h"', 'int main(void) {']
     structs = (("mtgr_batch", _lib.MtgrBatch), ("mtgr_block_params", _lib.MtgrBlockParams),
-               ("mtgr_token_mlp", _lib.MtgrTokenMlp), ("mtgr_head_params", _lib.MtgrHeadParams))
+               ("mtgr_token_mlp", _lib.MtgrTokenMlp), ("mtgr_head_params", _lib.MtgrHeadParams),
+               ("mtgr_block_grads", _lib.MtgrBlockGrads))
     for cname, cls in structs:
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
         for f, _ in cls._fields_:
@@ -67,7 +68,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert _lib.status_string(code) != "unknown status"
     assert _lib.status_string(99) == "unknown status"
     assert lib.mtgr_version() >= 100
@@ -179,3 +180,35 @@ def test_candidate_pass_workspace_sizes(lib):
     assert _lib.mtgr_stack_candidates_workspace_bytes(B, T, K, [p]) == one
     assert _lib.mtgr_stack_candidates_workspace_bytes(B, T, K, [p, p]) == one + up(K * 512 * 4)
     assert _lib.mtgr_stack_candidates_workspace_bytes(B, T, T + 1, [p]) == 0
+
+
+def test_training_workspace_sizes(lib):
+    # saved activations: X~, Q|K|V|U, O/N, G, G~ [T][d..4d] and Z1, H [T][d_ff],
+    # each region 256-byte aligned; 2 bytes per element on the bf16 path
+    p = _lib.MtgrBlockParams(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16, eps=1e-5, variant=0,
+                             gln1_gamma=16, gln1_beta=16, gln2_gamma=16, gln2_beta=16,
+                             w_qkvu=16, w1=16, w2=16)
+    T = 1000
+    al = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    want = sum(al(T * c * 2) for c in (512, 4 * 512, 512, 512, 512, 2048, 2048))
+    assert _lib.mtgr_block_saved_bytes(T, p) == want
+    b = _lib.MtgrBatch(B=2, T=T, q_capacity=9, kt_capacity=5)
+    ws = _lib.mtgr_block_bwd_workspace_bytes(T, p, b)
+    assert ws >= al(T * 512 * 2) + al(T * 2048 * 2) + al(T * 4 * 512 * 2) + al(10 * 4) + al(45 * 4)
+    p.variant = 1
+    assert _lib.mtgr_block_saved_bytes(T, p) > 0  # sizes are shape-only; the call itself refuses
+
+
+def test_training_entry_points_validate_on_the_host(lib):
+    p = _lib.MtgrBlockParams(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16, eps=1e-5, variant=2,
+                             gln1_gamma=16, gln1_beta=16, gln2_gamma=16, gln2_beta=16,
+                             w_qkvu=16, w1=16, w2=16)
+    b = _lib.MtgrBatch(B=0, T=0, seg_off=16, user_off=16, ts=16, counts=16, status=16)
+    g = _lib.MtgrBlockGrads()
+    # a variant block has no backward
+    assert lib.mtgr_hstu_block_fwd_train(ctypes.byref(p), ctypes.byref(b), None, None, None, 0,
+                                         None) == _lib.MTGR_ERR_UNSUPPORTED
+    p.variant = 0
+    # missing gradient outputs
+    assert lib.mtgr_hstu_block_bwd(ctypes.byref(p), ctypes.byref(b), None, None, None, None,
+                                   ctypes.byref(g), None, 0, None) == _lib.MTGR_ERR_INVALID_ARG
