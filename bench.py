@@ -66,6 +66,10 @@ def parse_args():
     ap.add_argument("--serving", action="store_true",
                     help="cached-context candidate scoring on the 512-user block workload: the "
                          "candidate pass against the aggregated pass (one JSON line)")
+    ap.add_argument("--backward", action="store_true",
+                    help="one training step of the block on the 512-user block workload: the "
+                         "forward keeping its activations, then the backward (one JSON line, "
+                         "each backward kernel class with its roofline)")
     ap.add_argument("--pipeline", action="store_true",
                     help="time token MLPs -> block -> CTR/CTCVR heads on the 512-user block "
                          "workload, each part with its roofline (one JSON line)")
@@ -782,6 +786,109 @@ def run_pipeline(args, local):
     print(json.dumps(line), flush=True)
 
 
+def run_backward(args, local):
+    """Training step of one bf16 block: pack, mask metadata, the forward that
+    keeps the backward's activations, and the backward (dX and every
+    parameter gradient), all through the C ABI, inputs and upstream gradient
+    resident in HBM."""
+    import generative_recommendation_ranking_b200 as mt
+    from generative_recommendation_ranking_b200 import _lib
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = synth.make_workload(2, seed=args.seed, B=args.users)
+    lens = wl["lens"]
+    B, T, d, H, dff = int(lens.shape[0]), int(lens.sum()), wl["d"], wl["H"], wl["d_ff"]
+    stream = torch.cuda.current_stream(dev)
+    batch = mt.PackedBatch(lens, wl["ts"], device=dev)
+    bw = mt.BlockWeights(wl["layers"][0], H, device=dev)
+    x = torch.from_numpy(wl["x"]).to(dev)
+    dy = torch.from_numpy(np.random.default_rng(args.seed + 1).standard_normal(
+        wl["x"].shape, dtype=np.float32)).to(dev)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    saved = torch.empty(_lib.mtgr_block_saved_bytes(T, bw.c), dtype=torch.uint8, device=dev)
+    bws = torch.empty(_lib.mtgr_block_bwd_workspace_bytes(T, bw.c, batch.c), dtype=torch.uint8,
+                      device=dev)
+    shapes = {"gln1_gamma": (4, d), "gln1_beta": (4, d), "w_qkvu": (4 * d, d),
+              "gln2_gamma": (4, d), "gln2_beta": (4, d), "w1": (dff, d), "w2": (d, dff)}
+    grads = {k: torch.empty(v, dtype=torch.float32, device=dev) for k, v in shapes.items()}
+    gc = _lib.MtgrBlockGrads(**{k: v.data_ptr() for k, v in grads.items()})
+
+    def step():
+        batch.pack(stream)
+        batch.build_meta(stream)
+        _lib.mtgr_hstu_block_fwd_train(bw.c, batch.c, x, y, saved, stream)
+        _lib.mtgr_hstu_block_bwd(bw.c, batch.c, x, saved, dy, dx, gc, bws, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    batch.check()
+    n = max(3, min(args.steps, 50))
+    timer = _lib.Timer()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    timer.attach()
+    ms = time_steps(step, n, stream) / n
+    timer.detach()
+    clk = clocks.stop()
+    batch.check()
+    per = timer.read()
+    V = int(batch.counts[2].item())
+    peaks, peak_src = load_peaks()
+    tkey = tensor_peak_key(ms * n / 1e3)
+    # algorithmic work per step of each class (bf16 block, dh = 64):
+    #   forward: projections 2 T (4 d^2 + 2 d d_ff), attention 4 d V
+    #   backward GEMMs dH, dG~, dX~: 2 T (d d_ff + d_ff d + 4 d^2); weight
+    #   gradients the same count; attention backward 10 d V (S, dP, dV, dK,
+    #   dQ: 2 dh FLOP each per visible pair and head)
+    gemm_flop = 2.0 * T * (d * dff + dff * d + 4 * d * d)
+    work = {"bwd_gemm": ("tensor", gemm_flop), "bwd_wgrad": ("tensor", gemm_flop),
+            "bwd_attention": ("tensor", 10.0 * d * V),
+            "attention": ("tensor", 4.0 * d * V),
+            "gemm_qkvu": ("tensor", 2.0 * T * 4 * d * d), "gemm_mlp1": ("tensor", 2.0 * T * d * dff),
+            "gemm_mlp2": ("tensor", 2.0 * T * d * dff),
+            # GroupLN backward, bytes per token: GLN_1 reads x, dX~, dY and
+            # writes dX (fp32: 16 d); GLN_2 with the gate reads G (bf16), dG~
+            # (fp32), U (f16), O/N (bf16) and writes dO~ (f16), dU (bf16): 14 d
+            "bwd_gln": ("hbm", T * d * (16.0 + 14.0))}
+    kernels = {}
+    for cls, (bound, w) in work.items():
+        t_ms, cnt = per[cls]
+        if cnt == 0:
+            continue
+        avg = t_ms / n
+        ach = w / (avg * 1e-3) / (1e12 if bound == "tensor" else 1e9)
+        peak = peaks[tkey] if bound == "tensor" else peaks["hbm_gbs"]
+        kernels[cls] = {"bound": bound, "ms_per_step": avg, "launches_per_step": cnt / n,
+                        "achieved": ach, "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                        "peak": peak, "frac": ach / peak, "share": t_ms / (ms * n)}
+    for cls in ("pack", "mask_meta", "gln", "bwd_rows"):
+        t_ms, cnt = per[cls]
+        if cnt:
+            kernels[cls] = {"ms_per_step": t_ms / n, "launches_per_step": cnt / n,
+                            "share": t_ms / (ms * n)}
+    bwd = [c for c in ("bwd_gemm", "bwd_wgrad", "bwd_attention", "bwd_gln") if c in kernels]
+    dom = max(bwd, key=lambda c: kernels[c]["share"])
+    k = kernels[dom]
+    total_flop = 3 * gemm_flop + 14.0 * d * V
+    line = {"metric": "HSTU-block training step (fwd + bwd) user-samples/s",
+            "value": B / (ms * 1e-3), "unit": "user-samples/s", "ms_per_step": ms, "steps": n,
+            "warmup": max(3, args.warmup), "higher_is_better": True, "n_gpus": 1,
+            "dtype": "bf16 (attention operands f16, fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": wl["name"], "users": B, "tokens": T, "d_model": d, "heads": H,
+                       "d_ff": dff, "layers": 1, "visible_pairs": V,
+                       "l2": "inputs larger than L2 (fp32 token features and gradient, 1.9 GB)"},
+            "step_tflops": total_flop / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"],
+                         "unit": k["unit"], "frac": k["frac"], "traffic": None, "kernel": dom,
+                         "peak_source": f"{peak_src} ({tkey if k['bound'] == 'tensor' else 'hbm_gbs'})"},
+            "kernels": kernels, "gpu_launches": int(sum(c for _, c in per.values()) / n),
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args) if args.impl == "ours" else (
@@ -795,6 +902,9 @@ def main():
         elif args.pipeline:
             if rank == 0:
                 run_pipeline(args, local)
+        elif args.backward:
+            if rank == 0:
+                run_backward(args, local)
         elif synth.WORKLOADS[args.config].kind == "sweep":
             if rank == 0:
                 run_sweep(args, local)

@@ -68,7 +68,7 @@ constexpr size_t SMEM_BYTES = 1024 + 4 * TILE_BYTES + 4 * TILE_BYTES + 4 * HALF_
                               (size_t)NUM_EPI_WARPS * 2 * STG_BYTES + 256;
 
 struct AttnBwdArgs {
-  int32_t d, H;
+  int32_t d, H, T;
   const int32_t* seg_off;
   const int32_t* qtile_desc;
   const int32_t* order;
@@ -223,6 +223,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // the dV / dK / dQ MMAs of round r (a q-tile), `first` of its item
       auto back = [&](int32_t r, bool first, uint32_t k_addr) -> bool {
         if (!mbar_wait(p_full, r & 1)) return false;
+        // an item's first dV / dK MMAs overwrite the accumulators: the
+        // previous item's must have been drained
+        if (first && !mbar_wait(dkv_free, (li & 1) ^ 1)) return false;
         if (!mbar_wait(&dq_free[r & 1], ((r >> 1) & 1) ^ 1)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQD + (r & 1) * 2 * TILE_BYTES);
@@ -250,11 +253,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const BwdItem it = load_bwd_item(a, w);
         const int kb = li & 1;
         if (!mbar_wait(&kv_full[kb], (li >> 1) & 1)) { timed_out = true; break; }
-        // dK / dV of the previous item drained before this item overwrites them
-        if (!mbar_wait(dkv_free, (li & 1) ^ 1)) { timed_out = true; break; }
         const uint32_t k_addr = smem_u32(sKV + kb * 2 * TILE_BYTES);
         const uint32_t v_addr = k_addr + TILE_BYTES;
-        const int32_t nq = it.e1 - it.e0, g0 = g;
+        const int32_t nq = it.e1 - it.e0;
         for (int32_t t = 0; t < nq; ++t, ++g) {
           const int st = g & 1;
           if (!mbar_wait(&qd_full[st], (g >> 1) & 1)) { timed_out = true; break; }
@@ -273,7 +274,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (timed_out) break;
         if (!back(g - 1, nq == 1, k_addr)) { timed_out = true; break; }
-        (void)g0;
         tc_commit(&kv_empty[kb]);
         tc_commit(dkv_full);
       }
@@ -389,9 +389,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          // rows past the user's end hold zeros (their A and dS rows are masked)
-          const int32_t y = it.us + qt * TM + quarter * 32;
+        // rows past the user's end hold zeros (their A and dS rows are
+        // masked); a block wholly past the last token is not sent
+        const int32_t y = it.us + qt * TM + quarter * 32;
+        if (lane == 0 && y < a.T) {
           tma_reduce_add_2d(&tm_dq, stg, it.h * DH, y);
           tma_reduce_add_2d(&tm_dq, stg + STG_BYTES, it.h * DH + 32, y);
           bulk_commit_group();
@@ -454,7 +455,7 @@ int launch_attn_bwd_tc(const mtgr_batch* bt, int32_t d, int32_t H, const void* q
   rc = make_tmap_2d(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)d, (uint64_t)bt->T,
                     (uint64_t)4 * d, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MTGR_OK) return rc;
-  AttnBwdArgs a{d, H, bt->seg_off, bt->qtile_desc, bt->order, csc_ptr, csc, bt->counts, bt->rt_cnt,
+  AttnBwdArgs a{d, H, bt->T, bt->seg_off, bt->qtile_desc, bt->order, csc_ptr, csc, bt->counts, bt->rt_cnt,
                 bt->rt_off, bt->rt_mask, bt->norm, bt->q_capacity,
                 static_cast<__nv_bfloat16*>(dz), bt->status};
   const int64_t items = (int64_t)bt->q_capacity * H;
