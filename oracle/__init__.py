@@ -30,6 +30,11 @@ from .mtgr import (  # noqa: F401
     group_layernorm_pooled,
     VARIANT_POOLED_GLN,
     VARIANT_SILU_QKVU,
+    VARIANT_RAB,
+    RAB_MAX_DIST,
+    RAB_TIME_BUCKETS,
+    rab_time_bucket,
+    rab_bias,
     hstu_attention,
     hstu_block,
     hstu_stack,

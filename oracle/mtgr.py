@@ -125,6 +125,41 @@ def group_layernorm(x: np.ndarray, group_id: np.ndarray, gamma: np.ndarray,
 #     attention and gating" (it also puts SiLU on U before the gate).
 VARIANT_POOLED_GLN = 1
 VARIANT_SILU_QKVU = 2
+#   VARIANT_RAB: HSTU's relative attention bias, a learned per-head bias added
+#     to every score before the SiLU, silu(q_i . k_j + rab_h(i, j)). The pages
+#     name the bias only through HSTU; the reading taken: rab_h(i, j) =
+#     w_pos[h][clip(i - j, -RAB_MAX_DIST, RAB_MAX_DIST) + RAB_MAX_DIST] +
+#     w_time[h][time_bucket(|t_i - t_j|)], with i, j the user-relative
+#     positions, time_bucket(0) = 0 and time_bucket(dt) = min(floor(log2 dt)
+#     + 1, RAB_TIME_BUCKETS - 1) for dt >= 1, and no time term (bucket 0)
+#     when either token is a U token, which carries no time.
+VARIANT_RAB = 4
+RAB_MAX_DIST = 128
+RAB_TIME_BUCKETS = 32
+
+
+def rab_time_bucket(dt: int) -> int:
+    """Bucket of an absolute time difference: 0 for 0, else the number of
+    binary digits of dt (floor(log2 dt) + 1), capped at RAB_TIME_BUCKETS - 1."""
+    dt = int(dt)
+    if dt <= 0:
+        return 0
+    return min(dt.bit_length(), RAB_TIME_BUCKETS - 1)
+
+
+def rab_bias(n_u: int, n_s: int, n_r: int, n_k: int, ts: np.ndarray, w_pos: np.ndarray,
+             w_time: np.ndarray, h: int) -> np.ndarray:
+    """The relative attention bias [N, N] of head h for one user (query i,
+    key j), by the VARIANT_RAB reading above, entry by entry."""
+    N = n_u + n_s + n_r + n_k
+    ts = np.asarray(ts, dtype=np.int64)
+    out = np.zeros((N, N), dtype=np.float64)
+    for i in range(N):
+        for j in range(N):
+            p = min(max(i - j, -RAB_MAX_DIST), RAB_MAX_DIST) + RAB_MAX_DIST
+            tb = 0 if (i < n_u or j < n_u) else rab_time_bucket(abs(int(ts[i]) - int(ts[j])))
+            out[i, j] = float(w_pos[h][p]) + float(w_time[h][tb])
+    return out
 
 
 def group_layernorm_pooled(x: np.ndarray, lens: np.ndarray, gamma: np.ndarray,
@@ -149,12 +184,14 @@ def group_layernorm_pooled(x: np.ndarray, lens: np.ndarray, gamma: np.ndarray,
 
 
 def hstu_attention(qkvu: np.ndarray, lens: np.ndarray, ts: np.ndarray, H: int,
-                   norm: np.ndarray | None = None) -> np.ndarray:
+                   norm: np.ndarray | None = None, rab: tuple | None = None) -> np.ndarray:
     """G = (silu(Q K^T) * M / N) V, gated by U, per user and head.
 
     Summary page, Method: V~ = silu(K^T Q) / (N_U+N_S+N_R+N_I) * M * V and the
     gate V~ (.) U of the update. ``qkvu`` is [T, 4d] with column blocks
     Q | K | V | U; head h owns columns [h*dh, (h+1)*dh) of each block.
+    ``rab`` = (w_pos [H, 2 RAB_MAX_DIST + 1], w_time [H, RAB_TIME_BUCKETS])
+    adds the relative attention bias of VARIANT_RAB to the scores.
     Returns G [T, d] in float64.
     """
     qkvu = np.asarray(qkvu, dtype=np.float64)
@@ -175,6 +212,8 @@ def hstu_attention(qkvu: np.ndarray, lens: np.ndarray, ts: np.ndarray, H: int,
         for h in range(H):
             c = slice(h * dh, (h + 1) * dh)
             scores = Q[s:e, c] @ K[s:e, c].T        # scores[i, j] = q_i . k_j
+            if rab is not None:
+                scores = scores + rab_bias(n_u, n_s, n_r, n_k, ts[s:e], rab[0], rab[1], h)
             A = silu(scores) * M / Nb
             out[s:e, c] = A @ V[s:e, c]
     return out * U
@@ -204,7 +243,8 @@ def hstu_block(x: np.ndarray, lens: np.ndarray, ts: np.ndarray, p: dict, H: int,
         qkvu = qkvu + np.asarray(p["b_qkvu"], np.float64)
     if variant & VARIANT_SILU_QKVU:
         qkvu = silu(qkvu)
-    g = hstu_attention(qkvu, lens, ts, H, norm)
+    rab = (p["rab_pos"], p["rab_time"]) if variant & VARIANT_RAB else None
+    g = hstu_attention(qkvu, lens, ts, H, norm, rab)
     gt = gln(g, p["gln2_gamma"], p["gln2_beta"])
     h = gt @ np.asarray(p["w1"], np.float64).T
     if p.get("b1") is not None:

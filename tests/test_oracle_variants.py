@@ -148,3 +148,88 @@ def test_pooled_block_constant_scores_reduce_to_masked_sum():
     gt = _pooled_torch(g, lens, p["gln2_gamma"], p["gln2_beta"], 1e-5)
     ref = x + _mlp(gt, p)
     np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-10)
+
+
+# ---------------------------------------------------------------- VARIANT_RAB
+def test_rab_time_bucket_is_the_binary_digit_count():
+    import math
+    assert oracle.rab_time_bucket(0) == 0
+    for dt in list(range(1, 70)) + [1000, 65535, 65536, 2 ** 29 + 3, 2 ** 40]:
+        want = min(int(math.floor(math.log2(dt))) + 1, oracle.RAB_TIME_BUCKETS - 1)
+        assert oracle.rab_time_bucket(dt) == want, dt
+
+
+def test_rab_bias_matches_hand_worked_user(golden):
+    g = golden("rab_tiny_user.txt")
+    n_u, n_s, n_r, n_k = g["lens"]
+    ts = np.array(g["ts"], np.int64)
+    bk = np.array(g["buckets"], np.int64)
+    H = 2
+    w_pos = np.tile(np.arange(2 * oracle.RAB_MAX_DIST + 1, dtype=np.float64), (H, 1))
+    w_time = np.tile(1000.0 * np.arange(oracle.RAB_TIME_BUCKETS), (H, 1))
+    w_time[1] *= 2.0  # the heads keep their own tables
+    for h in range(H):
+        got = oracle.rab_bias(n_u, n_s, n_r, n_k, ts, w_pos, w_time, h)
+        i, j = np.meshgrid(np.arange(6), np.arange(6), indexing="ij")
+        want = (i - j + oracle.RAB_MAX_DIST) + 1000.0 * (h + 1) * bk
+        np.testing.assert_array_equal(got, want)
+
+
+def test_rab_position_term_clips_far_pairs():
+    N = 300
+    ts = np.arange(N, dtype=np.int64)
+    w_pos = np.arange(2 * oracle.RAB_MAX_DIST + 1, dtype=np.float64)[None, :]
+    w_time = np.zeros((1, oracle.RAB_TIME_BUCKETS))
+    b = oracle.rab_bias(0, N, 0, 0, ts, w_pos, w_time, 0)
+    assert b[299, 0] == 2 * oracle.RAB_MAX_DIST and b[0, 299] == 0.0
+    assert b[150, 150 - oracle.RAB_MAX_DIST] == 2 * oracle.RAB_MAX_DIST
+    assert b[10, 10] == oracle.RAB_MAX_DIST
+
+
+def _rab_case(seed=0, H=2, dh=8):
+    rng = np.random.default_rng(seed)
+    lens = np.array([[2, 7, 4, 3], [1, 5, 0, 2], [0, 4, 3, 0]], np.int32)
+    ts = synth.make_timestamps(lens, rng)
+    qkvu = rng.standard_normal((int(lens.sum()), 4 * H * dh))
+    return lens, ts, qkvu, H
+
+
+def test_rab_zero_tables_reduce_to_the_plain_attention():
+    lens, ts, qkvu, H = _rab_case()
+    z = (np.zeros((H, 2 * oracle.RAB_MAX_DIST + 1)), np.zeros((H, oracle.RAB_TIME_BUCKETS)))
+    np.testing.assert_array_equal(oracle.hstu_attention(qkvu, lens, ts, H, rab=z),
+                                  oracle.hstu_attention(qkvu, lens, ts, H))
+
+
+def test_rab_constant_bias_with_zero_queries_closed_form():
+    # Q = 0 and rab = c everywhere: every visible weight is silu(c) / N, so
+    # G_i = silu(c) / N_b sum_j M_ij v_j (.) u_i, with M the mask's own matrix
+    lens, ts, qkvu, H = _rab_case(seed=1)
+    d = qkvu.shape[1] // 4
+    qkvu[:, :d] = 0.0
+    c = 0.7
+    rab = (np.full((H, 2 * oracle.RAB_MAX_DIST + 1), c), np.zeros((H, oracle.RAB_TIME_BUCKETS)))
+    g = oracle.hstu_attention(qkvu, lens, ts, H, rab=rab)
+    off = np.concatenate([[0], np.cumsum(lens.sum(1))])
+    sc = c / (1.0 + np.exp(-c))
+    for b in range(lens.shape[0]):
+        s, e = off[b], off[b + 1]
+        M = oracle.user_mask(*(int(v) for v in lens[b]), ts[s:e]).astype(np.float64)
+        want = sc / (e - s) * (M @ qkvu[s:e, 2 * d:3 * d]) * qkvu[s:e, 3 * d:]
+        np.testing.assert_allclose(g[s:e], want, rtol=1e-12, atol=1e-12)
+
+
+def test_rab_time_term_ignores_u_tokens_and_shifts_scores():
+    # a time table that only bucket 3 uses: exactly the pairs the fixture's
+    # bucket matrix marks 3 change, by silu(s + w) - silu(s) in their weight
+    lens = np.array([[1, 2, 2, 1]], np.int32)
+    ts = np.array([0, 5, 9, 12, 20, 13], np.int64)
+    H, dh = 1, 4
+    rng = np.random.default_rng(3)
+    qkvu = rng.standard_normal((6, 4 * dh))
+    w_time = np.zeros((H, oracle.RAB_TIME_BUCKETS))
+    w_time[0, 3] = 0.5
+    b = oracle.rab_bias(1, 2, 2, 1, ts, np.zeros((H, 2 * oracle.RAB_MAX_DIST + 1)), w_time, 0)
+    marked = np.array([[0, 0, 0, 0, 0, 0], [0, 0, 1, 1, 0, 0], [0, 1, 0, 0, 0, 1],
+                       [0, 1, 0, 0, 0, 0], [0, 0, 0, 0, 0, 1], [0, 0, 1, 0, 1, 0]], bool)
+    np.testing.assert_array_equal(b != 0, marked)
