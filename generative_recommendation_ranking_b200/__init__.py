@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     MTGR_F32,
     MTGR_VARIANT_POOLED_GLN,
     MTGR_VARIANT_SILU_QKVU,
+    MTGR_VARIANT_RAB,
     MTGRError,
     load,
     mtgr_block_workspace_bytes,

@@ -21,6 +21,9 @@ MTGR_ERR_CUDA = 2
 MTGR_ERR_UNSUPPORTED = 3
 MTGR_VARIANT_POOLED_GLN = 1
 MTGR_VARIANT_SILU_QKVU = 2
+MTGR_VARIANT_RAB = 4
+RAB_MAX_DIST = 128
+RAB_TIME_BUCKETS = 32
 MTGR_ERR_CAPACITY = 4
 MTGR_ERR_TIMEOUT = 5
 MTGR_ERR_DEVICE_VALIDATION = 6
@@ -65,7 +68,8 @@ class MtgrBlockParams(ctypes.Structure):
     _fields_ = [("d", c_i32), ("H", c_i32), ("d_ff", c_i32), ("dtype", c_i32), ("eps", c_float),
                 ("variant", c_i32), ("gln1_gamma", c_vp), ("gln1_beta", c_vp),
                 ("gln2_gamma", c_vp), ("gln2_beta", c_vp), ("w_qkvu", c_vp), ("w1", c_vp),
-                ("w2", c_vp), ("b_qkvu", c_vp), ("b1", c_vp), ("b2", c_vp)]
+                ("w2", c_vp), ("b_qkvu", c_vp), ("b1", c_vp), ("b2", c_vp),
+                ("rab_pos", c_vp), ("rab_time", c_vp)]
 
 
 class MtgrBlockGrads(ctypes.Structure):

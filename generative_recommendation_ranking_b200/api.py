@@ -128,7 +128,9 @@ class BlockWeights:
     ``dtype`` "bf16" keeps W_qkvu, W1, W2 in bf16 (tensor-core path); "f32"
     keeps everything in fp32 (CUDA-core path). GroupLN parameters are fp32.
     ``variant``: 0, or MTGR_VARIANT_* flags (bf16 only): pooled GroupLN
-    statistics, SiLU on the Q|K|V|U projections.
+    statistics, SiLU on the Q|K|V|U projections, the relative attention bias
+    (tables ``rab_pos`` [H, 2 RAB_MAX_DIST + 1] and ``rab_time``
+    [H, RAB_TIME_BUCKETS] in ``p``).
     """
 
     def __init__(self, p: dict, H: int, dtype: str = "bf16", device="cuda", eps: float = EPS,
@@ -145,7 +147,8 @@ class BlockWeights:
         self.t = dict(gln1_gamma=f32(p["gln1_gamma"]), gln1_beta=f32(p["gln1_beta"]),
                       gln2_gamma=f32(p["gln2_gamma"]), gln2_beta=f32(p["gln2_beta"]),
                       w_qkvu=w(p["w_qkvu"]), w1=w(p["w1"]), w2=w(p["w2"]),
-                      b_qkvu=f32(p.get("b_qkvu")), b1=f32(p.get("b1")), b2=f32(p.get("b2")))
+                      b_qkvu=f32(p.get("b_qkvu")), b1=f32(p.get("b1")), b2=f32(p.get("b2")),
+                      rab_pos=f32(p.get("rab_pos")), rab_time=f32(p.get("rab_time")))
         d = self.t["w_qkvu"].shape[1]
         d_ff = self.t["w1"].shape[0]
         ptr = {k: (None if v is None else v.data_ptr()) for k, v in self.t.items()}

@@ -47,7 +47,8 @@ int launch_attn_f32(const mtgr_batch* bt, int32_t d, int32_t H, const float* qkv
                     cudaStream_t s, float* obar = nullptr);
 int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
                    const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s,
-                   void* obar = nullptr);
+                   void* obar = nullptr, const float* rab_pos = nullptr,
+                   const float* rab_time = nullptr);
 int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
                        void* aux, void* out, int32_t* status, cudaStream_t s);
 int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const void* b,
@@ -102,7 +103,10 @@ int params_check(const mtgr_block_params* p) {
   if (p->d <= 0 || p->H <= 0 || p->d_ff <= 0 || p->d > kMaxD || p->d % p->H != 0)
     return MTGR_ERR_INVALID_ARG;
   if (!(p->eps >= 0.0f)) return MTGR_ERR_INVALID_ARG;
-  if (p->variant & ~(MTGR_VARIANT_POOLED_GLN | MTGR_VARIANT_SILU_QKVU)) return MTGR_ERR_INVALID_ARG;
+  if (p->variant & ~(MTGR_VARIANT_POOLED_GLN | MTGR_VARIANT_SILU_QKVU | MTGR_VARIANT_RAB))
+    return MTGR_ERR_INVALID_ARG;
+  if ((p->variant & MTGR_VARIANT_RAB) && (p->rab_pos == nullptr || p->rab_time == nullptr))
+    return MTGR_ERR_INVALID_ARG;
   if (p->variant != 0 && p->dtype != MTGR_BF16) return MTGR_ERR_UNSUPPORTED;
   if (p->gln1_gamma == nullptr || p->gln1_beta == nullptr || p->gln2_gamma == nullptr ||
       p->gln2_beta == nullptr || p->w_qkvu == nullptr || p->w1 == nullptr || p->w2 == nullptr)
@@ -200,7 +204,9 @@ int block_fwd_rows(const mtgr_block_params* p, const mtgr_batch* bt, int32_t row
   }
   {
     TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
-    if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, qkvu, MTGR_BF16, w.g, s)) != MTGR_OK)
+    const bool rab = (p->variant & MTGR_VARIANT_RAB) != 0;
+    if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, qkvu, MTGR_BF16, w.g, s, nullptr,
+                             rab ? p->rab_pos : nullptr, rab ? p->rab_time : nullptr)) != MTGR_OK)
       return rc;
   }
   {
@@ -1044,7 +1050,9 @@ int block_fwd_cand(const mtgr_block_params* p, const mtgr_batch* bt, int32_t K, 
   }
   {
     TimedScope tsc(MTGR_TIMER_ATTENTION, s, 1);
-    if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, qkvu, MTGR_BF16, w.g, s)) != MTGR_OK)
+    const bool rab = (p->variant & MTGR_VARIANT_RAB) != 0;
+    if ((rc = launch_attn_tc(bt, d, H, MTGR_F16, true, qkvu, MTGR_BF16, w.g, s, nullptr,
+                             rab ? p->rab_pos : nullptr, rab ? p->rab_time : nullptr)) != MTGR_OK)
       return rc;
   }
   {

@@ -97,7 +97,38 @@ struct AttnArgs {
   void* out;  // [T][d] f32 or bf16
   int32_t* status;
   uint16_t* obar;  // optional [T][d] bf16: O / N before the gate (training forward)
+  // relative attention bias (RAB kernels): per-head tables and the timestamps
+  const float* rab_pos;   // [H][2 MTGR_RAB_MAX_DIST + 1]
+  const float* rab_time;  // [H][MTGR_RAB_TIME_BUCKETS]
+  const int64_t* ts;      // [T]
 };
+
+// The relative attention bias of head h for query i (timestamp t_i, or none
+// for a U query) and the 16 keys [j0, j0 + 16) of one step, added to their
+// f32 scores (times `scale`: 1/2 when the scores arrive halved):
+// rab = pos[clip(i - j) + MAX] + time[bucket(|t_i - t_j|)], bucket 0 for a
+// pair with a U token, else the binary digit count of the difference.
+__device__ __forceinline__ void add_rab(uint32_t (&s)[16], const AttnArgs& a, int32_t h,
+                                        int32_t us, int32_t n_u, int32_t i, int64_t t_i,
+                                        int32_t j0, float scale) {
+  const float* wp = a.rab_pos + (int64_t)h * (2 * MTGR_RAB_MAX_DIST + 1);
+  const float* wt = a.rab_time + (int64_t)h * MTGR_RAB_TIME_BUCKETS;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const int32_t j = j0 + c;
+    int32_t dp = i - j;
+    dp = dp < -MTGR_RAB_MAX_DIST ? -MTGR_RAB_MAX_DIST : (dp > MTGR_RAB_MAX_DIST ? MTGR_RAB_MAX_DIST : dp);
+    int tb = 0;
+    if (i >= n_u && j >= n_u) {
+      const int64_t dt = t_i - __ldg(a.ts + us + j);
+      const uint64_t adt = (uint64_t)(dt < 0 ? -dt : dt);
+      tb = 64 - __clzll((long long)adt);
+      tb = tb > MTGR_RAB_TIME_BUCKETS - 1 ? MTGR_RAB_TIME_BUCKETS - 1 : tb;
+    }
+    const float b = __ldg(wp + dp + MTGR_RAB_MAX_DIST) + __ldg(wt + tb);
+    s[c] = __float_as_uint(fmaf(scale, b, __uint_as_float(s[c])));
+  }
+}
 
 struct Item {
   mtgr_work_item w;
@@ -180,8 +211,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
 
 // IN_BF16: Q/K/V/U are bf16 (V converted to f16 in shared memory before P V);
 // otherwise f16. HALVE: the scores still need the factor 1/2 of silu's
-// tanh form. OUT_F32: G written as f32, else bf16.
-template <bool IN_BF16, bool HALVE, bool OUT_F32>
+// tanh form. OUT_F32: G written as f32, else bf16. RAB: the relative
+// attention bias is added to the scores (block variant).
+template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -395,6 +427,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool two = it.w.nq == 2;
       const int32_t i = (it.w.qt0 + q) * TM + quarter * 32 + lane;  // user-relative row
       const int32_t cnt_i = i < it.w.n ? __ldg(a.rt_cnt + it.w.us + i) : 0;
+      const int64_t t_i = RAB && i < it.w.n ? __ldg(a.ts + it.w.us + i) : 0;
       UnionCursor cur;
       cur.init(a.entries, it.w);
       // the upcoming k-tile: index, whether it needs the per-element rules,
@@ -438,6 +471,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t (&cur_s)[16] = (k & 1) ? sb : sa;
             uint32_t (&ahead)[16] = (k & 1) ? sa : sb;
             if (k < 7) tmem_ld16(s_addr + 16 * (k + 1), ahead);
+            if (RAB)
+              add_rab(cur_s, a, it.h, it.w.us, it.w.n_u, i, t_i, kt * TN + 16 * k, HALVE ? 1.f : 0.5f);
             const uint64_t vv = k < 4 ? vis_lo : vis_hi;
             scores_to_h<HALVE>(cur_s, h + 8 * k, masked, (uint32_t)(vv >> (16 * (k & 3))));
             if (k < 7) {
@@ -597,9 +632,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool IN_BF16, bool HALVE, bool OUT_F32>
+template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB = false>
 int launch_t(const CUtensorMap& tm, const AttnArgs& a, int grid, cudaStream_t s) {
-  auto kern = attn_tc_kernel<IN_BF16, HALVE, OUT_F32>;
+  auto kern = attn_tc_kernel<IN_BF16, HALVE, OUT_F32, RAB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
       cudaSuccess)
     return MTGR_ERR_CUDA;
@@ -611,20 +646,25 @@ int launch_t(const CUtensorMap& tm, const AttnArgs& a, int grid, cudaStream_t s)
 
 // qkvu [T][4d] of 16-bit elements (bf16 or f16), dh = 64.
 int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype, bool q_prehalved,
-                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s, void* obar) {
+                   const void* qkvu, int32_t out_dtype, void* out, cudaStream_t s, void* obar,
+                   const float* rab_pos, const float* rab_time) {
   if (bt->q_capacity == 0 || bt->T == 0) return MTGR_OK;
   CUtensorMap tm;
   int rc = make_tmap_2d_16b(&tm, qkvu, (uint64_t)4 * d, (uint64_t)bt->T, (uint64_t)8 * d, DH, TM);
   if (rc != MTGR_OK) return rc;
   AttnArgs a{d, H, static_cast<const uint16_t*>(qkvu), bt->entries, bt->work, bt->counts,
              bt->rt_cnt, bt->rt_mask, bt->norm, bt->q_capacity, out, bt->status,
-             static_cast<uint16_t*>(obar)};
+             static_cast<uint16_t*>(obar), rab_pos, rab_time, bt->ts};
   const int64_t items = (int64_t)bt->q_capacity * H;
   const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
   const bool f32 = out_dtype == MTGR_F32;
   if (in_dtype == MTGR_BF16) {
     if (q_prehalved) return MTGR_ERR_UNSUPPORTED;
     return f32 ? launch_t<true, true, true>(tm, a, grid, s) : launch_t<true, true, false>(tm, a, grid, s);
+  }
+  if (rab_pos != nullptr) {  // the block's bias variant: f16, Q prehalved, bf16 G
+    if (in_dtype != MTGR_F16 || !q_prehalved || f32 || obar != nullptr) return MTGR_ERR_UNSUPPORTED;
+    return launch_t<false, false, false, true>(tm, a, grid, s);
   }
   if (in_dtype == MTGR_F16) {
     if (q_prehalved)

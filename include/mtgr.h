@@ -291,9 +291,22 @@ MTGR_API int mtgr_hstu_attention_fwd(const mtgr_batch* batch, int32_t d, int32_t
  *   MTGR_VARIANT_SILU_QKVU: Q, K, V, U = silu(X~ W_qkvu^T + b), HSTU's
  *     pointwise SiLU on the projections (one reading of the blog posts'
  *     "HSTU-style SiLU attention and gating"; it also gates with silu(U)).
+ *   MTGR_VARIANT_RAB: HSTU's relative attention bias, added to every score
+ *     before the SiLU: silu(q_i . k_j + rab_h(i, j)) with
+ *     rab_h(i, j) = rab_pos[h][clip(i - j, -MTGR_RAB_MAX_DIST,
+ *     MTGR_RAB_MAX_DIST) + MTGR_RAB_MAX_DIST] + rab_time[h][b(|t_i - t_j|)],
+ *     i, j the positions within the user, b(0) = 0 and b(dt) =
+ *     min(floor(log2 dt) + 1, MTGR_RAB_TIME_BUCKETS - 1), and bucket 0 when
+ *     either token is a U token (no time). The pages name this bias only
+ *     through HSTU; this is the reading taken. Positions are those of the
+ *     batch as given, so a candidate scored in a chunk of its own sees the
+ *     position term of its place in that chunk.
  */
 #define MTGR_VARIANT_POOLED_GLN 1
 #define MTGR_VARIANT_SILU_QKVU 2
+#define MTGR_VARIANT_RAB 4
+#define MTGR_RAB_MAX_DIST 128
+#define MTGR_RAB_TIME_BUCKETS 32
 
 /* Parameters of one HSTU block (device pointers; PyTorch Linear [out][in] layout). */
 typedef struct mtgr_block_params {
@@ -313,6 +326,8 @@ typedef struct mtgr_block_params {
   const float* b_qkvu;        /* [4d] or NULL */
   const float* b1;            /* [d_ff] or NULL */
   const float* b2;            /* [d] or NULL */
+  const float* rab_pos;       /* MTGR_VARIANT_RAB: [H][2 MTGR_RAB_MAX_DIST + 1], else unused */
+  const float* rab_time;      /* MTGR_VARIANT_RAB: [H][MTGR_RAB_TIME_BUCKETS], else unused */
 } mtgr_block_params;
 
 /* Workspace bytes of mtgr_hstu_block_fwd for T tokens (0 on invalid params). */

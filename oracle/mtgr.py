@@ -153,13 +153,15 @@ def rab_bias(n_u: int, n_s: int, n_r: int, n_k: int, ts: np.ndarray, w_pos: np.n
     key j), by the VARIANT_RAB reading above, entry by entry."""
     N = n_u + n_s + n_r + n_k
     ts = np.asarray(ts, dtype=np.int64)
-    out = np.zeros((N, N), dtype=np.float64)
-    for i in range(N):
-        for j in range(N):
-            p = min(max(i - j, -RAB_MAX_DIST), RAB_MAX_DIST) + RAB_MAX_DIST
-            tb = 0 if (i < n_u or j < n_u) else rab_time_bucket(abs(int(ts[i]) - int(ts[j])))
-            out[i, j] = float(w_pos[h][p]) + float(w_time[h][tb])
-    return out
+    idx = np.arange(N)
+    pos = np.clip(idx[:, None] - idx[None, :], -RAB_MAX_DIST, RAB_MAX_DIST) + RAB_MAX_DIST
+    dt = np.abs(ts[:, None] - ts[None, :])
+    # binary digit count of dt: frexp's exponent (exact for |dt| < 2^53), 0 for dt = 0
+    digits = np.frexp(dt.astype(np.float64))[1]
+    tb = np.where(dt == 0, 0, np.minimum(digits, RAB_TIME_BUCKETS - 1))
+    has_time = idx >= n_u
+    tb = np.where(has_time[:, None] & has_time[None, :], tb, 0)
+    return np.asarray(w_pos[h], np.float64)[pos] + np.asarray(w_time[h], np.float64)[tb]
 
 
 def group_layernorm_pooled(x: np.ndarray, lens: np.ndarray, gamma: np.ndarray,

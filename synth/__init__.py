@@ -13,6 +13,7 @@ from .workloads import (  # noqa: F401
     make_tokens,
     make_block_params,
     make_stack_params,
+    make_rab_tables,
     make_qkvu,
     make_workload,
     assemble_workload,

@@ -185,6 +185,15 @@ def make_block_params(d: int, d_ff: int, rng: np.random.Generator, dtype: str = 
     return p
 
 
+def make_rab_tables(H: int, rng: np.random.Generator, scale: float = 2.0, max_dist: int = 128,
+                    time_buckets: int = 32) -> tuple:
+    """Per-head relative attention bias tables, N(0, scale^2) float32:
+    positions [H, 2 max_dist + 1] and time buckets [H, time_buckets]."""
+    pos = (scale * rng.standard_normal((H, 2 * max_dist + 1))).astype(np.float32)
+    tim = (scale * rng.standard_normal((H, time_buckets))).astype(np.float32)
+    return pos, tim
+
+
 def make_stack_params(L: int, d: int, d_ff: int, rng: np.random.Generator, dtype: str = "bf16") -> list:
     return [make_block_params(d, d_ff, rng, dtype) for _ in range(L)]
 

@@ -80,3 +80,57 @@ def test_pooled_variant_rejected_on_candidate_rows():
     with pytest.raises(mt.MTGRError) as e:
         cc.score(w["ts"][n_ctx:], x[n_ctx:])
     assert e.value.status == mt._lib.MTGR_ERR_UNSUPPORTED
+
+
+def _with_rab(w, seed=5):
+    rng = np.random.default_rng(seed)
+    layers = []
+    for p in w["layers"]:
+        q = dict(p)
+        q["rab_pos"], q["rab_time"] = synth.make_rab_tables(w["H"], rng)
+        layers.append(q)
+    return layers
+
+
+@pytest.mark.parametrize("variant", [mt.MTGR_VARIANT_RAB, mt.MTGR_VARIANT_RAB | mt.MTGR_VARIANT_SILU_QKVU])
+def test_block_relative_attention_bias_matches_oracle(variant):
+    # ragged users (a 1000-token S run, tiles off the grid, a U-only user)
+    # and timestamp ties: every bucket and clip path of the bias
+    rng = np.random.default_rng(2)
+    lens = RAGGED
+    d, H, dff = 512, 8, 2048
+    ts = synth.make_timestamps(lens, rng)
+    x = synth.make_tokens(lens, d, rng)
+    w = dict(lens=lens, ts=ts, x=x, H=H, layers=[synth.make_block_params(d, dff, rng)])
+    layers = _with_rab(w)
+    b = mt.PackedBatch(lens, ts)
+    ws = [mt.BlockWeights(p, H, variant=variant) for p in layers]
+    y = to_host(mt.hstu_stack_forward(ws, b, torch.from_numpy(x).cuda()))
+    b.check()
+    ref = oracle.hstu_stack(x, lens, ts, layers, H, variant=variant)
+    assert_close_rms(y, ref, TOL_BF16, f"bias variant {variant}")
+    plain = oracle.hstu_stack(x, lens, ts, layers, H, variant=variant & ~mt.MTGR_VARIANT_RAB) - x
+    assert np.abs(plain - (ref - x)).max() > 0.1 * np.sqrt(np.mean(plain ** 2))
+
+
+def test_block_relative_attention_bias_full_workload_sampled_users():
+    w = synth.make_workload(2)
+    layers = _with_rab(w)
+    b = mt.PackedBatch(w["lens"], w["ts"])
+    ws = [mt.BlockWeights(p, w["H"], variant=mt.MTGR_VARIANT_RAB) for p in layers]
+    y = to_host(mt.hstu_stack_forward(ws, b, torch.from_numpy(w["x"]).cuda()))
+    b.check()
+    users = sample_users(w["lens"], k=2)
+    rows = user_rows(w["lens"], users)
+    ref = oracle.hstu_stack(w["x"][rows], w["lens"][users], w["ts"][rows], layers, w["H"],
+                            variant=mt.MTGR_VARIANT_RAB)
+    assert_close_rms(y[rows], ref, TOL_BF16, "bias variant, 512 users")
+
+
+def test_relative_attention_bias_needs_its_tables():
+    w = synth.make_workload(2, B=2)
+    b = mt.PackedBatch(w["lens"], w["ts"])
+    ws = [mt.BlockWeights(p, w["H"], variant=mt.MTGR_VARIANT_RAB) for p in w["layers"]]
+    with pytest.raises(mt.MTGRError) as e:
+        mt.hstu_stack_forward(ws, b, torch.from_numpy(w["x"]).cuda())
+    assert e.value.status == mt._lib.MTGR_ERR_INVALID_ARG

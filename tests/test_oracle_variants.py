@@ -233,3 +233,22 @@ def test_rab_time_term_ignores_u_tokens_and_shifts_scores():
     marked = np.array([[0, 0, 0, 0, 0, 0], [0, 0, 1, 1, 0, 0], [0, 1, 0, 0, 0, 1],
                        [0, 1, 0, 0, 0, 0], [0, 0, 0, 0, 0, 1], [0, 0, 1, 0, 1, 0]], bool)
     np.testing.assert_array_equal(b != 0, marked)
+
+
+def test_rab_bias_matches_the_entrywise_definition():
+    # brute force over every (i, j) of random small users against the scalar
+    # bucket function and the clip, ties and large gaps included
+    rng = np.random.default_rng(9)
+    H = 2
+    w_pos = rng.standard_normal((H, 2 * oracle.RAB_MAX_DIST + 1))
+    w_time = rng.standard_normal((H, oracle.RAB_TIME_BUCKETS))
+    for lens in ([3, 40, 9, 5], [0, 150, 2, 140], [1, 0, 0, 1]):
+        N = sum(lens)
+        ts = rng.integers(0, 3, N) * rng.integers(1, 1 << 40, N)
+        for h in range(H):
+            b = oracle.rab_bias(*lens, ts, w_pos, w_time, h)
+            for i in range(N):
+                for j in range(N):
+                    p = min(max(i - j, -oracle.RAB_MAX_DIST), oracle.RAB_MAX_DIST) + oracle.RAB_MAX_DIST
+                    tb = 0 if (i < lens[0] or j < lens[0]) else oracle.rab_time_bucket(abs(int(ts[i]) - int(ts[j])))
+                    assert b[i, j] == w_pos[h][p] + w_time[h][tb]
