@@ -151,6 +151,23 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int32_t w) {
   return it;
 }
 
+// The SiLU warps read an item's record, then their rows' rank-table indices
+// and the item's first tile entries, a chain of dependent loads at every
+// item start. These bring the lines into L1 ahead of time: the next record
+// at the start of an item, and, during its last k-tile, the lines that
+// record points to for this warp (the record is then an L1 hit).
+__device__ __forceinline__ void prefetch_record(const AttnArgs& a, int32_t w) {
+  prefetch_l1(a.work + w / a.H);
+}
+__device__ __forceinline__ void prefetch_item_rows(const AttnArgs& a, int32_t w, int q, int quarter) {
+  const Item nx = load_item(a, w);
+  const int qrow = nx.w.nq == 2 ? q : 0;  // one q-tile: both warps take its rows
+  const int32_t i0 = (nx.w.qt0 + qrow) * MTGR_TILE_M + quarter * 32;  // only rows of the user
+  if (i0 < nx.w.n) prefetch_l1(a.rt_cnt + nx.w.us + i0);
+  prefetch_l1(a.entries + nx.w.e0a);
+  if (nx.w.nq == 2) prefetch_l1(a.entries + nx.w.e0b);
+}
+
 __device__ __forceinline__ int32_t num_items(const AttnArgs& a) {
   const int64_t P = a.counts[3] < a.q_cap ? a.counts[3] : a.q_cap;
   return (int32_t)(P * a.H);
@@ -333,7 +350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // --------------------------------------------------- S issuer (MMA) --
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
-      int32_t g = 0, gb = 0, li = 0;
+      int32_t g = 0, li = 0;
+      int32_t gs_a = 0, gs_b = 0;  // rounds of the S_A, S_B slots
       Item nxt;
       if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
       for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
@@ -346,19 +364,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int st = g % KV_STAGES;
           if (!mbar_wait(&kv_full[st], (g / KV_STAGES) & 1)) { timed_out = true; break; }
           const uint32_t k_addr = smem_u32(sKV + st * 2 * TILE_BYTES);
-          for (int q = 0; q < (two ? 2 : 1); ++q) {
-            const int32_t r = q == 0 ? g : gb;
+          // two q-tiles: both slots, each with its own Q; one q-tile: the
+          // slots take alternate k-tiles, both with Q_A
+          const int q0 = two ? 0 : (t & 1), q1 = two ? 2 : q0 + 1;
+          for (int q = q0; q < q1; ++q) {
+            const int32_t r = q == 0 ? gs_a : gs_b;
             if (!mbar_wait(&s_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
             tc_fence_after();
-            const uint32_t q_addr = smem_u32(sQ + (2 * qb + q) * TILE_BYTES);
+            const uint32_t q_addr = smem_u32(sQ + (2 * qb + (two ? q : 0)) * TILE_BYTES);
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               tc_mma_ss(tmem + s_col(q), sdesc_sw128(q_addr + 32 * k, 16, 1024),
                         sdesc_sw128(k_addr + 32 * k, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
             }
             tc_commit(&s_full[q]);
+            if (q == 0) ++gs_a; else ++gs_b;
           }
-          if (two) ++gb;
           tc_commit(&kv_empty[st]);  // K read (V's reader commits separately)
         }
         if (!timed_out) tc_commit(&q_empty[qb]);
@@ -368,7 +389,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // -------------------------------------------------- PV issuer (MMA) --
     if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_f16(TM, DH, 0u, false, true);
-      int32_t g = 0, gb = 0, li = 0;
+      int32_t g = 0, li = 0;
+      int32_t gp_a = 0, gp_b = 0;  // rounds of the P_A, P_B slots
       Item nxt;
       if ((int32_t)blockIdx.x < n_items) nxt = load_item(a, blockIdx.x);
       for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
@@ -384,19 +406,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           const uint32_t v_addr = smem_u32(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
-          for (int q = 0; q < (two ? 2 : 1); ++q) {
-            const int32_t r = q == 0 ? g : gb;
+          // one q-tile: O_A and O_B accumulate alternate k-tiles (summed by
+          // the epilogue), each starting fresh at its first k-tile
+          const int q0 = two ? 0 : (t & 1), q1 = two ? 2 : q0 + 1;
+          const int32_t first_t = two ? 0 : q0;
+          for (int q = q0; q < q1; ++q) {
+            const int32_t r = q == 0 ? gp_a : gp_b;
             if (!mbar_wait(&p_full[q], r & 1)) { timed_out = true; break; }
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < TN / 16; ++k) {
               tc_mma_ts(tmem + o_col(q), tmem + p_col(q) + 8 * k,
                         sdesc_sw128(v_addr + 2048 * k, 16384, 1024), idesc_o,
-                        (t > 0 || k > 0) ? 1u : 0u);
+                        (t > first_t || k > 0) ? 1u : 0u);
             }
             tc_commit(&p_free[q]);
+            if (q == 0) ++gp_a; else ++gp_b;
           }
-          if (two) ++gb;
           tc_commit(&kv_empty[st]);
         }
         if (!timed_out) tc_commit(o_full);  // O complete (an item with no k-tiles: O unused)
@@ -418,14 +444,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t s_addr = tmem + lane_base + s_col(q);
     const uint32_t p_addr = tmem + lane_base + p_col(q);
     int32_t gq = 0;  // this q-tile slot's k-tile counter (barrier rounds)
-    int32_t gt = 0;  // k-tiles of two-q-tile items (rounds of the turn barriers)
+    int32_t gt = 0;  // turns on the sub-partition's MUFU pipe (rounds of the turn barriers)
     for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride) {
-      // no look-ahead copy of the next item here: the 64 registers of a
-      // row's scores leave no room for one
+      // no look-ahead copy of the next item in registers (a row's scores
+      // leave no room for one); its lines are prefetched into L1 instead
       const Item it = load_item(a, w);
-      if (q >= it.w.nq) continue;  // this item has no q-tile B
+      const bool has_next = w + stride < n_items;
+      if (lane == 0 && has_next) prefetch_record(a, w + stride);
+      // Two q-tiles: A takes q-tile A, B q-tile B, every k-tile. One q-tile:
+      // both take its rows, A the even and B the odd k-tiles of the union,
+      // so the item keeps both warps of a sub-partition (and its MUFU pipe)
+      // busy; their turns on the pipe alternate as for two q-tiles.
       const bool two = it.w.nq == 2;
-      const int32_t i = (it.w.qt0 + q) * TM + quarter * 32 + lane;  // user-relative row
+      const int qrow = two ? q : 0;  // the q-tile of this warp's rows
+      const int32_t i = (it.w.qt0 + qrow) * TM + quarter * 32 + lane;  // user-relative row
       const int32_t cnt_i = i < it.w.n ? __ldg(a.rt_cnt + it.w.us + i) : 0;
       const int64_t t_i = RAB && i < it.w.n ? __ldg(a.ts + it.w.us + i) : 0;
       UnionCursor cur;
@@ -438,7 +470,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto fetch = [&]() {
         int32_t ca, cb;
         kt_n = cur.next(ca, cb);
-        const int32_t code = q == 0 ? ca : cb;  // -1: EMPTY for this q-tile
+        const int32_t code = qrow == 0 ? ca : cb;  // -1: EMPTY for this q-tile
         masked_n = code < 0 || (code & 1) || kt_n * TN + TN > it.w.n;
         if (masked_n) {
           rt_lo_n = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN);
@@ -446,7 +478,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
       fetch();
-      for (int32_t t = 0; t < it.w.n_union; ++t, ++gq) {
+      for (int32_t t = 0; t < it.w.n_union; ++t) {
+        if (!two && (t & 1) != q) {  // the other warp's k-tile
+          if (t + 1 < it.w.n_union) fetch();
+          else if (lane == 0 && has_next) prefetch_item_rows(a, w + stride, q, quarter);
+          continue;
+        }
         const int32_t kt = kt_n;
         const bool masked = masked_n;
         const uint64_t rt_lo = rt_lo_n, rt_hi = rt_hi_n;
@@ -486,6 +523,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
         if (t + 1 < it.w.n_union) fetch();
+        else if (lane == 0 && has_next) prefetch_item_rows(a, w + stride, q, quarter);
         // The tanh of both q-tiles runs on the MUFU pipes (16 values per
         // clock per SM, one pipe per sub-partition), the bound of this
         // kernel. The A and B warps of one sub-partition (same lane quarter)
@@ -496,7 +534,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // pipe. Every wait is on a phase the other warp reaches without
         // waiting on this one (its previous turn), so the turns cannot
         // deadlock, and the two-slot rings keep each parity wait exact.
-        if (two && (q == 1 || gt > 0)) {
+        if (q == 1 || gt > 0) {
           uint64_t* bar = q == 0 ? &turn_a[2 * quarter + ((gt - 1) & 1)] : &turn_b[2 * quarter + (gt & 1)];
           const uint32_t par = q == 0 ? (((gt - 1) >> 1) & 1) : ((gt >> 1) & 1);
           if (!warp_wait(bar, par)) { timed_out = true; break; }
@@ -505,12 +543,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // P = h + h tanh(h) = silu(s), in place
 #pragma unroll
         for (int c = 0; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
-        if (two) {
-          reg_fence(h);  // hand over the turn only once this tile's tanh is done
-          __syncwarp();
-          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
-          ++gt;
-        }
+        reg_fence(h);  // hand over the turn only once this tile's tanh is done
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
+        ++gt;
         // P of the previous k-tile must have been consumed by its P V
         if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
         tc_fence_after();
@@ -520,6 +556,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[q]);
+        ++gq;
+      }
+      if (timed_out) break;
+      // one q-tile with an odd k-tile count: A took one turn more; B takes an
+      // empty turn so that the two keep alternating on the next item
+      if (!two && q == 1 && (it.w.n_union & 1)) {
+        if (!warp_wait(&turn_b[2 * quarter + (gt & 1)], (gt >> 1) & 1)) { timed_out = true; break; }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&turn_a[2 * quarter + (gt & 1)]);
+        ++gt;
       }
     }
     finish();
@@ -561,26 +607,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const bool empty = it.w.n_union <= 0;
       const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.w.b] : (float)it.w.n);
+      // one q-tile: O = O_A (even k-tiles) + O_B (odd k-tiles)
+      const bool sum_b = it.w.nq == 1 && it.w.n_union >= 2;
       for (int q = 0; q < it.w.nq; ++q) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tmem + lane_base + o_col(q), o0);
-        tmem_ld32(tmem + lane_base + o_col(q) + 32, o1);
-        tmem_ld_wait();
-        if (q == it.w.nq - 1) {  // all of O read: the next item may accumulate
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);
-        }
         const int32_t i = (it.w.qt0 + q) * TM + rr;
+        const int64_t row = it.w.us + i;
+        const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
         bool bad = false;  // a non-finite O: some P left the f16 range
-        if (i < it.w.n) {
-          const int64_t row = it.w.us + i;
-          const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {  // head columns [32 hf, 32 hf + 32)
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + o_col(q) + 32 * hf, o);
+          tmem_ld_wait();
+          if (sum_b) {
+            uint32_t ob[32];
+            tmem_ld32(tmem + lane_base + o_col(1) + 32 * hf, ob);
+            tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {  // columns [8k, 8k + 8) of the head
+            for (int c = 0; c < 32; ++c)
+              o[c] = __float_as_uint(__uint_as_float(o[c]) + __uint_as_float(ob[c]));
+          }
+          if (q == it.w.nq - 1 && hf == 1) {  // all of O read: the next item may accumulate
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+          }
+          if (i >= it.w.n) continue;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // columns [8k, 8k + 8) of the head
+            const int k = 4 * hf + kk;
             const uint4 x = *reinterpret_cast<const uint4*>(urow + ((k ^ (rr & 7)) << 4));
             const uint32_t uw[4] = {x.x, x.y, x.z, x.w};
-            float ov[8];
+            float ov[8], on[8];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               float u0, u1;
@@ -592,25 +650,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 u0 = __low2float(hh);
                 u1 = __high2float(hh);
               }
-              const int col = 8 * k + 2 * c;
-              const uint32_t r0 = col < 32 ? o0[col] : o1[col - 32];
-              const uint32_t r1 = col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32];
-              const float f0 = __uint_as_float(r0), f1 = __uint_as_float(r1);
+              const float f0 = __uint_as_float(o[8 * kk + 2 * c]), f1 = __uint_as_float(o[8 * kk + 2 * c + 1]);
               bad |= (f0 - f0) != 0.f || (f1 - f1) != 0.f;  // inf - inf, NaN - NaN: NaN
-              ov[2 * c] = __uint_as_float(r0) * inv_n * u0;
-              ov[2 * c + 1] = __uint_as_float(r1) * inv_n * u1;
+              on[2 * c] = f0 * inv_n;
+              on[2 * c + 1] = f1 * inv_n;
+              ov[2 * c] = on[2 * c] * u0;
+              ov[2 * c + 1] = on[2 * c + 1] * u1;
             }
-            if (a.obar != nullptr) {
-              uint32_t w[4];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int col = 8 * k + 2 * c;
-                const float x0 = __uint_as_float(col < 32 ? o0[col] : o1[col - 32]);
-                const float x1 = __uint_as_float(col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32]);
-                w[c] = cvt_bf16x2(x0 * inv_n, x1 * inv_n);
-              }
-              *reinterpret_cast<uint4*>(a.obar + row * d + it.h * DH + 8 * k) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+            if (a.obar != nullptr)
+              *reinterpret_cast<uint4*>(a.obar + row * d + it.h * DH + 8 * k) =
+                  make_uint4(cvt_bf16x2(on[0], on[1]), cvt_bf16x2(on[2], on[3]),
+                             cvt_bf16x2(on[4], on[5]), cvt_bf16x2(on[6], on[7]));
             if (OUT_F32) {
               float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * d + it.h * DH + 8 * k);
               op[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
