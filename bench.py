@@ -66,6 +66,10 @@ def parse_args():
     ap.add_argument("--serving", action="store_true",
                     help="cached-context candidate scoring on the 512-user block workload: the "
                          "candidate pass against the aggregated pass (one JSON line)")
+    ap.add_argument("--sweep-users", type=int, default=0,
+                    help="with --config 4: run the candidate sweep over this many users per "
+                         "launch (aggregated, cached-context and expanded legs), so that the "
+                         "cost per added candidate is not launch latency")
     ap.add_argument("--backward", action="store_true",
                     help="one training step of the block on the 512-user block workload: the "
                          "forward keeping its activations, then the backward (one JSON line, "
@@ -634,6 +638,114 @@ def run_sweep(args, local):
     print(json.dumps(line), flush=True)
 
 
+def expanded_rows(agg: dict, rows: int) -> dict:
+    """`rows` expanded rows [U, S, R, c] taken user by user, candidate by
+    candidate, from a many-user aggregated sweep batch: each row repeats its
+    user's U, S, R tokens and holds one of its candidates, with the
+    aggregated user's normaliser N = N_U + N_S + N_R + K."""
+    lens = np.asarray(agg["lens"])
+    n_u, n_s, n_r, K = (int(v) for v in lens[0])
+    n_ctx, n = n_u + n_s + n_r, n_u + n_s + n_r + K
+    xs, tss = [], []
+    for r in range(rows):
+        b, c = divmod(r, K)
+        s0 = b * n
+        xs += [agg["x"][s0:s0 + n_ctx], agg["x"][s0 + n_ctx + c:s0 + n_ctx + c + 1]]
+        tss += [agg["ts"][s0:s0 + n_ctx], agg["ts"][s0 + n_ctx + c:s0 + n_ctx + c + 1]]
+    out = dict(agg)
+    out["lens"] = np.tile(np.array([[n_u, n_s, n_r, 1]], np.int32), (rows, 1))
+    out["x"] = np.concatenate(xs, axis=0)
+    out["ts"] = np.concatenate(tss)
+    out["norm"] = np.full(rows, float(n), np.float32)
+    out["kind"] = "sweep_expanded"
+    return out
+
+
+def run_sweep_batched(args, local):
+    """The candidate sweep with many users per launch: B users of the sweep's
+    shape (N_U 24, S 1000, R 64, d_model 512, one block), each with K
+    candidates, K in 1, 8, 64, 512. Legs per K:
+      aggregated: pack + metadata + block over the B samples [U, S, R, c_1..c_K];
+      cached: the cached-context candidate pass (the B contexts computed once,
+        every layer's Q|K|V|U kept; per request only the candidate rows);
+      expanded: B K rows [U, S, R, c_i] at the same normaliser, timed on up to
+        4096 rows and scaled by the row count (rows are independent users of
+        equal length, so their cost is linear in the row count).
+    Reported: ms per step and per candidate for each leg, and the aggregated
+    pass's marginal cost per added candidate between K = 1 and K = 512."""
+    import generative_recommendation_ranking_b200 as mt
+    from generative_recommendation_ranking_b200 import _lib
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    B = args.sweep_users
+    n = max(5, min(args.steps, 30))
+    rows_out = []
+    for K in synth.WORKLOADS[4].sweep_k:
+        agg = synth.make_workload(4, seed=args.seed, k_override=K, B=B)
+        res = {"K": K, "candidates": B * K}
+        wsp = Workspace(agg, dev, stream)
+        for _ in range(max(3, args.warmup)):
+            wsp.step()
+        wsp.batch.check()
+        ms = time_steps(wsp.step, n, stream) / n
+        wsp.batch.check()
+        res["aggregated_ms"] = ms
+        res["aggregated_ms_per_candidate"] = ms / (B * K)
+        # cached contexts: the candidate pass over all B users
+        lens = agg["lens"]
+        x = wsp.x
+        gid = torch.from_numpy(np.repeat(np.tile(np.arange(4), B), lens.reshape(-1).astype(np.int64))).to(dev)
+        x_cand = x[gid == 3].contiguous()
+        cc = mt.BatchContextCache(wsp.layers, lens, agg["ts"], x, stream=stream)
+        cbatch = cc.candidate_batch(agg["ts"], stream)
+        cws = cc.workspace()
+        out = torch.empty(cc.k_total, agg["d"], dtype=torch.float32, device=dev)
+        c_layers = [l.c for l in wsp.layers]
+
+        def cand_step():
+            cbatch.pack(stream)
+            cbatch.build_meta(stream)
+            _lib.mtgr_stack_fwd_candidates(c_layers, cbatch.c, cc.k_total, cc.cache, cc.T, x_cand,
+                                           out, cws, stream)
+
+        for _ in range(max(3, args.warmup)):
+            cand_step()
+        cbatch.check()
+        ms = time_steps(cand_step, n, stream) / n
+        cbatch.check()
+        res["cached_ms"] = ms
+        res["cached_ms_per_candidate"] = ms / (B * K)
+        del cc, cbatch, cws, out, x_cand, wsp
+        torch.cuda.empty_cache()
+        # expanded rows, scaled linearly from at most 4096 rows
+        rows = min(B * K, 4096)
+        ex = Workspace(expanded_rows(agg, rows), dev, stream)
+        for _ in range(max(3, args.warmup)):
+            ex.step()
+        ex.batch.check()
+        ms = time_steps(ex.step, n, stream) / n
+        ex.batch.check()
+        res["expanded_rows_timed"] = rows
+        res["expanded_ms_per_candidate"] = ms / rows
+        res["expanded_ms"] = ms / rows * B * K
+        del ex
+        torch.cuda.empty_cache()
+        rows_out.append(res)
+    first, last = rows_out[0], rows_out[-1]
+    marginal = (last["aggregated_ms"] - first["aggregated_ms"]) / (B * (last["K"] - first["K"]))
+    line = {"metric": "candidate sweep, many users per launch: HSTU-block fwd ms per candidate, "
+                      "aggregated vs cached context vs expanded rows",
+            "unit": "ms", "higher_is_better": False, "data": "synthetic", "dtype": "bf16",
+            "config": {"workload": f"sweep_b{B}_d512", "users": B, "d_model": 512, "heads": 8,
+                       "d_ff": 2048, "n_u": 24, "s": 1000, "r": 64},
+            "sweep": rows_out,
+            "aggregated_marginal_ms_per_added_candidate": marginal,
+            "expanded_ms_per_candidate_at_k512": last["expanded_ms_per_candidate"],
+            "marginal_vs_expanded": marginal / last["expanded_ms_per_candidate"]}
+    print(json.dumps(line), flush=True)
+
+
 def run_serving(args, local):
     """Serving with cached contexts on the 512-user block workload: the
     contexts (U, S, R) of all users run once with every layer's Q|K|V|U kept;
@@ -907,7 +1019,10 @@ def main():
                 run_backward(args, local)
         elif synth.WORKLOADS[args.config].kind == "sweep":
             if rank == 0:
-                run_sweep(args, local)
+                if args.sweep_users > 0:
+                    run_sweep_batched(args, local)
+                else:
+                    run_sweep(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -94,3 +94,22 @@ def test_tensor_peak_follows_the_timed_region_length():
     assert bench.tensor_peak_key(bench.SUSTAINED_AFTER_S - 1e-3) == "bf16_tflops"
     assert bench.tensor_peak_key(bench.SUSTAINED_AFTER_S) == "bf16_tflops_sustained"
     assert bench.tensor_peak_key(30.0) == "bf16_tflops_sustained"
+
+
+def test_expanded_rows_of_a_many_user_sweep_batch():
+    # row r is user r // K's context with its candidate r % K, at the
+    # aggregated user's normaliser
+    import bench
+    import synth
+    K, B = 8, 3
+    agg = synth.make_workload(4, seed=1, k_override=K, B=B)
+    ex = bench.expanded_rows(agg, 11)
+    n_ctx, n = 1088, 1088 + K
+    assert ex["lens"].shape == (11, 4) and (ex["lens"][:, 3] == 1).all()
+    assert (ex["norm"] == n).all()
+    for r in (0, 7, 8, 10):
+        b, c = divmod(r, K)
+        row = ex["x"][r * (n_ctx + 1):(r + 1) * (n_ctx + 1)]
+        np.testing.assert_array_equal(row[:n_ctx], agg["x"][b * n:b * n + n_ctx])
+        np.testing.assert_array_equal(row[n_ctx], agg["x"][b * n + n_ctx + c])
+        np.testing.assert_array_equal(ex["ts"][r * (n_ctx + 1) + n_ctx], agg["ts"][b * n + n_ctx + c])
