@@ -376,60 +376,60 @@ def time_steps(fn, n, stream) -> float:
 
 
 def run_e2e(wsp: Workspace, steps: int, world: int, dev, users_total: int):
-    """The same step end to end through the C ABI with pinned host buffers:
-    every step copies its inputs host->device and its whole output back. Copies
-    in, compute and copies out run on three streams with two buffer sets, so
-    step k's output copy overlaps step k+1's input copy (PCIe is full duplex)."""
+    """The same step end to end through the C ABI's host-buffer entry
+    (mtgr_stack_fwd_host): every call copies the step's lengths, timestamps
+    and token features from pinned host memory into the device workspace,
+    packs, builds the mask metadata, runs the stack and copies the whole
+    output and the status word back. Steps alternate between two streams,
+    each with its own workspace, so one step's copies overlap the other's
+    kernels (PCIe is full duplex). Attention-only workloads keep the
+    device-pointer path (the host entry runs the block stack)."""
+    import generative_recommendation_ranking_b200 as mt
+    from generative_recommendation_ranking_b200 import _lib
     wl = wsp.wl
-    hx = torch.from_numpy(np.ascontiguousarray(wl["qkvu"] if wsp.kind == "attention" else wl["x"]))
-    hx = (hx.to(torch.bfloat16) if wsp.kind == "attention" else hx).pin_memory()
-    hl = torch.from_numpy(np.ascontiguousarray(wl["lens"])).pin_memory()
-    ht = torch.from_numpy(np.ascontiguousarray(wl["ts"])).pin_memory()
-    hout = [torch.empty(wsp.out.shape, dtype=wsp.out.dtype).pin_memory() for _ in range(2)]
-    dx = [torch.empty_like(wsp.x) for _ in range(2)]
-    dl = [torch.empty_like(wsp.batch.d_lens) for _ in range(2)]
-    dts = [torch.empty_like(wsp.batch.d_ts) for _ in range(2)]
-    dout = [torch.empty_like(wsp.out) for _ in range(2)]
-    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "cmp", "out")}
-    h2d = hx.numel() * hx.element_size() + hl.numel() * 4 + ht.numel() * 8
-    d2h = hout[0].numel() * hout[0].element_size()
+    if wsp.kind == "attention":
+        return None
+    hl = torch.from_numpy(np.ascontiguousarray(wl["lens"], np.int32)).pin_memory()
+    ht = torch.from_numpy(np.ascontiguousarray(wl["ts"], np.int64)).pin_memory()
+    hn = (torch.from_numpy(np.ascontiguousarray(wl["norm"], np.float32)).pin_memory()
+          if wl.get("norm") is not None else None)
+    hx = torch.from_numpy(np.ascontiguousarray(wl["x"], np.float32)).pin_memory()
+    hout = [torch.empty_like(hx).pin_memory() for _ in range(2)]
+    hst = [torch.zeros(1, dtype=torch.int32).pin_memory() for _ in range(2)]
+    c_layers = [l.c for l in wsp.layers]
+    nbytes = _lib.mtgr_stack_fwd_host_workspace_bytes(hl, c_layers)
+    dws = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    streams = [torch.cuda.Stream(dev) for _ in range(2)]
+    h2d = hl.numel() * 4 + ht.numel() * 8 + hx.numel() * 4 + (hn.numel() * 4 if hn is not None else 0)
+    d2h = hout[0].numel() * 4 + 4
 
     def run(n):
         for k in range(n):
             i = k & 1
-            s_in.wait_event(ev["cmp"][i])   # step k-2 has finished reading these inputs
-            with torch.cuda.stream(s_in):
-                dx[i].copy_(hx, non_blocking=True)
-                dl[i].copy_(hl, non_blocking=True)
-                dts[i].copy_(ht, non_blocking=True)
-            ev["in"][i].record(s_in)
-            s_cmp.wait_event(ev["in"][i])
-            s_cmp.wait_event(ev["out"][i])  # step k-2's output has been copied out
-            wsp.step(dl[i], dts[i], dx[i], dout[i], stream=s_cmp)
-            ev["cmp"][i].record(s_cmp)
-            s_out.wait_event(ev["cmp"][i])
-            with torch.cuda.stream(s_out):
-                hout[i].copy_(dout[i], non_blocking=True)
-            ev["out"][i].record(s_out)
+            _lib.mtgr_stack_fwd_host(c_layers, hl, ht, hn, hx, hout[i], hst[i], dws[i], streams[i])
 
     run(2)
     torch.cuda.synchronize(dev)
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    cur = torch.cuda.current_stream(dev)
+    ev[0].record(cur)
+    for st in streams:
+        st.wait_stream(cur)
     run(steps)
-    s_in.wait_stream(s_out)
-    e1.record(s_in)
+    for st in streams:
+        cur.wait_stream(st)
+    ev[1].record(cur)
     torch.cuda.synchronize(dev)
-    ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    wsp.batch.check()
+    ems = max_over_ranks(ev[0].elapsed_time(ev[1]), world, dev)
+    assert all(int(h.item()) == 0 for h in hst), "e2e device status"
     wsp.step()
     torch.cuda.synchronize(dev)
     assert torch.equal(hout[(steps - 1) & 1], wsp.out.cpu()), "e2e output mismatch"
     return {"value": users_total * steps / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ems / steps,
-            "pipelining": "3 streams (copy in / compute / copy out), 2 buffer sets"}
+            "path": "C ABI mtgr_stack_fwd_host (host buffers in, host buffers out)",
+            "pipelining": "2 streams, 2 workspaces: one step's copies overlap the other's kernels"}
 
 
 def run_ours(args, world, rank, local):

@@ -138,6 +138,9 @@ _SIGNATURES = {
     "mtgr_timer_read": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_double),
                                        ctypes.POINTER(ctypes.c_int64)]),
     "mtgr_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, c_vp, c_vp]),
+    "mtgr_stack_fwd_host_workspace_bytes": (c_size, [c_i32, c_vp, c_vp, c_i32]),
+    "mtgr_stack_fwd_host": (ctypes.c_int, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                           c_vp, c_size, c_vp]),
     "mtgr_block_saved_bytes": (c_size, [c_i32, ctypes.POINTER(MtgrBlockParams)]),
     "mtgr_hstu_block_fwd_train": (ctypes.c_int, [ctypes.POINTER(MtgrBlockParams),
                                                  ctypes.POINTER(MtgrBatch), c_vp, c_vp, c_vp,
@@ -395,3 +398,26 @@ def mtgr_hstu_block_bwd(p: MtgrBlockParams, batch: MtgrBatch, d_x_in, d_saved, d
     _check("mtgr_hstu_block_bwd", load().mtgr_hstu_block_bwd(
         ctypes.byref(p), ctypes.byref(batch), _ptr(d_x_in), _ptr(d_saved), _ptr(d_dy), _ptr(d_dx),
         ctypes.byref(grads), _ptr(d_ws), d_ws.numel() * d_ws.element_size(), _stream(stream)))
+
+
+def _layer_array(layers):
+    arr = (MtgrBlockParams * len(layers))(*layers)
+    return arr
+
+
+def mtgr_stack_fwd_host_workspace_bytes(h_lens, layers) -> int:
+    """h_lens: host int32 tensor [B, 4]; layers: MtgrBlockParams list."""
+    arr = _layer_array(layers)
+    return load().mtgr_stack_fwd_host_workspace_bytes(int(h_lens.shape[0]), _ptr(h_lens), arr,
+                                                      len(layers))
+
+
+def mtgr_stack_fwd_host(layers, h_lens, h_ts, h_norm, h_x_in, h_x_out, h_status, d_ws,
+                        stream=None) -> None:
+    """Host tensors (pinned) h_lens [B,4] int32, h_ts [T] int64, h_norm [B] float32 or None,
+    h_x_in / h_x_out [T, d] float32, h_status [1] int32; d_ws a device workspace."""
+    arr = _layer_array(layers)
+    _check("mtgr_stack_fwd_host", load().mtgr_stack_fwd_host(
+        arr, len(layers), int(h_lens.shape[0]), _ptr(h_lens), _ptr(h_ts), _ptr(h_norm),
+        _ptr(h_x_in), _ptr(h_x_out), _ptr(h_status), _ptr(d_ws),
+        d_ws.numel() * d_ws.element_size(), _stream(stream)))

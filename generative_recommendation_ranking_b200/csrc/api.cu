@@ -1161,6 +1161,173 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
                         d_status, as_stream(stream));
 }
 
+// ------------------------------------------------------- host-buffer forward --
+namespace {
+
+struct HostCaps {
+  int64_t T, q_cap, kt_cap, e_cap, rt_cap;
+};
+
+// Capacities of the mask metadata from the host lengths: q-tiles, the
+// largest per-user k-tile count, an upper bound on tile entries and the
+// rank-table entries (64-key groups holding R keys x (N_R + 1)).
+bool host_caps(int32_t B, const int32_t* lens, HostCaps* c) {
+  c->T = c->q_cap = c->kt_cap = c->e_cap = c->rt_cap = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t nu = lens[4 * b], ns = lens[4 * b + 1], nr = lens[4 * b + 2], nk = lens[4 * b + 3];
+    if (nu < 0 || ns < 0 || nr < 0 || nk < 0) return false;
+    const int64_t n = nu + ns + nr + nk;
+    const int64_t nt = (n + MTGR_TILE_M - 1) / MTGR_TILE_M;
+    c->T += n;
+    c->q_cap += nt;
+    c->kt_cap = nt > c->kt_cap ? nt : c->kt_cap;
+    c->e_cap += nt * nt;
+    const int64_t n_us = nu + ns, c_lo = n_us + nr;
+    const int64_t groups = nr > 0 ? (c_lo - 1) / 64 - n_us / 64 + 1 : 0;
+    c->rt_cap += groups * (nr + 1);
+  }
+  return c->T <= INT32_MAX && c->q_cap <= INT32_MAX && c->e_cap <= INT32_MAX &&
+         c->kt_cap <= kMaxKtCapacity;
+}
+
+struct HostWs {
+  int32_t* lens;
+  int64_t* ts;
+  float* norm;
+  float* x_in;
+  float* x_out;
+  int32_t* seg_off;
+  int32_t* user_off;
+  int8_t* group_id;
+  int32_t* status;
+  int32_t* qtile_desc;
+  int32_t* row_ptr;
+  int32_t* entries;
+  int32_t* order;
+  int64_t* counts;
+  int32_t* rt_cnt;
+  int64_t* rt_off;
+  uint64_t* rt_mask;
+  mtgr_work_item* work;
+  void* meta_ws;
+  void* stack_ws;
+  size_t stack_bytes;
+  size_t bytes;
+};
+
+HostWs host_ws_layout(int32_t B, const HostCaps& c, int32_t d, size_t stack_bytes, void* base) {
+  uint8_t* b = static_cast<uint8_t*>(base);
+  HostWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    uint8_t* p = b + off;
+    off += align_up(n > 0 ? n : 1, 256);
+    return p;
+  };
+  const size_t T = (size_t)c.T, q = (size_t)c.q_cap;
+  w.lens = reinterpret_cast<int32_t*>(take((size_t)B * 4 * 4));
+  w.ts = reinterpret_cast<int64_t*>(take(T * 8));
+  w.norm = reinterpret_cast<float*>(take((size_t)B * 4));
+  w.x_in = reinterpret_cast<float*>(take(T * d * 4));
+  w.x_out = reinterpret_cast<float*>(take(T * d * 4));
+  w.seg_off = reinterpret_cast<int32_t*>(take((4 * (size_t)B + 1) * 4));
+  w.user_off = reinterpret_cast<int32_t*>(take(((size_t)B + 1) * 4));
+  w.group_id = reinterpret_cast<int8_t*>(take(T));
+  w.status = reinterpret_cast<int32_t*>(take(4));
+  w.qtile_desc = reinterpret_cast<int32_t*>(take(q * 2 * 4));
+  w.row_ptr = reinterpret_cast<int32_t*>(take((q + 1) * 4));
+  w.entries = reinterpret_cast<int32_t*>(take((size_t)c.e_cap * 4));
+  w.order = reinterpret_cast<int32_t*>(take(q * 4));
+  w.counts = reinterpret_cast<int64_t*>(take(4 * 8));
+  w.rt_cnt = reinterpret_cast<int32_t*>(take(T * 4));
+  w.rt_off = reinterpret_cast<int64_t*>(take(((size_t)B + 1) * 8));
+  w.rt_mask = reinterpret_cast<uint64_t*>(take((size_t)c.rt_cap * 8));
+  w.work = reinterpret_cast<mtgr_work_item*>(take(q * sizeof(mtgr_work_item)));
+  w.meta_ws = take(mask_meta_ws_bytes((int32_t)c.q_cap, (int32_t)c.kt_cap));
+  w.stack_bytes = stack_bytes;
+  w.stack_ws = take(stack_bytes);
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+MTGR_API size_t mtgr_stack_fwd_host_workspace_bytes(int32_t B, const int32_t* h_lens,
+                                                    const mtgr_block_params* layers, int32_t L) {
+  if (B < 0 || (B > 0 && h_lens == nullptr) || layers == nullptr || L <= 0) return 0;
+  HostCaps c;
+  if (!host_caps(B, h_lens, &c)) return 0;
+  const size_t sb = mtgr_stack_workspace_bytes((int32_t)c.T, layers, L);
+  if (sb == 0 && c.T > 0) return 0;
+  return host_ws_layout(B, c, layers[0].d, sb, nullptr).bytes;
+}
+
+MTGR_API int mtgr_stack_fwd_host(const mtgr_block_params* layers, int32_t L, int32_t B,
+                                 const int32_t* h_lens, const int64_t* h_ts, const float* h_norm,
+                                 const float* h_x_in, float* h_x_out, int32_t* h_status,
+                                 void* d_ws, size_t ws_bytes, mtgr_stream_t stream) {
+  if (layers == nullptr || L <= 0 || B < 0 || (B > 0 && h_lens == nullptr) || h_status == nullptr ||
+      d_ws == nullptr || !aligned16(d_ws))
+    return MTGR_ERR_INVALID_ARG;
+  HostCaps c;
+  if (!host_caps(B, h_lens, &c)) return MTGR_ERR_INVALID_ARG;
+  if (c.T > 0 && (h_ts == nullptr || h_x_in == nullptr || h_x_out == nullptr))
+    return MTGR_ERR_INVALID_ARG;
+  const size_t sb = mtgr_stack_workspace_bytes((int32_t)c.T, layers, L);
+  if (sb == 0 && c.T > 0) return MTGR_ERR_INVALID_ARG;
+  const int32_t d = layers[0].d;
+  const HostWs w = host_ws_layout(B, c, d, sb, d_ws);
+  if (ws_bytes < w.bytes) return MTGR_ERR_CAPACITY;
+  const cudaStream_t s = as_stream(stream);
+  const size_t T = (size_t)c.T;
+  auto h2d = [&](void* dst, const void* src, size_t n) {
+    return n == 0 || cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  };
+  if (cudaMemsetAsync(w.status, 0, 4, s) != cudaSuccess) return MTGR_ERR_CUDA;
+  if (!h2d(w.lens, h_lens, (size_t)B * 16) || !h2d(w.ts, h_ts, T * 8) ||
+      (h_norm != nullptr && !h2d(w.norm, h_norm, (size_t)B * 4)) ||
+      !h2d(w.x_in, h_x_in, T * d * 4))
+    return MTGR_ERR_CUDA;
+  int rc = mtgr_pack_offsets(B, w.lens, (int32_t)c.T, w.seg_off, w.user_off, w.group_id, w.status,
+                             stream);
+  if (rc != MTGR_OK) return rc;
+  rc = mtgr_build_mask_meta(B, w.seg_off, w.ts, (int32_t)c.q_cap, (int32_t)c.kt_cap,
+                            (int32_t)c.e_cap, c.rt_cap, w.qtile_desc, w.row_ptr, w.entries, w.order,
+                            w.counts, w.rt_cnt, w.rt_off, w.rt_mask, w.work, w.meta_ws,
+                            mask_meta_ws_bytes((int32_t)c.q_cap, (int32_t)c.kt_cap), w.status,
+                            stream);
+  if (rc != MTGR_OK) return rc;
+  mtgr_batch bt{};
+  bt.B = B;
+  bt.T = (int32_t)c.T;
+  bt.q_capacity = (int32_t)c.q_cap;
+  bt.kt_capacity = (int32_t)c.kt_cap;
+  bt.seg_off = w.seg_off;
+  bt.user_off = w.user_off;
+  bt.group_id = w.group_id;
+  bt.ts = w.ts;
+  bt.qtile_desc = w.qtile_desc;
+  bt.row_ptr = w.row_ptr;
+  bt.entries = w.entries;
+  bt.order = w.order;
+  bt.counts = w.counts;
+  bt.rt_cnt = w.rt_cnt;
+  bt.rt_off = w.rt_off;
+  bt.rt_mask = w.rt_mask;
+  bt.work = w.work;
+  bt.norm = h_norm != nullptr ? w.norm : nullptr;
+  bt.status = w.status;
+  if (c.T > 0) {
+    rc = mtgr_stack_fwd(layers, L, &bt, w.x_in, w.x_out, w.stack_ws, w.stack_bytes, stream);
+    if (rc != MTGR_OK) return rc;
+    if (cudaMemcpyAsync(h_x_out, w.x_out, T * d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return MTGR_ERR_CUDA;
+  }
+  if (cudaMemcpyAsync(h_status, w.status, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MTGR_ERR_CUDA;
+  return MTGR_OK;
+}
+
 MTGR_API size_t mtgr_block_saved_bytes(int32_t T, const mtgr_block_params* p) {
   if (T < 0 || params_check(p) != MTGR_OK) return 0;
   return saved_layout(T, p, nullptr).bytes;

@@ -358,6 +358,33 @@ MTGR_API int mtgr_stack_fwd(const mtgr_block_params* layers, int32_t L, const mt
                             mtgr_stream_t stream);
 
 /*
+ * The whole forward from HOST buffers, for callers that keep their batches in
+ * host memory (a C serving process, or a pipeline that stages batches from
+ * disk): one call enqueues on `stream` the copies of the lengths, timestamps,
+ * optional normalisers and token features into the device workspace, the
+ * packing, the mask metadata, the L-block stack and the copies of the output
+ * rows and the status word back to the host. Nothing is allocated: the device
+ * workspace (mtgr_stack_fwd_host_workspace_bytes) holds the staged inputs,
+ * the batch, its metadata and the stack's workspace.
+ *   h_lens [B][4] int32, h_ts [T] int64, h_norm [B] float (or NULL),
+ *   h_x_in, h_x_out [T][d] float32: HOST memory, pinned (page-locked) for the
+ *     copies to be asynchronous; they must stay valid and untouched until
+ *     the stream has passed this call's work
+ *   h_status: host int32, written by the final copy (0 = ok, else a device
+ *     status such as MTGR_ERR_DEVICE_VALIDATION), valid once the stream has
+ *     synchronised
+ * T is the sum of h_lens (computed here, on the host). Calls sharing a
+ * workspace must be ordered; two workspaces on two streams let one call's
+ * copies overlap the other's kernels.
+ */
+MTGR_API size_t mtgr_stack_fwd_host_workspace_bytes(int32_t B, const int32_t* h_lens,
+                                                    const mtgr_block_params* layers, int32_t L);
+MTGR_API int mtgr_stack_fwd_host(const mtgr_block_params* layers, int32_t L, int32_t B,
+                                 const int32_t* h_lens, const int64_t* h_ts, const float* h_norm,
+                                 const float* h_x_in, float* h_x_out, int32_t* h_status,
+                                 void* d_ws, size_t ws_bytes, mtgr_stream_t stream);
+
+/*
  * Candidate-incremental scoring (serving). A user's U, S and R tokens never
  * attend to candidates (mask rules 1-3), so the context side of every layer
  * is computed once and candidates are scored against it afterwards, in one

@@ -131,3 +131,25 @@ def test_temporal_replay_bit_exact_on_gpu():
     y2 = _gpu_stack(w, x=x2)
     np.testing.assert_array_equal(y2[c], y[c])
     assert not np.array_equal(y2[late[0]], y[late[0]])
+
+
+def test_host_buffer_entry_matches_the_device_path():
+    # mtgr_stack_fwd_host (host lengths, timestamps, features in; host rows
+    # out) against the device-pointer stack on the same batch: bit-exact
+    from generative_recommendation_ranking_b200 import _lib
+    w = synth.make_workload(2, B=9, seed=6)
+    y_dev = _gpu_stack(w)
+    layers = [mt.BlockWeights(p, w["H"], dtype=w["dtype"]) for p in w["layers"]]
+    hl = torch.from_numpy(np.ascontiguousarray(w["lens"], np.int32)).pin_memory()
+    ht = torch.from_numpy(np.ascontiguousarray(w["ts"], np.int64)).pin_memory()
+    hx = torch.from_numpy(np.ascontiguousarray(w["x"], np.float32)).pin_memory()
+    ho = torch.full_like(hx, float("nan")).pin_memory()
+    hs = torch.full((1,), -1, dtype=torch.int32).pin_memory()
+    c_layers = [l.c for l in layers]
+    ws = torch.full((_lib.mtgr_stack_fwd_host_workspace_bytes(hl, c_layers),), 0xFF,
+                    dtype=torch.uint8, device="cuda")
+    for _ in range(2):  # a second call on the dirty workspace gives the same rows
+        _lib.mtgr_stack_fwd_host(c_layers, hl, ht, None, hx, ho, hs, ws)
+        torch.cuda.synchronize()
+        assert int(hs.item()) == 0
+        np.testing.assert_array_equal(ho.numpy(), y_dev)

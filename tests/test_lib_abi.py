@@ -212,3 +212,26 @@ def test_training_entry_points_validate_on_the_host(lib):
     # missing gradient outputs
     assert lib.mtgr_hstu_block_bwd(ctypes.byref(p), ctypes.byref(b), None, None, None, None,
                                    ctypes.byref(g), None, 0, None) == _lib.MTGR_ERR_INVALID_ARG
+
+
+def test_host_entry_workspace_and_validation(lib):
+    # the host-buffer forward sizes its workspace from the host lengths: the
+    # staged inputs, the batch and metadata at api.capacities, the stack's
+    # workspace; bad arguments are refused before any device work
+    import torch
+    p = _lib.MtgrBlockParams(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16, eps=1e-5, variant=0,
+                             gln1_gamma=16, gln1_beta=16, gln2_gamma=16, gln2_beta=16,
+                             w_qkvu=16, w1=16, w2=16)
+    lens = torch.tensor([[24, 300, 20, 32], [24, 1000, 100, 256], [0, 0, 0, 0]], dtype=torch.int32)
+    T = int(lens.sum())
+    q_cap, kt_cap, e_cap, rt_cap = api.capacities(lens.numpy())
+    need = _lib.mtgr_stack_fwd_host_workspace_bytes(lens, [p])
+    stack = _lib.mtgr_stack_workspace_bytes(T, [p])
+    at_least = T * 512 * 4 * 2 + T * 8 + e_cap * 4 + rt_cap * 8 + q_cap * 64 + stack
+    assert at_least <= need <= at_least + 64 * 256 + 8 * T + 4 * T + 64 * q_cap
+    bad = torch.tensor([[1, -2, 0, 0]], dtype=torch.int32)
+    assert _lib.mtgr_stack_fwd_host_workspace_bytes(bad, [p]) == 0
+    st = torch.zeros(1, dtype=torch.int32)
+    arr = _lib._layer_array([p])
+    assert lib.mtgr_stack_fwd_host(arr, 1, 3, lens.data_ptr(), None, None, None, None,
+                                   st.data_ptr(), None, 0, None) == _lib.MTGR_ERR_INVALID_ARG
