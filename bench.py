@@ -245,6 +245,18 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def dtype_label(wl: dict) -> str:
+    """The arithmetic the step computes in. bf16 blocks: bf16 GEMM operands
+    with fp32 accumulation and an fp32 residual stream; the attention takes
+    Q|K|V|U and its silu weights P in f16 and accumulates Q K^T and P V in
+    fp32."""
+    if wl["dtype"] == "f32":
+        return "f32"
+    if wl["kind"] == "attention":
+        return "bf16 (attention: Q|K|V|U bf16, P and V f16, fp32 accumulate)"
+    return "bf16 (GEMMs bf16 -> fp32 accumulate; attention Q|K|V|U and P f16, fp32 accumulate)"
+
+
 def rank_workload(args, world: int, rank: int):
     """This rank's workload and the global user count. One GPU: the workload
     itself. N GPUs: one global batch of N x B users drawn with the same seed
@@ -539,7 +551,7 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wl["dtype"], "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_label(wl), "data": "synthetic",
         "config": workload_config(wl, world, B_global),
         "masked_attn": {"tflops": att.get("achieved"),
                         "frac_of_bf16_peak": att.get("frac"),
