@@ -248,13 +248,14 @@ def run_reference(args, world, rank):
 def dtype_label(wl: dict) -> str:
     """The arithmetic the step computes in. bf16 blocks: bf16 GEMM operands
     with fp32 accumulation and an fp32 residual stream; the attention takes
-    Q|K|V|U and its silu weights P in f16 and accumulates Q K^T and P V in
-    fp32."""
+    Q|K|V|U and its silu weights P in f16, sums Q K^T in f16 (an overflow
+    sets MTGR_ERR_RANGE) and P V in fp32."""
     if wl["dtype"] == "f32":
         return "f32"
     if wl["kind"] == "attention":
         return "bf16 (attention: Q|K|V|U bf16, P and V f16, fp32 accumulate)"
-    return "bf16 (GEMMs bf16 -> fp32 accumulate; attention Q|K|V|U and P f16, fp32 accumulate)"
+    return ("bf16 (GEMMs bf16 -> fp32 accumulate; attention: Q|K|V|U f16, Q.K^T f16 accumulate "
+            "(overflow reported), P f16, P.V fp32 accumulate)")
 
 
 def rank_workload(args, world: int, rank: int):

@@ -58,7 +58,11 @@ constexpr int HALF_BYTES = TM * 64 * 2;  // 16 KB: 64 keys of A or dS for 128 qu
 constexpr int NUM_THREADS = 512;
 constexpr int SILU_WARP0 = 4, NUM_SILU_WARPS = 8;
 constexpr int EPI_WARP0 = SILU_WARP0 + NUM_SILU_WARPS, NUM_EPI_WARPS = 4;
-constexpr uint32_t REGS_CTRL = 56, REGS_SILU = 160, REGS_EPI = 136;
+// launched with 65536 / 512 = 128 per thread: the control and epilogue
+// warpgroups give registers back (setmaxnreg.dec may only lower a count), the
+// A/dS warps take them
+constexpr uint32_t REGS_CTRL = 56, REGS_SILU = 168, REGS_EPI = 120;
+static_assert(REGS_CTRL <= 128 && REGS_EPI <= 128 && REGS_SILU >= 128, "dec lowers, inc raises");
 static_assert(128u * (REGS_CTRL + 2 * REGS_SILU + REGS_EPI) <= 65536u, "register split over budget");
 constexpr uint32_t S_COL = 0, DP_COL = 128, DQ_COL = 256, DK_COL = 384, DV_COL = 448;
 constexpr uint32_t TMEM_COLS = 512;

@@ -34,17 +34,20 @@
 // TMEM (512 columns): S_A, S_B (128 each), P_A, P_B (64 each, f16 pairs),
 // O_A, O_B (64 each).
 //
-// Scores accumulate in fp32 in TMEM (for f16 and bf16 operands alike). P and
+// Scores accumulate in TMEM: in f16 for f16 operands (the block path; one
+// packed TMEM load brings a row's 128 scores to 64 registers), in fp32 for
+// bf16 operands and for the relative-attention-bias variant. P and
 // V enter the second MMA as f16 (11-bit significand) rather than bf16: the
 // unnormalised silu weights span a wide range and bf16 rounding of P alone
 // would put the max-abs error near the 2e-2 x RMS bound on heavy-tailed
 // outputs. silu(s) = h + h tanh(h), h = s/2, is computed on f16x2 pairs
 // (one MUFU tanh per two scores). When Q arrives pre-halved (block path, the
 // projection epilogue scales the Q columns by 0.5 exactly) h is the score.
-// A score whose silu leaves the f16 range (above 65504) makes P infinite; the
+// A score (or, with the f16 accumulator, a partial sum of one) beyond the
+// f16 range, or a silu weight above 65504, makes P infinite or NaN; the
 // epilogue finds the non-finite O and records MTGR_ERR_RANGE, so such inputs
-// are reported, never silently wrong. (Very negative scores saturate at
-// -65504 and give P = 0, which is silu's value to f16 precision there.)
+// are reported, never silently wrong. (Very negative fp32 scores saturate at
+// -65504 on conversion and give P = 0, silu's value to f16 precision there.)
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -229,10 +232,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
 // IN_BF16: Q/K/V/U are bf16 (V converted to f16 in shared memory before P V);
 // otherwise f16. HALVE: the scores still need the factor 1/2 of silu's
 // tanh form. OUT_F32: G written as f32, else bf16. RAB: the relative
-// attention bias is added to the scores (block variant).
-template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB = false>
+// attention bias is added to the scores (block variant). S_F32: the scores
+// accumulate in fp32 (required for bf16 operands, whose MMA has no f16
+// accumulator, and for the bias, added before the f16 rounding).
+template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB = false, bool S_F32 = IN_BF16 || RAB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
+  static_assert(S_F32 || (!IN_BF16 && !RAB), "bf16 operands and the bias need fp32 scores");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -349,7 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // --------------------------------------------------- S issuer (MMA) --
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false);
+      constexpr uint32_t idesc_s = idesc_f16(TM, TN, IN_BF16 ? 1u : 0u, false, false, !S_F32);
       int32_t g = 0, li = 0;
       int32_t gs_a = 0, gs_b = 0;  // rounds of the S_A, S_B slots
       Item nxt;
@@ -406,19 +412,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           const uint32_t v_addr = smem_u32(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
-          // one q-tile: O_A and O_B accumulate alternate k-tiles (summed by
-          // the epilogue), each starting fresh at its first k-tile
+          // one q-tile: P_A and P_B hold alternate k-tiles of the same rows;
+          // both accumulate into O_A, in k-tile order as for two q-tiles (the
+          // MMAs run in issue order), so the sums match a paired item's
           const int q0 = two ? 0 : (t & 1), q1 = two ? 2 : q0 + 1;
-          const int32_t first_t = two ? 0 : q0;
           for (int q = q0; q < q1; ++q) {
             const int32_t r = q == 0 ? gp_a : gp_b;
             if (!mbar_wait(&p_full[q], r & 1)) { timed_out = true; break; }
             tc_fence_after();
+            const uint32_t o_dst = tmem + o_col(two ? q : 0);
 #pragma unroll
             for (int k = 0; k < TN / 16; ++k) {
-              tc_mma_ts(tmem + o_col(q), tmem + p_col(q) + 8 * k,
+              tc_mma_ts(o_dst, tmem + p_col(q) + 8 * k,
                         sdesc_sw128(v_addr + 2048 * k, 16384, 1024), idesc_o,
-                        (t > first_t || k > 0) ? 1u : 0u);
+                        (t > 0 || k > 0) ? 1u : 0u);
             }
             tc_commit(&p_free[q]);
             if (q == 0) ++gp_a; else ++gp_b;
@@ -490,10 +497,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t r = static_cast<uint32_t>(gq);
         if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-        // f32 scores: 16-column steps, the load of step k + 1 in flight while
-        // step k is masked, scaled and converted to f16 pairs
         uint32_t h[64];
-        {
+        if (!S_F32) {
+          // f16 scores (f16 accumulator, one per column): one packed load
+          tmem_ld64_pack16(s_addr, h);
+          tmem_ld_wait();
+          reg_fence(h);
+        } else {
+          // f32 scores: 16-column steps, the load of step k + 1 in flight
+          // while step k is masked, scaled and converted to f16 pairs
           uint64_t vis_lo = 0, vis_hi = 0;
           if (masked) {
             vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
@@ -522,8 +534,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
+        uint64_t vis_lo = 0, vis_hi = 0;
+        if (!S_F32 && masked) {
+          vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
+          vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
+        }
         if (t + 1 < it.w.n_union) fetch();
         else if (lane == 0 && has_next) prefetch_item_rows(a, w + stride, q, quarter);
+        if (!S_F32) {
+          if (masked) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              h[c] &= pair_mask(static_cast<uint32_t>((c < 32 ? vis_lo : vis_hi) >> (2 * (c & 31))));
+          }
+          if (HALVE) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) h[c] = mul_f16x2(h[c], 0x38003800u);  // x 0.5, exact
+          }
+        }
         // The tanh of both q-tiles runs on the MUFU pipes (16 values per
         // clock per SM, one pipe per sub-partition), the bound of this
         // kernel. The A and B warps of one sub-partition (same lane quarter)
@@ -607,35 +635,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const bool empty = it.w.n_union <= 0;
       const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.w.b] : (float)it.w.n);
-      // one q-tile: O = O_A (even k-tiles) + O_B (odd k-tiles)
-      const bool sum_b = it.w.nq == 1 && it.w.n_union >= 2;
       for (int q = 0; q < it.w.nq; ++q) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tmem + lane_base + o_col(q), o0);
+        tmem_ld32(tmem + lane_base + o_col(q) + 32, o1);
+        tmem_ld_wait();
+        if (q == it.w.nq - 1) {  // all of O read: the next item may accumulate
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
         const int32_t i = (it.w.qt0 + q) * TM + rr;
-        const int64_t row = it.w.us + i;
-        const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
         bool bad = false;  // a non-finite O: some P left the f16 range
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {  // head columns [32 hf, 32 hf + 32)
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + o_col(q) + 32 * hf, o);
-          tmem_ld_wait();
-          if (sum_b) {
-            uint32_t ob[32];
-            tmem_ld32(tmem + lane_base + o_col(1) + 32 * hf, ob);
-            tmem_ld_wait();
+        if (i < it.w.n) {
+          const int64_t row = it.w.us + i;
+          const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              o[c] = __float_as_uint(__uint_as_float(o[c]) + __uint_as_float(ob[c]));
-          }
-          if (q == it.w.nq - 1 && hf == 1) {  // all of O read: the next item may accumulate
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(o_free);
-          }
-          if (i >= it.w.n) continue;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // columns [8k, 8k + 8) of the head
-            const int k = 4 * hf + kk;
+          for (int k = 0; k < 8; ++k) {  // columns [8k, 8k + 8) of the head
             const uint4 x = *reinterpret_cast<const uint4*>(urow + ((k ^ (rr & 7)) << 4));
             const uint32_t uw[4] = {x.x, x.y, x.z, x.w};
             float ov[8], on[8];
@@ -650,7 +666,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 u0 = __low2float(hh);
                 u1 = __high2float(hh);
               }
-              const float f0 = __uint_as_float(o[8 * kk + 2 * c]), f1 = __uint_as_float(o[8 * kk + 2 * c + 1]);
+              const int col = 8 * k + 2 * c;
+              const float f0 = __uint_as_float(col < 32 ? o0[col] : o1[col - 32]);
+              const float f1 = __uint_as_float(col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32]);
               bad |= (f0 - f0) != 0.f || (f1 - f1) != 0.f;  // inf - inf, NaN - NaN: NaN
               on[2 * c] = f0 * inv_n;
               on[2 * c + 1] = f1 * inv_n;
