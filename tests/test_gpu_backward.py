@@ -1,8 +1,9 @@
 """GPU parity of the HSTU block's backward pass (training) against the
 oracle's chain-rule gradients (oracle.hstu_block_backward): the fp32 path at
-1e-4 x RMS, the bf16 tensor-core path at 2e-2 x RMS, on small and ragged
-batches and on the 512-user block workload, every gradient tensor compared
-element by element against its own RMS."""
+1e-4 x RMS, the bf16 tensor-core path at the gradient bars of tests/_util.py
+(max-abs 5e-2 x RMS, RMS error 1e-2 x RMS), on small and ragged batches and
+on the 512-user block workload, every gradient tensor compared element by
+element against its own RMS."""
 
 import numpy as np
 import pytest
@@ -10,7 +11,8 @@ import torch
 
 import oracle
 import synth
-from _util import TOL_BF16, TOL_F32, assert_close_rms, oracle_backward_all_users, to_host
+from _util import (TOL_BF16_GRAD_MAX, TOL_BF16_GRAD_RMS, TOL_F32, assert_grads_close,
+                   oracle_backward_all_users, to_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -32,8 +34,12 @@ def _gpu_backward(lens, ts, x, p, H, dtype, dy, norm=None):
 
 
 def _compare(got, ref, tol, what):
-    for k in ref:
-        assert_close_rms(got[k], ref[k], tol, f"{what}: d{k}")
+    # fp32: max-abs and RMS error both within 1e-4 x RMS; bf16: the gradient
+    # bars of tests/_util.py
+    if tol == TOL_F32:
+        assert_grads_close(got, ref, TOL_F32, TOL_F32, what)
+    else:
+        assert_grads_close(got, ref, TOL_BF16_GRAD_MAX, TOL_BF16_GRAD_RMS, what)
 
 
 def test_fp32_block_backward_workload_full():
@@ -67,7 +73,7 @@ def test_bf16_block_backward_small_batch():
     y, y_inf, g = _gpu_backward(w["lens"], w["ts"], w["x"], w["layers"][0], w["H"], "bf16", dy)
     np.testing.assert_array_equal(y, y_inf)  # the training forward computes the same output
     ref = oracle.hstu_block_backward(w["x"], w["lens"], w["ts"], w["layers"][0], w["H"], dy)
-    _compare(g, ref, TOL_BF16, "bf16 block, 6 users")
+    _compare(g, ref, "bf16", "bf16 block, 6 users")
 
 
 def test_bf16_block_backward_ragged_edge_users():
@@ -87,7 +93,7 @@ def test_bf16_block_backward_ragged_edge_users():
     dy = rng.standard_normal(x.shape).astype(np.float32)
     _, _, g = _gpu_backward(lens, ts, x, p, H, "bf16", dy)
     ref = oracle.hstu_block_backward(x, lens, ts, p, H, dy)
-    _compare(g, ref, TOL_BF16, "bf16 block, ragged users")
+    _compare(g, ref, "bf16", "bf16 block, ragged users")
 
 
 def test_bf16_block_backward_full_workload():
@@ -99,4 +105,4 @@ def test_bf16_block_backward_full_workload():
     for k, v in g.items():
         assert np.isfinite(v).all(), k
     ref = oracle_backward_all_users(w, dy)
-    _compare(g, ref, TOL_BF16, "bf16 block, 512 users")
+    _compare(g, ref, "bf16", "bf16 block, 512 users")
