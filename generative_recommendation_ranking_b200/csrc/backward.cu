@@ -108,9 +108,11 @@ struct GlnBwdArgs {
   int32_t* status;      // f16 dO~ beyond +-65504: MTGR_ERR_RANGE
 };
 
-// One warp per token, VPL 8-element vectors per lane (d <= 256 VPL); the
-// per-group gamma/beta gradients are summed in shared memory and added to
-// the global sums once per block.
+// One warp per token, VPL 8-element vectors per lane (d <= 256 VPL), each
+// warp over a contiguous run of tokens. The per-group gamma/beta gradients
+// accumulate in registers while the group stays the same (the tokens of a
+// user's segment are consecutive), go to the block's shared-memory sums when
+// it changes, and the block adds those to the global sums once.
 template <typename Tx, int VPL, bool GATE, typename Tq, typename To, typename Tg, typename Tz>
 __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
   extern __shared__ float sacc[];  // [2][G][d]: dgamma, dbeta
@@ -123,6 +125,26 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
   const int64_t t_end = min((int64_t)a.T, t_begin + a.tokens_per_warp);
   const Tx* x = static_cast<const Tx*>(a.x);
   bool range_bad = false;
+  float acc_g[VPL][8], acc_b[VPL][8];
+#pragma unroll
+  for (int k = 0; k < VPL; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc_g[k][e] = acc_b[k][e] = 0.f;
+  int g_run = -1;  // group of the sums in acc_g / acc_b
+  auto flush = [&]() {
+    if (g_run < 0) return;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = lane + 32 * k;
+      if (vi >= nv) continue;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        atomicAdd(&sacc[(int64_t)g_run * d + 8 * vi + e], acc_g[k][e]);
+        atomicAdd(&sacc[(int64_t)(G + g_run) * d + 8 * vi + e], acc_b[k][e]);
+        acc_g[k][e] = acc_b[k][e] = 0.f;
+      }
+    }
+  };
   for (int64_t t = t_begin; t < t_end; ++t) {
     float xv[VPL][8], gv[VPL][8];
     float s = 0.f;
@@ -151,6 +173,10 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
     const float rstd = 1.0f / sqrtf(warp_sum(q) / (float)d + a.eps);
     int g = a.gid[t];
     g = g < 0 ? 0 : (g >= G ? G - 1 : g);
+    if (g != g_run) {
+      flush();
+      g_run = g;
+    }
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
@@ -162,8 +188,8 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
         for (int e = 0; e < 8; ++e) {
           const float xh = (xv[k][e] - mean) * rstd;
           const float dxh = gv[k][e] * gm[e];
-          atomicAdd(&sacc[(int64_t)g * d + 8 * vi + e], gv[k][e] * xh);
-          atomicAdd(&sacc[(int64_t)(G + g) * d + 8 * vi + e], gv[k][e]);
+          acc_g[k][e] = fmaf(gv[k][e], xh, acc_g[k][e]);
+          acc_b[k][e] += gv[k][e];
           s1 += dxh;
           s2 += dxh * xh;
           xv[k][e] = xh;   // keep xhat
@@ -202,6 +228,7 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
       }
     }
   }
+  flush();
   if (GATE && sizeof(Tg) == 2 && range_bad) set_status(a.status, MTGR_ERR_RANGE);
   __syncthreads();
   for (int i = threadIdx.x; i < G * d; i += blockDim.x) {

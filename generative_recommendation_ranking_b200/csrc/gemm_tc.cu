@@ -351,19 +351,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         if constexpr (EPI == kEpiSilu2) {
-          // two outputs per block: z through tmR from buffer 0, silu(z)
-          // through tmO from buffer 1, once both earlier stores have read them
-          if (lane == 0) bulk_wait_group_read<0>();
+          // two bf16 outputs per block, 2 KB each, in one staging buffer: z
+          // (through tmR) in its first half, silu(z) (through tmO) in its
+          // second; the buffers alternate as for one output
+          uint8_t* sb = stg + buf * STG_BYTES;
+          if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait();
-          epilogue_silu2(args, col0, r, stg, stg + STG_BYTES, lane);
+          epilogue_silu2(args, col0, r, sb, sb + STG_BYTES / 2, lane);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmR, stg, col0, row0);
-            tma_store_2d(&tmO, stg + STG_BYTES, col0, row0);
+            tma_store_2d(&tmR, sb, col0, row0);
+            tma_store_2d(&tmO, sb + STG_BYTES / 2, col0, row0);
             bulk_commit_group();
           }
           continue;
