@@ -154,23 +154,6 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int32_t w) {
   return it;
 }
 
-// The SiLU warps read an item's record, then their rows' rank-table indices
-// and the item's first tile entries, a chain of dependent loads at every
-// item start. These bring the lines into L1 ahead of time: the next record
-// at the start of an item, and, during its last k-tile, the lines that
-// record points to for this warp (the record is then an L1 hit).
-__device__ __forceinline__ void prefetch_record(const AttnArgs& a, int32_t w) {
-  prefetch_l1(a.work + w / a.H);
-}
-__device__ __forceinline__ void prefetch_item_rows(const AttnArgs& a, int32_t w, int q, int quarter) {
-  const Item nx = load_item(a, w);
-  const int qrow = nx.w.nq == 2 ? q : 0;  // one q-tile: both warps take its rows
-  const int32_t i0 = (nx.w.qt0 + qrow) * MTGR_TILE_M + quarter * 32;  // only rows of the user
-  if (i0 < nx.w.n) prefetch_l1(a.rt_cnt + nx.w.us + i0);
-  prefetch_l1(a.entries + nx.w.e0a);
-  if (nx.w.nq == 2) prefetch_l1(a.entries + nx.w.e0b);
-}
-
 __device__ __forceinline__ int32_t num_items(const AttnArgs& a) {
   const int64_t P = a.counts[3] < a.q_cap ? a.counts[3] : a.q_cap;
   return (int32_t)(P * a.H);
@@ -370,14 +353,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int st = g % KV_STAGES;
           if (!mbar_wait(&kv_full[st], (g / KV_STAGES) & 1)) { timed_out = true; break; }
           const uint32_t k_addr = smem_u32(sKV + st * 2 * TILE_BYTES);
-          // two q-tiles: both slots, each with its own Q; one q-tile: the
-          // slots take alternate k-tiles, both with Q_A
-          const int q0 = two ? 0 : (t & 1), q1 = two ? 2 : q0 + 1;
-          for (int q = q0; q < q1; ++q) {
+          for (int q = 0; q < (two ? 2 : 1); ++q) {
             const int32_t r = q == 0 ? gs_a : gs_b;
             if (!mbar_wait(&s_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
             tc_fence_after();
-            const uint32_t q_addr = smem_u32(sQ + (2 * qb + (two ? q : 0)) * TILE_BYTES);
+            const uint32_t q_addr = smem_u32(sQ + (2 * qb + q) * TILE_BYTES);
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               tc_mma_ss(tmem + s_col(q), sdesc_sw128(q_addr + 32 * k, 16, 1024),
@@ -412,15 +392,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           const uint32_t v_addr = smem_u32(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
-          // one q-tile: P_A and P_B hold alternate k-tiles of the same rows;
-          // both accumulate into O_A, in k-tile order as for two q-tiles (the
-          // MMAs run in issue order), so the sums match a paired item's
-          const int q0 = two ? 0 : (t & 1), q1 = two ? 2 : q0 + 1;
-          for (int q = q0; q < q1; ++q) {
+          for (int q = 0; q < (two ? 2 : 1); ++q) {
             const int32_t r = q == 0 ? gp_a : gp_b;
             if (!mbar_wait(&p_full[q], r & 1)) { timed_out = true; break; }
             tc_fence_after();
-            const uint32_t o_dst = tmem + o_col(two ? q : 0);
+            const uint32_t o_dst = tmem + o_col(q);
 #pragma unroll
             for (int k = 0; k < TN / 16; ++k) {
               tc_mma_ts(o_dst, tmem + p_col(q) + 8 * k,
@@ -451,20 +427,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t s_addr = tmem + lane_base + s_col(q);
     const uint32_t p_addr = tmem + lane_base + p_col(q);
     int32_t gq = 0;  // this q-tile slot's k-tile counter (barrier rounds)
-    int32_t gt = 0;  // turns on the sub-partition's MUFU pipe (rounds of the turn barriers)
+    int32_t gt = 0;  // k-tiles of two-q-tile items (rounds of the turn barriers)
     for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride) {
-      // no look-ahead copy of the next item in registers (a row's scores
-      // leave no room for one); its lines are prefetched into L1 instead
+      // no look-ahead copy of the next item here: the 64 registers of a
+      // row's scores leave no room for one
       const Item it = load_item(a, w);
-      const bool has_next = w + stride < n_items;
-      if (lane == 0 && has_next) prefetch_record(a, w + stride);
-      // Two q-tiles: A takes q-tile A, B q-tile B, every k-tile. One q-tile:
-      // both take its rows, A the even and B the odd k-tiles of the union,
-      // so the item keeps both warps of a sub-partition (and its MUFU pipe)
-      // busy; their turns on the pipe alternate as for two q-tiles.
+      if (q >= it.w.nq) continue;  // this item has no q-tile B
       const bool two = it.w.nq == 2;
-      const int qrow = two ? q : 0;  // the q-tile of this warp's rows
-      const int32_t i = (it.w.qt0 + qrow) * TM + quarter * 32 + lane;  // user-relative row
+      const int32_t i = (it.w.qt0 + q) * TM + quarter * 32 + lane;  // user-relative row
       const int32_t cnt_i = i < it.w.n ? __ldg(a.rt_cnt + it.w.us + i) : 0;
       const int64_t t_i = RAB && i < it.w.n ? __ldg(a.ts + it.w.us + i) : 0;
       UnionCursor cur;
@@ -477,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto fetch = [&]() {
         int32_t ca, cb;
         kt_n = cur.next(ca, cb);
-        const int32_t code = qrow == 0 ? ca : cb;  // -1: EMPTY for this q-tile
+        const int32_t code = q == 0 ? ca : cb;  // -1: EMPTY for this q-tile
         masked_n = code < 0 || (code & 1) || kt_n * TN + TN > it.w.n;
         if (masked_n) {
           rt_lo_n = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN);
@@ -486,11 +456,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       fetch();
       for (int32_t t = 0; t < it.w.n_union; ++t) {
-        if (!two && (t & 1) != q) {  // the other warp's k-tile
-          if (t + 1 < it.w.n_union) fetch();
-          else if (lane == 0 && has_next) prefetch_item_rows(a, w + stride, q, quarter);
-          continue;
-        }
         const int32_t kt = kt_n;
         const bool masked = masked_n;
         const uint64_t rt_lo = rt_lo_n, rt_hi = rt_hi_n;
@@ -540,7 +505,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
         }
         if (t + 1 < it.w.n_union) fetch();
-        else if (lane == 0 && has_next) prefetch_item_rows(a, w + stride, q, quarter);
         if (!S_F32) {
           if (masked) {
 #pragma unroll
@@ -562,7 +526,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // pipe. Every wait is on a phase the other warp reaches without
         // waiting on this one (its previous turn), so the turns cannot
         // deadlock, and the two-slot rings keep each parity wait exact.
-        if (q == 1 || gt > 0) {
+        if (two && (q == 1 || gt > 0)) {
           uint64_t* bar = q == 0 ? &turn_a[2 * quarter + ((gt - 1) & 1)] : &turn_b[2 * quarter + (gt & 1)];
           const uint32_t par = q == 0 ? (((gt - 1) >> 1) & 1) : ((gt >> 1) & 1);
           if (!warp_wait(bar, par)) { timed_out = true; break; }
@@ -571,10 +535,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // P = h + h tanh(h) = silu(s), in place
 #pragma unroll
         for (int c = 0; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
-        reg_fence(h);  // hand over the turn only once this tile's tanh is done
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
-        ++gt;
+        if (two) {
+          reg_fence(h);  // hand over the turn only once this tile's tanh is done
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
+          ++gt;
+        }
         // P of the previous k-tile must have been consumed by its P V
         if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
         tc_fence_after();
@@ -585,15 +551,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[q]);
         ++gq;
-      }
-      if (timed_out) break;
-      // one q-tile with an odd k-tile count: A took one turn more; B takes an
-      // empty turn so that the two keep alternating on the next item
-      if (!two && q == 1 && (it.w.n_union & 1)) {
-        if (!warp_wait(&turn_b[2 * quarter + (gt & 1)], (gt >> 1) & 1)) { timed_out = true; break; }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&turn_a[2 * quarter + (gt & 1)]);
-        ++gt;
       }
     }
     finish();

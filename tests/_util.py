@@ -134,34 +134,42 @@ def oracle_backward_all_users(w, dy, procs=None, chunk=8):
 
 # bf16 backward: gradient tensors inherit the per-element error of the
 # forward's saved bf16/f16 activations (about 0.5% of an element), which sums
-# over tokens do not dilute; the bar takes the maximum over up to 10^6
-# elements at about 5 sigma (max-abs) and the bulk at 2 sigma (RMS error)
-TOL_BF16_GRAD_MAX = 5e-2
+# over tokens do not dilute. Bars: the RMS error of a tensor within 1e-2 of
+# its RMS (the bulk, about 2 sigma), and its largest error within 2e-2 of its
+# largest element (the tail: gradient tensors are heavy-tailed, their largest
+# elements 10-20 x RMS, and each element carries its own relative error)
 TOL_BF16_GRAD_RMS = 1e-2
+TOL_BF16_GRAD_PEAK = 2e-2
 
 
 def grad_errors(gpu, ref):
-    """(max-abs error, RMS error), both divided by the oracle tensor's RMS."""
+    """(max-abs error / max|ref|, RMS error / RMS(ref), max-abs error / RMS(ref))."""
     g = np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
-    rms = float(np.sqrt(np.mean(r ** 2))) if r.size else 0.0
+    if not r.size:
+        return 0.0, 0.0, 0.0
+    rms = float(np.sqrt(np.mean(r ** 2)))
+    peak = float(np.max(np.abs(r)))
     d = g - r
-    return (float(np.max(np.abs(d))) / max(rms, 1e-300) if r.size else 0.0,
-            float(np.sqrt(np.mean(d ** 2))) / max(rms, 1e-300) if r.size else 0.0)
+    mx = float(np.max(np.abs(d)))
+    return (mx / max(peak, 1e-300), float(np.sqrt(np.mean(d ** 2))) / max(rms, 1e-300),
+            mx / max(rms, 1e-300))
 
 
-def assert_grads_close(got: dict, ref: dict, max_tol: float, rms_tol: float, what: str):
-    """Every gradient tensor of ``ref`` against ``got``: finite, max-abs error
-    <= max_tol x RMS and RMS error <= rms_tol x RMS; prints each tensor's two
-    errors so the margins stay on record."""
+def assert_grads_close(got: dict, ref: dict, peak_tol: float, rms_tol: float, what: str):
+    """Every gradient tensor of ``ref`` against ``got``: finite, largest error
+    <= peak_tol x its largest element and RMS error <= rms_tol x its RMS;
+    prints each tensor's errors (also the largest error over the RMS) so the
+    margins stay on record."""
     report = []
     for k in ref:
         g = np.asarray(got[k], np.float64)
         assert g.shape == np.shape(ref[k]), (k, g.shape, np.shape(ref[k]))
         assert np.isfinite(g).all(), f"{what}: d{k} has non-finite values"
-        mx, rm = grad_errors(g, ref[k])
-        report.append(f"d{k} max {mx:.2e} rms {rm:.2e}")
+        pk, rm, mx = grad_errors(g, ref[k])
+        report.append(f"d{k} peak {pk:.2e} rms {rm:.2e} max/rms {mx:.2e}")
     print(f"{what}: " + "; ".join(report))
     for k in ref:
-        mx, rm = grad_errors(got[k], ref[k])
-        assert mx <= max_tol and rm <= rms_tol, f"{what}: d{k} max {mx:.2e} (<= {max_tol}) rms {rm:.2e} (<= {rms_tol})"
+        pk, rm, _ = grad_errors(got[k], ref[k])
+        assert pk <= peak_tol and rm <= rms_tol, \
+            f"{what}: d{k} peak {pk:.2e} (<= {peak_tol}) rms {rm:.2e} (<= {rms_tol})"
