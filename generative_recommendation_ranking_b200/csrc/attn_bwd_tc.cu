@@ -305,32 +305,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           vis = visible_bits(it.u, rt_word(it.u, a.rt_mask, cnt_i, j0), i, j0);
         }
         if (!warp_wait(s_full, g & 1)) { timed_out = true; break; }
-        // the previous q-tile's dV / dK / dQ MMAs have read A and dS
-        if (g > 0 && !warp_wait(p_free, (g - 1) & 1)) { timed_out = true; break; }
         tc_fence_after();
-        uint8_t* pa_row = sA + half * HALF_BYTES;
-        uint8_t* pd_row = sDS + half * HALF_BYTES;
-        // 16 keys at a time: S and dP from TMEM, A and dS (f16 pairs) to
-        // shared memory as two 16-byte chunks each
+        // A and dS of the 64 keys, in registers (f16 pairs), 8 keys at a time
+        // from S and dP in TMEM: this overlaps the previous q-tile's dV / dK /
+        // dQ MMAs, which still read the shared-memory copies
+        uint32_t pa[32], pd[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[16], dr[16];
-          tmem_ld16(tmem + lane_base + S_COL + 64 * half + 16 * c, sr);
-          tmem_ld16(tmem + lane_base + DP_COL + 64 * half + 16 * c, dr);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t sr[8], dr[8];
+          tmem_ld8(tmem + lane_base + S_COL + 64 * half + 8 * c, sr);
+          tmem_ld8(tmem + lane_base + DP_COL + 64 * half + 8 * c, dr);
           tmem_ld_wait();
-          if (c == 3) {
-            // S and dP are all in registers: the next q-tile's MMAs may overwrite them
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_free);
-          }
-          uint32_t pa[8], pd[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 4; ++k) {
             float av[2], dv[2];
 #pragma unroll
             for (int z = 0; z < 2; ++z) {
-              const int col = 16 * c + 2 * k + z;
+              const int col = 8 * c + 2 * k + z;
               const float h = __uint_as_float(sr[2 * k + z]);   // s / 2
               const float dp = __uint_as_float(dr[2 * k + z]);
               const float t = tanh_approx_f32(h);
@@ -340,16 +331,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               av[z] = on ? silu * it.inv_n : 0.f;
               dv[z] = on ? dp * it.inv_n * sg : 0.f;
             }
-            pa[k] = cvt_f16x2(av[0], av[1]);
-            pd[k] = cvt_f16x2(dv[0], dv[1]);
+            pa[4 * c + k] = cvt_f16x2(av[0], av[1]);
+            pd[4 * c + k] = cvt_f16x2(dv[0], dv[1]);
           }
+        }
+        // S and dP are in registers: the next q-tile's MMAs may overwrite them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // the previous q-tile's dV / dK / dQ MMAs have read A and dS
+        if (g > 0 && !warp_wait(p_free, (g - 1) & 1)) { timed_out = true; break; }
+        uint8_t* pa_row = sA + half * HALF_BYTES;
+        uint8_t* pd_row = sDS + half * HALF_BYTES;
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            *reinterpret_cast<uint4*>(pa_row + sw128(row, 2 * c + v)) =
-                make_uint4(pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
-            *reinterpret_cast<uint4*>(pd_row + sw128(row, 2 * c + v)) =
-                make_uint4(pd[4 * v], pd[4 * v + 1], pd[4 * v + 2], pd[4 * v + 3]);
-          }
+        for (int c = 0; c < 8; ++c) {
+          *reinterpret_cast<uint4*>(pa_row + sw128(row, c)) =
+              make_uint4(pa[4 * c], pa[4 * c + 1], pa[4 * c + 2], pa[4 * c + 3]);
+          *reinterpret_cast<uint4*>(pd_row + sw128(row, c)) =
+              make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
