@@ -79,6 +79,8 @@ constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);  // 512
 // the single-thread roles need few, the SiLU warps hold a row's 64 packed
 // scores. 128 x (80 + 152 + 152 + 128) = 65536.
 constexpr uint32_t REGS_CTRL = 80, REGS_SILU = 152;
+// tanh pairs a SiLU warp still computes after handing the MUFU turn over
+constexpr int HANDOFF_PAIRS = 8;
 static_assert(128u * (REGS_CTRL + 2 * REGS_SILU + 128u) <= 65536u, "register split over budget");
 __host__ __device__ constexpr uint32_t s_col(int q) { return 128u * q; }        // S_A, S_B
 __host__ __device__ constexpr uint32_t p_col(int q) { return 256u + 64u * q; }  // P_A, P_B
@@ -183,9 +185,12 @@ struct UnionCursor {
   }
 };
 
-// Keep-mask of one f16 pair from its two visibility bits (bit 0: low half).
-__device__ __forceinline__ uint32_t pair_mask(uint32_t bits) {
-  return ((bits & 1u) ? 0x0000ffffu : 0u) | ((bits & 2u) ? 0xffff0000u : 0u);
+// h[p] &= the keep-mask of f16 pair p (p < 16) from the visibility word w
+// of its 32 columns.
+__device__ __forceinline__ void mask_pairs16(uint32_t* h, uint32_t w) {
+  const PairMasks pm(w);
+#pragma unroll
+  for (int p = 0; p < 16; ++p) h[p] &= pm(p);
 }
 
 // h = s / 2 (or s, when the scores arrive halved) for 16 consecutive keys of
@@ -463,6 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
         uint32_t h[64];
+        uint64_t vis_lo = 0, vis_hi = 0;  // this row's visible columns, masked tiles
         if (!S_F32) {
           // f16 scores (f16 accumulator, one per column): one packed load
           tmem_ld64_pack16(s_addr, h);
@@ -471,7 +477,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else {
           // f32 scores: 16-column steps, the load of step k + 1 in flight
           // while step k is masked, scaled and converted to f16 pairs
-          uint64_t vis_lo = 0, vis_hi = 0;
           if (masked) {
             vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
             vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
@@ -499,7 +504,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
-        uint64_t vis_lo = 0, vis_hi = 0;
         if (!S_F32 && masked) {
           vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
           vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
@@ -507,9 +511,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (t + 1 < it.w.n_union) fetch();
         if (!S_F32) {
           if (masked) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              h[c] &= pair_mask(static_cast<uint32_t>((c < 32 ? vis_lo : vis_hi) >> (2 * (c & 31))));
+            mask_pairs16(h, static_cast<uint32_t>(vis_lo));
+            mask_pairs16(h + 16, static_cast<uint32_t>(vis_lo >> 32));
+            mask_pairs16(h + 32, static_cast<uint32_t>(vis_hi));
+            mask_pairs16(h + 48, static_cast<uint32_t>(vis_hi >> 32));
           }
           if (HALVE) {
 #pragma unroll
@@ -532,15 +537,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!warp_wait(bar, par)) { timed_out = true; break; }
           reg_fence(h);  // the arithmetic below may not move above the wait
         }
-        // P = h + h tanh(h) = silu(s), in place
+        // P = h + h tanh(h) = silu(s), in place, as one straight run of
+        // tanh/FMA pairs (a branch inside it costs more than it saves). The
+        // turn goes to the other warp with the last HANDOFF_PAIRS pairs still
+        // to compute, so its wake-up (about 190 cycles from the barrier
+        // arrive) overlaps their tanh.
 #pragma unroll
-        for (int c = 0; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
+        for (int c = 0; c < 64 - HANDOFF_PAIRS; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
         if (two) {
-          reg_fence(h);  // hand over the turn only once this tile's tanh is done
+#pragma unroll
+          for (int c = 0; c < 64 - HANDOFF_PAIRS; ++c) asm volatile("" : "+r"(h[c]));
           __syncwarp();
           if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
           ++gt;
         }
+#pragma unroll
+        for (int c = 64 - HANDOFF_PAIRS; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
         // P of the previous k-tile must have been consumed by its P V
         if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
         tc_fence_after();

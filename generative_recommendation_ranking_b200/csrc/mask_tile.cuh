@@ -61,4 +61,24 @@ __device__ __forceinline__ uint64_t visible_bits(const UserSpan& u, uint64_t rt,
   return vis & range_bits(0, u.n - j0);  // keys past the user's end
 }
 
+// Keep-masks of 16 f16 pairs from a 32-bit visibility word w (bit 2p: the
+// low half of pair p, bit 2p + 1: its high half). With sh[k] = w << (7 - k),
+// bit 8m + k of w is the sign bit of byte m of sh[k]; one byte permute with
+// sign replication (selector nibbles 8 | m for the low half, 12 | m for the
+// high half) spreads bits 2p and 2p + 1, both in byte m = p / 4, over the
+// pair's 16-bit halves: one instruction per pair plus seven shifts per word.
+struct PairMasks {
+  uint32_t sh[8];
+  __device__ __forceinline__ explicit PairMasks(uint32_t w) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sh[k] = w << (7 - k);
+  }
+  __device__ __forceinline__ uint32_t operator()(int p) const {
+    const uint32_t sel = 0xcc88u + 0x1111u * static_cast<uint32_t>(p >> 2);  // cc88 dd99 eeaa ffbb
+    uint32_t m;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(sh[2 * (p & 3)]), "r"(sh[2 * (p & 3) + 1]), "r"(sel));
+    return m;
+  }
+};
+
 }  // namespace mtgr
