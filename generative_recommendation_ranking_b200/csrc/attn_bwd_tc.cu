@@ -28,10 +28,14 @@
 // Warps (512 threads, registers re-split by setmaxnreg):
 //   0        TMA producer: K_j, V_j per item (two item buffers); Q_i, dO~_i per
 //            q-tile (two stages)
-//   1        MMA issuer (one thread): S/dP of q-tile t+1 go ahead of the
-//            dV/dK/dQ of q-tile t, so the tensor pipe works while the SiLU
-//            warps turn S, dP into A, dS
-//   2, 3     idle (complete warpgroup 0)
+//   1        dV/dK/dQ issuer (one thread): the MMAs that read A and dS
+//   2        S/dP issuer (one thread): S/dP of q-tile t+1 are issued as soon
+//            as the A/dS warps hold q-tile t's in registers, so the tensor
+//            pipe works while they turn S, dP into A, dS. Two issuers, because
+//            an MMA issue returns only once the pipe takes it and every
+//            barrier wait costs the waiting thread: each one's waits overlap
+//            the other's MMAs
+//   3        idle (completes warpgroup 0)
 //   4-11     A and dS: warp w takes TMEM lane quarter w % 4 (32 query rows)
 //            and key half (w - 4) / 4 (64 keys)
 //   12-15    epilogue: each q-tile's dQ part to the fp32 dQ buffer; at the
@@ -160,7 +164,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_dq);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], 2);  // one commit from each MMA issuer
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], 1);
       mbar_init(&dq_full[i], 1);
@@ -218,8 +222,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     } else if (warp == 1 && lane == 0) {
-      // -------------------------------------------------------- MMA issuer --
-      constexpr uint32_t idesc_s = idesc_f16(TM, TN, 0u, false, false);   // S, dP
+      // ------------------------------------------- dV / dK / dQ issuer (MMA) --
       constexpr uint32_t idesc_kv = idesc_f16(TN, DH, 0u, true, true);    // dV, dK
       constexpr uint32_t idesc_q = idesc_f16(TM, DH, 0u, false, true);    // dQ
       const uint32_t a_addr = smem_u32(sA), ds_addr = smem_u32(sDS);
@@ -258,6 +261,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kb = li & 1;
         if (!mbar_wait(&kv_full[kb], (li >> 1) & 1)) { timed_out = true; break; }
         const uint32_t k_addr = smem_u32(sKV + kb * 2 * TILE_BYTES);
+        const int32_t nq = it.e1 - it.e0;
+        for (int32_t t = 0; t < nq; ++t, ++g) {
+          if (!back(g, t == 0, k_addr)) { timed_out = true; break; }
+        }
+        if (timed_out) break;
+        tc_commit(&kv_empty[kb]);  // K read by the dQ MMAs
+        tc_commit(dkv_full);
+      }
+    } else if (warp == 2 && lane == 0) {
+      // ------------------------------------------------ S / dP issuer (MMA) --
+      constexpr uint32_t idesc_s = idesc_f16(TM, TN, 0u, false, false);
+      int32_t g = 0, li = 0;
+      for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride, ++li) {
+        const BwdItem it = load_bwd_item(a, w);
+        const int kb = li & 1;
+        if (!mbar_wait(&kv_full[kb], (li >> 1) & 1)) { timed_out = true; break; }
+        const uint32_t k_addr = smem_u32(sKV + kb * 2 * TILE_BYTES);
         const uint32_t v_addr = k_addr + TILE_BYTES;
         const int32_t nq = it.e1 - it.e0;
         for (int32_t t = 0; t < nq; ++t, ++g) {
@@ -274,12 +294,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       sdesc_sw128(v_addr + 32 * k, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
           }
           tc_commit(s_full);
-          if (t > 0 && !back(g - 1, t - 1 == 0, k_addr)) { timed_out = true; break; }
         }
         if (timed_out) break;
-        if (!back(g - 1, nq == 1, k_addr)) { timed_out = true; break; }
-        tc_commit(&kv_empty[kb]);
-        tc_commit(dkv_full);
+        tc_commit(&kv_empty[kb]);  // K and V read by the S / dP MMAs
       }
     }
     finish();
@@ -294,51 +311,78 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride) {
       const BwdItem it = load_bwd_item(a, w);
       const int32_t j0 = it.kt * TN + 64 * half;  // first key of this warp's half
+      const bool kt_ragged = it.kt * TN + TN > it.u.n;
+      // The per-pair metadata is a chain of dependent loads (tile code, then
+      // the row's rank count, then its rank-table word), each an L2 round
+      // trip. It runs one pair ahead: the next code is loaded a pair early,
+      // the next rank count before this pair's math and the next rank-table
+      // word after it, so no load is waited on directly.
+      auto is_masked = [&](int32_t code) {
+        return (code & 1) || (code >> 1) * TM + TM > it.u.n || kt_ragged;
+      };
+      int32_t code_c = __ldg(a.csc + it.e0);
+      int32_t code_n = it.e0 + 1 < it.e1 ? __ldg(a.csc + it.e0 + 1) : 0;
+      uint64_t rt_c = 0;
+      if (is_masked(code_c)) {
+        const int32_t i0 = (code_c >> 1) * TM + row;
+        rt_c = rt_word(it.u, a.rt_mask, i0 < it.u.n ? __ldg(a.rt_cnt + it.us + i0) : 0, j0);
+      }
       for (int32_t e = it.e0; e < it.e1; ++e, ++g) {
-        const int32_t code = __ldg(a.csc + e);
-        const int32_t qt = code >> 1;
-        const int32_t i = qt * TM + row;
-        const bool masked = (code & 1) || qt * TM + TM > it.u.n || it.kt * TN + TN > it.u.n;
-        uint64_t vis = ~0ull;
-        if (masked) {
-          const int32_t cnt_i = i < it.u.n ? __ldg(a.rt_cnt + it.us + i) : 0;
-          vis = visible_bits(it.u, rt_word(it.u, a.rt_mask, cnt_i, j0), i, j0);
-        }
+        const int32_t code = code_c;
+        const int32_t i = (code >> 1) * TM + row;
+        const bool masked = is_masked(code);
+        const bool has_next = e + 1 < it.e1;
+        const int32_t code_nn = e + 2 < it.e1 ? __ldg(a.csc + e + 2) : 0;
+        const int32_t i_n = (code_n >> 1) * TM + row;
+        const bool masked_n = has_next && is_masked(code_n);
+        const int32_t cnt_n = masked_n && i_n < it.u.n ? __ldg(a.rt_cnt + it.us + i_n) : 0;
+        const uint64_t vis = masked ? visible_bits(it.u, rt_c, i, j0) : ~0ull;
         if (!warp_wait(s_full, g & 1)) { timed_out = true; break; }
         tc_fence_after();
-        // A and dS of the 64 keys, in registers (f16 pairs), 8 keys at a time
-        // from S and dP in TMEM: this overlaps the previous q-tile's dV / dK /
-        // dQ MMAs, which still read the shared-memory copies
+        // A and dS of the 64 keys, in registers (f16 pairs), 16 keys at a
+        // time from S and dP in TMEM: this overlaps the previous q-tile's
+        // dV / dK / dQ MMAs, which still read the shared-memory copies.
+        // With h = s / 2 in f16 pairs and t = tanh(h) (the forward's form):
+        // A = h (1 + t) / N, dS = dP / N (1 + t) / 2 (1 + h (1 - t)).
         uint32_t pa[32], pd[32];
+        const float inv_n = it.inv_n;
+        const uint32_t inv_n2 = cvt_f16x2(inv_n, inv_n);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t sr[8], dr[8];
-          tmem_ld8(tmem + lane_base + S_COL + 64 * half + 8 * c, sr);
-          tmem_ld8(tmem + lane_base + DP_COL + 64 * half + 8 * c, dr);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[16], dr[16];
+          tmem_ld16(tmem + lane_base + S_COL + 64 * half + 16 * c, sr);
+          tmem_ld16(tmem + lane_base + DP_COL + 64 * half + 16 * c, dr);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float av[2], dv[2];
-#pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const int col = 8 * c + 2 * k + z;
-              const float h = __uint_as_float(sr[2 * k + z]);   // s / 2
-              const float dp = __uint_as_float(dr[2 * k + z]);
-              const float t = tanh_approx_f32(h);
-              const float silu = fmaf(h, t, h);
-              const float sg = 0.5f * (1.0f + t) * fmaf(h, 1.0f - t, 1.0f);  // silu'(s)
-              const bool on = (vis >> col) & 1ull;
-              av[z] = on ? silu * it.inv_n : 0.f;
-              dv[z] = on ? dp * it.inv_n * sg : 0.f;
-            }
-            pa[4 * c + k] = cvt_f16x2(av[0], av[1]);
-            pd[4 * c + k] = cvt_f16x2(dv[0], dv[1]);
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t h2 = cvt_f16x2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
+            const uint32_t t2 = tanh_f16x2(h2);
+            pa[8 * c + k] = mul_f16x2(fma_f16x2(h2, t2, h2), inv_n2);
+            const uint32_t omt = fma_f16x2(t2, 0xbc00bc00u, 0x3c003c00u);   // 1 - t
+            const uint32_t u2 = fma_f16x2(h2, omt, 0x3c003c00u);             // 1 + h (1 - t)
+            const uint32_t opt = fma_f16x2(t2, 0x38003800u, 0x38003800u);    // (1 + t) / 2
+            const uint32_t dpn = cvt_f16x2(__uint_as_float(dr[2 * k]) * inv_n,
+                                           __uint_as_float(dr[2 * k + 1]) * inv_n);
+            pd[8 * c + k] = mul_f16x2(dpn, mul_f16x2(opt, u2));
           }
         }
         // S and dP are in registers: the next q-tile's MMAs may overwrite them
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
+        if (masked) {
+          const PairMasks lo(static_cast<uint32_t>(vis)), hi(static_cast<uint32_t>(vis >> 32));
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const uint32_t ml = lo(p), mh = hi(p);
+            pa[p] &= ml;
+            pd[p] &= ml;
+            pa[16 + p] &= mh;
+            pd[16 + p] &= mh;
+          }
+        }
+        // the next pair's rank-table word (its rank count has arrived)
+        const uint64_t rt_n = masked_n ? rt_word(it.u, a.rt_mask, cnt_n, j0) : 0ull;
         // the previous q-tile's dV / dK / dQ MMAs have read A and dS
         if (g > 0 && !warp_wait(p_free, (g - 1) & 1)) { timed_out = true; break; }
         uint8_t* pa_row = sA + half * HALF_BYTES;
@@ -353,6 +397,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
+        code_c = code_n;
+        code_n = code_nn;
+        rt_c = rt_n;
       }
     }
     finish();
