@@ -48,6 +48,7 @@ struct GemmArgs {
   int32_t* status;
   const int32_t* row_map;  // row-map form: output row of each a row (-1: dropped)
   int out_rows;            // row-map form: rows of out
+  const uint16_t* aux_in;  // dSiLU form: Z1, bf16 [M][N]
 };
 
 __device__ __forceinline__ float u32_as_f(uint32_t v) { return __uint_as_float(v); }
@@ -99,14 +100,13 @@ __device__ __forceinline__ float silu_grad_fast(float z) {
 }
 
 // Backward of the MLP's SiLU: dZ1 = dH (.) silu'(Z1) for 32 columns of one
-// row, Z1 read from the staging block (bf16, as the TMA load left it) and
-// the result written over it.
-__device__ __forceinline__ void epilogue_dsilu(const uint32_t (&acc)[32], uint8_t* stg, int r) {
+// row, Z1 from registers (bf16 pairs), the result to the staging block.
+__device__ __forceinline__ void epilogue_dsilu(const uint32_t (&acc)[32], const uint4 (&z)[4],
+                                               uint8_t* stg, int r) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint4* p = reinterpret_cast<uint4*>(stg + stg_off<MTGR_BF16>(r, c));
-    const uint4 z4 = *p;
-    const uint32_t zw[4] = {z4.x, z4.y, z4.z, z4.w};
+    const uint32_t zw[4] = {z[c].x, z[c].y, z[c].z, z[c].w};
     uint32_t w[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -142,10 +142,6 @@ __device__ __forceinline__ void epilogue_silu2(const GemmArgs& a, int col0, cons
 template <int EPI, int OUT>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
                                                uint8_t* stg, int r) {
-  if constexpr (EPI == kEpiDSilu) {
-    epilogue_dsilu(acc, stg, r);
-    return;
-  }
   float v[32];
   epilogue_math<EPI, OUT>(a, col0, acc, v);
   if (OUT == MTGR_F16) {
@@ -234,7 +230,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmO);
-    if (EPI == MTGR_EPI_RESID || EPI == kEpiDSilu || EPI == kEpiSilu2) tma_prefetch_desc(&tmR);
+    if (EPI == MTGR_EPI_RESID || EPI == kEpiSilu2) tma_prefetch_desc(&tmR);
     for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&rbar[i], 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -306,6 +302,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0, chunk = 0;
     bool prev_scatter = false;  // row-map form: the last chunk left row by row
+    if constexpr (EPI == kEpiDSilu) {
+      // Z1, the second input, comes by plain loads: each lane's 64 bytes of
+      // a block (its row, 32 columns) into a four-block register ring,
+      // loaded four blocks ahead of use and across tile boundaries, so the
+      // DRAM latency hides behind the MMAs instead of stalling every block.
+      // Every tile takes eight ring steps (blocks past N load nothing), so
+      // a block's slot is its column block index mod 4.
+      uint4 zr[4][4];
+      int lt = blockIdx.x, lc = 0;  // the next block to load
+      auto load_next = [&](uint4 (&z)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (lt < num_tiles) {
+          const int m = (lt / n_tiles) * BM + quarter * 32 + lane;
+          const int col = (lt % n_tiles) * BN + lc * 32;
+          if (m < M && col < N) {
+            const uint4* p = reinterpret_cast<const uint4*>(args.aux_in + (size_t)m * N + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) z[i] = __ldg(p + i);
+          }
+        }
+        if (++lc == BN / 32) { lc = 0; lt += gridDim.x; }
+      };
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) load_next(zr[sl]);
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int mb = tile / n_tiles, nb = tile % n_tiles;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
+        if (!ok) { timed_out = true; break; }
+        tc_fence_after();
+        const int row0 = mb * BM + quarter * 32;
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = nb * BN + c * 32;
+          if (col0 < N) {
+            uint8_t* sb = stg + (chunk & 1) * STG_BYTES;
+            // the TMA store that last read this buffer (two blocks ago) must be done
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            uint32_t r[32];
+            tmem_ld32(t_row + c * 32, r);
+            tmem_ld_wait();
+            epilogue_dsilu(r, zr[c & 3], sb, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmO, sb, col0, row0);
+              bulk_commit_group();
+            }
+            ++chunk;
+          }
+          load_next(zr[c & 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    } else
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile / n_tiles, nb = tile % n_tiles;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
@@ -375,9 +431,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
         // a second input block arrives by TMA into the staging block: the
-        // fp32 residual, or the bf16 pre-activation of the SiLU backward
-        constexpr bool kAuxIn = EPI == MTGR_EPI_RESID || EPI == kEpiDSilu;
-        constexpr uint32_t kAuxBytes = EPI == MTGR_EPI_RESID ? STG_BYTES : STG_BYTES / 2;
+        // fp32 residual
+        constexpr bool kAuxIn = EPI == MTGR_EPI_RESID;
+        constexpr uint32_t kAuxBytes = STG_BYTES;
         if (kAuxIn && lane == 0) {
           mbar_arrive_expect_tx(&rbar[2 * ew + buf], kAuxBytes);
           tma_load_2d(&tmR, &rbar[2 * ew + buf], sb, col0, row0);
@@ -480,7 +536,7 @@ int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const 
   rc = make_tmap_2d(&tr, aux, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N, (uint64_t)M,
                     (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc != MTGR_OK) return rc;
-  GemmArgs args{M, N, K, bias, nullptr, out, 0, status, nullptr, 0};
+  GemmArgs args{M, N, K, bias, nullptr, out, 0, status, nullptr, 0, static_cast<const uint16_t*>(aux)};
   if (epi == kEpiDSilu) return launch_t<kEpiDSilu, MTGR_BF16>(ta, tb, to, tr, args, s);
   if (epi == kEpiSilu2) return launch_t<kEpiSilu2, MTGR_BF16>(ta, tb, to, tr, args, s);
   return MTGR_ERR_UNSUPPORTED;
