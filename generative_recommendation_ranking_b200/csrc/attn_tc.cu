@@ -68,20 +68,41 @@ constexpr int TM = MTGR_TILE_M;  // 128 query rows per q-tile
 constexpr int TN = MTGR_TILE_N;  // 128 keys per k-tile
 constexpr int KV_STAGES = 4;
 constexpr int TILE_BYTES = TM * DH * 2;  // 16 KB (one Q, K, V or U tile)
-constexpr int NUM_SILU_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
-// Four warpgroups: 0 = TMA producer, S issuer, PV issuer (warp 3 idle);
-// 1 = SiLU of q-tile A; 2 = SiLU of q-tile B; 3 = epilogue.
 constexpr int SILU_WARP0 = 4;
-constexpr int EPI_WARP0 = SILU_WARP0 + NUM_SILU_WARPS;
-constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);  // 512
-// Registers per thread after the split (launched with 65536 / 512 = 128):
-// the single-thread roles need few, the SiLU warps hold a row's 64 packed
-// scores. 128 x (80 + 152 + 152 + 128) = 65536.
-constexpr uint32_t REGS_CTRL = 80, REGS_SILU = 152;
+// Warpgroups: 0 = TMA producer, S issuer, PV issuer (warp 3 idle); then the
+// SiLU warps; last, the epilogue. SPLIT = 1: one SiLU warp per TMEM lane
+// quarter and q-tile covers all 128 keys of a k-tile (warpgroups 1 / 2 for
+// q-tiles A / B). SPLIT = 2: two warps share each row, one per 64-key half
+// (warpgroups 1 / 2: A / B, first half; 3 / 4: A / B, second half), so four
+// SiLU warps interleave on each sub-partition: their waits and TMEM round
+// trips hide behind one another's work instead of idling the MUFU pipe.
+template <int SPLIT>
+struct Layout {
+  static constexpr int kSiluWarps = 8 * SPLIT;
+  static constexpr int kEpiWarp0 = SILU_WARP0 + kSiluWarps;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + NUM_EPI_WARPS);  // 512 or 768
+  static constexpr int kPairs = 64 / SPLIT;  // f16 score pairs per SiLU warp and k-tile
+  static constexpr int kWords = 2 / SPLIT;   // 64-key visibility words per SiLU warp
+  // Registers per thread after the split, within the launch's 65536 /
+  // kThreads each (128 or 80; all of the block's registers are drawn at
+  // launch, and setmaxnreg.inc can only take from that pool):
+  // 128 x (80 + 152 + 152 + 128) = 65536; 128 x (48 + 4 x 88 + 80) = 61440.
+  static constexpr uint32_t kRegsCtrl = SPLIT == 1 ? 80 : 48;
+  static constexpr uint32_t kRegsSilu = SPLIT == 1 ? 152 : 88;
+  static constexpr uint32_t kRegsEpi = SPLIT == 1 ? 128 : 80;
+  static constexpr uint32_t kLaunchRegs = SPLIT == 1 ? 128 : 80;
+  static constexpr uint32_t kSplitRegs = 128u * (kRegsCtrl + 2u * SPLIT * kRegsSilu + kRegsEpi);
+  static_assert(kSplitRegs <= kLaunchRegs * kThreads, "register split over the launch's registers");
+  static_assert(kLaunchRegs * kThreads <= 65536u, "launch registers");
+};
 // tanh pairs a SiLU warp still computes after handing the MUFU turn over
 constexpr int HANDOFF_PAIRS = 8;
-static_assert(128u * (REGS_CTRL + 2 * REGS_SILU + 128u) <= 65536u, "register split over budget");
+// the layout of the f16-score kernels (the block's path)
+#ifndef MTGR_ATTN_SPLIT_F16
+#define MTGR_ATTN_SPLIT_F16 2
+#endif
+constexpr int kSplitF16 = MTGR_ATTN_SPLIT_F16;
 __host__ __device__ constexpr uint32_t s_col(int q) { return 128u * q; }        // S_A, S_B
 __host__ __device__ constexpr uint32_t p_col(int q) { return 256u + 64u * q; }  // P_A, P_B
 __host__ __device__ constexpr uint32_t o_col(int q) { return 384u + 64u * q; }  // O_A, O_B
@@ -223,10 +244,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
 // attention bias is added to the scores (block variant). S_F32: the scores
 // accumulate in fp32 (required for bf16 operands, whose MMA has no f16
 // accumulator, and for the bias, added before the f16 rounding).
-template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB = false, bool S_F32 = IN_BF16 || RAB>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB, int SPLIT, bool S_F32 = IN_BF16 || RAB>
+__global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
+  using L = Layout<SPLIT>;
   static_assert(S_F32 || (!IN_BF16 && !RAB), "bf16 operands and the bias need fp32 scores");
+  static_assert(SPLIT == 1 || !S_F32, "the split layout serves the f16-score form");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -248,10 +271,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* u_full = o_free + 1;
   uint64_t* u_empty = u_full + 1;
   // Turns on each SM sub-partition's MUFU pipe, one barrier pair per A/B
-  // warp pair sharing it: [sub-partition][slot]
-  uint64_t* turn_b = u_empty + 1;  // [4][2] A's tanh of a k-tile done: B's turn
-  uint64_t* turn_a = turn_b + 8;   // [4][2] B's tanh of a k-tile done: A's turn
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn_a + 8);
+  // warp pair sharing it: [key half][sub-partition][slot]
+  uint64_t* turn_b = u_empty + 1;        // A's tanh of a k-tile done: B's turn
+  uint64_t* turn_a = turn_b + 8 * SPLIT;  // B's tanh of a k-tile done: A's turn
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn_a + 8 * SPLIT);
 
   const int warp = warp_id(), lane = lane_id();
   if (warp == 0 && lane == 0) {
@@ -260,8 +283,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], NUM_SILU_WARPS / 2);
-      mbar_init(&p_full[i], NUM_SILU_WARPS / 2);
+      mbar_init(&s_free[i], L::kSiluWarps / 2);
+      mbar_init(&p_full[i], L::kSiluWarps / 2);
       mbar_init(&p_free[i], 1);
     }
     for (int s = 0; s < KV_STAGES; ++s) {
@@ -273,7 +296,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(o_free, NUM_EPI_WARPS);
     mbar_init(u_full, 1);
     mbar_init(u_empty, NUM_EPI_WARPS);
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 8 * SPLIT; ++i) {
       mbar_init(&turn_b[i], 1);
       mbar_init(&turn_a[i], 1);
     }
@@ -303,7 +326,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   if (warp < SILU_WARP0) {
-  setmaxnreg_dec<REGS_CTRL>();
+  setmaxnreg_dec<L::kRegsCtrl>();
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
@@ -418,24 +441,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   finish();
-  } else if (warp < EPI_WARP0) {
-    setmaxnreg_inc<REGS_SILU>();
+  } else if (warp < L::kEpiWarp0) {
+    setmaxnreg_inc<L::kRegsSilu>();
     // -------------------------------------------------------- SiLU warps --
-    // Warps 4-7 take q-tile A of every item, warps 8-11 q-tile B; each warp
-    // covers 32 query rows (its TMEM lane quarter) across all 128 keys of a
-    // k-tile. S goes to registers in one step and is released at once; the
-    // next k-tile's entry and rule-2 words are fetched while this one's
-    // tanh runs.
+    // Each SiLU warp covers 32 query rows (its TMEM lane quarter) of one
+    // q-tile slot (A or B) across its keys of a k-tile: all 128 (SPLIT 1)
+    // or one 64-key half (SPLIT 2). S goes to registers in one step and is
+    // released at once; the next k-tile's entry and rule-2 words are fetched
+    // while this one's tanh runs.
+    constexpr int NP = L::kPairs;
     const int quarter = warp & 3;
-    const int q = (warp - SILU_WARP0) >> 2;  // 0: q-tile A, 1: q-tile B
+    const int idx = warp - SILU_WARP0;
+    const int q = (idx >> 2) & 1;  // 0: q-tile A, 1: q-tile B
+    const int half = idx >> 3;     // key half (SPLIT 2), else 0
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + s_col(q);
-    const uint32_t p_addr = tmem + lane_base + p_col(q);
+    const uint32_t s_addr = tmem + lane_base + s_col(q) + static_cast<uint32_t>(half * 2 * NP);
+    const uint32_t p_addr = tmem + lane_base + p_col(q) + static_cast<uint32_t>(half * NP);
+    const int tb = 8 * half + 2 * quarter;  // this warp pair's turn barriers
     int32_t gq = 0;  // this q-tile slot's k-tile counter (barrier rounds)
     int32_t gt = 0;  // k-tiles of two-q-tile items (rounds of the turn barriers)
     for (int32_t w = blockIdx.x; w < n_items && !timed_out; w += stride) {
-      // no look-ahead copy of the next item here: the 64 registers of a
-      // row's scores leave no room for one
+      // no look-ahead copy of the next item here: the registers of a row's
+      // scores leave no room for one
       const Item it = load_item(a, w);
       if (q >= it.w.nq) continue;  // this item has no q-tile B
       const bool two = it.w.nq == 2;
@@ -445,41 +472,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       UnionCursor cur;
       cur.init(a.entries, it.w);
       // the upcoming k-tile: index, whether it needs the per-element rules,
-      // and its two rule-2 words
+      // and the rule-2 words of this warp's keys
       int32_t kt_n = 0;
       bool masked_n = false;
-      uint64_t rt_lo_n = 0, rt_hi_n = 0;
+      uint64_t rt_n[L::kWords];
+#pragma unroll
+      for (int k = 0; k < L::kWords; ++k) rt_n[k] = 0;
       auto fetch = [&]() {
         int32_t ca, cb;
         kt_n = cur.next(ca, cb);
         const int32_t code = q == 0 ? ca : cb;  // -1: EMPTY for this q-tile
         masked_n = code < 0 || (code & 1) || kt_n * TN + TN > it.w.n;
         if (masked_n) {
-          rt_lo_n = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN);
-          rt_hi_n = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN + 64);
+#pragma unroll
+          for (int k = 0; k < L::kWords; ++k)
+            rt_n[k] = rt_word(UserSpan(it.w), a.rt_mask, cnt_i, kt_n * TN + 64 * (half + k));
         }
       };
       fetch();
       for (int32_t t = 0; t < it.w.n_union; ++t) {
         const int32_t kt = kt_n;
         const bool masked = masked_n;
-        const uint64_t rt_lo = rt_lo_n, rt_hi = rt_hi_n;
+        uint64_t rt[L::kWords];
+#pragma unroll
+        for (int k = 0; k < L::kWords; ++k) rt[k] = rt_n[k];
         const uint32_t r = static_cast<uint32_t>(gq);
         if (!warp_wait(&s_full[q], r & 1)) { timed_out = true; break; }
         tc_fence_after();
-        uint32_t h[64];
-        uint64_t vis_lo = 0, vis_hi = 0;  // this row's visible columns, masked tiles
-        if (!S_F32) {
+        uint32_t h[NP];
+        uint64_t vis[L::kWords];  // this row's visible columns, masked tiles
+#pragma unroll
+        for (int k = 0; k < L::kWords; ++k) vis[k] = 0;
+        if constexpr (!S_F32) {
           // f16 scores (f16 accumulator, one per column): one packed load
-          tmem_ld64_pack16(s_addr, h);
+          if constexpr (SPLIT == 1) tmem_ld64_pack16(s_addr, h);
+          else tmem_ld32_pack16(s_addr, h);
           tmem_ld_wait();
           reg_fence(h);
         } else {
           // f32 scores: 16-column steps, the load of step k + 1 in flight
           // while step k is masked, scaled and converted to f16 pairs
           if (masked) {
-            vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
-            vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
+            vis[0] = visible_bits(UserSpan(it.w), rt[0], i, kt * TN);
+            vis[1] = visible_bits(UserSpan(it.w), rt[1], i, kt * TN + 64);
           }
           uint32_t sa[16], sb[16];
           tmem_ld16(s_addr, sa);
@@ -492,7 +527,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (k < 7) tmem_ld16(s_addr + 16 * (k + 1), ahead);
             if (RAB)
               add_rab(cur_s, a, it.h, it.w.us, it.w.n_u, i, t_i, kt * TN + 16 * k, HALVE ? 1.f : 0.5f);
-            const uint64_t vv = k < 4 ? vis_lo : vis_hi;
+            const uint64_t vv = vis[k >> 2];
             scores_to_h<HALVE>(cur_s, h + 8 * k, masked, (uint32_t)(vv >> (16 * (k & 3))));
             if (k < 7) {
               tmem_ld_wait();
@@ -504,35 +539,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
-        if (!S_F32 && masked) {
-          vis_lo = visible_bits(UserSpan(it.w), rt_lo, i, kt * TN);
-          vis_hi = visible_bits(UserSpan(it.w), rt_hi, i, kt * TN + 64);
+        if constexpr (!S_F32) {
+          if (masked) {
+#pragma unroll
+            for (int k = 0; k < L::kWords; ++k)
+              vis[k] = visible_bits(UserSpan(it.w), rt[k], i, kt * TN + 64 * (half + k));
+          }
         }
         if (t + 1 < it.w.n_union) fetch();
-        if (!S_F32) {
+        if constexpr (!S_F32) {
           if (masked) {
-            mask_pairs16(h, static_cast<uint32_t>(vis_lo));
-            mask_pairs16(h + 16, static_cast<uint32_t>(vis_lo >> 32));
-            mask_pairs16(h + 32, static_cast<uint32_t>(vis_hi));
-            mask_pairs16(h + 48, static_cast<uint32_t>(vis_hi >> 32));
+#pragma unroll
+            for (int k = 0; k < L::kWords; ++k) {
+              mask_pairs16(h + 32 * k, static_cast<uint32_t>(vis[k]));
+              mask_pairs16(h + 32 * k + 16, static_cast<uint32_t>(vis[k] >> 32));
+            }
           }
           if (HALVE) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) h[c] = mul_f16x2(h[c], 0x38003800u);  // x 0.5, exact
+            for (int c = 0; c < NP; ++c) h[c] = mul_f16x2(h[c], 0x38003800u);  // x 0.5, exact
           }
         }
         // The tanh of both q-tiles runs on the MUFU pipes (16 values per
-        // clock per SM, one pipe per sub-partition), the bound of this
-        // kernel. The A and B warps of one sub-partition (same lane quarter)
-        // share its pipe; within a two-q-tile item they take turns, A(0)
-        // B(0) A(1) B(1) ...: each one's loads, stores and waits then
-        // overlap the other's tanh instead of coinciding with it. The turns
-        // are per warp pair, so a slow warp elsewhere does not idle this
-        // pipe. Every wait is on a phase the other warp reaches without
-        // waiting on this one (its previous turn), so the turns cannot
-        // deadlock, and the two-slot rings keep each parity wait exact.
+        // clock per SM, one pipe per sub-partition). The A and B warps of
+        // one sub-partition and key half (same lane quarter) share its pipe;
+        // within a two-q-tile item they take turns, A(0) B(0) A(1) B(1) ...:
+        // each one's loads, stores and waits then overlap the other's tanh
+        // instead of coinciding with it. The turns are per warp pair, so a
+        // slow warp elsewhere does not idle this pipe. Every wait is on a
+        // phase the other warp reaches without waiting on this one (its
+        // previous turn), so the turns cannot deadlock, and the two-slot
+        // rings keep each parity wait exact.
         if (two && (q == 1 || gt > 0)) {
-          uint64_t* bar = q == 0 ? &turn_a[2 * quarter + ((gt - 1) & 1)] : &turn_b[2 * quarter + (gt & 1)];
+          uint64_t* bar = q == 0 ? &turn_a[tb + ((gt - 1) & 1)] : &turn_b[tb + (gt & 1)];
           const uint32_t par = q == 0 ? (((gt - 1) >> 1) & 1) : ((gt >> 1) & 1);
           if (!warp_wait(bar, par)) { timed_out = true; break; }
           reg_fence(h);  // the arithmetic below may not move above the wait
@@ -543,21 +582,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // to compute, so its wake-up (about 190 cycles from the barrier
         // arrive) overlaps their tanh.
 #pragma unroll
-        for (int c = 0; c < 64 - HANDOFF_PAIRS; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
+        for (int c = 0; c < NP - HANDOFF_PAIRS; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
         if (two) {
 #pragma unroll
-          for (int c = 0; c < 64 - HANDOFF_PAIRS; ++c) asm volatile("" : "+r"(h[c]));
+          for (int c = 0; c < NP - HANDOFF_PAIRS; ++c) asm volatile("" : "+r"(h[c]));
           __syncwarp();
-          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[2 * quarter + (gt & 1)] : &turn_a[2 * quarter + (gt & 1)]);
+          if (lane == 0) mbar_arrive(q == 0 ? &turn_b[tb + (gt & 1)] : &turn_a[tb + (gt & 1)]);
           ++gt;
         }
 #pragma unroll
-        for (int c = 64 - HANDOFF_PAIRS; c < 64; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
+        for (int c = NP - HANDOFF_PAIRS; c < NP; ++c) h[c] = fma_f16x2(h[c], tanh_f16x2(h[c]), h[c]);
         // P of the previous k-tile must have been consumed by its P V
         if (!warp_wait(&p_free[q], (r & 1) ^ 1)) { timed_out = true; break; }
         tc_fence_after();
-        tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(h));
-        tmem_st32(p_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(h + 32));
+#pragma unroll
+        for (int k = 0; k < NP / 32; ++k)
+          tmem_st32(p_addr + 32 * k, *reinterpret_cast<const uint32_t(*)[32]>(h + 32 * k));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -568,8 +608,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     finish();
   } else {
     // ---------------------------------------------------- epilogue warps --
+    if constexpr (SPLIT != 1) setmaxnreg_dec<L::kRegsEpi>();
     const int quarter = warp & 3;
-    const int et = (warp - EPI_WARP0) * 32 + lane;  // 0..127
+    const int et = (warp - L::kEpiWarp0) * 32 + lane;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int rr = quarter * 32 + lane;  // row within each q-tile
     int32_t g = 0, li = 0;
@@ -605,57 +646,60 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool empty = it.w.n_union <= 0;
       const float inv_n = empty ? 0.f : 1.0f / (a.norm ? a.norm[it.w.b] : (float)it.w.n);
       for (int q = 0; q < it.w.nq; ++q) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tmem + lane_base + o_col(q), o0);
-        tmem_ld32(tmem + lane_base + o_col(q) + 32, o1);
-        tmem_ld_wait();
-        if (q == it.w.nq - 1) {  // all of O read: the next item may accumulate
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);
-        }
         const int32_t i = (it.w.qt0 + q) * TM + rr;
+        const int64_t row = it.w.us + i;
+        const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
         bool bad = false;  // a non-finite O: some P left the f16 range
-        if (i < it.w.n) {
-          const int64_t row = it.w.us + i;
-          const uint8_t* urow = sU + q * TILE_BYTES + rr * 128;
+        // O in two 32-column halves (32 registers live at a time)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {  // columns [8k, 8k + 8) of the head
-            const uint4 x = *reinterpret_cast<const uint4*>(urow + ((k ^ (rr & 7)) << 4));
-            const uint32_t uw[4] = {x.x, x.y, x.z, x.w};
-            float ov[8], on[8];
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + o_col(q) + 32 * hc, o);
+          tmem_ld_wait();
+          if (hc == 1 && q == it.w.nq - 1) {  // all of O read: the next item may accumulate
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+          }
+          if (i < it.w.n) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float u0, u1;
-              if (IN_BF16) {
-                u0 = __uint_as_float(uw[c] << 16);
-                u1 = __uint_as_float(uw[c] & 0xffff0000u);
-              } else {
-                const __half2 hh = *reinterpret_cast<const __half2*>(&uw[c]);
-                u0 = __low2float(hh);
-                u1 = __high2float(hh);
+            for (int kk = 0; kk < 4; ++kk) {  // columns [8k, 8k + 8) of the head
+              const int k = 4 * hc + kk;
+              const uint4 x = *reinterpret_cast<const uint4*>(urow + ((k ^ (rr & 7)) << 4));
+              const uint32_t uw[4] = {x.x, x.y, x.z, x.w};
+              float ov[8], on[8];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                float u0, u1;
+                if (IN_BF16) {
+                  u0 = __uint_as_float(uw[c] << 16);
+                  u1 = __uint_as_float(uw[c] & 0xffff0000u);
+                } else {
+                  const __half2 hh = *reinterpret_cast<const __half2*>(&uw[c]);
+                  u0 = __low2float(hh);
+                  u1 = __high2float(hh);
+                }
+                const float f0 = __uint_as_float(o[8 * kk + 2 * c]);
+                const float f1 = __uint_as_float(o[8 * kk + 2 * c + 1]);
+                bad |= (f0 - f0) != 0.f || (f1 - f1) != 0.f;  // inf - inf, NaN - NaN: NaN
+                on[2 * c] = f0 * inv_n;
+                on[2 * c + 1] = f1 * inv_n;
+                ov[2 * c] = on[2 * c] * u0;
+                ov[2 * c + 1] = on[2 * c + 1] * u1;
               }
-              const int col = 8 * k + 2 * c;
-              const float f0 = __uint_as_float(col < 32 ? o0[col] : o1[col - 32]);
-              const float f1 = __uint_as_float(col + 1 < 32 ? o0[col + 1] : o1[col + 1 - 32]);
-              bad |= (f0 - f0) != 0.f || (f1 - f1) != 0.f;  // inf - inf, NaN - NaN: NaN
-              on[2 * c] = f0 * inv_n;
-              on[2 * c + 1] = f1 * inv_n;
-              ov[2 * c] = on[2 * c] * u0;
-              ov[2 * c + 1] = on[2 * c + 1] * u1;
-            }
-            if (a.obar != nullptr)
-              *reinterpret_cast<uint4*>(a.obar + row * d + it.h * DH + 8 * k) =
-                  make_uint4(cvt_bf16x2(on[0], on[1]), cvt_bf16x2(on[2], on[3]),
-                             cvt_bf16x2(on[4], on[5]), cvt_bf16x2(on[6], on[7]));
-            if (OUT_F32) {
-              float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * d + it.h * DH + 8 * k);
-              op[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
-              op[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
-            } else {
-              uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * d + it.h * DH + 8 * k);
-              *op = make_uint4(cvt_bf16x2(ov[0], ov[1]), cvt_bf16x2(ov[2], ov[3]),
-                               cvt_bf16x2(ov[4], ov[5]), cvt_bf16x2(ov[6], ov[7]));
+              if (a.obar != nullptr)
+                *reinterpret_cast<uint4*>(a.obar + row * d + it.h * DH + 8 * k) =
+                    make_uint4(cvt_bf16x2(on[0], on[1]), cvt_bf16x2(on[2], on[3]),
+                               cvt_bf16x2(on[4], on[5]), cvt_bf16x2(on[6], on[7]));
+              if (OUT_F32) {
+                float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * d + it.h * DH + 8 * k);
+                op[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
+                op[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+              } else {
+                uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * d + it.h * DH + 8 * k);
+                *op = make_uint4(cvt_bf16x2(ov[0], ov[1]), cvt_bf16x2(ov[2], ov[3]),
+                                 cvt_bf16x2(ov[4], ov[5]), cvt_bf16x2(ov[6], ov[7]));
+              }
             }
           }
         }
@@ -669,13 +713,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB = false>
+template <bool IN_BF16, bool HALVE, bool OUT_F32, bool RAB, int SPLIT>
 int launch_t(const CUtensorMap& tm, const AttnArgs& a, int grid, cudaStream_t s) {
-  auto kern = attn_tc_kernel<IN_BF16, HALVE, OUT_F32, RAB>;
+  using L = Layout<SPLIT>;
+  auto kern = attn_tc_kernel<IN_BF16, HALVE, OUT_F32, RAB, SPLIT>;
+  // The register re-split (setmaxnreg) draws on the registers the block is
+  // launched with; a build whose kernel got fewer per thread than the split
+  // assumes would leave the SiLU warps waiting for registers, so it is
+  // refused here instead of launched.
+  static int checked = 0;  // 1 ok, -1 refused
+  if (checked == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return MTGR_ERR_CUDA;
+    checked = (uint32_t)fa.numRegs * (uint32_t)L::kThreads >= L::kSplitRegs ? 1 : -1;
+  }
+  if (checked < 0) return MTGR_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
       cudaSuccess)
     return MTGR_ERR_CUDA;
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tm, a);
+  kern<<<grid, L::kThreads, SMEM_BYTES, s>>>(tm, a);
   return launch_status();
 }
 
@@ -697,16 +753,19 @@ int launch_attn_tc(const mtgr_batch* bt, int32_t d, int32_t H, int32_t in_dtype,
   const bool f32 = out_dtype == MTGR_F32;
   if (in_dtype == MTGR_BF16) {
     if (q_prehalved) return MTGR_ERR_UNSUPPORTED;
-    return f32 ? launch_t<true, true, true>(tm, a, grid, s) : launch_t<true, true, false>(tm, a, grid, s);
+    return f32 ? launch_t<true, true, true, false, 1>(tm, a, grid, s)
+               : launch_t<true, true, false, false, 1>(tm, a, grid, s);
   }
   if (rab_pos != nullptr) {  // the block's bias variant: f16, Q prehalved, bf16 G
     if (in_dtype != MTGR_F16 || !q_prehalved || f32 || obar != nullptr) return MTGR_ERR_UNSUPPORTED;
-    return launch_t<false, false, false, true>(tm, a, grid, s);
+    return launch_t<false, false, false, true, 1>(tm, a, grid, s);
   }
   if (in_dtype == MTGR_F16) {
     if (q_prehalved)
-      return f32 ? launch_t<false, false, true>(tm, a, grid, s) : launch_t<false, false, false>(tm, a, grid, s);
-    return f32 ? launch_t<false, true, true>(tm, a, grid, s) : launch_t<false, true, false>(tm, a, grid, s);
+      return f32 ? launch_t<false, false, true, false, kSplitF16>(tm, a, grid, s)
+                 : launch_t<false, false, false, false, kSplitF16>(tm, a, grid, s);
+    return f32 ? launch_t<false, true, true, false, kSplitF16>(tm, a, grid, s)
+               : launch_t<false, true, false, false, kSplitF16>(tm, a, grid, s);
   }
   return MTGR_ERR_UNSUPPORTED;
 }
