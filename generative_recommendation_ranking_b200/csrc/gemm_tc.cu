@@ -31,6 +31,29 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+// CG = 1: one CTA per 128 x 256 tile. CG = 2: a cluster of two CTAs (two
+// SMs) per 256 x 256 tile with pair MMAs (M = 256): each CTA keeps its 128
+// rows of A and 128 of the 256 B columns in its own shared memory, so an
+// SM's operand reads per MMA fall from 12 KB to 8 KB (the single-CTA main
+// loop is bound by shared-memory bandwidth: an M = 128, N = 256 MMA takes
+// about 165 cycles instead of 128).
+// CTA pairs for reductions of at least this length: measured on the
+// 512-user block step, pairs take MLP2 (K = 2048) from 0.831 to 0.807 ms and
+// the backward's dG~ / dX~ GEMMs down by a similar share, but slow the
+// K = 512 projections by 7% (a tile's main loop is then short, and the pair
+// waits for the slower CTA's loads and for both epilogues). The row-map
+// form stays on single CTAs.
+constexpr int kPairMinK = 1024;
+
+template <int CG>
+struct GemmShape {
+  static constexpr int kStages = CG == 1 ? STAGES : 6;  // the same 192 KB of stages
+  static constexpr int kBRows = BN / CG;                 // B columns (rows of b) per CTA
+  static constexpr int kBBytes = kBRows * BK * 2;
+  static constexpr int kStageBytes = A_BYTES + kBBytes;  // per CTA
+  static constexpr int kTileM = BM * CG;
+  static_assert(kStages * kStageBytes == STAGES * STAGE_BYTES, "stage memory");
+};
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int NUM_THREADS = 192;
@@ -201,30 +224,38 @@ __device__ __forceinline__ void rowmap_scatter(const GemmArgs& a, int col0, cons
   }
 }
 
-template <int EPI, int OUT, bool ROWMAP>
+template <int EPI, int OUT, bool ROWMAP, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    GemmArgs args) {
+  using G = GemmShape<CG>;
+  constexpr int NST = G::kStages;
+  static_assert(CG == 1 || !ROWMAP, "the row-map form runs on single CTAs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  uint8_t* sStg = sB + STAGES * B_BYTES;  // [EPI_WARPS][2][STG_BYTES]
+  uint8_t* sB = smem + NST * A_BYTES;
+  uint8_t* sStg = sB + NST * G::kBBytes;  // [EPI_WARPS][2][STG_BYTES]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + EPI_WARPS * 2 * STG_BYTES);
   uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* acc_full = bars + 2 * STAGES;
-  uint64_t* acc_empty = bars + 2 * STAGES + 2;
-  uint64_t* rbar = bars + 2 * STAGES + 4;  // [EPI_WARPS][2] residual block landed
+  uint64_t* empty = bars + NST;
+  uint64_t* acc_full = bars + 2 * NST;
+  uint64_t* acc_empty = bars + 2 * NST + 2;
+  uint64_t* rbar = bars + 2 * NST + 4;  // [EPI_WARPS][2] residual block landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 2 * EPI_WARPS);
 
   const int warp = warp_id(), lane = lane_id();
   const int M = args.M, N = args.N, K = args.K;
   const int n_tiles = (N + BN - 1) / BN;
-  const int num_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int num_tiles = ((M + G::kTileM - 1) / G::kTileM) * n_tiles;
   const int kblocks = K / BK;
+  // CTA pairs: rank 0 (the leader) issues the pair MMAs; both CTAs load their
+  // halves and drain their own 128 accumulator rows
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int tile0 = CG == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tstride = CG == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
@@ -232,22 +263,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmO);
     if (EPI == MTGR_EPI_RESID || EPI == kEpiSilu2) tma_prefetch_desc(&tmR);
     for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&rbar[i], 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], CG * EPI_WARPS);  // the pair's epilogue warps (leader's barrier)
     }
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_cg2(tmem_slot, TMEM_COLS);
+      tmem_relinquish_cg2();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync();  // both CTAs' barriers initialised
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   bool timed_out = false;
@@ -256,23 +293,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !timed_out; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles && !timed_out; tile += tstride) {
         const int mb = tile / n_tiles, nb = tile % n_tiles;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { timed_out = true; break; }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(&tmA, &full[stage], sA + stage * A_BYTES, kb * BK, mb * BM);
-          tma_load_2d(&tmB, &full[stage], sB + stage * B_BYTES, kb * BK, nb * BN);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if constexpr (CG == 2) {
+            // both CTAs' halves complete on the leader's barrier, which the
+            // leader arms for the bytes of both
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * G::kStageBytes);
+            const uint32_t fb = mapa_shared(&full[stage], 0);
+            tma_load_2d_cg2(&tmA, fb, sA + stage * A_BYTES, kb * BK, mb * G::kTileM + (int)rank * BM);
+            tma_load_2d_cg2(&tmB, fb, sB + stage * G::kBBytes, kb * BK, nb * BN + (int)rank * G::kBRows);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+            tma_load_2d(&tmA, &full[stage], sA + stage * A_BYTES, kb * BK, mb * BM);
+            tma_load_2d(&tmB, &full[stage], sB + stage * B_BYTES, kb * BK, nb * BN);
+          }
+          if (++stage == NST) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(BM, BN, 1u, false, false);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_f16(G::kTileM, BN, 1u, false, false);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !timed_out; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles && !timed_out; tile += tstride) {
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { timed_out = true; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
@@ -280,22 +326,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(&full[stage], phase)) { timed_out = true; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * G::kBBytes);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            tc_mma_ss(d_tmem, sdesc_sw128(a_addr + 32 * k, 16, 1024),
-                      sdesc_sw128(b_addr + 32 * k, 16, 1024), idesc, (kb | k) != 0 ? 1u : 0u);
+            const uint64_t ad = sdesc_sw128(a_addr + 32 * k, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + 32 * k, 16, 1024);
+            if constexpr (CG == 2) tc_mma_ss_cg2(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            else tc_mma_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if constexpr (CG == 2) tc_commit_cg2(&empty[stage], 0x3);
+          else tc_commit(&empty[stage]);
+          if (++stage == NST) { stage = 0; phase ^= 1; }
         }
         if (timed_out) break;
-        tc_commit(&acc_full[acc]);
+        if constexpr (CG == 2) tc_commit_cg2(&acc_full[acc], 0x3);
+        else tc_commit(&acc_full[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
     }
   } else {
     // epilogue warp ew drains accumulator rows [32 quarter, 32 quarter + 32)
+    // of its CTA; the accumulator is released on the leader's barrier
+    auto release_acc = [&](uint64_t* bar) {
+      if constexpr (CG == 2) {
+        if (rank == 0) mbar_arrive(bar);
+        else mbar_arrive_cluster(mapa_shared(bar, 0));
+      } else {
+        mbar_arrive(bar);
+      }
+    };
     const int quarter = warp & 3;
     const int ew = warp - 2;
     uint8_t* stg = sStg + ew * 2 * STG_BYTES;
@@ -310,12 +369,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Every tile takes eight ring steps (blocks past N load nothing), so
       // a block's slot is its column block index mod 4.
       uint4 zr[4][4];
-      int lt = blockIdx.x, lc = 0;  // the next block to load
+      int lt = tile0, lc = 0;  // the next block to load
       auto load_next = [&](uint4 (&z)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
         if (lt < num_tiles) {
-          const int m = (lt / n_tiles) * BM + quarter * 32 + lane;
+          const int m = (lt / n_tiles) * G::kTileM + (int)rank * BM + quarter * 32 + lane;
           const int col = (lt % n_tiles) * BN + lc * 32;
           if (m < M && col < N) {
             const uint4* p = reinterpret_cast<const uint4*>(args.aux_in + (size_t)m * N + col);
@@ -323,16 +382,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < 4; ++i) z[i] = __ldg(p + i);
           }
         }
-        if (++lc == BN / 32) { lc = 0; lt += gridDim.x; }
+        if (++lc == BN / 32) { lc = 0; lt += tstride; }
       };
 #pragma unroll
       for (int sl = 0; sl < 4; ++sl) load_next(zr[sl]);
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles; tile += tstride) {
         const int mb = tile / n_tiles, nb = tile % n_tiles;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
         if (!ok) { timed_out = true; break; }
         tc_fence_after();
-        const int row0 = mb * BM + quarter * 32;
+        const int row0 = mb * G::kTileM + (int)rank * BM + quarter * 32;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
@@ -358,16 +417,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (lane == 0) release_acc(&acc_empty[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
     } else
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = tile0; tile < num_tiles; tile += tstride) {
       const int mb = tile / n_tiles, nb = tile % n_tiles;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
       if (!ok) { timed_out = true; break; }
       tc_fence_after();
-      const int row0 = mb * BM + quarter * 32;
+      const int row0 = mb * G::kTileM + (int)rank * BM + quarter * 32;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c, ++chunk) {
@@ -456,33 +515,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (timed_out) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (lane == 0) release_acc(&acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
     if (lane == 0) bulk_wait_group<0>();  // stores complete before the CTA retires
   }
   if (timed_out) set_status(args.status, MTGR_ERR_TIMEOUT);
-  __syncthreads();
+  // a pair retires together: the leader's MMAs read the other CTA's shared
+  // memory and the other CTA arrives on the leader's barriers
+  tc_fence_before();
+  if constexpr (CG == 2) cluster_sync();
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (CG == 2) tmem_dealloc_cg2(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-template <int EPI, int OUT, bool ROWMAP = false>
+template <int EPI, int OUT, bool ROWMAP = false, int CG = 1>
 int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
              const CUtensorMap& tr, const GemmArgs& args, cudaStream_t s) {
-  auto kern = gemm_tc_kernel<EPI, OUT, ROWMAP>;
+  auto kern = gemm_tc_kernel<EPI, OUT, ROWMAP, CG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
       cudaSuccess)
     return MTGR_ERR_CUDA;
-  const int tiles = ((args.M + BM - 1) / BM) * ((args.N + BN - 1) / BN);
-  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
+  const int tiles = ((args.M + BM * CG - 1) / (BM * CG)) * ((args.N + BN - 1) / BN);
+  if constexpr (CG == 1) {
+    const int units = device_sm_count();
+    const int grid = tiles < units ? tiles : units;
+    kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // The pairs are persistent: launch no more than can be resident at once
+    // (a GPC with an odd number of SMs leaves one unpaired), so none waits
+    // for a second wave.
+    static int resident = 0;
+    if (resident == 0) {
+      cfg.gridDim = dim3(device_sm_count());
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return MTGR_ERR_CUDA;
+      resident = n;
+    }
+    const int pairs = tiles < resident ? tiles : resident;
+    cfg.gridDim = dim3(2 * pairs);
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, tr, args) != cudaSuccess) return MTGR_ERR_CUDA;
+  }
   return launch_status();
 }
 
 }  // namespace
+
+template <int EPI, int OUT>
+int launch_cg(int cg, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+              const CUtensorMap& tr, const GemmArgs& args, cudaStream_t s) {
+  return cg == 2 ? launch_t<EPI, OUT, false, 2>(ta, tb, to, tr, args, s)
+                 : launch_t<EPI, OUT, false, 1>(ta, tb, to, tr, args, s);
+}
 
 // a [M][K] bf16, b [N][K] bf16; K % 64 == 0, N % 32 == 0, rows 16-byte aligned.
 int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const float* bias, int epi,
@@ -492,7 +591,8 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
   CUtensorMap ta, tb, to, tr;
   int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
   if (rc != MTGR_OK) return rc;
-  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
+  const int cg = K >= kPairMinK ? 2 : 1;
+  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN / cg);
   if (rc != MTGR_OK) return rc;
   if (out_dtype == MTGR_F32) {
     rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)M,
@@ -509,13 +609,13 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
     if (rc != MTGR_OK) return rc;
   }
   GemmArgs args{M, N, K, bias, resid, out, q_cols, status, nullptr, 0};
-  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_NONE, MTGR_F16>(ta, tb, to, tr, args, s);
-  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_NONE, MTGR_BF16>(ta, tb, to, tr, args, s);
-  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_NONE, MTGR_F32>(ta, tb, to, tr, args, s);
-  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F16) return launch_t<MTGR_EPI_SILU, MTGR_F16>(ta, tb, to, tr, args, s);
-  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_t<MTGR_EPI_SILU, MTGR_BF16>(ta, tb, to, tr, args, s);
-  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_SILU, MTGR_F32>(ta, tb, to, tr, args, s);
-  if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_t<MTGR_EPI_RESID, MTGR_F32>(ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_cg<MTGR_EPI_NONE, MTGR_F16>(cg, ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_cg<MTGR_EPI_NONE, MTGR_BF16>(cg, ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F32) return launch_cg<MTGR_EPI_NONE, MTGR_F32>(cg, ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F16) return launch_cg<MTGR_EPI_SILU, MTGR_F16>(cg, ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_BF16) return launch_cg<MTGR_EPI_SILU, MTGR_BF16>(cg, ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_SILU && out_dtype == MTGR_F32) return launch_cg<MTGR_EPI_SILU, MTGR_F32>(cg, ta, tb, to, tr, args, s);
+  if (epi == MTGR_EPI_RESID && out_dtype == MTGR_F32) return launch_cg<MTGR_EPI_RESID, MTGR_F32>(cg, ta, tb, to, tr, args, s);
   return MTGR_ERR_UNSUPPORTED;
 }
 
@@ -528,7 +628,8 @@ int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const 
   CUtensorMap ta, tb, to, tr;
   int rc = make_tmap_2d_16b(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM);
   if (rc != MTGR_OK) return rc;
-  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN);
+  const int cg = K >= kPairMinK ? 2 : 1;
+  rc = make_tmap_2d_16b(&tb, b, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN / cg);
   if (rc != MTGR_OK) return rc;
   rc = make_tmap_2d(&to, out, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N, (uint64_t)M,
                     (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -537,8 +638,8 @@ int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const 
                     (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc != MTGR_OK) return rc;
   GemmArgs args{M, N, K, bias, nullptr, out, 0, status, nullptr, 0, static_cast<const uint16_t*>(aux)};
-  if (epi == kEpiDSilu) return launch_t<kEpiDSilu, MTGR_BF16>(ta, tb, to, tr, args, s);
-  if (epi == kEpiSilu2) return launch_t<kEpiSilu2, MTGR_BF16>(ta, tb, to, tr, args, s);
+  if (epi == kEpiDSilu) return launch_cg<kEpiDSilu, MTGR_BF16>(cg, ta, tb, to, tr, args, s);
+  if (epi == kEpiSilu2) return launch_cg<kEpiSilu2, MTGR_BF16>(cg, ta, tb, to, tr, args, s);
   return MTGR_ERR_UNSUPPORTED;
 }
 
