@@ -303,9 +303,10 @@ KERNEL_SRC = {"attention": "attn_tc.cu", "gemm_qkvu": "gemm_tc.cu", "gemm_mlp1":
               "mask_meta": "pack_meta.cu"}
 
 
-def ncu_traffic(cls: str):
+def ncu_traffic(cls: str, workload: str = None):
     """Per-launch DRAM bytes of a kernel class from the committed ncu summary,
-    or None when absent or when the kernel source changed since the capture."""
+    or None when absent, when the kernel source changed since the capture, or
+    when the record is for another workload than `workload`."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -313,6 +314,8 @@ def ncu_traffic(cls: str):
         d = json.load(f)
     e = d.get(cls)
     if not e or e.get("src_sha") != src_sha(KERNEL_SRC[cls]):
+        return None
+    if workload is not None and e.get("workload") != workload:
         return None
     return e.get("bytes_per_launch")
 
@@ -530,7 +533,7 @@ def run_ours(args, world, rank, local):
                                        "peak_source": f"MUFU tanh 16/clk/SM x {n_sm} SMs x {sm_mhz:.0f} MHz"}
     dom = max((c for c in work if c in kernels), key=lambda c: kernels[c]["share"])
     k = kernels[dom]
-    traffic = ncu_traffic(dom)
+    traffic = ncu_traffic(dom, wl["name"])
     roofline = {"bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"], "unit": k["unit"],
                 "frac": k["frac"], "traffic": traffic, "kernel": dom,
                 "peak_source": f"{peak_src} ({tensor_key if k['bound'] == 'tensor' else 'hbm_gbs'}; "

@@ -22,7 +22,8 @@ def _fake_root(tmp_path, src_text, recorded_sha):
     (csrc / "attn_tc.cu").write_text(src_text)
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(
-        {"attention": {"bytes_per_launch": 12345, "src_sha": recorded_sha}}))
+        {"attention": {"bytes_per_launch": 12345, "src_sha": recorded_sha,
+                       "workload": "block_bf16_b512_d512"}}))
     return str(tmp_path)
 
 
@@ -35,6 +36,14 @@ def test_traffic_only_while_the_source_matches(tmp_path, monkeypatch):
     assert bench.ncu_traffic("attention") is None
     monkeypatch.setattr(bench, "ROOT", str(tmp_path / "missing"))
     assert bench.ncu_traffic("attention") is None
+
+
+def test_traffic_only_for_the_captured_workload(tmp_path, monkeypatch):
+    text = "// kernel source\n"
+    sha = hashlib.sha256(text.encode()).hexdigest()[:16]
+    monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path / "a", text, sha))
+    assert bench.ncu_traffic("attention", "block_bf16_b512_d512") == 12345
+    assert bench.ncu_traffic("attention", "attn_bf16_b256_d256") is None
 
 
 def test_committed_traffic_record_names_a_kernel_class_with_a_source():
