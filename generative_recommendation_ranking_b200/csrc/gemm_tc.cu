@@ -56,9 +56,21 @@ struct GemmShape {
 };
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARPS = 4;
 constexpr int STG_BYTES = 4096;  // one 32x32 staging block (fp32; 16-bit uses half)
+// Epilogue warps of each form. The dSiLU form (backward of MLP1's SiLU) does
+// a tanh and a few FMAs per element on top of the drain, and at K = 512 its
+// four warps, one per sub-partition, could not keep up with the MMAs; it runs
+// eight, two per TMEM lane quarter, each draining 128 of the 256 columns.
+// Its output is 16-bit, so its staging blocks are 2 KB and the eight warps'
+// double buffers take the same 32 KB as four warps' 4 KB ones.
+template <int EPI>
+struct EpiShape {
+  static constexpr int kWarps = EPI == kEpiDSilu ? 8 : EPI_WARPS;
+  static constexpr int kThreads = 64 + 32 * kWarps;
+  static constexpr int kStg = EPI == kEpiDSilu ? STG_BYTES / 2 : STG_BYTES;
+  static_assert(kWarps * kStg == EPI_WARPS * STG_BYTES, "staging memory");
+};
 constexpr size_t SMEM_BYTES =
     1024 + (size_t)STAGES * STAGE_BYTES + (size_t)EPI_WARPS * 2 * STG_BYTES + 256;
 
@@ -225,7 +237,7 @@ __device__ __forceinline__ void rowmap_scatter(const GemmArgs& a, int col0, cons
 }
 
 template <int EPI, int OUT, bool ROWMAP, int CG>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    GemmArgs args) {
@@ -269,7 +281,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], CG * EPI_WARPS);  // the pair's epilogue warps (leader's barrier)
+      mbar_init(&acc_empty[a], CG * EpiShape<EPI>::kWarps);  // the pair's epilogue warps (leader's barrier)
     }
     fence_barrier_init();
   }
@@ -357,7 +369,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     const int quarter = warp & 3;
     const int ew = warp - 2;
-    uint8_t* stg = sStg + ew * 2 * STG_BYTES;
+    uint8_t* stg = sStg + ew * 2 * EpiShape<EPI>::kStg;
     int acc = 0;
     uint32_t acc_phase = 0, chunk = 0;
     bool prev_scatter = false;  // row-map form: the last chunk left row by row
@@ -366,8 +378,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // a block (its row, 32 columns) into a four-block register ring,
       // loaded four blocks ahead of use and across tile boundaries, so the
       // DRAM latency hides behind the MMAs instead of stalling every block.
-      // Every tile takes eight ring steps (blocks past N load nothing), so
-      // a block's slot is its column block index mod 4.
+      // Each warp drains NB = 4 blocks of a tile (column half grp of its
+      // lane quarter); every tile takes NB ring steps (blocks past N load
+      // nothing), so a block's slot is its index among the warp's blocks.
+      constexpr int NB = (BN / 32) / (EpiShape<EPI>::kWarps / 4);
+      static_assert(NB == 4, "one ring slot per block of a tile");
+      const int grp = ew >> 2;
       uint4 zr[4][4];
       int lt = tile0, lc = 0;  // the next block to load
       auto load_next = [&](uint4 (&z)[4]) {
@@ -375,14 +391,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = 0; i < 4; ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
         if (lt < num_tiles) {
           const int m = (lt / n_tiles) * G::kTileM + (int)rank * BM + quarter * 32 + lane;
-          const int col = (lt % n_tiles) * BN + lc * 32;
+          const int col = (lt % n_tiles) * BN + (grp * NB + lc) * 32;
           if (m < M && col < N) {
             const uint4* p = reinterpret_cast<const uint4*>(args.aux_in + (size_t)m * N + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i) z[i] = __ldg(p + i);
           }
         }
-        if (++lc == BN / 32) { lc = 0; lt += tstride; }
+        if (++lc == NB) { lc = 0; lt += tstride; }
       };
 #pragma unroll
       for (int sl = 0; sl < 4; ++sl) load_next(zr[sl]);
@@ -394,17 +410,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int row0 = mb * G::kTileM + (int)rank * BM + quarter * 32;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int cc = 0; cc < NB; ++cc) {
+          const int c = grp * NB + cc;
           const int col0 = nb * BN + c * 32;
           if (col0 < N) {
-            uint8_t* sb = stg + (chunk & 1) * STG_BYTES;
+            uint8_t* sb = stg + (chunk & 1) * EpiShape<EPI>::kStg;
             // the TMA store that last read this buffer (two blocks ago) must be done
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
             uint32_t r[32];
             tmem_ld32(t_row + c * 32, r);
             tmem_ld_wait();
-            epilogue_dsilu(r, zr[c & 3], sb, lane);
+            epilogue_dsilu(r, zr[cc], sb, lane);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -413,7 +430,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             ++chunk;
           }
-          load_next(zr[c & 3]);
+          load_next(zr[cc]);
         }
         tc_fence_before();
         __syncwarp();
@@ -544,10 +561,10 @@ int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to
   if constexpr (CG == 1) {
     const int units = device_sm_count();
     const int grid = tiles < units ? tiles : units;
-    kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
+    kern<<<grid, EpiShape<EPI>::kThreads, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
   } else {
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.blockDim = dim3(EpiShape<EPI>::kThreads);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
