@@ -146,14 +146,27 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
     }
   };
   for (int64_t t = t_begin; t < t_end; ++t) {
-    float xv[VPL][8], gv[VPL][8];
-    float s = 0.f;
+    // every input of the token at once (none depends on the statistics),
+    // so a token costs one memory round trip, not two
+    float xv[VPL][8], gv[VPL][8], e1[VPL][8], e2[VPL][8];
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
       const int vi = lane + 32 * k;
       if (vi < nv) {
         ld8(x + t * d + 8 * vi, xv[k]);
         ld8(a.dy + t * d + 8 * vi, gv[k]);
+        if (GATE) {
+          ld8(static_cast<const Tq*>(a.qkvu) + t * 4 * d + 3 * d + 8 * vi, e1[k]);  // U
+          ld8(static_cast<const To*>(a.obar) + t * d + 8 * vi, e2[k]);             // O~
+        } else if (a.dres != nullptr) {
+          ld8(a.dres + t * d + 8 * vi, e1[k]);
+        }
+      }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      if (lane + 32 * k < nv) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) s += xv[k][e];
       }
@@ -207,20 +220,16 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
       for (int e = 0; e < 8; ++e) dx[e] = (gv[k][e] - m1 - xv[k][e] * m2) * rstd;
       if (!GATE) {
         if (a.dres != nullptr) {
-          float r[8];
-          ld8(a.dres + t * d + 8 * vi, r);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dx[e] += r[e];
+          for (int e = 0; e < 8; ++e) dx[e] += e1[k][e];
         }
         st8(a.dx + t * d + 8 * vi, dx);
       } else {
-        float u[8], ob[8], dob[8], du[8];
-        ld8(static_cast<const Tq*>(a.qkvu) + t * 4 * d + 3 * d + 8 * vi, u);
-        ld8(static_cast<const To*>(a.obar) + t * d + 8 * vi, ob);
+        float dob[8], du[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          dob[e] = dx[e] * u[e];
-          du[e] = dx[e] * ob[e];
+          dob[e] = dx[e] * e1[k][e];
+          du[e] = dx[e] * e2[k][e];
           range_bad |= !(fabsf(dob[e]) <= 65504.f);
         }
         st8(static_cast<Tg*>(a.dobar) + t * d + 8 * vi, dob);
