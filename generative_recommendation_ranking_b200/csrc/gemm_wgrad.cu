@@ -15,7 +15,8 @@
 // so the work is split "stream-K": the (tile, 64-token block) space is cut
 // into one contiguous range per CTA, and each CTA adds every partial tile it
 // finishes into the fp32 output with TMA reduce-add stores
-// (cp.reduce.async.bulk.tensor ... .add). The caller zeroes the output first
+// (cp.reduce.async.bulk.tensor ... .add); with few tiles, a slab schedule
+// replaces the contiguous ranges (SegCursor). The caller zeroes the output first
 // unless it accumulates. Roles as in the block's forward GEMM: warp 0 TMA
 // producer, one thread of warp 1 issues the MMAs, warps 2-5 drain the
 // double-buffered TMEM accumulator.
@@ -50,11 +51,21 @@ struct WgradArgs {
   int kblocks;        // ceil(T / BK)
   int n_tiles;        // tiles along N
   int64_t total;      // tiles * kblocks: the stream-K work space
+  int tiles;          // output tiles
+  int slabs;          // > 0: slab schedule (grid = tiles * slabs), else stream-K
   int32_t* status;
 };
 
 // The CTA's range [g0, g1) of the work space, split into runs that stay
-// inside one output tile.
+// inside one output tile. Stream-K cuts the space into one contiguous range
+// per CTA, so at any moment the CTAs read scattered token ranges and the L2
+// catches only part of the operand re-reads (each token block is read by
+// every tile: 2.4x the compulsory DRAM bytes measured on dW2 of the block).
+// When the output has few tiles (at most half as many as SMs), the slab
+// schedule runs tiles x slabs CTAs instead: CTA c takes tile c % tiles over
+// token slab c / tiles, so the CTAs of one slab, launched together, stream
+// the same tokens at the same time and each token block crosses DRAM about
+// once. It leaves SMs % tiles SMs idle.
 struct Segment {
   int tile, kb0, n;
 };
@@ -62,9 +73,15 @@ struct SegCursor {
   int64_t g, g1;
   int kblocks;
   __device__ __forceinline__ SegCursor(const WgradArgs& a) {
-    g = a.total * blockIdx.x / gridDim.x;
-    g1 = a.total * (blockIdx.x + 1) / gridDim.x;
     kblocks = a.kblocks;
+    if (a.slabs > 0) {
+      const int tile = (int)blockIdx.x % a.tiles, slab = (int)blockIdx.x / a.tiles;
+      g = (int64_t)tile * kblocks + (int64_t)kblocks * slab / a.slabs;
+      g1 = (int64_t)tile * kblocks + (int64_t)kblocks * (slab + 1) / a.slabs;
+    } else {
+      g = a.total * blockIdx.x / gridDim.x;
+      g1 = a.total * (blockIdx.x + 1) / gridDim.x;
+    }
   }
   __device__ __forceinline__ bool next(Segment& s) {
     if (g >= g1) return false;
@@ -251,9 +268,12 @@ int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const
   args.n_tiles = (N + BN - 1) / BN;
   const int64_t tiles = (int64_t)((M + BM - 1) / BM) * args.n_tiles;
   args.total = tiles * args.kblocks;
+  args.tiles = (int)tiles;
   args.status = status;
   const int64_t sms = device_sm_count();
-  const int grid = (int)(args.total < sms ? args.total : sms);
+  const int64_t slabs = sms / tiles;
+  args.slabs = slabs >= 2 ? (int)slabs : 0;
+  const int grid = args.slabs > 0 ? (int)(tiles * slabs) : (int)(args.total < sms ? args.total : sms);
   if (cudaFuncSetAttribute(gemm_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
     return MTGR_ERR_CUDA;
