@@ -77,6 +77,16 @@ def test_workload_config_describes_the_block_workload():
     assert "larger than L2" in c["l2"]
 
 
+def test_small_workloads_flush_l2():
+    # a workload whose inputs fit in L2 is timed with the L2 flushed between
+    # steps, and its config says so; the 512-user block workload is not
+    small, big = synth.make_workload(0), synth.make_workload(2)
+    assert bench.needs_flush(small) and not bench.needs_flush(big)
+    assert bench.input_bytes(big) == int(np.asarray(big["lens"]).sum()) * 512 * 4
+    assert bench.FLUSH_BYTES > bench.L2_BYTES
+    assert "flushed" in bench.workload_config(small, 1)["l2"]
+
+
 def test_default_flags(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py"])
     a = bench.parse_args()
