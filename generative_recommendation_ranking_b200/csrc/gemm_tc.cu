@@ -10,7 +10,8 @@
 // tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM), warps 2-5 drain
 // the accumulator (tcgen05.ld), apply the epilogue, stage 32x32 blocks in
 // swizzled shared memory and write them with TMA tensor stores (the residual
-// of the last projection arrives the same way, by TMA load). The 512 TMEM
+// of the last projection comes by plain loads into a register ring, ahead of
+// use). The 512 TMEM
 // columns hold two accumulators so the epilogue of tile i overlaps the main
 // loop of tile i+1.
 #include <cuda.h>
@@ -96,9 +97,8 @@ __device__ __forceinline__ uint32_t stg_off(int r, int c) {
                          : (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
-// Epilogue math of 32 consecutive columns [col0, col0+32) of one row; the
-// result goes to row `r` of the staging block `stg` (holding the residual
-// block on entry for EPI_RESID).
+// Epilogue math of 32 consecutive columns [col0, col0+32) of one row (the
+// residual form adds its residual block afterwards, epilogue_resid_regs).
 template <int EPI, int OUT>
 __device__ __forceinline__ void epilogue_math(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
                                               float (&v)[32]) {
@@ -194,10 +194,6 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, cons
     for (int c = 0; c < 8; ++c) {
       float4* p = reinterpret_cast<float4*>(stg + stg_off<OUT>(r, c));
       float4 x = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-      if (EPI == MTGR_EPI_RESID) {
-        const float4 y = *p;
-        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
-      }
       *p = x;
     }
   } else {
@@ -211,6 +207,20 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int col0, cons
       }
       *reinterpret_cast<uint4*>(stg + stg_off<OUT>(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+  }
+}
+
+// The residual form with the residual block in registers (res: this lane's
+// row, 32 fp32 columns): v = acc (+ bias) + res, to row `r` of `stg`.
+__device__ __forceinline__ void epilogue_resid_regs(const GemmArgs& a, int col0, const uint32_t (&acc)[32],
+                                                    const float4 (&res)[8], uint8_t* stg, int r) {
+  float v[32];
+  epilogue_math<MTGR_EPI_RESID, MTGR_F32>(a, col0, acc, v);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 x = make_float4(v[4 * c] + res[c].x, v[4 * c + 1] + res[c].y, v[4 * c + 2] + res[c].z,
+                                 v[4 * c + 3] + res[c].w);
+    *reinterpret_cast<float4*>(stg + stg_off<MTGR_F32>(r, c)) = x;
   }
 }
 
@@ -255,8 +265,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
   uint64_t* empty = bars + NST;
   uint64_t* acc_full = bars + 2 * NST;
   uint64_t* acc_empty = bars + 2 * NST + 2;
-  uint64_t* rbar = bars + 2 * NST + 4;  // [EPI_WARPS][2] residual block landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 2 * EPI_WARPS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
 
   const int warp = warp_id(), lane = lane_id();
   const int M = args.M, N = args.N, K = args.K;
@@ -273,8 +282,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmO);
-    if (EPI == MTGR_EPI_RESID || EPI == kEpiSilu2) tma_prefetch_desc(&tmR);
-    for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&rbar[i], 1);
+    if (EPI == kEpiSilu2) tma_prefetch_desc(&tmR);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -358,11 +366,12 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
     }
   } else {
     // epilogue warp ew drains accumulator rows [32 quarter, 32 quarter + 32)
-    // of its CTA; the accumulator is released on the leader's barrier
+    // of its CTA; the accumulator is released on the leader's barrier (its
+    // TMEM loads have completed, so the remote arrive needs no ordering)
     auto release_acc = [&](uint64_t* bar) {
       if constexpr (CG == 2) {
         if (rank == 0) mbar_arrive(bar);
-        else mbar_arrive_cluster(mapa_shared(bar, 0));
+        else mbar_arrive_cluster_relaxed(mapa_shared(bar, 0));
       } else {
         mbar_arrive(bar);
       }
@@ -431,6 +440,66 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
             ++chunk;
           }
           load_next(zr[cc]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release_acc(&acc_empty[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    } else if constexpr (EPI == MTGR_EPI_RESID && OUT == MTGR_F32 && !ROWMAP) {
+      // The fp32 residual comes by plain loads into a register ring: each
+      // lane's 128 bytes of a block (its row, 32 columns), RB blocks ahead of
+      // use and across tile boundaries, so its DRAM latency hides behind the
+      // blocks drained meanwhile instead of stalling every block.
+      constexpr int NB = BN / 32;
+      constexpr int RB = 2;  // measured as fast as 4 (one DRAM latency is about two blocks)
+      static_assert(NB % RB == 0, "a block's ring slot is its index within the tile mod RB");
+      float4 rs[RB][8];
+      int lt = tile0, lc = 0;  // the next block to load
+      auto load_next = [&](float4 (&z)[8]) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lt < num_tiles) {
+          const int m = (lt / n_tiles) * G::kTileM + (int)rank * BM + quarter * 32 + lane;
+          const int col = (lt % n_tiles) * BN + lc * 32;
+          if (m < M && col < N) {
+            const float4* p = reinterpret_cast<const float4*>(args.resid + (size_t)m * N + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) z[i] = __ldg(p + i);
+          }
+        }
+        if (++lc == NB) { lc = 0; lt += tstride; }
+      };
+#pragma unroll
+      for (int sl = 0; sl < RB; ++sl) load_next(rs[sl]);
+      for (int tile = tile0; tile < num_tiles; tile += tstride) {
+        const int mb = tile / n_tiles, nb = tile % n_tiles;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
+        if (!ok) { timed_out = true; break; }
+        tc_fence_after();
+        const int row0 = mb * G::kTileM + (int)rank * BM + quarter * 32;
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll
+        for (int c = 0; c < NB; ++c) {
+          const int col0 = nb * BN + c * 32;
+          if (col0 < N) {
+            uint8_t* sb = stg + (chunk & 1) * STG_BYTES;
+            // the TMA store that last read this buffer (two blocks ago) must be done
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            uint32_t r[32];
+            tmem_ld32(t_row + c * 32, r);
+            tmem_ld_wait();
+            epilogue_resid_regs(args, col0, r, rs[c % RB], sb, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmO, sb, col0, row0);
+              bulk_commit_group();
+            }
+            ++chunk;
+          }
+          load_next(rs[c % RB]);
         }
         tc_fence_before();
         __syncwarp();
@@ -506,21 +575,9 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
         // the TMA store that last read this buffer (two blocks ago) must be done
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
-        // a second input block arrives by TMA into the staging block: the
-        // fp32 residual
-        constexpr bool kAuxIn = EPI == MTGR_EPI_RESID;
-        constexpr uint32_t kAuxBytes = STG_BYTES;
-        if (kAuxIn && lane == 0) {
-          mbar_arrive_expect_tx(&rbar[2 * ew + buf], kAuxBytes);
-          tma_load_2d(&tmR, &rbar[2 * ew + buf], sb, col0, row0);
-        }
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        if (kAuxIn && !__all_sync(0xffffffffu, mbar_wait(&rbar[2 * ew + buf], (chunk >> 1) & 1))) {
-          timed_out = true;
-          break;
-        }
         epilogue_chunk<EPI, OUT>(args, col0, r, sb, lane);
         fence_proxy_async_smem();
         __syncwarp();
@@ -619,12 +676,10 @@ int launch_gemm_tc(int M, int N, int K, const void* a, const void* b, const floa
                       (uint64_t)N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (rc != MTGR_OK) return rc;
-  tr = to;
-  if (epi == MTGR_EPI_RESID) {
-    rc = make_tmap_2d(&tr, resid, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)N, (uint64_t)M,
-                      (uint64_t)N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc != MTGR_OK) return rc;
-  }
+  tr = to;  // not read by these forms
+  // the residual is read by 16-byte loads along its rows (N % 32 == 0)
+  if (epi == MTGR_EPI_RESID && (resid == nullptr || (reinterpret_cast<uintptr_t>(resid) & 15) != 0))
+    return MTGR_ERR_INVALID_ARG;
   GemmArgs args{M, N, K, bias, resid, out, q_cols, status, nullptr, 0};
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_F16) return launch_cg<MTGR_EPI_NONE, MTGR_F16>(cg, ta, tb, to, tr, args, s);
   if (epi == MTGR_EPI_NONE && out_dtype == MTGR_BF16) return launch_cg<MTGR_EPI_NONE, MTGR_BF16>(cg, ta, tb, to, tr, args, s);

@@ -199,9 +199,13 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+// Arrive on an mbarrier of another CTA of the cluster (shared::cluster
+// address), without release ordering. A release arrive at cluster scope waits
+// like a memory barrier; where the arrive only announces that TMEM data was
+// read (tcgen05.wait::ld done), nothing needs ordering and the relaxed form
+// costs no stall.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                    bar_cluster_addr)
                : "memory");
 }

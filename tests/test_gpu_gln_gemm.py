@@ -96,6 +96,21 @@ def test_gemm_silu_and_residual_epilogues():
     assert_close_rms(to_host(y), y_ref, TOL_F32, "residual epilogue")
 
 
+def test_gemm_residual_single_cta_ragged():
+    # the residual form on single CTAs (K < 1024) with M and N off the tile
+    # grid: the residual ring skips rows past M and column blocks past N
+    rng = np.random.default_rng(16)
+    M, N, K = 700, 288, 512
+    a = _bf16(rng.standard_normal((M, K)))
+    b = _bf16(rng.uniform(-1, 1, (N, K)) * np.sqrt(3 / K))
+    x = rng.standard_normal((M, N)).astype(np.float32) * 2
+    dev = torch.device("cuda")
+    y = mt.gemm(torch.from_numpy(a).to(dev).bfloat16(), torch.from_numpy(b).to(dev).bfloat16(),
+                epi=mt.MTGR_EPI_RESID, resid=torch.from_numpy(x).to(dev), out_dtype=torch.float32)
+    y_ref = a.astype(np.float64) @ b.astype(np.float64).T + x
+    assert_close_rms(to_host(y), y_ref, TOL_F32, "residual epilogue, single CTAs")
+
+
 def test_gemm_f32_simt_path():
     rng = np.random.default_rng(7)
     a = rng.standard_normal((208, 64)).astype(np.float32)
