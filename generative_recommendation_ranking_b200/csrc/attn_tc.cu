@@ -97,7 +97,7 @@ struct Layout {
   static_assert(kLaunchRegs * kThreads <= 65536u, "launch registers");
 };
 // tanh pairs a SiLU warp still computes after handing the MUFU turn over
-constexpr int HANDOFF_PAIRS = 8;
+constexpr int HANDOFF_PAIRS = 4;
 // the layout of the f16-score kernels (the block's path)
 #ifndef MTGR_ATTN_SPLIT_F16
 #define MTGR_ATTN_SPLIT_F16 2
