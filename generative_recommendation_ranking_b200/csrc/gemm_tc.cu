@@ -38,13 +38,15 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 // SM's operand reads per MMA fall from 12 KB to 8 KB (the single-CTA main
 // loop is bound by shared-memory bandwidth: an M = 128, N = 256 MMA takes
 // about 165 cycles instead of 128).
-// CTA pairs for reductions of at least this length: measured on the
-// 512-user block step, pairs take MLP2 (K = 2048) from 0.831 to 0.807 ms and
-// the backward's dG~ / dX~ GEMMs down by a similar share, but slow the
-// K = 512 projections by 7% (a tile's main loop is then short, and the pair
-// waits for the slower CTA's loads and for both epilogues). The row-map
-// form stays on single CTAs.
-constexpr int kPairMinK = 1024;
+// CTA pairs for reductions of at least this length. Measured on the 512-user
+// block step: pairs take MLP2 (K = 2048) from 0.831 to 0.807 ms and the
+// backward's dG~ / dX~ GEMMs down by a similar share. At K = 512 a pair
+// tile's main loop is short enough that four epilogue warps draining 256
+// columns each became the bound (pairs were 7% slower); with eight epilogue
+// warps for the 16-bit outputs (EpiShape) pairs take the Q|K|V|U projection
+// from 0.860 to 0.76 ms and MLP1 from 0.926 to 0.80 ms. The row-map form
+// stays on single CTAs.
+constexpr int kPairMinK = 512;
 
 template <int CG>
 struct GemmShape {
@@ -59,17 +61,23 @@ constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int EPI_WARPS = 4;
 constexpr int STG_BYTES = 4096;  // one 32x32 staging block (fp32; 16-bit uses half)
-// Epilogue warps of each form. The dSiLU form (backward of MLP1's SiLU) does
-// a tanh and a few FMAs per element on top of the drain, and at K = 512 its
-// four warps, one per sub-partition, could not keep up with the MMAs; it runs
-// eight, two per TMEM lane quarter, each draining 128 of the 256 columns.
-// Its output is 16-bit, so its staging blocks are 2 KB and the eight warps'
+// Epilogue warps of each form. Eight warps, two per TMEM lane quarter, each
+// draining 128 of a tile's 256 columns, where four could not keep up with
+// the MMAs:
+// - the dSiLU form (backward of MLP1's SiLU), which does a tanh and a few
+//   FMAs per element on top of the drain;
+// - the 16-bit outputs on CTA pairs, whose K = 512 main loop is short.
+// (On single CTAs eight measured slower for the 16-bit forms: their main
+// loop is bound by shared-memory bandwidth, which more epilogue traffic
+// slows further.) The 16-bit staging blocks are 2 KB, so the eight warps'
 // double buffers take the same 32 KB as four warps' 4 KB ones.
-template <int EPI>
+template <int EPI, int OUT, int CG>
 struct EpiShape {
-  static constexpr int kWarps = EPI == kEpiDSilu ? 8 : EPI_WARPS;
+  static constexpr bool kEight =
+      EPI == kEpiDSilu || (CG == 2 && OUT != MTGR_F32 && EPI != kEpiSilu2 && EPI != MTGR_EPI_RESID);
+  static constexpr int kWarps = kEight ? 8 : EPI_WARPS;
   static constexpr int kThreads = 64 + 32 * kWarps;
-  static constexpr int kStg = EPI == kEpiDSilu ? STG_BYTES / 2 : STG_BYTES;
+  static constexpr int kStg = kEight ? STG_BYTES / 2 : STG_BYTES;
   static_assert(kWarps * kStg == EPI_WARPS * STG_BYTES, "staging memory");
 };
 constexpr size_t SMEM_BYTES =
@@ -247,7 +255,7 @@ __device__ __forceinline__ void rowmap_scatter(const GemmArgs& a, int col0, cons
 }
 
 template <int EPI, int OUT, bool ROWMAP, int CG>
-__global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
+__global__ void __launch_bounds__(EpiShape<EPI, OUT, CG>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    GemmArgs args) {
@@ -289,7 +297,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], CG * EpiShape<EPI>::kWarps);  // the pair's epilogue warps (leader's barrier)
+      mbar_init(&acc_empty[a], CG * EpiShape<EPI, OUT, CG>::kWarps);  // the pair's epilogue warps (leader's barrier)
     }
     fence_barrier_init();
   }
@@ -378,7 +386,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
     };
     const int quarter = warp & 3;
     const int ew = warp - 2;
-    uint8_t* stg = sStg + ew * 2 * EpiShape<EPI>::kStg;
+    uint8_t* stg = sStg + ew * 2 * EpiShape<EPI, OUT, CG>::kStg;
     int acc = 0;
     uint32_t acc_phase = 0, chunk = 0;
     bool prev_scatter = false;  // row-map form: the last chunk left row by row
@@ -390,7 +398,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
       // Each warp drains NB = 4 blocks of a tile (column half grp of its
       // lane quarter); every tile takes NB ring steps (blocks past N load
       // nothing), so a block's slot is its index among the warp's blocks.
-      constexpr int NB = (BN / 32) / (EpiShape<EPI>::kWarps / 4);
+      constexpr int NB = (BN / 32) / (EpiShape<EPI, OUT, CG>::kWarps / 4);
       static_assert(NB == 4, "one ring slot per block of a tile");
       const int grp = ew >> 2;
       uint4 zr[4][4];
@@ -423,7 +431,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
           const int c = grp * NB + cc;
           const int col0 = nb * BN + c * 32;
           if (col0 < N) {
-            uint8_t* sb = stg + (chunk & 1) * EpiShape<EPI>::kStg;
+            uint8_t* sb = stg + (chunk & 1) * EpiShape<EPI, OUT, CG>::kStg;
             // the TMA store that last read this buffer (two blocks ago) must be done
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
@@ -514,15 +522,18 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
       tc_fence_after();
       const int row0 = mb * G::kTileM + (int)rank * BM + quarter * 32;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+      constexpr int NBW = (BN / 32) / (EpiShape<EPI, OUT, CG>::kWarps / 4);
+      const int grp = ew >> 2;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c, ++chunk) {
+      for (int cc = 0; cc < NBW; ++cc, ++chunk) {
+        const int c = grp * NBW + cc;
         const int col0 = nb * BN + c * 32;
         if (col0 >= N) break;
         const int buf = chunk & 1;
         if (ROWMAP) {
           // 32 rows whose destinations are 32 consecutive rows leave by one
           // TMA store, like the plain form; any other group row by row
-          uint8_t* sb = stg + buf * STG_BYTES;
+          uint8_t* sb = stg + buf * EpiShape<EPI, OUT, CG>::kStg;
           if (lane == 0) {
             if (prev_scatter) bulk_wait_group_read<0>();  // chunk - 1 committed no store
             else bulk_wait_group_read<1>();
@@ -555,7 +566,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
           // two bf16 outputs per block, 2 KB each, in one staging buffer: z
           // (through tmR) in its first half, silu(z) (through tmO) in its
           // second; the buffers alternate as for one output
-          uint8_t* sb = stg + buf * STG_BYTES;
+          uint8_t* sb = stg + buf * EpiShape<EPI, OUT, CG>::kStg;
           if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
           uint32_t r[32];
@@ -571,7 +582,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::kThreads, 1)
           }
           continue;
         }
-        uint8_t* sb = stg + buf * STG_BYTES;
+        uint8_t* sb = stg + buf * EpiShape<EPI, OUT, CG>::kStg;
         // the TMA store that last read this buffer (two blocks ago) must be done
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
@@ -618,10 +629,10 @@ int launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to
   if constexpr (CG == 1) {
     const int units = device_sm_count();
     const int grid = tiles < units ? tiles : units;
-    kern<<<grid, EpiShape<EPI>::kThreads, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
+    kern<<<grid, EpiShape<EPI, OUT, CG>::kThreads, SMEM_BYTES, s>>>(ta, tb, to, tr, args);
   } else {
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(EpiShape<EPI>::kThreads);
+    cfg.blockDim = dim3(EpiShape<EPI, OUT, CG>::kThreads);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
