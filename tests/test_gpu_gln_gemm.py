@@ -77,6 +77,31 @@ def test_gemm_qkvu_epilogue_f16_with_halved_q(M, N, K):
     assert_close_rms(to_host(out), ref, 4e-3, "gemm f16 out")  # f16 rounding: 2^-11 x max|out|
 
 
+@pytest.mark.parametrize("M,N", [(1, 32), (100, 288), (257, 512), (700, 96)])
+@pytest.mark.parametrize("form", ["f16", "bf16", "silu_bf16"])
+def test_gemm_16bit_pairs_ragged(M, N, form):
+    # K = 512 runs on CTA pairs with eight epilogue warps, each on half of a
+    # tile's columns: M below one pair tile or off the 256-row grid, N off
+    # the 256-column grid (one warp group's columns all past N)
+    rng = np.random.default_rng(M * 7 + N)
+    K = 512
+    a = _bf16(rng.standard_normal((M, K)))
+    b = _bf16(rng.standard_normal((N, K)) / np.sqrt(K))
+    bias = rng.standard_normal(N).astype(np.float32) * 0.1
+    dev = torch.device("cuda")
+    epi = mt.MTGR_EPI_SILU if form == "silu_bf16" else mt.MTGR_EPI_NONE
+    dt = torch.float16 if form == "f16" else torch.bfloat16
+    out = mt.gemm(torch.from_numpy(a).to(dev).bfloat16(), torch.from_numpy(b).to(dev).bfloat16(),
+                  torch.from_numpy(bias).to(dev), epi=epi, out_dtype=dt)
+    ref = a.astype(np.float64) @ b.astype(np.float64).T + bias
+    if form == "silu_bf16":
+        ref = oracle.silu(ref)
+    if form == "f16":
+        assert_close_rms(to_host(out), ref, 4e-3, f"gemm f16 {M}x{N}")  # 2^-11 x max|out|
+    else:
+        assert_close_bf16_out(to_host(out), ref, f"gemm {form} {M}x{N}")
+
+
 def test_gemm_silu_and_residual_epilogues():
     rng = np.random.default_rng(6)
     M, d, dff = 1500, 512, 2048
