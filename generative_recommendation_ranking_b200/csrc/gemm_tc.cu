@@ -7,13 +7,14 @@
 // Design: a persistent kernel, one CTA per SM, 128x256 output tiles, 64-deep
 // k-blocks staged by TMA (128-byte swizzle) through a 4-stage mbarrier
 // pipeline. Warp 0 issues TMA loads, one thread of warp 1 issues
-// tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM), warps 2-5 drain
-// the accumulator (tcgen05.ld), apply the epilogue, stage 32x32 blocks in
-// swizzled shared memory and write them with TMA tensor stores (the residual
-// of the last projection comes by plain loads into a register ring, ahead of
-// use). The 512 TMEM
-// columns hold two accumulators so the epilogue of tile i overlaps the main
-// loop of tile i+1.
+// tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM), and the
+// epilogue warps (from warp 2) drain the accumulator (tcgen05.ld), apply the
+// epilogue, stage 32x32 blocks in swizzled shared memory and write them with
+// TMA tensor stores. The residual of the last projection comes by plain loads
+// into a register ring, ahead of use. The 512 TMEM columns hold two
+// accumulators so the epilogue of tile i overlaps the main loop of tile i+1.
+// Reductions of K >= 512 run on CTA pairs (M = 256 tiles, below), with eight
+// epilogue warps for the 16-bit outputs.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
