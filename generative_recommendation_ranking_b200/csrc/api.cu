@@ -53,7 +53,7 @@ int launch_gemm_tc_aux(int M, int N, int K, const void* a, const void* b, const 
                        void* aux, void* out, int32_t* status, cudaStream_t s);
 int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const void* b,
                       int64_t ldb, float* out, bool accumulate, int32_t* status, cudaStream_t s);
-int launch_gln_bwd(int32_t T, int32_t d, bool bf16, const void* x, const float* dy,
+int launch_gln_bwd(int32_t T, int32_t d, bool bf16, const void* x, const void* dy, bool dy_bf16,
                    const int8_t* gid, int32_t G, const float* gamma, float eps, float* dgamma,
                    float* dbeta, float* dx, const float* dres, const void* qkvu, const void* obar,
                    void* dobar, void* dz, int32_t* status, cudaStream_t s);
@@ -311,7 +311,7 @@ struct BwdWs {
   void* w1t;     // bf16 W1^T [d][d_ff]
   void* wt;      // bf16 W^T [d][4d]
   void* dz1;     // dZ1 [T][d_ff] (bf16 or fp32)
-  float* dgt;    // dG~, then dX~ [T][d] fp32
+  void* dgt;     // dG~, then dX~ [T][d]: bf16 on the bf16 path, else fp32
   void* dobar;   // dO~ [T][d] (f16 or fp32)
   void* dz;      // dZ = [dQ|dK|dV|dU] [T][4d] (bf16 or fp32)
   float* dq;     // fp32 dQ accumulator [T][d] (bf16 blocks)
@@ -334,7 +334,7 @@ BwdWs bwd_layout(int32_t T, const mtgr_block_params* p, const mtgr_batch* bt, vo
     w.wt = b + off;  off += align_up(d * 4 * d * 2, 256);
   }
   w.dz1 = b + off;   off += align_up(t * f * e, 256);
-  w.dgt = reinterpret_cast<float*>(b + off); off += align_up(t * d * 4, 256);
+  w.dgt = b + off;   off += align_up(t * d * 4, 256);
   w.dobar = b + off; off += align_up(t * d * e, 256);
   w.dz = b + off;    off += align_up(t * 4 * d * e, 256);
   if (bf) {
@@ -450,13 +450,13 @@ int block_bwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
     }
     {  // dG~ = dZ1 W1
       TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);
-      if ((rc = launch_gemm_tc(T, d, dff, w.dz1, w.w1t, nullptr, MTGR_EPI_NONE, nullptr, 0, MTGR_F32,
+      if ((rc = launch_gemm_tc(T, d, dff, w.dz1, w.w1t, nullptr, MTGR_EPI_NONE, nullptr, 0, MTGR_BF16,
                                w.dgt, bt->status, s)) != MTGR_OK)
         return rc;
     }
     {  // GroupLN_2 and the gate: dO~ (f16), dU into dZ
       TimedScope tsc(MTGR_TIMER_BWD_GLN, s, 1);
-      if ((rc = launch_gln_bwd(T, d, true, sv.g, w.dgt, bt->group_id, 4, p->gln2_gamma, p->eps,
+      if ((rc = launch_gln_bwd(T, d, true, sv.g, w.dgt, true, bt->group_id, 4, p->gln2_gamma, p->eps,
                                gr->gln2_gamma, gr->gln2_beta, nullptr, nullptr, sv.qkvu, sv.obar,
                                w.dobar, w.dz, bt->status, s)) != MTGR_OK)
         return rc;
@@ -480,7 +480,7 @@ int block_bwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
     }
     {  // dX~ = dZ W
       TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);
-      if ((rc = launch_gemm_tc(T, d, 4 * d, w.dz, w.wt, nullptr, MTGR_EPI_NONE, nullptr, 0, MTGR_F32,
+      if ((rc = launch_gemm_tc(T, d, 4 * d, w.dz, w.wt, nullptr, MTGR_EPI_NONE, nullptr, 0, MTGR_BF16,
                                w.dgt, bt->status, s)) != MTGR_OK)
         return rc;
     }
@@ -509,12 +509,12 @@ int block_bwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
     {
       TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);  // dG~ = dZ1 W1
       if ((rc = launch_gemm_f32_strided(T, d, dff, dz1f, dff, 1, static_cast<const float*>(p->w1), d,
-                                        1, MTGR_EPI_NONE, nullptr, w.dgt, s)) != MTGR_OK)
+                                        1, MTGR_EPI_NONE, nullptr, static_cast<float*>(w.dgt), s)) != MTGR_OK)
         return rc;
     }
     {
       TimedScope tsc(MTGR_TIMER_BWD_GLN, s, 1);
-      if ((rc = launch_gln_bwd(T, d, false, sv.g, w.dgt, bt->group_id, 4, p->gln2_gamma, p->eps,
+      if ((rc = launch_gln_bwd(T, d, false, sv.g, w.dgt, false, bt->group_id, 4, p->gln2_gamma, p->eps,
                                gr->gln2_gamma, gr->gln2_beta, nullptr, nullptr, sv.qkvu, sv.obar,
                                w.dobar, w.dz, bt->status, s)) != MTGR_OK)
         return rc;
@@ -536,13 +536,13 @@ int block_bwd(const mtgr_block_params* p, const mtgr_batch* bt, const float* x_i
       TimedScope tsc(MTGR_TIMER_BWD_GEMM, s, 1);  // dX~ = dZ W
       if ((rc = launch_gemm_f32_strided(T, d, 4 * d, dzf, 4 * d, 1,
                                         static_cast<const float*>(p->w_qkvu), d, 1, MTGR_EPI_NONE,
-                                        nullptr, w.dgt, s)) != MTGR_OK)
+                                        nullptr, static_cast<float*>(w.dgt), s)) != MTGR_OK)
         return rc;
     }
   }
   {  // GroupLN_1 and the residual: dX = GLN_1 backward of dX~ + dY
     TimedScope tsc(MTGR_TIMER_BWD_GLN, s, 1);
-    if ((rc = launch_gln_bwd(T, d, false, x_in, w.dgt, bt->group_id, 4, p->gln1_gamma, p->eps,
+    if ((rc = launch_gln_bwd(T, d, false, x_in, w.dgt, p->dtype == MTGR_BF16, bt->group_id, 4, p->gln1_gamma, p->eps,
                              gr->gln1_gamma, gr->gln1_beta, dx, dy, nullptr, nullptr, nullptr,
                              nullptr, bt->status, s)) != MTGR_OK)
       return rc;

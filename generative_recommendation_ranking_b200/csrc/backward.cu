@@ -87,7 +87,7 @@ __device__ __forceinline__ void st8(__half* p, const float (&v)[8]) {
 // --------------------------------------------------------- GroupLN backward --
 struct GlnBwdArgs {
   int32_t T, d, G;
-  const float* dy;      // [T][d] gradient of the GroupLN output
+  const void* dy;       // [T][d] gradient of the GroupLN output (Ty)
   const void* x;        // [T][d] GroupLN input (Tx)
   const int8_t* gid;    // [T]
   const float* gamma;   // [G][d]
@@ -113,7 +113,7 @@ struct GlnBwdArgs {
 // accumulate in registers while the group stays the same (the tokens of a
 // user's segment are consecutive), go to the block's shared-memory sums when
 // it changes, and the block adds those to the global sums once.
-template <typename Tx, int VPL, bool GATE, typename Tq, typename To, typename Tg, typename Tz>
+template <typename Tx, typename Ty, int VPL, bool GATE, typename Tq, typename To, typename Tg, typename Tz>
 __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
   extern __shared__ float sacc[];  // [2][G][d]: dgamma, dbeta
   const int d = a.d, G = a.G, nv = d >> 3;
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(256) gln_bwd_kernel(GlnBwdArgs a) {
       const int vi = lane + 32 * k;
       if (vi < nv) {
         ld8(x + t * d + 8 * vi, xv[k]);
-        ld8(a.dy + t * d + 8 * vi, gv[k]);
+        ld8(static_cast<const Ty*>(a.dy) + t * d + 8 * vi, gv[k]);
         if (GATE) {
           ld8(static_cast<const Tq*>(a.qkvu) + t * 4 * d + 3 * d + 8 * vi, e1[k]);  // U
           ld8(static_cast<const To*>(a.obar) + t * d + 8 * vi, e2[k]);             // O~
@@ -567,7 +567,7 @@ int grid_for(int64_t n, int threads) {
 // GroupLN backward. Plain: dx = GLN backward of dy (+ dres). Gate form: see
 // GlnBwdArgs. dgamma/dbeta [G][d] are zeroed here. bf16 selects the bf16
 // block's types (x bf16, U f16, O~ bf16, dO~ f16, dU bf16), else all fp32.
-int launch_gln_bwd(int32_t T, int32_t d, bool bf16, const void* x, const float* dy,
+int launch_gln_bwd(int32_t T, int32_t d, bool bf16, const void* x, const void* dy, bool dy_bf16,
                    const int8_t* gid, int32_t G, const float* gamma, float eps, float* dgamma,
                    float* dbeta, float* dx, const float* dres, const void* qkvu, const void* obar,
                    void* dobar, void* dz, int32_t* status, cudaStream_t s) {
@@ -588,7 +588,8 @@ int launch_gln_bwd(int32_t T, int32_t d, bool bf16, const void* x, const float* 
   const bool gate = obar != nullptr;
 #define MTGR_GLN_BWD(TX, V, GT, TQ, TO, TG, TZ)                                                  \
   do {                                                                                           \
-    auto k = gln_bwd_kernel<TX, V, GT, TQ, TO, TG, TZ>;                                          \
+    auto k = dy_bf16 ? gln_bwd_kernel<TX, __nv_bfloat16, V, GT, TQ, TO, TG, TZ>                  \
+                     : gln_bwd_kernel<TX, float, V, GT, TQ, TO, TG, TZ>;                         \
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=       \
         cudaSuccess)                                                                             \
       return MTGR_ERR_CUDA;                                                                      \
