@@ -618,9 +618,11 @@ typedef struct mtgr_block_grads {
  * bf16 blocks run the contractions on tcgen05 tensor cores (the attention's
  * with f16 operands, its dO~ = dG (.) U in f16: values beyond 65504 set
  * MTGR_ERR_RANGE in the batch status, values below 2^-14 lose precision as
- * f16 subnormals, so scale the loss as usual for f16 training); fp32 blocks
- * on CUDA cores. Weight gradients are sums over all tokens accumulated in
- * fp32 in an order that varies from run to run.
+ * f16 subnormals, so scale the loss as usual for f16 training), and keep the
+ * gradients of the GroupLN outputs (dG~, dX~) in bf16 between a GEMM and the
+ * GroupLN backward that reads them; fp32 blocks run on CUDA cores in fp32
+ * throughout. Weight gradients are sums over all tokens accumulated in fp32
+ * in an order that varies from run to run.
  */
 MTGR_API size_t mtgr_block_bwd_workspace_bytes(int32_t T, const mtgr_block_params* p,
                                                const mtgr_batch* batch);
