@@ -267,8 +267,8 @@ __global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
   uint64_t* p_full = s_free + 2;             // [A, B]
   uint64_t* p_free = p_full + 2;             // [A, B]
   uint64_t* o_full = p_free + 2;
-  uint64_t* o_free = o_full + 1;
-  uint64_t* u_full = o_free + 1;
+  uint64_t* o_free = o_full + 1;             // [A, B]: each q-tile's O read by the epilogue
+  uint64_t* u_full = o_free + 2;
   uint64_t* u_empty = u_full + 1;
   // Turns on each SM sub-partition's MUFU pipe, one barrier pair per A/B
   // warp pair sharing it: [key half][sub-partition][slot]
@@ -293,7 +293,8 @@ __global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
       mbar_init(&v_ready[s], NUM_EPI_WARPS);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_free, NUM_EPI_WARPS);
+    mbar_init(&o_free[0], NUM_EPI_WARPS);
+    mbar_init(&o_free[1], NUM_EPI_WARPS);
     mbar_init(u_full, 1);
     mbar_init(u_empty, NUM_EPI_WARPS);
     for (int i = 0; i < 8 * SPLIT; ++i) {
@@ -411,7 +412,6 @@ __global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
         const Item it = nxt;
         if (w + stride < n_items) nxt = load_item(a, w + stride);
         const bool two = it.w.nq == 2;
-        if (!mbar_wait(o_free, (li & 1) ^ 1)) { timed_out = true; break; }
         for (int32_t t = 0; t < it.w.n_union && !timed_out; ++t, ++g) {
           const int st = g % KV_STAGES;
           // V landed (and, for bf16 inputs, was converted to f16)
@@ -422,6 +422,8 @@ __global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
           const uint32_t v_addr = smem_u32(sKV + st * 2 * TILE_BYTES + TILE_BYTES);
           for (int q = 0; q < (two ? 2 : 1); ++q) {
             const int32_t r = q == 0 ? gp_a : gp_b;
+            // the item's first P V into O_q: the previous item's O_q has been read
+            if (t == 0 && !mbar_wait(&o_free[q], (li & 1) ^ 1)) { timed_out = true; break; }
             if (!mbar_wait(&p_full[q], r & 1)) { timed_out = true; break; }
             tc_fence_after();
             const uint32_t o_dst = tmem + o_col(q);
@@ -656,10 +658,10 @@ __global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
           uint32_t o[32];
           tmem_ld32(tmem + lane_base + o_col(q) + 32 * hc, o);
           tmem_ld_wait();
-          if (hc == 1 && q == it.w.nq - 1) {  // all of O read: the next item may accumulate
+          if (hc == 1) {  // all of O_q read: the next item may accumulate into it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(o_free);
+            if (lane == 0) mbar_arrive(&o_free[q]);
           }
           if (i < it.w.n) {
 #pragma unroll
@@ -704,6 +706,11 @@ __global__ void __launch_bounds__(Layout<SPLIT>::kThreads, 1)
           }
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, MTGR_ERR_RANGE);
+      }
+      // every item completes one phase of both O slots
+      if (it.w.nq == 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[1]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(u_empty);  // U of this item consumed
