@@ -62,28 +62,53 @@ struct WgradArgs {
 // catches only part of the operand re-reads (each token block is read by
 // every tile: 2.4x the compulsory DRAM bytes measured on dW2 of the block).
 // When the output has few tiles (at most half as many as SMs), the slab
-// schedule runs tiles x slabs CTAs instead: CTA c takes tile c % tiles over
-// token slab c / tiles, so the CTAs of one slab, launched together, stream
-// the same tokens at the same time and each token block crosses DRAM about
-// once. It leaves SMs % tiles SMs idle.
+// schedule cuts the tokens into slabs and the work into (tile, slab) units,
+// slab-major: unit u is tile u % tiles over slab u / tiles, and CTA c takes
+// units c, c + gridDim.x, ... The CTAs running at any moment then cover a
+// few slabs for all tiles, so they stream the same tokens at about the same
+// time and each token block crosses DRAM about once. The slab count makes
+// tiles x slabs a multiple of the SM count (37 slabs for 32 tiles on 148
+// SMs), so every SM gets the same work; each unit's partial tile goes out by
+// reduce-add.
 struct Segment {
   int tile, kb0, n;
 };
 struct SegCursor {
   int64_t g, g1;
   int kblocks;
+  // slab schedule: the units (tile, slab), slab-major, CTA c taking units
+  // c, c + gridDim.x, ...
+  int64_t u, units;
+  int tiles, slabs;
   __device__ __forceinline__ SegCursor(const WgradArgs& a) {
     kblocks = a.kblocks;
+    slabs = a.slabs;
+    tiles = a.tiles;
+    u = blockIdx.x;
+    units = (int64_t)a.tiles * a.slabs;
     if (a.slabs > 0) {
-      const int tile = (int)blockIdx.x % a.tiles, slab = (int)blockIdx.x / a.tiles;
-      g = (int64_t)tile * kblocks + (int64_t)kblocks * slab / a.slabs;
-      g1 = (int64_t)tile * kblocks + (int64_t)kblocks * (slab + 1) / a.slabs;
+      g = g1 = 0;
     } else {
       g = a.total * blockIdx.x / gridDim.x;
       g1 = a.total * (blockIdx.x + 1) / gridDim.x;
     }
   }
   __device__ __forceinline__ bool next(Segment& s) {
+    if (slabs > 0) {
+      for (; u < units; u += gridDim.x) {
+        const int tile = (int)(u % tiles), slab = (int)(u / tiles);
+        const int kb0 = (int)((int64_t)kblocks * slab / slabs);
+        const int kb1 = (int)((int64_t)kblocks * (slab + 1) / slabs);
+        if (kb1 > kb0) {
+          s.tile = tile;
+          s.kb0 = kb0;
+          s.n = kb1 - kb0;
+          u += gridDim.x;
+          return true;
+        }
+      }
+      return false;
+    }
     if (g >= g1) return false;
     s.tile = (int)(g / kblocks);
     s.kb0 = (int)(g - (int64_t)s.tile * kblocks);
@@ -271,9 +296,21 @@ int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const
   args.tiles = (int)tiles;
   args.status = status;
   const int64_t sms = device_sm_count();
-  const int64_t slabs = sms / tiles;
-  args.slabs = slabs >= 2 ? (int)slabs : 0;
-  const int grid = args.slabs > 0 ? (int)(tiles * slabs) : (int)(args.total < sms ? args.total : sms);
+  // slabs so that tiles x slabs is a multiple of the SM count: every CTA
+  // then takes the same number of (tile, slab) units
+  int64_t gcd = tiles, r = sms;
+  while (r != 0) { const int64_t t2 = gcd % r; gcd = r; r = t2; }
+  const int64_t even = sms / gcd;  // lcm(tiles, sms) / tiles
+  int64_t slabs = 0, grid64 = 0;
+  if (tiles * 2 <= sms && even <= 64 && even * BK <= T) {
+    slabs = even;
+    grid64 = sms;
+  } else if (sms / tiles >= 2) {
+    slabs = sms / tiles;
+    grid64 = tiles * slabs;
+  }
+  args.slabs = (int)slabs;
+  const int grid = slabs > 0 ? (int)grid64 : (int)(args.total < sms ? args.total : sms);
   if (cudaFuncSetAttribute(gemm_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
     return MTGR_ERR_CUDA;
