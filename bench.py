@@ -282,6 +282,7 @@ def rank_workload(args, world: int, rank: int):
 
 L2_BYTES = 126 * 10**6   # the B200's L2
 FLUSH_BYTES = 256 * 2**20
+E2E_STREAMS = 3  # host-buffer leg: streams (and workspaces) the steps rotate over
 
 
 def input_bytes(wl: dict) -> int:
@@ -428,10 +429,14 @@ def run_e2e(wsp: Workspace, steps: int, world: int, dev, users_total: int):
     (mtgr_stack_fwd_host): every call copies the step's lengths, timestamps
     and token features from pinned host memory into the device workspace,
     packs, builds the mask metadata, runs the stack and copies the whole
-    output and the status word back. Steps alternate between two streams,
-    each with its own workspace, so one step's copies overlap the other's
-    kernels (PCIe is full duplex). Attention-only workloads keep the
-    device-pointer path (the host entry runs the block stack)."""
+    output and the status word back. Steps rotate over E2E_STREAMS streams,
+    each with its own workspace and output buffer. On one stream a step's
+    input copy waits for the output copy of the step before it there, so
+    with three streams one step's input copy, another's kernels and a third's
+    output copy run at once and both directions of the (full-duplex) PCIe
+    link stay busy; two leave each direction idle while a stream turns
+    around. Attention-only workloads keep the device-pointer path (the host
+    entry runs the block stack)."""
     import generative_recommendation_ranking_b200 as mt
     from generative_recommendation_ranking_b200 import _lib
     wl = wsp.wl
@@ -442,21 +447,21 @@ def run_e2e(wsp: Workspace, steps: int, world: int, dev, users_total: int):
     hn = (torch.from_numpy(np.ascontiguousarray(wl["norm"], np.float32)).pin_memory()
           if wl.get("norm") is not None else None)
     hx = torch.from_numpy(np.ascontiguousarray(wl["x"], np.float32)).pin_memory()
-    hout = [torch.empty_like(hx).pin_memory() for _ in range(2)]
-    hst = [torch.zeros(1, dtype=torch.int32).pin_memory() for _ in range(2)]
+    hout = [torch.empty_like(hx).pin_memory() for _ in range(E2E_STREAMS)]
+    hst = [torch.zeros(1, dtype=torch.int32).pin_memory() for _ in range(E2E_STREAMS)]
     c_layers = [l.c for l in wsp.layers]
     nbytes = _lib.mtgr_stack_fwd_host_workspace_bytes(hl, c_layers)
-    dws = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-    streams = [torch.cuda.Stream(dev) for _ in range(2)]
+    dws = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(E2E_STREAMS)]
+    streams = [torch.cuda.Stream(dev) for _ in range(E2E_STREAMS)]
     h2d = hl.numel() * 4 + ht.numel() * 8 + hx.numel() * 4 + (hn.numel() * 4 if hn is not None else 0)
     d2h = hout[0].numel() * 4 + 4
 
     def run(n):
         for k in range(n):
-            i = k & 1
+            i = k % E2E_STREAMS
             _lib.mtgr_stack_fwd_host(c_layers, hl, ht, hn, hx, hout[i], hst[i], dws[i], streams[i])
 
-    run(2)
+    run(E2E_STREAMS)
     torch.cuda.synchronize(dev)
     barrier(world)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -473,11 +478,12 @@ def run_e2e(wsp: Workspace, steps: int, world: int, dev, users_total: int):
     assert all(int(h.item()) == 0 for h in hst), "e2e device status"
     wsp.step()
     torch.cuda.synchronize(dev)
-    assert torch.equal(hout[(steps - 1) & 1], wsp.out.cpu()), "e2e output mismatch"
+    assert torch.equal(hout[(steps - 1) % E2E_STREAMS], wsp.out.cpu()), "e2e output mismatch"
     return {"value": users_total * steps / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ems / steps,
             "path": "C ABI mtgr_stack_fwd_host (host buffers in, host buffers out)",
-            "pipelining": "2 streams, 2 workspaces: one step's copies overlap the other's kernels"}
+            "pipelining": f"{E2E_STREAMS} streams, {E2E_STREAMS} workspaces: one step's input copy, "
+                          "another's kernels and a third's output copy overlap"}
 
 
 def run_ours(args, world, rank, local):
