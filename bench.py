@@ -1017,10 +1017,11 @@ def run_backward(args, local):
             "attention": ("tensor", 4.0 * d * V),
             "gemm_qkvu": ("tensor", 2.0 * T * 4 * d * d), "gemm_mlp1": ("tensor", 2.0 * T * d * dff),
             "gemm_mlp2": ("tensor", 2.0 * T * d * dff),
-            # GroupLN backward, bytes per token: GLN_1 reads x, dX~, dY and
-            # writes dX (fp32: 16 d); GLN_2 with the gate reads G (bf16), dG~
-            # (fp32), U (f16), O/N (bf16) and writes dO~ (f16), dU (bf16): 14 d
-            "bwd_gln": ("hbm", T * d * (16.0 + 14.0))}
+            # GroupLN backward, bytes per token: GLN_1 reads x (fp32), dX~
+            # (bf16), dY (fp32) and writes dX (fp32): 14 d; GLN_2 with the
+            # gate reads G (bf16), dG~ (bf16), U (f16), O/N (bf16) and writes
+            # dO~ (f16), dU (bf16): 12 d
+            "bwd_gln": ("hbm", T * d * (14.0 + 12.0))}
     kernels = {}
     for cls, (bound, w) in work.items():
         t_ms, cnt = per[cls]
