@@ -10,16 +10,24 @@
 // operand in blocks of 64 contiguous m (or n) values, LBO = 8 KB apart, with
 // 8-token groups SBO = 1 KB apart.
 //
+// The kernel runs on CTA pairs (tcgen05.mma.cta_group::2): a pair tile is
+// 256 x 256, each CTA loading its 128 rows of A and its 128 columns of B per
+// 64-token block, so an SM moves 32 KB of operands through shared memory per
+// block instead of 48 KB (a single CTA's 128 x 256 tile). The single-CTA
+// form was bound by that shared-memory traffic (TMA writes plus MMA reads),
+// not by the tensor pipe.
+//
 // The reduction dimension (T, hundreds of thousands of tokens) is far longer
-// than the output has tiles (a 2048 x 512 gradient is 32 tiles of 128 x 256),
+// than the output has tiles (a 2048 x 512 gradient is 16 pair tiles),
 // so the work is split "stream-K": the (tile, 64-token block) space is cut
 // into one contiguous range per CTA, and each CTA adds every partial tile it
 // finishes into the fp32 output with TMA reduce-add stores
 // (cp.reduce.async.bulk.tensor ... .add); with few tiles, a slab schedule
 // replaces the contiguous ranges (SegCursor). The caller zeroes the output first
 // unless it accumulates. Roles as in the block's forward GEMM: warp 0 TMA
-// producer, one thread of warp 1 issues the MMAs, warps 2-5 drain the
-// double-buffered TMEM accumulator.
+// producer, one thread of warp 1 of the leader CTA issues the pair MMAs,
+// warps 2-5 of each CTA drain its 128 rows of the double-buffered TMEM
+// accumulator.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -32,11 +40,13 @@ namespace mtgr {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+// A pair tile is PAIR_M x BN: each CTA of the pair holds BM of its rows (its
+// half of the A operand) and BN / 2 of its columns (its half of B).
+constexpr int BM = 128, PAIR_M = 2 * BM, BN = 256, BH = BN / 2, BK = 64, STAGES = 6;
 constexpr int BOX = 64;                     // MN values per TMA box (128 bytes)
 constexpr int BOX_BYTES = BOX * BK * 2;     // 8 KB
 constexpr int A_BYTES = BM * BK * 2;        // 2 boxes
-constexpr int B_BYTES = BN * BK * 2;        // 4 boxes
+constexpr int B_BYTES = BH * BK * 2;        // 2 boxes
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
@@ -49,53 +59,56 @@ constexpr size_t SMEM_BYTES =
 struct WgradArgs {
   int M, N;
   int kblocks;        // ceil(T / BK)
-  int n_tiles;        // tiles along N
+  int n_tiles;        // pair tiles along N
   int64_t total;      // tiles * kblocks: the stream-K work space
-  int tiles;          // output tiles
-  int slabs;          // > 0: slab schedule (grid = tiles * slabs), else stream-K
+  int tiles;          // output pair tiles (PAIR_M x BN)
+  int slabs;          // > 0: slab schedule, else stream-K
   int32_t* status;
 };
 
-// The CTA's range [g0, g1) of the work space, split into runs that stay
+// The pair's range [g0, g1) of the work space, split into runs that stay
 // inside one output tile. Stream-K cuts the space into one contiguous range
-// per CTA, so at any moment the CTAs read scattered token ranges and the L2
+// per pair, so at any moment the pairs read scattered token ranges and the L2
 // catches only part of the operand re-reads (each token block is read by
 // every tile: 2.4x the compulsory DRAM bytes measured on dW2 of the block).
-// When the output has few tiles (at most half as many as SMs), the slab
+// When the output has few tiles (at most half as many as pairs), the slab
 // schedule cuts the tokens into slabs and the work into (tile, slab) units,
-// slab-major: unit u is tile u % tiles over slab u / tiles, and CTA c takes
-// units c, c + gridDim.x, ... The CTAs running at any moment then cover a
-// few slabs for all tiles, so they stream the same tokens at about the same
+// slab-major: unit u is tile u % tiles over slab u / tiles, and pair p takes
+// units p, p + pairs, ... The pairs running at any moment then cover a few
+// slabs for all tiles, so they stream the same tokens at about the same
 // time and each token block crosses DRAM about once. The slab count makes
-// tiles x slabs a multiple of the SM count (37 slabs for 32 tiles on 148
-// SMs), so every SM gets the same work; each unit's partial tile goes out by
-// reduce-add.
+// tiles x slabs a multiple of the pair count (37 slabs for 16 tiles on 74
+// pairs), so every pair gets the same work; each unit's partial tile goes
+// out by reduce-add.
 struct Segment {
   int tile, kb0, n;
 };
 struct SegCursor {
   int64_t g, g1;
   int kblocks;
-  // slab schedule: the units (tile, slab), slab-major, CTA c taking units
-  // c, c + gridDim.x, ...
+  // slab schedule: the units (tile, slab), slab-major, pair p taking units
+  // p, p + pairs, ...
   int64_t u, units;
   int tiles, slabs;
+  int64_t pair, pairs;  // both CTAs of a pair walk the pair's units
   __device__ __forceinline__ SegCursor(const WgradArgs& a) {
     kblocks = a.kblocks;
     slabs = a.slabs;
     tiles = a.tiles;
-    u = blockIdx.x;
+    pair = blockIdx.x >> 1;
+    pairs = gridDim.x >> 1;
+    u = pair;
     units = (int64_t)a.tiles * a.slabs;
     if (a.slabs > 0) {
       g = g1 = 0;
     } else {
-      g = a.total * blockIdx.x / gridDim.x;
-      g1 = a.total * (blockIdx.x + 1) / gridDim.x;
+      g = a.total * pair / pairs;
+      g1 = a.total * (pair + 1) / pairs;
     }
   }
   __device__ __forceinline__ bool next(Segment& s) {
     if (slabs > 0) {
-      for (; u < units; u += gridDim.x) {
+      for (; u < units; u += pairs) {
         const int tile = (int)(u % tiles), slab = (int)(u / tiles);
         const int kb0 = (int)((int64_t)kblocks * slab / slabs);
         const int kb1 = (int)((int64_t)kblocks * (slab + 1) / slabs);
@@ -103,7 +116,7 @@ struct SegCursor {
           s.tile = tile;
           s.kb0 = kb0;
           s.n = kb1 - kb0;
-          u += gridDim.x;
+          u += pairs;
           return true;
         }
       }
@@ -136,6 +149,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
 
   const int warp = warp_id(), lane = lane_id();
+  // rank 0 of the pair (the leader) issues the pair MMAs; both CTAs load
+  // their halves of each stage and drain their own 128 accumulator rows
+  const uint32_t rank = cluster_ctarank();
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -146,16 +162,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], EPI_WARPS);
+      mbar_init(&acc_empty[a], 2 * EPI_WARPS);  // the pair's epilogue warps (leader's barrier)
     }
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_cg2(tmem_slot, TMEM_COLS);
+    tmem_relinquish_cg2();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   bool timed_out = false;
@@ -167,26 +183,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       SegCursor cur(args);
       Segment sg;
       while (!timed_out && cur.next(sg)) {
-        const int m0 = (sg.tile / args.n_tiles) * BM, n0 = (sg.tile % args.n_tiles) * BN;
+        const int m0 = (sg.tile / args.n_tiles) * PAIR_M + (int)rank * BM;
+        const int n0 = (sg.tile % args.n_tiles) * BN + (int)rank * BH;
         for (int kb = sg.kb0; kb < sg.kb0 + sg.n; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { timed_out = true; break; }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          // both CTAs' halves complete on the leader's barrier, which the
+          // leader arms for the bytes of both
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          const uint32_t fb = mapa_shared(&full[stage], 0);
           uint8_t* a = sA + stage * A_BYTES;
           uint8_t* b = sB + stage * B_BYTES;
 #pragma unroll
-          for (int j = 0; j < BM / BOX; ++j)
-            tma_load_2d(&tmA, &full[stage], a + j * BOX_BYTES, m0 + j * BOX, kb * BK);
+          for (int j = 0; j < BM / BOX; ++j) tma_load_2d_cg2(&tmA, fb, a + j * BOX_BYTES, m0 + j * BOX, kb * BK);
 #pragma unroll
-          for (int j = 0; j < BN / BOX; ++j)
-            tma_load_2d(&tmB, &full[stage], b + j * BOX_BYTES, n0 + j * BOX, kb * BK);
+          for (int j = 0; j < BH / BOX; ++j) tma_load_2d_cg2(&tmB, fb, b + j * BOX_BYTES, n0 + j * BOX, kb * BK);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // bf16 operands, both MN-major, fp32 accumulator
-      constexpr uint32_t idesc = idesc_f16(BM, BN, 1u, true, true);
+    if (lane == 0 && rank == 0) {
+      // bf16 operands, both MN-major, fp32 accumulator; M = 256 over the pair
+      constexpr uint32_t idesc = idesc_f16(PAIR_M, BN, 1u, true, true);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       SegCursor cur(args);
@@ -203,19 +221,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // 16 tokens = two 8-token groups of 1 KB each
-            tc_mma_ss(d_tmem, sdesc_sw128(a_addr + 2048 * k, BOX_BYTES, 1024),
-                      sdesc_sw128(b_addr + 2048 * k, BOX_BYTES, 1024), idesc, (i | k) != 0 ? 1u : 0u);
+            tc_mma_ss_cg2(d_tmem, sdesc_sw128(a_addr + 2048 * k, BOX_BYTES, 1024),
+                          sdesc_sw128(b_addr + 2048 * k, BOX_BYTES, 1024), idesc, (i | k) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          tc_commit_cg2(&empty[stage], 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (timed_out) break;
-        tc_commit(&acc_full[acc]);
+        tc_commit_cg2(&acc_full[acc], 0x3);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
     }
   } else {
     // epilogue warp ew adds accumulator rows [32 quarter, 32 quarter + 32)
+    // of its CTA; the accumulator is released on the leader's barrier (its
+    // TMEM loads have completed, so the remote arrive needs no ordering)
+    auto release_acc = [&](uint64_t* bar) {
+      if (rank == 0) mbar_arrive(bar);
+      else mbar_arrive_cluster_relaxed(mapa_shared(bar, 0));
+    };
     const int quarter = warp & 3;
     const int ew = warp - 2;
     uint8_t* stg = sStg + ew * 2 * STG_BYTES;
@@ -224,7 +248,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     SegCursor cur(args);
     Segment sg;
     while (cur.next(sg)) {
-      const int m0 = (sg.tile / args.n_tiles) * BM, n0 = (sg.tile % args.n_tiles) * BN;
+      const int m0 = (sg.tile / args.n_tiles) * PAIR_M + (int)rank * BM;
+      const int n0 = (sg.tile % args.n_tiles) * BN;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase))) { timed_out = true; break; }
       tc_fence_after();
       const int row0 = m0 + quarter * 32;
@@ -254,16 +279,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (lane == 0) release_acc(&acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
     if (lane == 0) bulk_wait_group<0>();  // reductions complete before the CTA retires
   }
   if (timed_out) set_status(args.status, MTGR_ERR_TIMEOUT);
-  __syncthreads();
+  // a pair retires together: the leader's MMAs read the other CTA's shared
+  // memory and the other CTA arrives on the leader's barriers
+  tc_fence_before();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_cg2(tmem_base, TMEM_COLS);
   }
 }
 
@@ -291,30 +319,53 @@ int launch_gemm_wgrad(int M, int N, int64_t T, const void* a, int64_t lda, const
   args.N = N;
   args.kblocks = (int)((T + BK - 1) / BK);
   args.n_tiles = (N + BN - 1) / BN;
-  const int64_t tiles = (int64_t)((M + BM - 1) / BM) * args.n_tiles;
+  const int64_t tiles = (int64_t)((M + PAIR_M - 1) / PAIR_M) * args.n_tiles;
   args.total = tiles * args.kblocks;
   args.tiles = (int)tiles;
   args.status = status;
-  const int64_t sms = device_sm_count();
-  // slabs so that tiles x slabs is a multiple of the SM count: every CTA
-  // then takes the same number of (tile, slab) units
-  int64_t gcd = tiles, r = sms;
-  while (r != 0) { const int64_t t2 = gcd % r; gcd = r; r = t2; }
-  const int64_t even = sms / gcd;  // lcm(tiles, sms) / tiles
-  int64_t slabs = 0, grid64 = 0;
-  if (tiles * 2 <= sms && even <= 64 && even * BK <= T) {
-    slabs = even;
-    grid64 = sms;
-  } else if (sms / tiles >= 2) {
-    slabs = sms / tiles;
-    grid64 = tiles * slabs;
-  }
-  args.slabs = (int)slabs;
-  const int grid = slabs > 0 ? (int)grid64 : (int)(args.total < sms ? args.total : sms);
   if (cudaFuncSetAttribute(gemm_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
     return MTGR_ERR_CUDA;
-  gemm_wgrad_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, to, args);
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // The pairs are persistent: no more than can be resident at once (a GPC
+  // with an odd number of SMs leaves one SM unpaired).
+  static int resident = 0;
+  if (resident == 0) {
+    cfg.gridDim = dim3(device_sm_count());
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_wgrad_kernel, &cfg) != cudaSuccess || n <= 0)
+      return MTGR_ERR_CUDA;
+    resident = n;
+  }
+  const int64_t np = resident;
+  // slabs so that tiles x slabs is a multiple of the pair count: every pair
+  // then takes the same number of (tile, slab) units
+  int64_t gcd = tiles, r = np;
+  while (r != 0) { const int64_t t2 = gcd % r; gcd = r; r = t2; }
+  const int64_t even = np / gcd;  // lcm(tiles, pairs) / tiles
+  int64_t slabs = 0, pairs = 0;
+  if (tiles * 2 <= np && even <= 64 && even * BK <= T) {
+    slabs = even;
+    pairs = np;
+  } else if (np / tiles >= 2) {
+    slabs = np / tiles;
+    pairs = tiles * slabs;
+  } else {
+    pairs = args.total < np ? args.total : np;
+  }
+  args.slabs = (int)slabs;
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  if (cudaLaunchKernelEx(&cfg, gemm_wgrad_kernel, ta, tb, to, args) != cudaSuccess) return MTGR_ERR_CUDA;
   return launch_status();
 }
 
