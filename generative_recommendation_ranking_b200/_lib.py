@@ -132,6 +132,8 @@ _SIGNATURES = {
                                             c_i32, c_vp, c_vp, c_vp, c_size, c_vp]),
     "mtgr_gemm": (ctypes.c_int, [c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32,
                                  c_i32, c_vp, c_vp, c_vp]),
+    "mtgr_gemm_wgrad": (ctypes.c_int, [c_i32, c_i32, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i32,
+                                       c_vp, c_vp]),
     "mtgr_timer_create": (c_vp, []),
     "mtgr_timer_destroy": (None, [c_vp]),
     "mtgr_timer_attach": (ctypes.c_int, [c_vp]),
@@ -371,6 +373,14 @@ def mtgr_gemm(d_a, d_b, d_bias, epi, d_resid, q_cols, d_out, d_status, stream=No
     _check("mtgr_gemm", load().mtgr_gemm(
         M, N, K, dtype_code(d_a.dtype), _ptr(d_a), _ptr(d_b), _ptr(d_bias), epi, _ptr(d_resid),
         q_cols, dtype_code(d_out.dtype), _ptr(d_out), _ptr(d_status), _stream(stream)))
+
+
+def mtgr_gemm_wgrad(d_a, d_b, d_out, accumulate, d_status, stream=None):
+    T, M = d_a.shape
+    N = d_b.shape[1]
+    _check("mtgr_gemm_wgrad", load().mtgr_gemm_wgrad(
+        M, N, T, _ptr(d_a), d_a.stride(0), _ptr(d_b), d_b.stride(0), _ptr(d_out),
+        1 if accumulate else 0, _ptr(d_status), _stream(stream)))
 
 
 def mtgr_selftest_bounded_wait(limit_ns: int, d_status, stream=None) -> None:

@@ -263,6 +263,18 @@ def gemm(a: torch.Tensor, b: torch.Tensor, bias=None, epi: int = 0, resid=None, 
     return out
 
 
+def gemm_wgrad(a: torch.Tensor, b: torch.Tensor, out=None, status=None, stream=None) -> torch.Tensor:
+    """out [M, N] fp32 (+)= a^T b; a [T, M] and b [T, N] bf16, token-major.
+    With ``out`` given the sums are added to it, else a zeroed one is made."""
+    acc = out is not None
+    if out is None:
+        out = torch.empty(a.shape[1], b.shape[1], dtype=torch.float32, device=a.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=a.device)
+    _lib.mtgr_gemm_wgrad(a, b, out, acc, status, stream)
+    return out
+
+
 class ContextCache:
     """One user's context tokens (U, S, R) run once through a bf16 stack, with
     every layer's Q|K|V|U kept on the device, so that the user's candidates

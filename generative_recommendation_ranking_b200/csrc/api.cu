@@ -1161,6 +1161,21 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
                         d_status, as_stream(stream));
 }
 
+MTGR_API int mtgr_gemm_wgrad(int32_t M, int32_t N, int64_t T, const void* d_a, int64_t lda,
+                             const void* d_b, int64_t ldb, float* d_out, int32_t accumulate,
+                             int32_t* d_status, mtgr_stream_t stream) {
+  if (M < 0 || N < 0 || T < 0 || d_status == nullptr) return MTGR_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return MTGR_OK;
+  if (d_out == nullptr || (T > 0 && (d_a == nullptr || d_b == nullptr))) return MTGR_ERR_INVALID_ARG;
+  if (lda < M || ldb < N || lda % 8 != 0 || ldb % 8 != 0 || N % 4 != 0) return MTGR_ERR_INVALID_ARG;
+  if (T > INT32_MAX) return MTGR_ERR_INVALID_ARG;
+  if (!aligned16(d_a) || !aligned16(d_b) || !aligned16(d_out)) return MTGR_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return MTGR_ERR_UNSUPPORTED;
+  TimedScope tsc(MTGR_TIMER_BWD_WGRAD, as_stream(stream), 1);
+  return launch_gemm_wgrad(M, N, T, d_a, lda, d_b, ldb, d_out, accumulate != 0, d_status,
+                           as_stream(stream));
+}
+
 // ------------------------------------------------------- host-buffer forward --
 namespace {
 

@@ -539,6 +539,28 @@ MTGR_API int mtgr_gemm(int32_t M, int32_t N, int32_t K, int32_t ab_dtype, const 
                        mtgr_stream_t stream);
 
 /*
+ * Weight-gradient GEMM of the block's backward, exposed for testing: the
+ * gradient of a Linear layer's weight is a sum over tokens of two activation
+ * rows (summary page, "Method": the block's projections, their gradients by
+ * the chain rule),
+ *   out[m][n] (+)= sum_t a[t][m] * b[t][n]
+ * a [T][lda] and b [T][ldb] bf16, token-major as the forward wrote them
+ * (the first M, resp. N, values of each row are used); out [M][N] fp32,
+ * row-major. accumulate == 0 zeroes out first; otherwise the sums are added
+ * to what it holds. Runs on tcgen05 CTA pairs with fp32 reduce-add of
+ * partial tiles, so the summation order over tokens varies from run to run
+ * (results agree to fp32 rounding). lda, ldb: multiples of 8 elements, at
+ * least M, N; N a multiple of 4; pointers 16-byte aligned. The caller owns
+ * every buffer. Returns MTGR_ERR_INVALID_ARG for a bad size, stride,
+ * alignment or a NULL pointer, MTGR_ERR_UNSUPPORTED off sm_100;
+ * MTGR_ERR_TIMEOUT is written to d_status if a wait inside the kernel runs
+ * out. Timer class MTGR_TIMER_BWD_WGRAD.
+ */
+MTGR_API int mtgr_gemm_wgrad(int32_t M, int32_t N, int64_t T, const void* d_a, int64_t lda,
+                             const void* d_b, int64_t ldb, float* d_out, int32_t accumulate,
+                             int32_t* d_status, mtgr_stream_t stream);
+
+/*
  * Kernel timing. A timer attached to the calling host thread makes every
  * entry point bracket its kernels with CUDA events on its stream and count
  * them, per class: MTGR_TIMER_PACK (2 kernels per call), MTGR_TIMER_MASK_META

@@ -90,6 +90,18 @@ def test_host_validation_without_device(lib):
     assert lib.mtgr_stack_fwd_candidates(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
     assert lib.mtgr_candidate_heads(None, None, 0, None, None, None, 0, None) == E
     assert lib.mtgr_stack_fwd_rows(None, 0, None, 0, None, 0, None, None, None, 0, None) == E
+    # weight-gradient GEMM: sizes, strides, alignment and the status word are
+    # checked before any device work (the stand-in addresses are never read)
+    f = 0x100000
+    wg = lib.mtgr_gemm_wgrad
+    assert wg(-1, 32, 64, f, 8, f, 32, f, 0, f, None) == E            # negative M
+    assert wg(64, 32, 64, f, 32, f, 32, f, 0, f, None) == E           # lda < M
+    assert wg(60, 32, 64, f, 60, f, 32, f, 0, f, None) == E           # lda not a multiple of 8
+    assert wg(64, 30, 64, f, 64, f, 32, f, 0, f, None) == E           # N not a multiple of 4
+    assert wg(64, 32, 64, f + 2, 64, f, 32, f, 0, f, None) == E       # unaligned a
+    assert wg(64, 32, 64, f, 64, f, 32, None, 0, f, None) == E        # no output
+    assert wg(64, 32, 64, f, 64, f, 32, f, 0, None, None) == E        # no status word
+    assert wg(0, 32, 64, None, 8, None, 32, None, 0, f, None) == _lib.MTGR_OK  # empty output
 
 
 def _params(d=512, H=8, d_ff=2048, dtype=_lib.MTGR_BF16):
