@@ -320,7 +320,8 @@ def src_sha(name: str) -> str:
 
 KERNEL_SRC = {"attention": "attn_tc.cu", "gemm_qkvu": "gemm_tc.cu", "gemm_mlp1": "gemm_tc.cu",
               "gemm_mlp2": "gemm_tc.cu", "gln": "gln.cu", "pack": "pack_meta.cu",
-              "mask_meta": "pack_meta.cu"}
+              "mask_meta": "pack_meta.cu", "bwd_attention": "attn_bwd_tc.cu",
+              "bwd_wgrad": "gemm_wgrad.cu"}
 
 
 def ncu_traffic(cls: str, workload: str = None):
@@ -1051,7 +1052,9 @@ def run_backward(args, local):
                        "l2": "inputs larger than L2 (fp32 token features and gradient, 1.9 GB)"},
             "step_tflops": total_flop / (ms * 1e-3) / 1e12,
             "roofline": {"bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"],
-                         "unit": k["unit"], "frac": k["frac"], "traffic": None, "kernel": dom,
+                         "unit": k["unit"], "frac": k["frac"],
+                         "traffic": ncu_traffic(dom, wl["name"]) if dom in KERNEL_SRC else None,
+                         "kernel": dom,
                          "peak_source": f"{peak_src} ({tkey if k['bound'] == 'tensor' else 'hbm_gbs'})"},
             "kernels": kernels, "gpu_launches": int(sum(c for _, c in per.values()) / n),
             "clocks": clk}
