@@ -324,10 +324,11 @@ KERNEL_SRC = {"attention": "attn_tc.cu", "gemm_qkvu": "gemm_tc.cu", "gemm_mlp1":
               "bwd_wgrad": "gemm_wgrad.cu"}
 
 
-def ncu_traffic(cls: str, workload: str = None):
+def ncu_traffic(cls: str, workload: str = None, users: int = None):
     """Per-launch DRAM bytes of a kernel class from the committed ncu summary,
     or None when absent, when the kernel source changed since the capture, or
-    when the record is for another workload than `workload`."""
+    when the record is for another workload than `workload` or another user
+    count than `users` (a --users override keeps the workload's name)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -337,6 +338,8 @@ def ncu_traffic(cls: str, workload: str = None):
     if not e or e.get("src_sha") != src_sha(KERNEL_SRC[cls]):
         return None
     if workload is not None and e.get("workload") != workload:
+        return None
+    if users is not None and e.get("users") != users:
         return None
     return e.get("bytes_per_launch")
 
@@ -574,7 +577,7 @@ def run_ours(args, world, rank, local):
                                        "peak_source": f"MUFU tanh 16/clk/SM x {n_sm} SMs x {sm_mhz:.0f} MHz"}
     dom = max((c for c in work if c in kernels), key=lambda c: kernels[c]["share"])
     k = kernels[dom]
-    traffic = ncu_traffic(dom, wl["name"])
+    traffic = ncu_traffic(dom, wl["name"], int(wl["lens"].shape[0]))
     roofline = {"bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"], "unit": k["unit"],
                 "frac": k["frac"], "traffic": traffic, "kernel": dom,
                 "peak_source": f"{peak_src} ({tensor_key if k['bound'] == 'tensor' else 'hbm_gbs'}; "
@@ -1053,7 +1056,7 @@ def run_backward(args, local):
             "step_tflops": total_flop / (ms * 1e-3) / 1e12,
             "roofline": {"bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"],
                          "unit": k["unit"], "frac": k["frac"],
-                         "traffic": ncu_traffic(dom, wl["name"]) if dom in KERNEL_SRC else None,
+                         "traffic": ncu_traffic(dom, wl["name"], B) if dom in KERNEL_SRC else None,
                          "kernel": dom,
                          "peak_source": f"{peak_src} ({tkey if k['bound'] == 'tensor' else 'hbm_gbs'})"},
             "kernels": kernels, "gpu_launches": int(sum(c for _, c in per.values()) / n),

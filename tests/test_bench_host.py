@@ -23,7 +23,7 @@ def _fake_root(tmp_path, src_text, recorded_sha):
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(
         {"attention": {"bytes_per_launch": 12345, "src_sha": recorded_sha,
-                       "workload": "block_bf16_b512_d512"}}))
+                       "workload": "block_bf16_b512_d512", "users": 512}}))
     return str(tmp_path)
 
 
@@ -44,6 +44,9 @@ def test_traffic_only_for_the_captured_workload(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path / "a", text, sha))
     assert bench.ncu_traffic("attention", "block_bf16_b512_d512") == 12345
     assert bench.ncu_traffic("attention", "attn_bf16_b256_d256") is None
+    # a --users override keeps the workload's name: the user count decides
+    assert bench.ncu_traffic("attention", "block_bf16_b512_d512", 512) == 12345
+    assert bench.ncu_traffic("attention", "block_bf16_b512_d512", 128) is None
 
 
 def test_committed_traffic_record_names_a_kernel_class_with_a_source():
@@ -51,7 +54,7 @@ def test_committed_traffic_record_names_a_kernel_class_with_a_source():
         rec = json.load(f)
     for cls, e in rec.items():
         assert cls in bench.KERNEL_SRC, cls
-        assert e["bytes_per_launch"] > 0 and len(e["src_sha"]) == 16
+        assert e["bytes_per_launch"] > 0 and len(e["src_sha"]) == 16 and e["users"] > 0
         assert os.path.exists(os.path.join(ROOT, "profiles", os.path.basename(e["source"])))
 
 
